@@ -1,0 +1,161 @@
+// kernels.h -- host-side launch interface between the C ABI (api.cu) and the
+// kernel files.  Internal to the library.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace kv2d {
+
+// Kernel stages the optional event profiler tells apart.
+enum ProfStage {
+    kProfWinStats = 0,
+    kProfPass1,
+    kProfLseMerge,
+    kProfPass2,
+    kProfChan,
+    kProfSegSelect,
+    kProfBudget,
+    kProfPack,
+    kProfAppend,
+    kProfDecode,
+    kProfStages
+};
+
+// Records a CUDA event pair around one launch when profiling is on
+// (defined in api.cu; a no-op otherwise).
+void prof_begin(cudaStream_t s, int stage);
+void prof_end(cudaStream_t s, int stage);
+
+struct UnitShape {
+    int32_t Hkv, Hq, G, W, GW, GWpad;
+    int32_t S, r, c;
+    float c2;   // softmax scale * log2(e)
+};
+
+// ---- scoring (score.cu)
+struct ScoreLaunch {
+    SeqPlan plan;
+    UnitShape shp;
+    int batch;
+    DenseView dv;
+    const __half* qw;          // [B][Hq][W][d]
+    CUtensorMap qmap;          // 2-D map over qw rows, box 64 x 64
+    CUtensorMap kmap;          // 4-D map over K, box 64 x (128 | 16)
+    int paged;
+    int max_region;            // longest region of the call (tokens)
+    int max_nseg;
+    // workspace
+    float* a;                  // [units][d]
+    float2* part;              // [units][GWpad][nsplit1]
+    int nsplit1, kps1;
+    float* lse2;               // [units][GWpad]
+    float* s;                  // [units][s_stride]
+    int64_t s_stride;
+    int nsplit2, kps2;
+    double* g;                 // [units][g_stride]
+    uint8_t* cidx;             // [units][g_stride][c]
+    int64_t g_stride;
+    uint32_t* status;
+    // debug
+    float* dbg_a;
+    float* dbg_lse;
+    float* dbg_s;
+    double* dbg_g;
+    int64_t dbg_stride;
+};
+cudaError_t launch_scoring(const ScoreLaunch& L, cudaStream_t stream);
+int score_pass1_smem_bytes();
+int score_pass2_smem_bytes(int gwpad);
+
+// ---- selection (select.cu)
+struct SelectLaunch {
+    SeqPlan plan;
+    UnitShape shp;
+    int batch, max_nseg;
+    int64_t bytes[4];          // payload bytes per strategy
+    int32_t order[4];          // strategies by (bytes, id)
+    int all_full;              // beta >= 1
+    const float* s;
+    int64_t s_stride;
+    const double* g;
+    int64_t g_stride;
+    uint8_t* tidx;             // [units][max_nseg][r]
+    double* E;                 // [units][max_nseg][4]
+    uint8_t* hull;             // [units][max_nseg][8]: nv, verts[4]
+    double* eff;               // [units][max_nseg][3]
+    int32_t* dbytes;           // [units][max_nseg][3]
+    uint8_t* strat;            // [units][max_nseg]
+    int32_t* unit_ok;          // [units]
+    // compressed cache
+    uint64_t* desc;            // [units][max_segs]
+    int32_t max_segs;
+    int32_t* n_segs;
+    int64_t* used_bytes;
+    int32_t* comp_end;
+    int64_t arena_stride;
+    uint32_t* status;
+    double* dbg_E;
+    int32_t dbg_seg_stride;
+};
+cudaError_t launch_selection(const SelectLaunch& L, cudaStream_t stream);
+
+// ---- packing (pack.cu)
+struct PackLaunch {
+    SeqPlan plan;
+    UnitShape shp;
+    int batch, max_nseg;
+    DenseView dv;
+    const uint8_t* tidx;
+    const uint8_t* cidx;
+    int64_t g_stride;
+    const uint8_t* strat;
+    const int32_t* unit_ok;
+    const uint64_t* desc;
+    int32_t max_segs;
+    uint8_t* arena;
+    int64_t arena_stride;
+    uint32_t* status;
+};
+cudaError_t launch_pack(const PackLaunch& L, cudaStream_t stream);
+
+// ---- append and decode (decode.cu)
+struct AppendLaunch {
+    int batch, Hkv;
+    DenseView dv;
+    __half* k;
+    __half* v;
+    const __half* k_new;
+    const __half* v_new;
+    int32_t* seq_len;
+    uint32_t* status;
+};
+cudaError_t launch_append(const AppendLaunch& L, cudaStream_t stream);
+
+struct DecodeLaunch {
+    UnitShape shp;
+    int batch;
+    float scale_log2;
+    DenseView dv;
+    const uint8_t* arena;
+    int64_t arena_stride;
+    const uint64_t* desc;
+    int32_t max_segs;
+    const int32_t* n_segs;
+    const int64_t* used_bytes;
+    const int32_t* comp_end;
+    const int32_t* seq_len;
+    const __half* q;
+    __half* out;
+    int nsplit;
+    float* part;               // [units][nsplit][G][d + 2]
+    uint32_t* ticket;          // [units]
+    uint32_t* status;
+};
+cudaError_t launch_decode(const DecodeLaunch& L, cudaStream_t stream);
+int decode_split_count(int units, int64_t max_seq_len, int num_sms);
+
+}  // namespace kv2d

@@ -1,0 +1,130 @@
+// pack.cu -- packed KV format of the compressed segments (sm_100a).
+//
+// MosaicKV ("MosaicKV: Serving Long-Context LLM with Dynamic Two-D KV Cache
+// Compression", Fig. 6: packed KV format and flexible KV encoding) stores the
+// mixed-strategy segments in a packed layout that attention reads directly.
+// The pages give no byte layout; this library uses, per segment, sections
+// zero-padded to 16 bytes:
+//   FULL : K[S][d] | V[S][d]
+//   TOK  : tidx[r] | K[r][d] | V[r][d]
+//   CH   : cidx[S][c] | Kval[S][c] | V[S][d]
+//   BOTH : tidx[r] | cidx[r][c] | Kval[r][c] | V[r][d]
+// with Kval[t][j] = K[t][cidx[t][j]], uint8 indices ascending and tidx
+// segment-relative.  One CTA writes one segment: whole K / V rows move as
+// 16-byte vectors, index and Kval sections as consecutive bytes / halves.
+#include "kernels.h"
+
+namespace kv2d {
+
+namespace {
+
+struct PackArgs {
+    SeqPlan plan;
+    int Hkv, S, r, c, max_nseg;
+    DenseView dv;
+    const uint8_t* tidx;
+    const uint8_t* cidx;
+    int64_t g_stride;
+    const uint8_t* strat;
+    const int32_t* unit_ok;
+    const uint64_t* desc;
+    int32_t max_segs;
+    uint8_t* arena;
+    int64_t arena_stride;
+    uint32_t* status;
+};
+
+__device__ __forceinline__ void copy_rows(const __half* base, const DenseView& dv, int b, int h,
+                                          int t0, const int* toks, int ntok, uint8_t* dst,
+                                          uint32_t* status) {
+    for (int idx = threadIdx.x; idx < ntok * 16; idx += blockDim.x) {
+        const int i = idx >> 4, ch = idx & 15;
+        const __half* row = dense_row(dv, base, b, h, t0 + toks[i], status);
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (row) v = *reinterpret_cast<const uint4*>(row + ch * 8);
+        *reinterpret_cast<uint4*>(dst + i * 256 + ch * 16) = v;
+    }
+}
+
+__global__ void __launch_bounds__(128) pack_kernel(const __grid_constant__ PackArgs A) {
+    const int j = blockIdx.x, u = blockIdx.y;
+    const int b = u / A.Hkv, h = u % A.Hkv;
+    if (j >= A.plan.nseg[b] || !A.unit_ok[u]) return;
+    const int S = A.S, r = A.r, c = A.c;
+    const int64_t slot = static_cast<int64_t>(u) * A.max_nseg + j;
+    const int st = A.strat[slot];
+    const int segbase = A.plan.r0[b] / S;
+    const uint64_t d = A.desc[static_cast<int64_t>(u) * A.max_segs + segbase + j];
+    uint8_t* out = A.arena + static_cast<int64_t>(u) * A.arena_stride +
+                   static_cast<int64_t>(d & 0xffffffffull) * 16;
+    const int t0 = A.plan.r0[b] + j * S;
+    __shared__ int toks[256];
+    const bool sparse_tok = (st == KV2D_TOK || st == KV2D_BOTH);
+    const int ntok = sparse_tok ? r : S;
+    for (int i = threadIdx.x; i < ntok; i += blockDim.x)
+        toks[i] = sparse_tok ? A.tidx[slot * r + i] : i;
+    __syncthreads();
+    int64_t o = 0;
+    if (sparse_tok) {
+        for (int i = threadIdx.x; i < pad16(r); i += blockDim.x)
+            out[i] = (i < r) ? static_cast<uint8_t>(toks[i]) : 0;
+        o = pad16(r);
+    }
+    if (st == KV2D_FULL || st == KV2D_TOK) {
+        copy_rows(A.dv.k, A.dv, b, h, t0, toks, ntok, out + o, A.status);
+        o += static_cast<int64_t>(ntok) * 256;
+    } else {
+        const int n = ntok * c;
+        const uint8_t* cbase = A.cidx + (static_cast<int64_t>(u) * A.g_stride + static_cast<int64_t>(j) * S) * c;
+        for (int i = threadIdx.x; i < pad16(n); i += blockDim.x) {
+            uint8_t val = 0;
+            if (i < n) val = cbase[static_cast<int64_t>(toks[i / c]) * c + i % c];
+            out[o + i] = val;
+        }
+        o += pad16(n);
+        uint16_t* kv = reinterpret_cast<uint16_t*>(out + o);
+        for (int i = threadIdx.x; i < pad16(2 * n) / 2; i += blockDim.x) {
+            uint16_t val = 0;
+            if (i < n) {
+                const int tk = toks[i / c];
+                const int ch = cbase[static_cast<int64_t>(tk) * c + i % c];
+                const __half* row = dense_row(A.dv, A.dv.k, b, h, t0 + tk, A.status);
+                if (row) val = __half_as_ushort(row[ch]);
+            }
+            kv[i] = val;
+        }
+        o += pad16(2 * n);
+    }
+    copy_rows(A.dv.v, A.dv, b, h, t0, toks, ntok, out + o, A.status);
+}
+
+}  // namespace
+
+cudaError_t launch_pack(const PackLaunch& L, cudaStream_t stream) {
+    if (L.max_nseg <= 0) return cudaSuccess;
+    PackArgs a;
+    a.plan = L.plan;
+    a.Hkv = L.shp.Hkv;
+    a.S = L.shp.S;
+    a.r = L.shp.r;
+    a.c = L.shp.c;
+    a.max_nseg = L.max_nseg;
+    a.dv = L.dv;
+    a.tidx = L.tidx;
+    a.cidx = L.cidx;
+    a.g_stride = L.g_stride;
+    a.strat = L.strat;
+    a.unit_ok = L.unit_ok;
+    a.desc = L.desc;
+    a.max_segs = L.max_segs;
+    a.arena = L.arena;
+    a.arena_stride = L.arena_stride;
+    a.status = L.status;
+    dim3 grid(L.max_nseg, L.batch * L.shp.Hkv);
+    prof_begin(stream, kProfPack);
+    pack_kernel<<<grid, 128, 0, stream>>>(a);
+    prof_end(stream, kProfPack);
+    return cudaGetLastError();
+}
+
+}  // namespace kv2d

@@ -1,0 +1,760 @@
+// score.cu -- per-unit scoring of the KV cache (sm_100a).
+//
+// MosaicKV ("MosaicKV: Serving Long-Context LLM with Dynamic Two-D KV Cache
+// Compression", Core claim and Fig. 6 Stage-1) identifies important elements
+// of every KV vector; Kara ("KARA: Efficient Reasoning LLM Serving via
+// Sliding-Window KV Cache Compression", "What carries the argument") scores
+// keys by the attention that all queries of a recent window give them.
+// The kernels here compute, per unit (sequence b, KV head h):
+//   win_stats : a_d = mean_{G*W window rows} |q_d|
+//   pass 1    : lse of every window row over the causal region, from a
+//               tcgen05 product Q_w K^T (M = 128 window rows, N = 128 keys),
+//               split over key ranges -> per-split (max, sum) partials
+//   lse merge : combines the partials in split order
+//   pass 2    : s_t = sum_rows exp(l - lse) from the transposed product
+//               K Q_w^T (M = 128 keys, N = window rows) so that each TMEM lane
+//               owns one key and sums over queries in-thread
+//   chan      : per key: top-c channels of |k_d| a_d and g_t in fp64
+// Both products take their operands from shared memory written by TMA with
+// the 128-byte swizzle; the fp32 accumulators live in tensor memory.
+#include "kernels.h"
+
+namespace kv2d {
+
+namespace {
+
+constexpr int kPassThreads = 320;    // 8 epilogue warps, 1 TMA warp, 1 MMA warp
+constexpr int kStage = 128 * 256;    // one K tile: 128 keys x 128 fp16
+constexpr int kP1Stages = 4;
+constexpr uint32_t kNegInf = 0xff800000u;
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+    return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// Issues the TMA loads of one 128-key tile starting at token t0 into dst
+// (two 16 KB halves of 64 channels; rows in token order).
+__device__ __forceinline__ void load_key_tile(uint8_t* dst, const CUtensorMap* kmap,
+                                              uint64_t* bar, const DenseView& dv, int paged,
+                                              int b, int h, int t0, int T, uint32_t* status) {
+    if (!paged) {
+        tma_load_4d(dst, kmap, bar, 0, t0, h, b);
+        tma_load_4d(dst + 16384, kmap, bar, 64, t0, h, b);
+        return;
+    }
+    for (int j = 0; j < 8; ++j) {
+        int t = t0 + 16 * j;
+        int lb = t / dv.block_size;
+        int phys = -1;
+        if (lb < dv.max_blocks) phys = dv.block_table[static_cast<int64_t>(b) * dv.max_blocks + lb];
+        if (phys < 0 || phys >= dv.num_blocks) {
+            if (t < T) set_status(status, KV2D_DEV_BLOCK_TABLE);
+            phys = 0;
+        }
+        int row = t % dv.block_size;
+        tma_load_4d(dst + j * 2048, kmap, bar, 0, row, h, phys);
+        tma_load_4d(dst + 16384 + j * 2048, kmap, bar, 64, row, h, phys);
+    }
+}
+
+// ------------------------------------------------------------ win_stats
+
+__global__ void win_stats_kernel(const __half* __restrict__ qw, int Hq, int G, int W, int Hkv,
+                                 float* __restrict__ a, float* __restrict__ dbg_a) {
+    const int u = blockIdx.x;
+    const int b = u / Hkv, h = u % Hkv;
+    const int x = threadIdx.x;
+    const int rows = G * W;
+    const __half* base = qw + (static_cast<int64_t>(b) * Hq + static_cast<int64_t>(h) * G) * W *
+                                  kHeadDim;
+    float acc = 0.f;
+    for (int row = 0; row < rows; ++row)
+        acc += fabsf(__half2float(base[static_cast<int64_t>(row) * kHeadDim + x]));
+    float v = acc / static_cast<float>(rows);
+    a[static_cast<int64_t>(u) * kHeadDim + x] = v;
+    if (dbg_a) dbg_a[static_cast<int64_t>(u) * kHeadDim + x] = v;
+}
+
+// --------------------------------------------------------------- pass 1
+
+struct Pass1Args {
+    SeqPlan plan;
+    UnitShape shp;
+    DenseView dv;
+    int paged;
+    int kps, nsplit;
+    float2* part;
+    uint32_t* status;
+};
+
+__global__ void __launch_bounds__(kPassThreads, 1)
+    score_pass1_kernel(const __grid_constant__ CUtensorMap qmap,
+                       const __grid_constant__ CUtensorMap kmap, const __grid_constant__ Pass1Args A) {
+    const int sp = blockIdx.x, mt = blockIdx.y, u = blockIdx.z;
+    const int Hkv = A.shp.Hkv, W = A.shp.W, GW = A.shp.GW, GWpad = A.shp.GWpad;
+    const int b = u / Hkv, h = u % Hkv;
+    const int T = A.plan.T[b], r0 = A.plan.r0[b];
+    const int k_lo = r0 + sp * A.kps;
+    const int k_hi = min(T, k_lo + A.kps);
+    const int nt = k_hi > k_lo ? (k_hi - k_lo + kKeyTile - 1) / kKeyTile : 0;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    if (nt == 0) {
+        if (tid < 128) {
+            int rho = mt * 128 + tid;
+            if (rho < GW)
+                A.part[(static_cast<int64_t>(u) * GWpad + rho) * A.nsplit + sp] =
+                    make_float2(__uint_as_float(kNegInf), 0.f);
+        }
+        return;
+    }
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = align1024(smem_raw);
+    uint8_t* q_s = smem;                                   // 32 KB
+    uint8_t* k_s = smem + 32768;                           // stages
+    uint64_t* full = reinterpret_cast<uint64_t*>(k_s + kP1Stages * kStage);
+    uint64_t* empty = full + kP1Stages;
+    uint64_t* tfull = empty + kP1Stages;
+    uint64_t* tempty = tfull + 2;
+    uint64_t* qbar = tempty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(qbar + 1);
+    float* xm = reinterpret_cast<float*>(tmem_slot + 4);
+    float* xl = xm + 128;
+
+    if (tid == 0) {
+        for (int i = 0; i < kP1Stages; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&tfull[i], 1);
+            mbar_init(&tempty[i], 128);
+        }
+        mbar_init(qbar, 1);
+        mbar_fence_init();
+    }
+    if (warp == 9) {
+        tmem_alloc(tmem_slot, 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 8) {
+        if (lane == 0) {
+            tma_prefetch_desc(&qmap);
+            tma_prefetch_desc(&kmap);
+            const int qrow0 = (b * A.shp.Hq + h * A.shp.G) * W + mt * 128;
+            mbar_expect_tx(qbar, 32768);
+            for (int hf = 0; hf < 2; ++hf)
+                for (int rb = 0; rb < 2; ++rb)
+                    tma_load_2d(q_s + hf * 16384 + rb * 8192, &qmap, qbar, hf * 64, qrow0 + rb * 64);
+            for (int i = 0; i < nt; ++i) {
+                const int s = i % kP1Stages;
+                if (i >= kP1Stages && !mbar_wait(&empty[s], ((i / kP1Stages) - 1) & 1, A.status))
+                    break;
+                mbar_expect_tx(&full[s], kStage);
+                load_key_tile(k_s + s * kStage, &kmap, &full[s], A.dv, A.paged, b, h,
+                              k_lo + i * kKeyTile, T, A.status);
+            }
+        }
+    } else if (warp == 9) {
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_f16_f32(128, 128);
+            const uint32_t qa = smem_u32(q_s);
+            bool ok = mbar_wait(qbar, 0, A.status);
+            for (int i = 0; ok && i < nt; ++i) {
+                const int s = i % kP1Stages, buf = i & 1;
+                if (!mbar_wait(&full[s], (i / kP1Stages) & 1, A.status)) break;
+                if (i >= 2 && !mbar_wait(&tempty[buf], ((i >> 1) - 1) & 1, A.status)) break;
+                tc_fence_after();
+                const uint32_t ka = smem_u32(k_s + s * kStage);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                    umma_f16(tmem + buf * 128, sw128_kmajor_desc(qa + off),
+                             sw128_kmajor_desc(ka + off), idesc, kk > 0 ? 1u : 0u);
+                }
+                umma_commit(&empty[s]);
+                umma_commit(&tfull[buf]);
+            }
+        }
+    } else {
+        // epilogue: warps 0-3 take even tiles (TMEM columns 0..127), warps
+        // 4-7 odd tiles (columns 128..255); thread <-> window row.
+        const int wg = warp >> 2, lg = warp & 3;
+        const int row = lg * 32 + lane;
+        const int rho = mt * 128 + row;
+        const int pw = (rho < GW) ? (T - W + (rho % W)) : -1;   // last key the row sees
+        const int lim = min(pw, k_hi - 1);
+        const float c2 = A.shp.c2;
+        float m = __uint_as_float(kNegInf), l = 0.f;
+        for (int i = wg; i < nt; i += 2) {
+            if (!mbar_wait(&tfull[wg], (i >> 1) & 1, A.status)) break;
+            tc_fence_after();
+            const int t_base = k_lo + i * kKeyTile;
+            const uint32_t taddr = tmem + (static_cast<uint32_t>(lg * 32) << 16) + wg * 128;
+            const bool whole = (t_base + kKeyTile - 1 <= lim);
+#pragma unroll 1
+            for (int half = 0; half < 2; ++half) {
+                uint32_t ra[32], rb[32];
+                tmem_ld32(taddr + half * 64, ra);
+                tmem_ld32(taddr + half * 64 + 32, rb);
+                tmem_ld_wait();
+                float x[64];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    x[j] = __uint_as_float(ra[j]) * c2;
+                    x[32 + j] = __uint_as_float(rb[j]) * c2;
+                }
+                if (!whole) {
+                    const int t0 = t_base + half * 64;
+#pragma unroll
+                    for (int j = 0; j < 64; ++j)
+                        if (t0 + j > lim) x[j] = __uint_as_float(kNegInf);
+                }
+                float mx = x[0];
+#pragma unroll
+                for (int j = 1; j < 64; ++j) mx = fmaxf(mx, x[j]);
+                if (mx > m) {
+                    l = (l == 0.f) ? 0.f : l * fast_exp2(m - mx);
+                    m = mx;
+                }
+                if (m != __uint_as_float(kNegInf)) {
+                    float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+                    for (int j = 0; j < 64; j += 2) {
+                        acc0 += fast_exp2(x[j] - m);
+                        acc1 += fast_exp2(x[j + 1] - m);
+                    }
+                    l += acc0 + acc1;
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&tempty[wg]);
+        }
+        if (wg == 1) {
+            xm[row] = m;
+            xl[row] = l;
+        }
+        named_bar_sync(1, 256);
+        if (wg == 0 && rho < GW) {
+            const float m1 = xm[row], l1 = xl[row];
+            const float M = fmaxf(m, m1);
+            float L = 0.f;
+            if (M != __uint_as_float(kNegInf)) {
+                if (l > 0.f) L += l * fast_exp2(m - M);
+                if (l1 > 0.f) L += l1 * fast_exp2(m1 - M);
+            }
+            A.part[(static_cast<int64_t>(u) * GWpad + rho) * A.nsplit + sp] = make_float2(M, L);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 9) tmem_dealloc(tmem, 256);
+}
+
+// ------------------------------------------------------------ lse merge
+
+__global__ void lse_merge_kernel(const float2* __restrict__ part, int nsplit, int GW, int GWpad,
+                                 int Hkv, int Hq, int G, int W, float* __restrict__ lse2,
+                                 float* __restrict__ dbg_lse) {
+    const int u = blockIdx.x;
+    const int rho = threadIdx.x;
+    if (rho >= GWpad) return;
+    float out = __int_as_float(0x7f800000);   // +inf: padded rows weigh nothing
+    if (rho < GW) {
+        const float2* p = part + (static_cast<int64_t>(u) * GWpad + rho) * nsplit;
+        float M = __uint_as_float(kNegInf);
+        for (int s = 0; s < nsplit; ++s) M = fmaxf(M, p[s].x);
+        float L = 0.f;
+        for (int s = 0; s < nsplit; ++s)
+            if (p[s].y > 0.f) L += p[s].y * exp2f(p[s].x - M);
+        out = M + log2f(L);
+        if (dbg_lse) {
+            const int b = u / Hkv, h = u % Hkv;
+            const int g = rho / W, i = rho % W;
+            dbg_lse[(static_cast<int64_t>(b) * Hq + h * G + g) * W + i] =
+                out * 0.69314718055994531f;
+        }
+    }
+    lse2[static_cast<int64_t>(u) * GWpad + rho] = out;
+}
+
+// --------------------------------------------------------------- pass 2
+
+struct Pass2Args {
+    SeqPlan plan;
+    UnitShape shp;
+    DenseView dv;
+    int paged;
+    int kps, nstages, nqc, Nc;
+    const float* lse2;
+    float* s;
+    int64_t s_stride;
+    float* dbg_s;
+    int64_t dbg_stride;
+    uint32_t* status;
+};
+
+__global__ void __launch_bounds__(kPassThreads, 1)
+    score_pass2_kernel(const __grid_constant__ CUtensorMap qmap,
+                       const __grid_constant__ CUtensorMap kmap, const __grid_constant__ Pass2Args A) {
+    const int sp = blockIdx.x, u = blockIdx.y;
+    const int Hkv = A.shp.Hkv, W = A.shp.W, GWpad = A.shp.GWpad;
+    const int b = u / Hkv, h = u % Hkv;
+    const int T = A.plan.T[b], r0 = A.plan.r0[b];
+    const int r_end = r0 + A.plan.nseg[b] * A.shp.S;
+    const int k_lo = r0 + sp * A.kps;
+    const int k_hi = min(r_end, k_lo + A.kps);
+    const int nt = k_hi > k_lo ? (k_hi - k_lo + kKeyTile - 1) / kKeyTile : 0;
+    if (nt == 0) return;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int NS = A.nstages, nqc = A.nqc, Nc = A.Nc;
+    const bool split_cols = (nqc == 2);          // both WGs on every tile
+    const uint32_t ncols = split_cols ? 512u : (Nc == 256 ? 512u : 256u);
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = align1024(smem_raw);
+    uint8_t* q_s = smem;                                  // GWpad x 256 B
+    uint8_t* k_s = smem + GWpad * 256;
+    float* lse_s = reinterpret_cast<float*>(k_s + NS * kStage);
+    int* wpos_s = reinterpret_cast<int*>(lse_s + GWpad);
+    float* sb = reinterpret_cast<float*>(wpos_s + GWpad);
+    uint64_t* full = reinterpret_cast<uint64_t*>(sb + 128);
+    uint64_t* empty = full + 4;
+    uint64_t* tfull = empty + 4;
+    uint64_t* tempty = tfull + 2;
+    uint64_t* qbar = tempty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(qbar + 1);
+
+    for (int i = tid; i < GWpad; i += kPassThreads) {
+        lse_s[i] = A.lse2[static_cast<int64_t>(u) * GWpad + i];
+        wpos_s[i] = i % W;
+    }
+    if (tid == 0) {
+        for (int i = 0; i < NS; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&tfull[i], 1);
+            mbar_init(&tempty[i], split_cols ? 256 : 128);
+        }
+        mbar_init(qbar, 1);
+        mbar_fence_init();
+    }
+    if (warp == 9) {
+        tmem_alloc(tmem_slot, ncols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 8) {
+        if (lane == 0) {
+            tma_prefetch_desc(&qmap);
+            tma_prefetch_desc(&kmap);
+            const int qrow0 = (b * A.shp.Hq + h * A.shp.G) * W;
+            mbar_expect_tx(qbar, GWpad * 256);
+            for (int qc = 0; qc < nqc; ++qc)
+                for (int hf = 0; hf < 2; ++hf)
+                    for (int rb = 0; rb < Nc / 64; ++rb)
+                        tma_load_2d(q_s + qc * Nc * 256 + hf * Nc * 128 + rb * 8192, &qmap, qbar,
+                                    hf * 64, qrow0 + qc * Nc + rb * 64);
+            for (int i = 0; i < nt; ++i) {
+                const int s = i % NS;
+                if (i >= NS && !mbar_wait(&empty[s], ((i / NS) - 1) & 1, A.status)) break;
+                mbar_expect_tx(&full[s], kStage);
+                load_key_tile(k_s + s * kStage, &kmap, &full[s], A.dv, A.paged, b, h,
+                              k_lo + i * kKeyTile, T, A.status);
+            }
+        }
+    } else if (warp == 9) {
+        if (lane == 0) {
+            const uint32_t idesc = idesc_f16_f32(128, Nc);
+            const uint32_t qa = smem_u32(q_s);
+            bool ok = mbar_wait(qbar, 0, A.status);
+            for (int i = 0; ok && i < nt; ++i) {
+                const int s = i % NS;
+                const int buf = split_cols ? 0 : (i & 1);
+                if (!mbar_wait(&full[s], (i / NS) & 1, A.status)) break;
+                if (split_cols) {
+                    if (i >= 1 && !mbar_wait(&tempty[0], (i - 1) & 1, A.status)) break;
+                } else if (i >= 2 && !mbar_wait(&tempty[buf], ((i >> 1) - 1) & 1, A.status)) {
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t ka = smem_u32(k_s + s * kStage);
+                for (int qc = 0; qc < nqc; ++qc) {
+                    const uint32_t dcol = split_cols ? qc * Nc : buf * Nc;
+                    const uint32_t qb = qa + qc * Nc * 256;
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint32_t aoff = (kk >> 2) * 16384 + (kk & 3) * 32;
+                        const uint32_t boff = (kk >> 2) * (Nc * 128) + (kk & 3) * 32;
+                        umma_f16(tmem + dcol, sw128_kmajor_desc(ka + aoff),
+                                 sw128_kmajor_desc(qb + boff), idesc, kk > 0 ? 1u : 0u);
+                    }
+                }
+                umma_commit(&empty[s]);
+                umma_commit(&tfull[buf]);
+            }
+        }
+    } else {
+        // epilogue: thread <-> key (TMEM lane), loop over query columns.
+        const int wg = warp >> 2, lg = warp & 3;
+        const int row = lg * 32 + lane;
+        const float c2 = A.shp.c2;
+        const int tw = T - W;                 // keys <= tw are seen by every row
+        const int step = split_cols ? 1 : 2;
+        for (int i = split_cols ? 0 : wg; i < nt; i += step) {
+            const int buf = split_cols ? 0 : wg;
+            const int k = split_cols ? i : (i >> 1);
+            if (!mbar_wait(&tfull[buf], k & 1, A.status)) break;
+            tc_fence_after();
+            const int t = k_lo + i * kKeyTile + row;
+            const int qc = split_cols ? wg : 0;
+            const uint32_t taddr = tmem + (static_cast<uint32_t>(lg * 32) << 16) +
+                                   (split_cols ? qc * Nc : buf * Nc);
+            const int col0 = qc * Nc;
+            const int need = t - tw;          // row visible iff wpos >= need
+            float sacc = 0.f;
+#pragma unroll 1
+            for (int cc = 0; cc < Nc; cc += 64) {
+                uint32_t ra[32], rb[32];
+                tmem_ld32(taddr + cc, ra);
+                const bool two = (cc + 32 < Nc);
+                if (two) tmem_ld32(taddr + cc + 32, rb);
+                tmem_ld_wait();
+                const float4* l4 = reinterpret_cast<const float4*>(lse_s + col0 + cc);
+                float a0 = 0.f, a1 = 0.f;
+                if (need <= 0) {
+#pragma unroll
+                    for (int j = 0; j < 32; j += 4) {
+                        const float4 lz = l4[j >> 2];
+                        a0 += fast_exp2(__uint_as_float(ra[j]) * c2 - lz.x);
+                        a1 += fast_exp2(__uint_as_float(ra[j + 1]) * c2 - lz.y);
+                        a0 += fast_exp2(__uint_as_float(ra[j + 2]) * c2 - lz.z);
+                        a1 += fast_exp2(__uint_as_float(ra[j + 3]) * c2 - lz.w);
+                    }
+                    if (two) {
+#pragma unroll
+                        for (int j = 0; j < 32; j += 4) {
+                            const float4 lz = l4[(32 + j) >> 2];
+                            a0 += fast_exp2(__uint_as_float(rb[j]) * c2 - lz.x);
+                            a1 += fast_exp2(__uint_as_float(rb[j + 1]) * c2 - lz.y);
+                            a0 += fast_exp2(__uint_as_float(rb[j + 2]) * c2 - lz.z);
+                            a1 += fast_exp2(__uint_as_float(rb[j + 3]) * c2 - lz.w);
+                        }
+                    }
+                } else {
+                    const int* wp = wpos_s + col0 + cc;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const float e = fast_exp2(__uint_as_float(ra[j]) * c2 - lse_s[col0 + cc + j]);
+                        a0 += (wp[j] >= need) ? e : 0.f;
+                    }
+                    if (two) {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            const float e =
+                                fast_exp2(__uint_as_float(rb[j]) * c2 - lse_s[col0 + cc + 32 + j]);
+                            a1 += (wp[32 + j] >= need) ? e : 0.f;
+                        }
+                    }
+                }
+                sacc += a0 + a1;
+            }
+            tc_fence_before();
+            if (split_cols) {
+                if (wg == 1) sb[row] = sacc;
+                named_bar_sync(1, 256);
+                if (wg == 0) sacc = sacc + sb[row];
+                named_bar_sync(2, 256);
+            }
+            mbar_arrive(&tempty[buf]);
+            if ((!split_cols || wg == 0) && t < k_hi) {
+                const int64_t rel = t - r0;
+                A.s[static_cast<int64_t>(u) * A.s_stride + rel] = sacc;
+                if (A.dbg_s) A.dbg_s[static_cast<int64_t>(u) * A.dbg_stride + rel] = sacc;
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 9) tmem_dealloc(tmem, ncols);
+}
+
+// ------------------------------------------------- channel top-c and g_t
+
+// Bitonic sort of 128 keys into descending order, fully unrolled so that
+// every index is a compile-time constant and the array stays in registers.
+__device__ __forceinline__ void sort128_desc(uint32_t (&v)[128]) {
+#pragma unroll
+    for (int k = 2; k <= 128; k <<= 1) {
+#pragma unroll
+        for (int j = k >> 1; j > 0; j >>= 1) {
+#pragma unroll
+            for (int i = 0; i < 128; ++i) {
+                const int l = i ^ j;
+                if (l > i) {
+                    const uint32_t a = v[i], c = v[l];
+                    const uint32_t hi = max(a, c), lo = min(a, c);
+                    if ((i & k) == 0) {
+                        v[i] = hi;
+                        v[l] = lo;
+                    } else {
+                        v[i] = lo;
+                        v[l] = hi;
+                    }
+                }
+            }
+        }
+    }
+}
+
+struct ChanArgs {
+    SeqPlan plan;
+    int Hkv, S, c;
+    DenseView dv;
+    const float* a;
+    double* g;
+    uint8_t* cidx;
+    int64_t g_stride;
+    double* dbg_g;
+    int64_t dbg_stride;
+    uint32_t* status;
+};
+
+// One thread per key.  The block's 128 key rows sit in shared memory with
+// their 16-byte chunks XOR-swizzled by (row & 7), so that 8 consecutive
+// threads reading the same logical chunk hit 8 different bank groups.
+//
+// Selection: f_x = fp32(|k_x| * a_x) is the correctly rounded value of the
+// exact product e_x = |k_x| * a_x, so it is monotone in e_x.  Sorting the
+// 32-bit keys (f_x with its low 7 bits replaced by 127 - x) gives the order
+// (trunc(f) desc, x asc).  Let v be the truncated value of the c-th key:
+// channels above v are in, channels below are out, and channels equal to v
+// are ranked exactly by (e desc, x asc) in fp64 when they straddle the cut.
+__global__ void __launch_bounds__(128) chan_kernel(const __grid_constant__ ChanArgs A) {
+    const int u = blockIdx.y;
+    const int b = u / A.Hkv, h = u % A.Hkv;
+    const int r0 = A.plan.r0[b];
+    const int ntok = A.plan.nseg[b] * A.S;
+    const int base = blockIdx.x * 128;
+    if (base >= ntok) return;
+    __shared__ __align__(16) uint8_t rows[128 * 256];
+    __shared__ float as[128];
+    const int tid = threadIdx.x;
+    as[tid] = A.a[static_cast<int64_t>(u) * kHeadDim + tid];
+    for (int idx = tid; idx < 128 * 16; idx += 128) {
+        const int rr = idx >> 4, ch = idx & 15;
+        uint4 val = make_uint4(0, 0, 0, 0);
+        if (base + rr < ntok) {
+            const __half* src = dense_row(A.dv, A.dv.k, b, h, r0 + base + rr, A.status);
+            if (src) val = *reinterpret_cast<const uint4*>(src + ch * 8);
+        }
+        *reinterpret_cast<uint4*>(rows + rr * 256 + ((ch ^ (rr & 7)) << 4)) = val;
+    }
+    __syncthreads();
+    const int t = base + tid;
+    if (t >= ntok) return;
+    const uint8_t* myrow = rows + tid * 256;
+    const int sw = tid & 7;
+    const int c = A.c;
+
+    uint32_t key[128];
+#pragma unroll
+    for (int ch = 0; ch < 16; ++ch) {
+        const uint4 q = *reinterpret_cast<const uint4*>(myrow + ((ch ^ sw) << 4));
+        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int x = ch * 8 + e * 2 + hh;
+                const uint16_t hb = static_cast<uint16_t>(hh ? (w[e] >> 16) : (w[e] & 0xffff));
+                const float mag = fabsf(__half2float(__ushort_as_half(hb)));
+                const float f = __fmul_rn(mag, as[x]);
+                key[x] = (__float_as_uint(f) & 0xFFFFFF80u) | static_cast<uint32_t>(127 - x);
+            }
+        }
+    }
+    sort128_desc(key);
+    uint32_t kc = 0;
+#pragma unroll
+    for (int i = 0; i < 128; ++i)
+        if (i == c - 1) kc = key[i];
+    const uint32_t v = kc >> 7;
+    int n_gt = 0, n_eq = 0;
+    uint32_t m0 = 0, m1 = 0, m2 = 0, m3 = 0;
+#pragma unroll
+    for (int i = 0; i < 128; ++i) {
+        const uint32_t tv = key[i] >> 7;
+        n_gt += (tv > v);
+        n_eq += (tv == v);
+        if (i < c) {
+            const int x = 127 - static_cast<int>(key[i] & 127u);
+            const uint32_t bit = 1u << (x & 31);
+            m0 |= (x >> 5) == 0 ? bit : 0u;
+            m1 |= (x >> 5) == 1 ? bit : 0u;
+            m2 |= (x >> 5) == 2 ? bit : 0u;
+            m3 |= (x >> 5) == 3 ? bit : 0u;
+        }
+    }
+    auto elem = [&](int x) -> float {
+        const int ch = x >> 3, within = x & 7;
+        const uint16_t hb = *reinterpret_cast<const uint16_t*>(myrow + ((ch ^ sw) << 4) + within * 2);
+        return fabsf(__half2float(__ushort_as_half(hb)));
+    };
+    if (n_gt + n_eq > c) {
+        // exact ranking of the channels whose truncated key equals v
+        const int need = c - n_gt;
+        for (int x = 0; x < 128; ++x) {
+            const float f = __fmul_rn(elem(x), as[x]);
+            if ((__float_as_uint(f) >> 7) != v) continue;
+            const double ex = __dmul_rn(static_cast<double>(elem(x)), static_cast<double>(as[x]));
+            int rank = 0;
+            for (int y = 0; y < 128; ++y) {
+                if (y == x) continue;
+                const float fy = __fmul_rn(elem(y), as[y]);
+                if ((__float_as_uint(fy) >> 7) != v) continue;
+                const double ey =
+                    __dmul_rn(static_cast<double>(elem(y)), static_cast<double>(as[y]));
+                rank += (ey > ex) || (ey == ex && y < x);
+            }
+            const uint32_t bit = 1u << (x & 31);
+            const uint32_t set = rank < need ? bit : 0u;
+            const int w = x >> 5;
+            if (w == 0) m0 = (m0 & ~bit) | set;
+            else if (w == 1) m1 = (m1 & ~bit) | set;
+            else if (w == 2) m2 = (m2 & ~bit) | set;
+            else m3 = (m3 & ~bit) | set;
+        }
+    }
+    const int64_t slot = static_cast<int64_t>(u) * A.g_stride + t;
+    uint8_t* out = A.cidx + slot * c;
+    int k = 0;
+    double tot = 0.0, drop = 0.0;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+        const uint32_t mw = (w == 0) ? m0 : (w == 1) ? m1 : (w == 2) ? m2 : m3;
+#pragma unroll 4
+        for (int bit = 0; bit < 32; ++bit) {
+            const int x = w * 32 + bit;
+            const double e = __dmul_rn(static_cast<double>(elem(x)), static_cast<double>(as[x]));
+            tot = __dadd_rn(tot, e);
+            if ((mw >> bit) & 1u) out[k++] = static_cast<uint8_t>(x);
+            else drop = __dadd_rn(drop, e);
+        }
+    }
+    const double gv = tot > 0.0 ? __ddiv_rn(drop, tot) : 0.0;
+    A.g[slot] = gv;
+    if (A.dbg_g) A.dbg_g[static_cast<int64_t>(u) * A.dbg_stride + t] = gv;
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------ host
+
+int score_pass1_smem_bytes() {
+    return 1024 + 32768 + kP1Stages * kStage + 256 + 1024;
+}
+
+int score_pass2_smem_bytes(int gwpad) {
+    const int ns = gwpad <= 256 ? 4 : 2;
+    return 1024 + gwpad * 256 + ns * kStage + gwpad * 8 + 512 + 256;
+}
+
+cudaError_t launch_scoring(const ScoreLaunch& L, cudaStream_t stream) {
+    const int units = L.batch * L.shp.Hkv;
+    prof_begin(stream, kProfWinStats);
+    win_stats_kernel<<<units, kHeadDim, 0, stream>>>(L.qw, L.shp.Hq, L.shp.G, L.shp.W, L.shp.Hkv,
+                                                      L.a, L.dbg_a);
+    prof_end(stream, kProfWinStats);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+
+    Pass1Args p1;
+    p1.plan = L.plan;
+    p1.shp = L.shp;
+    p1.dv = L.dv;
+    p1.paged = L.paged;
+    p1.kps = L.kps1;
+    p1.nsplit = L.nsplit1;
+    p1.part = L.part;
+    p1.status = L.status;
+    const int smem1 = score_pass1_smem_bytes();
+    e = cudaFuncSetAttribute(score_pass1_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem1);
+    if (e != cudaSuccess) return e;
+    dim3 g1(L.nsplit1, L.shp.GWpad / 128, units);
+    prof_begin(stream, kProfPass1);
+    score_pass1_kernel<<<g1, kPassThreads, smem1, stream>>>(L.qmap, L.kmap, p1);
+    prof_end(stream, kProfPass1);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+
+    prof_begin(stream, kProfLseMerge);
+    lse_merge_kernel<<<units, L.shp.GWpad, 0, stream>>>(L.part, L.nsplit1, L.shp.GW, L.shp.GWpad,
+                                                         L.shp.Hkv, L.shp.Hq, L.shp.G, L.shp.W,
+                                                         L.lse2, L.dbg_lse);
+    prof_end(stream, kProfLseMerge);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+
+    Pass2Args p2;
+    p2.plan = L.plan;
+    p2.shp = L.shp;
+    p2.dv = L.dv;
+    p2.paged = L.paged;
+    p2.kps = L.kps2;
+    p2.nstages = L.shp.GWpad <= 256 ? 4 : 2;
+    p2.nqc = L.shp.GWpad <= 256 ? 1 : 2;
+    p2.Nc = L.shp.GWpad / p2.nqc;
+    p2.lse2 = L.lse2;
+    p2.s = L.s;
+    p2.s_stride = L.s_stride;
+    p2.dbg_s = L.dbg_s;
+    p2.dbg_stride = L.dbg_stride;
+    p2.status = L.status;
+    const int smem2 = score_pass2_smem_bytes(L.shp.GWpad);
+    e = cudaFuncSetAttribute(score_pass2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem2);
+    if (e != cudaSuccess) return e;
+    dim3 g2(L.nsplit2, units);
+    prof_begin(stream, kProfPass2);
+    score_pass2_kernel<<<g2, kPassThreads, smem2, stream>>>(L.qmap, L.kmap, p2);
+    prof_end(stream, kProfPass2);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+
+    ChanArgs ca;
+    ca.plan = L.plan;
+    ca.Hkv = L.shp.Hkv;
+    ca.S = L.shp.S;
+    ca.c = L.shp.c;
+    ca.dv = L.dv;
+    ca.a = L.a;
+    ca.g = L.g;
+    ca.cidx = L.cidx;
+    ca.g_stride = L.g_stride;
+    ca.dbg_g = L.dbg_g;
+    ca.dbg_stride = L.dbg_stride;
+    ca.status = L.status;
+    dim3 gc((L.max_nseg * L.shp.S + 127) / 128, units);
+    if (gc.x > 0) {
+        prof_begin(stream, kProfChan);
+        chan_kernel<<<gc, 128, 0, stream>>>(ca);
+        prof_end(stream, kProfChan);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace kv2d

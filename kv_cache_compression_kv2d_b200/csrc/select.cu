@@ -1,0 +1,407 @@
+// select.cu -- per-segment strategy generation under a byte budget (sm_100a).
+//
+// MosaicKV ("MosaicKV: Serving Long-Context LLM with Dynamic Two-D KV Cache
+// Compression", Fig. 5: segment partitioning and compression-strategy
+// generation) chooses one compression pattern per KV-cache segment.  The
+// pages define no criterion; this library reads it as minimising lost
+// attention mass under a byte budget:
+//   seg_select (one warp per segment):
+//     R_j = top-r tokens by s_t (ties to the lower token), ascending;
+//     E_FULL = 0, E_TOK = sum_{t not in R} s_t, E_CH = sum_t s_t g_t,
+//     E_BOTH = E_TOK + sum_{t in R} s_t g_t        (fp64, ascending t);
+//     lower convex hull of (bytes, E) over the four strategies.
+//   budget (one CTA per unit):
+//     starts every segment at its cheapest hull point and applies hull steps
+//     in (efficiency desc, segment asc, step asc) order while they fit the
+//     budget, stopping at the first that does not.  The stopping step is
+//     found exactly with a byte-weighted radix select over the 96-bit keys
+//     (~bits(eff), 4 * segment + step); then per-segment strategies, payload
+//     offsets (block scan) and descriptors are written.
+// Every fp64 sum, product and quotient uses the _rn intrinsics so that no
+// multiply-add is fused and the results are bit-identical to the same
+// operations done one at a time in IEEE double precision.
+#include "kernels.h"
+
+namespace kv2d {
+
+namespace {
+
+constexpr int kSegWarps = 8;
+
+struct SegArgs {
+    SeqPlan plan;
+    int Hkv, S, r, max_nseg;
+    int64_t bytes[4];
+    int32_t order[4];
+    const float* s;
+    int64_t s_stride;
+    const double* g;
+    int64_t g_stride;
+    uint8_t* tidx;
+    double* E;
+    uint8_t* hull;
+    double* eff;
+    int32_t* dbytes;
+    double* dbg_E;
+    int32_t dbg_seg_stride;
+};
+
+__global__ void __launch_bounds__(kSegWarps * 32) seg_select_kernel(const __grid_constant__ SegArgs A) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int u = blockIdx.y;
+    const int b = u / A.Hkv;
+    const int j = blockIdx.x * kSegWarps + warp;
+    if (j >= A.plan.nseg[b]) return;
+    __shared__ float ss[kSegWarps][256];
+    __shared__ double gs[kSegWarps][256];
+    __shared__ uint8_t kept[kSegWarps][256];
+    const int S = A.S, r = A.r;
+    const int64_t t0 = static_cast<int64_t>(j) * S;
+    for (int t = lane; t < S; t += 32) {
+        ss[warp][t] = A.s[static_cast<int64_t>(u) * A.s_stride + t0 + t];
+        gs[warp][t] = A.g[static_cast<int64_t>(u) * A.g_stride + t0 + t];
+    }
+    __syncwarp();
+    const int64_t slot = static_cast<int64_t>(u) * A.max_nseg + j;
+    int before = 0;
+    for (int tb = 0; tb < S; tb += 32) {
+        const int t = tb + lane;
+        bool kp = false;
+        if (t < S) {
+            const float v = ss[warp][t];
+            int rank = 0;
+            for (int t2 = 0; t2 < S; ++t2) {
+                const float v2 = ss[warp][t2];
+                rank += (v2 > v) || (v2 == v && t2 < t);
+            }
+            kp = rank < r;
+            kept[warp][t] = kp ? 1 : 0;
+        }
+        const uint32_t bal = __ballot_sync(0xffffffffu, kp);
+        if (kp) {
+            const int pos = before + __popc(bal & ((1u << lane) - 1u));
+            A.tidx[slot * r + pos] = static_cast<uint8_t>(t);
+        }
+        before += __popc(bal);
+    }
+    __syncwarp();
+    if (lane != 0) return;
+
+    double etok = 0.0, ech = 0.0, ekept = 0.0;
+    for (int t = 0; t < S; ++t)
+        if (!kept[warp][t]) etok = __dadd_rn(etok, static_cast<double>(ss[warp][t]));
+    for (int t = 0; t < S; ++t)
+        ech = __dadd_rn(ech, __dmul_rn(static_cast<double>(ss[warp][t]), gs[warp][t]));
+    for (int t = 0; t < S; ++t)
+        if (kept[warp][t])
+            ekept = __dadd_rn(ekept, __dmul_rn(static_cast<double>(ss[warp][t]), gs[warp][t]));
+    double E[4];
+    E[KV2D_FULL] = 0.0;
+    E[KV2D_TOK] = etok;
+    E[KV2D_CH] = ech;
+    E[KV2D_BOTH] = __dadd_rn(etok, ekept);
+    for (int k = 0; k < 4; ++k) A.E[slot * 4 + k] = E[k];
+    if (A.dbg_E)
+        for (int k = 0; k < 4; ++k)
+            A.dbg_E[(static_cast<int64_t>(u) * A.dbg_seg_stride + j) * 4 + k] = E[k];
+
+    // lower convex hull over (bytes, E), options visited by (bytes, id)
+    int hv[4];
+    int nh = 0;
+    hv[nh++] = A.order[0];
+    for (int i = 1; i < 4; ++i) {
+        const int o = A.order[i];
+        const int last = hv[nh - 1];
+        if (E[o] >= E[last]) continue;
+        if (A.bytes[o] == A.bytes[last]) {
+            hv[nh - 1] = o;
+            continue;
+        }
+        while (nh >= 2) {
+            const int pa = hv[nh - 2], pb = hv[nh - 1];
+            const double lhs = __dmul_rn(__dsub_rn(E[pa], E[pb]),
+                                         static_cast<double>(A.bytes[o] - A.bytes[pb]));
+            const double rhs = __dmul_rn(__dsub_rn(E[pb], E[o]),
+                                         static_cast<double>(A.bytes[pb] - A.bytes[pa]));
+            if (lhs <= rhs) --nh;
+            else break;
+        }
+        hv[nh++] = o;
+    }
+    uint8_t* H = A.hull + slot * 8;
+    H[0] = static_cast<uint8_t>(nh);
+    for (int k = 0; k < 4; ++k) H[1 + k] = static_cast<uint8_t>(k < nh ? hv[k] : 0);
+    for (int k = 1; k < nh; ++k) {
+        const int64_t db = A.bytes[hv[k]] - A.bytes[hv[k - 1]];
+        A.dbytes[slot * 3 + k - 1] = static_cast<int32_t>(db);
+        A.eff[slot * 3 + k - 1] =
+            __ddiv_rn(__dsub_rn(E[hv[k - 1]], E[hv[k]]), static_cast<double>(db));
+    }
+}
+
+// ---------------------------------------------------------------- budget
+
+constexpr int kBudgetThreads = 1024;
+
+struct BudgetArgs {
+    SeqPlan plan;
+    int Hkv, S, max_nseg;
+    int64_t bytes[4];
+    int all_full;
+    const uint8_t* hull;
+    const double* eff;
+    const int32_t* dbytes;
+    uint8_t* strat;
+    int32_t* unit_ok;
+    uint64_t* desc;
+    int32_t max_segs;
+    int32_t* n_segs;
+    int64_t* used_bytes;
+    int32_t* comp_end;
+    int64_t arena_stride;
+    uint32_t* status;
+};
+
+__device__ __forceinline__ long long block_sum(long long v, long long* red) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    __syncthreads();
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    long long t = 0;
+    if (warp == 0) {
+        t = (lane < (blockDim.x >> 5)) ? red[lane] : 0;
+        for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+        if (lane == 0) red[32] = t;
+    }
+    __syncthreads();
+    return red[32];
+}
+
+// Exclusive block scan; returns this thread's prefix and writes the block
+// total to *total.
+__device__ __forceinline__ long long block_exscan(long long v, long long* red, long long* total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    long long inc = v;
+    for (int o = 1; o < 32; o <<= 1) {
+        const long long n = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += n;
+    }
+    __syncthreads();
+    if (lane == 31) red[warp] = inc;
+    __syncthreads();
+    if (warp == 0) {
+        long long w = (lane < (blockDim.x >> 5)) ? red[lane] : 0;
+        long long wi = w;
+        for (int o = 1; o < 32; o <<= 1) {
+            const long long n = __shfl_up_sync(0xffffffffu, wi, o);
+            if (lane >= o) wi += n;
+        }
+        red[lane] = wi - w;            // exclusive warp offsets
+        if (lane == 31) red[32] = wi;  // total
+    }
+    __syncthreads();
+    const long long res = red[warp] + inc - v;
+    *total = red[32];
+    return res;
+}
+
+__device__ __forceinline__ uint64_t upg_hi(double eff) {
+    return ~static_cast<uint64_t>(__double_as_longlong(eff));
+}
+
+__global__ void __launch_bounds__(kBudgetThreads) budget_kernel(const __grid_constant__ BudgetArgs A) {
+    const int u = blockIdx.x;
+    const int b = u / A.Hkv, h = u % A.Hkv;
+    const int nseg = A.plan.nseg[b];
+    const int tid = threadIdx.x;
+    if (nseg == 0) {
+        if (tid == 0) A.unit_ok[u] = 1;
+        return;
+    }
+    __shared__ unsigned long long hist[256];
+    __shared__ long long red[33];
+    __shared__ uint64_t s_phi;
+    __shared__ uint32_t s_plo;
+    __shared__ long long s_below;
+    __shared__ int s_mode;            // 0 all full, 1 all steps, 2 threshold
+    const uint8_t* H = A.hull + static_cast<int64_t>(u) * A.max_nseg * 8;
+    const double* EF = A.eff + static_cast<int64_t>(u) * A.max_nseg * 3;
+    const int32_t* DB = A.dbytes + static_cast<int64_t>(u) * A.max_nseg * 3;
+
+    long long base_p = 0, wsum_p = 0;
+    for (int j = tid; j < nseg; j += kBudgetThreads) {
+        const int nv = H[j * 8];
+        base_p += A.bytes[H[j * 8 + 1]];
+        for (int k = 1; k < nv; ++k) wsum_p += DB[j * 3 + k - 1];
+    }
+    const long long base = block_sum(base_p, red);
+    const long long wsum = block_sum(wsum_p, red);
+    const long long rem = A.plan.Bu[b] - base;
+    if (tid == 0) {
+        s_mode = A.all_full ? 0 : (wsum <= rem ? 1 : 2);
+        s_phi = 0;
+        s_plo = 0;
+        s_below = 0;
+    }
+    __syncthreads();
+    const int mode = s_mode;
+    if (mode == 2) {
+        for (int dp = 0; dp < 12; ++dp) {
+            for (int i = tid; i < 256; i += kBudgetThreads) hist[i] = 0;
+            __syncthreads();
+            const uint64_t phi = s_phi;
+            const uint32_t plo = s_plo;
+            for (int j = tid; j < nseg; j += kBudgetThreads) {
+                const int nv = H[j * 8];
+                for (int k = 1; k < nv; ++k) {
+                    const uint64_t hi = upg_hi(EF[j * 3 + k - 1]);
+                    const uint32_t lo = static_cast<uint32_t>(j * 4 + k);
+                    bool match;
+                    int digit;
+                    if (dp < 8) {
+                        const int sh = 64 - 8 * dp;   // bits above the digit
+                        match = (dp == 0) || ((hi >> sh) == (phi >> sh));
+                        digit = static_cast<int>((hi >> (56 - 8 * dp)) & 255u);
+                    } else {
+                        const int dl = dp - 8;
+                        const int sh = 32 - 8 * dl;
+                        match = (hi == phi) && (dl == 0 || (lo >> sh) == (plo >> sh));
+                        digit = static_cast<int>((lo >> (24 - 8 * dl)) & 255u);
+                    }
+                    if (match)
+                        atomicAdd(&hist[digit], static_cast<unsigned long long>(DB[j * 3 + k - 1]));
+                }
+            }
+            __syncthreads();
+            if (tid == 0) {
+                long long cum = s_below;
+                int v = 0;
+                for (; v < 255; ++v) {
+                    if (cum + static_cast<long long>(hist[v]) > rem) break;
+                    cum += static_cast<long long>(hist[v]);
+                }
+                s_below = cum;
+                if (dp < 8) s_phi |= static_cast<uint64_t>(v) << (56 - 8 * dp);
+                else s_plo |= static_cast<uint32_t>(v) << (24 - 8 * (dp - 8));
+            }
+            __syncthreads();
+        }
+    }
+    const uint64_t phi = s_phi;
+    const uint32_t plo = s_plo;
+
+    // strategies and their total bytes
+    long long tot_p = 0;
+    uint8_t* ST = A.strat + static_cast<int64_t>(u) * A.max_nseg;
+    for (int j = tid; j < nseg; j += kBudgetThreads) {
+        const int nv = H[j * 8];
+        int st;
+        if (mode == 0) {
+            st = KV2D_FULL;
+        } else {
+            int level = nv - 1;
+            if (mode == 2) {
+                level = 0;
+                for (int k = 1; k < nv; ++k) {
+                    const uint64_t hi = upg_hi(EF[j * 3 + k - 1]);
+                    const uint32_t lo = static_cast<uint32_t>(j * 4 + k);
+                    if (hi < phi || (hi == phi && lo < plo)) level = k;
+                }
+            }
+            st = H[j * 8 + 1 + level];
+        }
+        ST[j] = static_cast<uint8_t>(st);
+        tot_p += A.bytes[st];
+    }
+    const long long total = block_sum(tot_p, red);
+    const long long used0 = A.used_bytes[u];
+    const int segbase = A.plan.r0[b] / A.S;
+    if (used0 + total > A.arena_stride || segbase + nseg > A.max_segs) {
+        if (tid == 0) {
+            set_status(A.status, KV2D_DEV_CAPACITY);
+            A.unit_ok[u] = 0;
+        }
+        return;
+    }
+    long long carry = used0;
+    for (int j0 = 0; j0 < nseg; j0 += kBudgetThreads) {
+        const int j = j0 + tid;
+        const long long nb = (j < nseg) ? A.bytes[ST[j]] : 0;
+        long long chunk_total;
+        const long long off = carry + block_exscan(nb, red, &chunk_total);
+        if (j < nseg) {
+            const uint64_t d = (static_cast<uint64_t>(off >> 4) & 0xffffffffull) |
+                               (static_cast<uint64_t>(ST[j]) << 32);
+            A.desc[static_cast<int64_t>(u) * A.max_segs + segbase + j] = d;
+        }
+        carry += chunk_total;
+        __syncthreads();
+    }
+    if (tid == 0) {
+        A.used_bytes[u] = used0 + total;
+        A.n_segs[u] = segbase + nseg;
+        if (h == 0) A.comp_end[b] = A.plan.r0[b] + nseg * A.S;
+        A.unit_ok[u] = 1;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_selection(const SelectLaunch& L, cudaStream_t stream) {
+    const int units = L.batch * L.shp.Hkv;
+    if (L.max_nseg > 0) {
+        SegArgs sa;
+        sa.plan = L.plan;
+        sa.Hkv = L.shp.Hkv;
+        sa.S = L.shp.S;
+        sa.r = L.shp.r;
+        sa.max_nseg = L.max_nseg;
+        for (int k = 0; k < 4; ++k) {
+            sa.bytes[k] = L.bytes[k];
+            sa.order[k] = L.order[k];
+        }
+        sa.s = L.s;
+        sa.s_stride = L.s_stride;
+        sa.g = L.g;
+        sa.g_stride = L.g_stride;
+        sa.tidx = L.tidx;
+        sa.E = L.E;
+        sa.hull = L.hull;
+        sa.eff = L.eff;
+        sa.dbytes = L.dbytes;
+        sa.dbg_E = L.dbg_E;
+        sa.dbg_seg_stride = L.dbg_seg_stride;
+        dim3 grid((L.max_nseg + kSegWarps - 1) / kSegWarps, units);
+        prof_begin(stream, kProfSegSelect);
+        seg_select_kernel<<<grid, kSegWarps * 32, 0, stream>>>(sa);
+        prof_end(stream, kProfSegSelect);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    BudgetArgs ba;
+    ba.plan = L.plan;
+    ba.Hkv = L.shp.Hkv;
+    ba.S = L.shp.S;
+    ba.max_nseg = L.max_nseg;
+    for (int k = 0; k < 4; ++k) ba.bytes[k] = L.bytes[k];
+    ba.all_full = L.all_full;
+    ba.hull = L.hull;
+    ba.eff = L.eff;
+    ba.dbytes = L.dbytes;
+    ba.strat = L.strat;
+    ba.unit_ok = L.unit_ok;
+    ba.desc = L.desc;
+    ba.max_segs = L.max_segs;
+    ba.n_segs = L.n_segs;
+    ba.used_bytes = L.used_bytes;
+    ba.comp_end = L.comp_end;
+    ba.arena_stride = L.arena_stride;
+    ba.status = L.status;
+    prof_begin(stream, kProfBudget);
+    budget_kernel<<<units, kBudgetThreads, 0, stream>>>(ba);
+    prof_end(stream, kProfBudget);
+    return cudaGetLastError();
+}
+
+}  // namespace kv2d

@@ -13,9 +13,9 @@ Distribution (one attention layer):
   * planted high-affinity tokens: k_t += 4 * mu_h / |mu_h| for a fraction of
     the tokens (uniform without replacement, or one per stratum).
   * optional segment classes (mix4) so that every strategy wins somewhere:
-    dense-mass segments (half their tokens planted), dense-mass segments whose
-    planted key energy sits in c channels, few-heavy segments (<= r planted)
-    and plain segments.
+    3% dense-mass segments (half their tokens planted), 5% dense-mass
+    segments whose keys keep their energy in c channels (the others x0.02),
+    30% few-heavy segments (1..r planted) and 62% plain segments.
 Everything is generated in fp32 with a seeded torch.Generator on the target
 device and rounded to fp16 once.
 """
@@ -129,44 +129,40 @@ def _keys_for_sequence(wl, T, mu_dir, outl, g, device, b):
     if wl.segment_mix:
         S = wl.segment_len
         nseg = T // S
-        # class per (h, j): 0 dense-mass, 1 dense-mass channel-concentrated,
-        # 2 few-heavy, 3 plain.  3% / 3% / 40% / 54%.
+        # class per (h, j): 0 dense-mass (half the tokens planted), 1 dense-mass
+        # with every key's energy in c channels, 2 few-heavy (1..r planted),
+        # 3 plain.  3% / 5% / 30% / 62%.
         u = torch.rand((H, max(nseg, 1)), generator=g, device=device)
         cls = torch.full_like(u, 3, dtype=torch.int64)
-        cls[u < 0.46] = 2
-        cls[u < 0.06] = 1
+        cls[u < 0.38] = 2
+        cls[u < 0.08] = 1
         cls[u < 0.03] = 0
+        ar = torch.arange(S, device=device)
         for h in range(H):
-            for c_id in (0, 1, 2):
-                segs = torch.nonzero(cls[h, :nseg] == c_id).flatten()
-                if segs.numel() == 0:
-                    continue
-                if c_id == 2:
-                    cnt = torch.randint(1, wl.r + 1, (segs.numel(),), generator=g, device=device)
-                    off = torch.rand((segs.numel(), S), generator=g, device=device).argsort(dim=1)
-                    mask = torch.arange(S, device=device)[None, :] < cnt[:, None]
-                    pos = (segs[:, None] * S + off)[mask]
-                    k[h, pos] += wl.planted_gain * mu_dir[h]
-                else:
-                    off = torch.rand((segs.numel(), S), generator=g, device=device).argsort(dim=1)
-                    pos = (segs[:, None] * S + off[:, : S // 2]).flatten()
-                    if c_id == 0:
-                        k[h, pos] += wl.planted_gain * mu_dir[h]
-                    else:
-                        ch = torch.rand((segs.numel(), d), generator=g,
-                                        device=device).argsort(dim=1)[:, : wl.c]
-                        for si in range(segs.numel()):
-                            rows = segs[si] * S + off[si, : S // 2]
-                            keep = ch[si]
-                            sub = k[h, rows]
-                            energy = torch.zeros(d, device=device)
-                            energy[keep] = 1.0
-                            # planted energy confined to the c channels, the
-                            # other channels of those keys scaled x0.05
-                            sub = sub * (0.05 + 0.95 * energy)
-                            sub = sub + wl.planted_gain * 2.0 * mu_dir[h] * energy
-                            k[h, rows] = sub
-        # the remaining planted budget goes uniform
+            segs = torch.nonzero(cls[h, :nseg] == 2).flatten()
+            if segs.numel():
+                cnt = torch.randint(1, wl.r + 1, (segs.numel(),), generator=g, device=device)
+                off = torch.rand((segs.numel(), S), generator=g, device=device).argsort(dim=1)
+                pos = (segs[:, None] * S + off)[ar[None, :] < cnt[:, None]]
+                k[h, pos] += wl.planted_gain * mu_dir[h]
+            segs = torch.nonzero(cls[h, :nseg] == 0).flatten()
+            if segs.numel():
+                off = torch.rand((segs.numel(), S), generator=g, device=device).argsort(dim=1)
+                pos = (segs[:, None] * S + off[:, : S // 2]).flatten()
+                k[h, pos] += wl.planted_gain * mu_dir[h]
+            segs = torch.nonzero(cls[h, :nseg] == 1).flatten()
+            if segs.numel():
+                n1 = segs.numel()
+                ch = torch.rand((n1, d), generator=g, device=device).argsort(dim=1)[:, : wl.c]
+                mask = torch.zeros((n1, d), device=device)
+                mask.scatter_(1, ch, 1.0)
+                rows = segs[:, None] * S + ar[None, :]                     # [n1][S]
+                k[h, rows] = k[h, rows] * (0.02 + 0.98 * mask)[:, None, :]
+                dirc = mu_dir[h][None, :] * mask
+                dirc = dirc / dirc.norm(dim=1, keepdim=True)
+                off = torch.rand((n1, S), generator=g, device=device).argsort(dim=1)[:, : S // 2]
+                pos = segs[:, None] * S + off                               # [n1][S/2]
+                k[h, pos] += 2.0 * wl.planted_gain * dirc[:, None, :]
     if n_pl > 0 and not wl.segment_mix:
         for h in range(H):
             if wl.planted_layout == "stratified":

@@ -1,0 +1,218 @@
+"""CUDA path vs the fp64 CPU oracle, element by element, through the C ABI.
+
+Sizes are chosen so that the oracle finishes in seconds while the kernels
+still see several tiles, ragged tails, padded window rows (G*W not a multiple
+of 128), both pass-2 column modes (G*W <= 256 and > 256), paged and
+contiguous dense views, and a region that starts after earlier compressions.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from kv_cache_compression_kv2d_b200 import binding as B
+from kv_cache_compression_kv2d_b200 import synth
+from kv_cache_compression_kv2d_b200.synth import Workload
+
+from tests import gpu_harness as H
+
+pytestmark = pytest.mark.gpu
+
+CASES = {
+    "tiny": synth.WORKLOADS["tiny"],
+    "ragged_multi": Workload("ragged_multi", 3, 2, 4, 128, 1537, 64, 24, 0.3, ragged_min=700),
+    "paged": Workload("paged", 3, 2, 4, 128, 1400, 64, 32, 0.25, ragged_min=600, block_size=16),
+    "gw512_s128": Workload("gw512_s128", 1, 2, 4, 128, 2048 + 77, 128, 128, 0.15),
+    "g8_gw384": Workload("g8_gw384", 2, 1, 8, 128, 1100, 32, 48, 0.3),
+    "g2_small_rc": Workload("g2_small_rc", 2, 2, 2, 128, 999, 16, 64, 0.35, keep_tokens=3,
+                            keep_channels=20),
+    "mix4": Workload("mix4", 2, 2, 4, 128, 2048, 64, 64, 0.15, segment_mix=True),
+}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    from kv_cache_compression_kv2d_b200 import build
+    build.build()
+    assert torch.cuda.is_available()
+    B.lib()
+
+
+def _run(wl, seed=0, budget=None, extra=0, **kw):
+    batch = synth.generate(wl, seed=seed, device="cpu", extra_capacity=extra)
+    dev = H.to_device(batch)
+    p = H.params_for(wl, budget=budget, **kw)
+    run = H.make_run(wl, dev, p)
+    return run
+
+
+def _check_all_units(orc, run, independent=True):
+    strats = []
+    for b in range(run.wl.batch):
+        for h in range(run.wl.num_kv_heads):
+            res = H.check_compress_unit(orc, run, b, h, independent=independent)
+            if res is not None:
+                strats.extend(res["strat"].tolist())
+    return strats
+
+
+def _check_decode(orc, run, q=None):
+    q = run.batch.q if q is None else q
+    out = H.gpu_decode(run, q).float().cpu().numpy()
+    worst = 0.0
+    for b in range(run.wl.batch):
+        for h in range(run.wl.num_kv_heads):
+            ref = H.oracle_decode_unit(orc, run, b, h, q)
+            G = run.wl.group
+            got = out[b, h * G:(h + 1) * G]
+            worst = max(worst, float(np.max(np.abs(got - ref))))
+    assert worst <= H.TOL_OUT, f"decode max abs err {worst}"
+    return worst
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_compress_and_decode_parity(orc, name):
+    wl = CASES[name]
+    run = _run(wl)
+    H.compress(run)
+    strats = _check_all_units(orc, run)
+    assert len(strats) > 0
+    _check_decode(orc, run)
+
+
+def test_mix4_spans_all_strategies(orc):
+    run = _run(CASES["mix4"])
+    H.compress(run)
+    strats = _check_all_units(orc, run, independent=False)
+    assert set(strats) == {0, 1, 2, 3}, f"strategies seen: {sorted(set(strats))}"
+
+
+def test_decode_on_oracle_arena(orc):
+    """Decode fed with the oracle's own packed arena (independent scoring),
+    uploaded into a fresh compressed cache."""
+    wl = CASES["ragged_multi"]
+    run = _run(wl, seed=3)
+    p = run.p
+    po = H.oracle_params(orc, p)
+    cc = B.CompressedCache(p, wl.batch, run.batch.capacity)
+    S = wl.segment_len
+    for b in range(wl.batch):
+        T = int(run.batch.seq_len[b])
+        nseg = T // S
+        for h in range(wl.num_kv_heads):
+            u = b * wl.num_kv_heads + h
+            K16, V16 = H.unit_inputs(run, b, h, 0, T)
+            ref = orc.compress_unit(po, T, 0, K16, V16, H.unit_qw(run, b, h))
+            assert ref["status"] == 0
+            base = u * cc.arena_stride
+            cc.arena[base:base + ref["used"]] = torch.from_numpy(ref["arena"]).cuda()
+            d = (ref["offs"] // 16).astype(np.uint64) | (ref["strat"].astype(np.uint64) << np.uint64(32))
+            cc.desc[u, :nseg] = torch.from_numpy(d.view(np.int64)).cuda()
+            cc.n_segs[u] = nseg
+            cc.used_bytes[u] = ref["used"]
+        cc.comp_end[b] = nseg * S
+    q = run.batch.q
+    out = H.gpu_decode(run, q, cc=cc).float().cpu().numpy()
+    for b in range(wl.batch):
+        for h in range(wl.num_kv_heads):
+            ref = H.oracle_decode_unit(orc, run, b, h, q, cc=cc)
+            G = wl.group
+            assert np.max(np.abs(out[b, h * G:(h + 1) * G] - ref)) <= H.TOL_OUT
+
+
+def test_full_budget_equals_dense_attention(orc):
+    wl = CASES["tiny"].with_(budget=1.0)
+    run = _run(wl, budget=1.0)
+    H.compress(run)
+    strats = _check_all_units(orc, run, independent=False)
+    assert set(strats) == {0}
+    q = run.batch.q
+    out = H.gpu_decode(run, q).float()
+    T = int(run.batch.seq_len[0])
+    K = run.batch.k[0, :, :T].float()
+    V = run.batch.v[0, :, :T].float()
+    G = wl.group
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        q[0].float().view(wl.num_kv_heads, G, 1, wl.head_dim),
+        K[:, None], V[:, None], scale=float(run.p.scale)).view(wl.num_q_heads, wl.head_dim)
+    assert float((out[0] - ref).abs().max()) <= H.TOL_OUT
+
+
+def test_keep_all_channels_is_token_only(orc):
+    wl = CASES["ragged_multi"]
+    run = _run(wl, keep_channels=128)
+    H.compress(run)
+    strats = _check_all_units(orc, run, independent=False)
+    assert set(strats) <= {0, 1}
+    _check_decode(orc, run)
+
+
+def test_append_then_periodic_compress(orc):
+    """Decode steps append tokens; a second compression covers the trailing
+    region [comp_end, seq_len) only, appending to the same arenas."""
+    wl = CASES["paged"]
+    steps = 150
+    run = _run(wl, extra=steps + 16)
+    H.compress(run)
+    _check_all_units(orc, run)
+    ws = B.workspace(256)
+    for step in range(steps):
+        k, v, q = synth.decode_tokens(wl, step, device="cuda", mu=run.batch.mu)
+        B.kv2d_append(run.p, wl.batch, run.dv, k, v, run.seq_len, ws)
+        if step in (0, steps - 1):
+            torch.cuda.synchronize()
+            _check_decode(orc, run, q)
+    torch.cuda.synchronize()
+    assert B.kv2d_read_status(ws) == 0
+    seq = run.seq_len.cpu().tolist()
+    assert seq == [int(x) + steps for x in run.batch.seq_len.tolist()]
+    # appended rows landed in the dense view
+    k, v, _ = synth.decode_tokens(wl, steps - 1, device="cuda", mu=run.batch.mu)
+    for b in range(wl.batch):
+        kr, vr = synth.dense_rows(run.batch, b, 1, seq[b] - 1, seq[b])
+        assert torch.equal(kr[0], k[b, 1]) and torch.equal(vr[0], v[b, 1])
+    # the window queries of the second compression: fresh draws
+    g = torch.Generator(device="cuda")
+    g.manual_seed(99)
+    run.batch.qw = (run.batch.mu.repeat_interleave(wl.group, 0)[None, :, None, :] +
+                    torch.randn(run.batch.qw.shape, generator=g, device="cuda")).to(torch.float16)
+    H.compress(run, seq_host=seq)
+    assert any(ce > 0 for ce in run.dbg["ce_before"])
+    _check_all_units(orc, run)
+    _, _, q = synth.decode_tokens(wl, steps, device="cuda", mu=run.batch.mu)
+    _check_decode(orc, run, q)
+
+
+def test_decode_is_deterministic(orc):
+    run = _run(CASES["mix4"])
+    H.compress(run)
+    q = run.batch.q
+    a = H.gpu_decode(run, q)
+    b = H.gpu_decode(run, q)
+    assert torch.equal(a, b)
+
+
+def test_compress_is_deterministic(orc):
+    wl = CASES["g8_gw384"]
+    r1 = _run(wl, seed=5)
+    H.compress(r1)
+    r2 = _run(wl, seed=5)
+    H.compress(r2)
+    assert torch.equal(r1.cc.arena, r2.cc.arena)
+    assert torch.equal(r1.cc.desc, r2.cc.desc)
+    assert torch.equal(r1.dbg["s"], r2.dbg["s"])
+
+
+def test_llama8b_32k_layer_all_units(orc):
+    """Full-size Llama-3-8B-shaped layer (8 KV heads, 32K tokens, budget
+    20%): every unit against the oracle, in the launch configuration the
+    benchmark times."""
+    wl = synth.WORKLOADS["llama3_8b_32k"]
+    run = _run(wl)
+    H.compress(run)
+    from oracle.oracle import parallel_map  # noqa: F401  (threads inside the C oracle)
+    units = [(b, h) for b in range(wl.batch) for h in range(wl.num_kv_heads)]
+    res = parallel_map(lambda bh: H.check_compress_unit(orc, run, bh[0], bh[1]), units)
+    assert all(r is not None for r in res)
+    _check_decode(orc, run)
