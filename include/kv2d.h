@@ -237,6 +237,34 @@ KV2D_API kv2d_status kv2d_decode_attn(const kv2d_params* p, int batch, const kv2
                              int32_t max_seq_len_host, const void* q, void* out, void* ws,
                              size_t ws_bytes, void* stream);
 
+/* kv2d_decode_attn_noalloc -- the same decode attention as kv2d_decode_attn,
+ * for callers that cannot obtain device memory at all: a plugin that runs
+ * inside a host process which owns every allocation, a runtime whose memory
+ * plan is fixed before the first request, or code that must not call
+ * cudaMalloc because that call can synchronise the device in the middle of a
+ * latency-critical loop.  There is no counterpart on the pages; it is an
+ * interface convenience only.
+ *   It takes no workspace.  Its split partials and per-unit tickets live in
+ *   a fixed 8 MiB array in the library's own device memory, which every GPU
+ *   that loads the library holds until the process exits.  Calls whose
+ *   scratch would exceed 8 MiB (units x splits x G x (d + 2) x 4 bytes plus
+ *   a few hundred bytes) return KV2D_ERR_WORKSPACE before launching.
+ *   The first call on each device looks up the array's device address with
+ *   the CUDA runtime; make that first call outside any stream capture.
+ *   All calls on a device share the one array and each leaves its partials
+ *   behind; the tickets are cleared at the start of every call.  Calls whose
+ *   kernels overlap on the GPU (two streams, or two host threads) race on the
+ *   array and give wrong results: serialise them.
+ *   status_dev: optional device uint32; device-side faults OR their
+ *   KV2D_DEV_* bits into it (NULL: they are not reported).
+ * Other arguments, layouts and errors as kv2d_decode_attn.  Allocates no
+ * memory: no cudaMalloc / cudaFree and no allocating library call. */
+KV2D_API kv2d_status kv2d_decode_attn_noalloc(const kv2d_params* p, int batch,
+                                              const kv2d_ccache* cc, const kv2d_dense* kv,
+                                              const int32_t* seq_len_dev, int32_t max_seq_len_host,
+                                              const void* q, void* out, uint32_t* status_dev,
+                                              void* stream);
+
 /* Synchronises stream, returns the device status bits of ws in *bits and
  * clears them.  KV2D_ERR_DEVICE_FAULT if any bit was set. */
 KV2D_API kv2d_status kv2d_read_status(void* ws, void* stream, uint32_t* bits);

@@ -55,7 +55,7 @@ class kv2d_debug(C.Structure):
 EXPORTS = ["kv2d_segment_bytes", "kv2d_arena_bytes", "kv2d_workspace_bytes", "kv2d_compress",
            "kv2d_append", "kv2d_decode_attn", "kv2d_read_status", "kv2d_last_error",
            "kv2d_version", "kv2d_profile_enable", "kv2d_profile_read",
-           "kv2d_profile_stage_name"]
+           "kv2d_profile_stage_name", "kv2d_decode_attn_noalloc"]
 
 _lib = None
 
@@ -85,6 +85,10 @@ def lib():
                                        C.c_void_p, C.c_int32, C.c_void_p, C.c_void_p, C.c_void_p,
                                        C.c_size_t, C.c_void_p]
         L.kv2d_decode_attn.restype = C.c_int
+        L.kv2d_decode_attn_noalloc.argtypes = [P(kv2d_params), C.c_int, P(kv2d_ccache),
+                                               P(kv2d_dense), C.c_void_p, C.c_int32, C.c_void_p,
+                                               C.c_void_p, C.c_void_p, C.c_void_p]
+        L.kv2d_decode_attn_noalloc.restype = C.c_int
         L.kv2d_read_status.argtypes = [C.c_void_p, C.c_void_p, P(C.c_uint32)]
         L.kv2d_read_status.restype = C.c_int
         L.kv2d_last_error.argtypes = []
@@ -211,6 +215,16 @@ def kv2d_profile_read() -> dict:
     for i in range(n):
         out[lib().kv2d_profile_stage_name(i).decode()] = (float(ms[i]), int(n_l[i]))
     return out
+
+
+def kv2d_decode_attn_noalloc(p, batch, cc, dense_view, seq_len_dev, max_seq_len_host, q, out,
+                             status_dev=None, stream=None, check=True) -> int:
+    """kv2d_decode_attn without a workspace: for callers that cannot allocate
+    device memory (scratch is the library's fixed per-GPU array)."""
+    rc = lib().kv2d_decode_attn_noalloc(C.byref(p), int(batch), C.byref(cc), C.byref(dense_view),
+                                        _ptr(seq_len_dev), int(max_seq_len_host), _ptr(q),
+                                        _ptr(out), _ptr(status_dev), _stream(stream))
+    return _check(rc) if check else rc
 
 
 def kv2d_read_status(ws, stream=None) -> int:

@@ -282,6 +282,46 @@ void prof_end(cudaStream_t s, int stage) {
 }  // namespace kv2d
 
 namespace {
+// ---- fixed device scratch for kv2d_decode_attn_noalloc
+//
+// The array lives in every GPU's global memory from the moment the library's
+// module is loaded on that GPU until the process exits.  Host code must not
+// take its address directly (the host-side name is only a stand-in); the
+// device address comes from cudaGetSymbolAddress, once per device.
+
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;   // 8 MiB per GPU
+constexpr int kNoAllocMaxDevices = 64;
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+
+}  // namespace
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+
+// Device address of the scratch array on the current device, resolved on
+// the first call per device.
+kv2d_status noalloc_scratch(void** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(KV2D_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    if (dev < 0 || dev >= kNoAllocMaxDevices)
+        return fail(KV2D_ERR_UNSUPPORTED, "device ordinal %d beyond %d", dev, kNoAllocMaxDevices);
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void* ptr = nullptr;
+        e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+        if (e != cudaSuccess || !ptr)
+            return fail(KV2D_ERR_CUDA, "cudaGetSymbolAddress of the decode scratch: %s",
+                        cudaGetErrorString(e));
+        g_noalloc_ptr[dev] = ptr;
+    }
+    *out = g_noalloc_ptr[dev];
+    return KV2D_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -612,6 +652,67 @@ kv2d_status kv2d_decode_attn(const kv2d_params* p, int batch, const kv2d_ccache*
     L.part = reinterpret_cast<float*>(w + WL.part);
     L.ticket = reinterpret_cast<uint32_t*>(w + WL.ticket);
     L.status = reinterpret_cast<uint32_t*>(w);
+    cudaError_t e = launch_decode(L, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail(KV2D_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
+    return ok();
+}
+
+kv2d_status kv2d_decode_attn_noalloc(const kv2d_params* p, int batch, const kv2d_ccache* cc,
+                                     const kv2d_dense* kv, const int32_t* seq_len_dev,
+                                     int32_t max_seq_len_host, const void* q, void* out,
+                                     uint32_t* status_dev, void* stream) {
+    kv2d_status st = check_params(p);
+    if (st != KV2D_OK) return st;
+    const UnitShape sh = shape_of(p);
+    if (sh.G != 2 && sh.G != 4 && sh.G != 8)
+        return fail(KV2D_ERR_UNSUPPORTED, "decode runs G = Hq/Hkv in {2, 4, 8}, got %d", sh.G);
+    if (batch < 1 || batch > KV2D_MAX_BATCH)
+        return fail(KV2D_ERR_INVALID_ARG, "batch %d not in [1, %d]", batch, KV2D_MAX_BATCH);
+    if ((st = check_dense(p, batch, kv)) != KV2D_OK) return st;
+    if (!cc || !cc->arena || !cc->desc || !cc->n_segs || !cc->used_bytes || !cc->comp_end)
+        return fail(KV2D_ERR_INVALID_ARG, "compressed cache has a NULL pointer");
+    if (!aligned(cc->arena, 256) || cc->arena_stride % 256)
+        return fail(KV2D_ERR_INVALID_ARG, "arena must be 256-byte aligned with a multiple-of-256 stride");
+    if (!seq_len_dev || !q || !out || !aligned(q, 16) || !aligned(out, 16))
+        return fail(KV2D_ERR_INVALID_ARG, "seq_len / q / out must be 16-byte aligned device pointers");
+    if (status_dev && !aligned(status_dev, 4))
+        return fail(KV2D_ERR_INVALID_ARG, "status_dev must be 4-byte aligned");
+    if (max_seq_len_host < 0 || max_seq_len_host > dense_capacity(kv))
+        return fail(KV2D_ERR_INVALID_ARG, "max_seq_len %d outside [0, capacity]", max_seq_len_host);
+    const int64_t units = static_cast<int64_t>(batch) * sh.Hkv;
+    const int nsplit =
+        std::min(kMaxSplitDec, decode_split_count(static_cast<int>(units), max_seq_len_host, num_sms()));
+    Carver c;
+    c.take(256);                                               // status word
+    const size_t ticket_off = c.take(units * 4);
+    const size_t part_off = c.take(units * nsplit * sh.G * (kHeadDim + 2) * 4);
+    if (c.off > kNoAllocScratchBytes)
+        return fail(KV2D_ERR_WORKSPACE,
+                    "decode needs %zu bytes of scratch for %lld units x %d splits; the built-in "
+                    "scratch holds %zu bytes",
+                    c.off, static_cast<long long>(units), nsplit, kNoAllocScratchBytes);
+    void* scratch = nullptr;
+    if ((st = noalloc_scratch(&scratch)) != KV2D_OK) return st;
+    uint8_t* w = static_cast<uint8_t*>(scratch);
+    DecodeLaunch L;
+    L.shp = sh;
+    L.batch = batch;
+    L.scale_log2 = sh.c2;
+    L.dv = view_of(p, kv);
+    L.arena = static_cast<const uint8_t*>(cc->arena);
+    L.arena_stride = cc->arena_stride;
+    L.desc = static_cast<const uint64_t*>(cc->desc);
+    L.max_segs = cc->max_segs;
+    L.n_segs = cc->n_segs;
+    L.used_bytes = cc->used_bytes;
+    L.comp_end = cc->comp_end;
+    L.seq_len = seq_len_dev;
+    L.q = static_cast<const __half*>(q);
+    L.out = static_cast<__half*>(out);
+    L.nsplit = nsplit;
+    L.part = reinterpret_cast<float*>(w + part_off);
+    L.ticket = reinterpret_cast<uint32_t*>(w + ticket_off);   // zeroed by launch_decode
+    L.status = status_dev ? status_dev : reinterpret_cast<uint32_t*>(w);
     cudaError_t e = launch_decode(L, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return fail(KV2D_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
     return ok();
