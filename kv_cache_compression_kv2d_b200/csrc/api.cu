@@ -249,7 +249,7 @@ bool g_prof_on = false;
 std::vector<ProfRec> g_prof_open;      // begun, not yet ended (one per stage)
 std::vector<ProfRec> g_prof_done;
 
-const char* const kStageNames[kProfStages] = {"win_stats", "score_pass1", "lse_merge",
+const char* const kStageNames[kProfStages] = {"win_stats", "score_pass1", "unit_stats",
                                               "score_pass2", "chan_topc", "seg_select",
                                               "budget", "pack", "append", "decode"};
 
@@ -472,13 +472,14 @@ kv2d_status kv2d_compress(const kv2d_params* p, int batch, const int32_t* seq_le
         }
         if (r != CUDA_SUCCESS) return fail(KV2D_ERR_CUDA, "key tensor map encode failed (%d)", int(r));
     }
+    // Grids fill whole waves: pass 1 runs two CTAs per SM, pass 2 one.
     const int nsm = num_sms();
     const int mtiles = sh.GWpad / 128;
     {
         const int64_t max_tiles = (max_region + kKeyTile - 1) / kKeyTile;
-        int ns = static_cast<int>((2 * nsm + units * mtiles - 1) / (units * mtiles));
-        ns = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>({static_cast<int64_t>(ns), max_tiles,
-                                                                       static_cast<int64_t>(kMaxSplit1)})));
+        const int groups = units * mtiles;
+        int64_t ns = std::max(1, (2 * nsm) / groups);
+        ns = std::max<int64_t>(1, std::min<int64_t>({ns, max_tiles, static_cast<int64_t>(kMaxSplit1)}));
         const int64_t tiles_per = (max_tiles + ns - 1) / ns;
         SL.kps1 = static_cast<int>(tiles_per * kKeyTile);
         SL.nsplit1 = static_cast<int>((max_tiles + tiles_per - 1) / tiles_per);
@@ -486,8 +487,8 @@ kv2d_status kv2d_compress(const kv2d_params* p, int batch, const int32_t* seq_le
     {
         const int64_t seg_tok = static_cast<int64_t>(max_nseg) * sh.S;
         const int64_t max_tiles = (seg_tok + kKeyTile - 1) / kKeyTile;
-        int ns = (2 * nsm + units - 1) / units;
-        ns = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(ns, max_tiles)));
+        int64_t ns = std::max(1, nsm / units);
+        ns = std::max<int64_t>(1, std::min<int64_t>(ns, max_tiles));
         const int64_t tiles_per = (max_tiles + ns - 1) / ns;
         SL.kps2 = static_cast<int>(tiles_per * kKeyTile);
         SL.nsplit2 = static_cast<int>((max_tiles + tiles_per - 1) / tiles_per);

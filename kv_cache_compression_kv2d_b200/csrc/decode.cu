@@ -279,6 +279,7 @@ constexpr int64_t kTailBytes = 2 * kHeadDim * 2;   // K + V row of one dense tok
 
 template <int G>
 __global__ void __launch_bounds__(kDecThreads) decode_kernel(const __grid_constant__ DecodeArgs A) {
+    constexpr int TB = 32 / G;                     // tokens per warp step
     const int sp = blockIdx.x, u = blockIdx.y;
     const int b = u / A.Hkv, h = u % A.Hkv;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -286,14 +287,16 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(const __grid_consta
     __shared__ float p_s[kDecWarps][32];
     __shared__ float wm[kDecWarps][G], wl[kDecWarps][G];
     __shared__ __align__(16) float wo[kDecWarps][G][kHeadDim];
-    __shared__ int rng[4];
+    __shared__ long long hdr[4];       // lo, hi, U, ce | ntail
+    __shared__ int cnt[2];
     __shared__ int is_last;
+    __shared__ float sc[64][G];
 
-    // ---- this CTA's share of the unit's bytes
+    // ---- this CTA's share [lo, hi) of the unit's bytes: packed arena, then
+    // the dense tail at 512 bytes per token
     if (tid == 0) {
         int T = A.seq_len[b];
         int ce = A.comp_end[b];
-        const int nsg = A.n_segs[u];
         const int64_t U = A.used_bytes[u];
         const int cap = A.dv.block_table ? A.dv.max_blocks * A.dv.block_size : A.dv.capacity;
         if (T < 0 || T > cap || ce < 0 || ce > T) {
@@ -301,28 +304,13 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(const __grid_consta
             T = max(0, min(T, cap));
             ce = max(0, min(ce, T));
         }
-        const int ntail = T - ce;
-        const int64_t Wt = U + static_cast<int64_t>(ntail) * kTailBytes;
-        const int64_t lo = Wt * sp / A.nsplit, hi = Wt * (sp + 1) / A.nsplit;
-        const uint64_t* D = A.desc + static_cast<int64_t>(u) * A.max_segs;
-        auto first_at_or_after = [&](int64_t x) {
-            int a = 0, z = nsg;
-            while (a < z) {
-                const int mid = (a + z) >> 1;
-                if (static_cast<int64_t>(D[mid] & 0xffffffffull) * 16 < x) a = mid + 1;
-                else z = mid;
-            }
-            return a;
-        };
-        rng[0] = first_at_or_after(lo);
-        rng[1] = first_at_or_after(hi);
-        auto tail_at_or_after = [&](int64_t x) {
-            if (x <= U) return 0;
-            const int64_t i = (x - U + kTailBytes - 1) / kTailBytes;
-            return static_cast<int>(i < ntail ? i : static_cast<int64_t>(ntail));
-        };
-        rng[2] = ce + tail_at_or_after(lo);
-        rng[3] = ce + tail_at_or_after(hi);
+        const int64_t Wt = U + static_cast<int64_t>(T - ce) * kTailBytes;
+        hdr[0] = Wt * sp / A.nsplit;
+        hdr[1] = Wt * (sp + 1) / A.nsplit;
+        hdr[2] = U;
+        hdr[3] = (static_cast<long long>(ce) << 32) | static_cast<unsigned>(T - ce);
+        cnt[0] = 0;
+        cnt[1] = 0;
     }
     for (int i = tid; i < G * kHeadDim; i += kDecThreads) {
         const int g = i / kHeadDim, x = i % kHeadDim;
@@ -330,7 +318,36 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(const __grid_consta
             __half2float(A.q[(static_cast<int64_t>(b) * A.Hq + h * G + g) * kHeadDim + x]) * A.c2;
     }
     __syncthreads();
-    const int j_lo = rng[0], j_hi = rng[1], t_lo = rng[2], t_hi = rng[3];
+    const int64_t lo = hdr[0], hi = hdr[1], U = hdr[2];
+    const int ce = static_cast<int>(hdr[3] >> 32), ntail = static_cast<int>(hdr[3] & 0xffffffff);
+    const int nsg = A.n_segs[u];
+    const uint64_t* D = A.desc + static_cast<int64_t>(u) * A.max_segs;
+    {
+        // segments whose first byte lies below lo / below hi (offsets ascend)
+        int c_lo = 0, c_hi = 0;
+        for (int j = tid; j < nsg; j += kDecThreads) {
+            const int64_t off = static_cast<int64_t>(D[j] & 0xffffffffull) * 16;
+            c_lo += off < lo;
+            c_hi += off < hi;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            c_lo += __shfl_xor_sync(0xffffffffu, c_lo, o);
+            c_hi += __shfl_xor_sync(0xffffffffu, c_hi, o);
+        }
+        if (lane == 0) {
+            atomicAdd(&cnt[0], c_lo);
+            atomicAdd(&cnt[1], c_hi);
+        }
+    }
+    __syncthreads();
+    const int j_lo = cnt[0], j_hi = cnt[1];
+    auto tail_at_or_after = [&](int64_t x) -> int {
+        if (x <= U) return 0;
+        const int64_t i = (x - U + kTailBytes - 1) / kTailBytes;
+        return static_cast<int>(i < ntail ? i : static_cast<int64_t>(ntail));
+    };
+    const int t_lo = ce + tail_at_or_after(lo), t_hi = ce + tail_at_or_after(hi);
 
     WarpState<G> st;
 #pragma unroll
@@ -346,37 +363,56 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(const __grid_consta
 #pragma unroll
         for (int e = 0; e < 4; ++e) qr[g][e] = q_s[(lane * 4 + e) * G + g];
 
+    // ---- work items: (segment, block of TB tokens) in order, then tail blocks;
+    // item i goes to warp i % 8.  A segment has ceil(ntok / TB) blocks.
     const uint8_t* ubase = A.arena + static_cast<int64_t>(u) * A.arena_stride;
-    const uint64_t* D = A.desc + static_cast<int64_t>(u) * A.max_segs;
-    const int nseg_items = j_hi - j_lo;
-    const int ntail_items = (t_hi - t_lo + 15) / 16;
     float* ps = p_s[warp];
-    for (int it = warp; it < nseg_items + ntail_items; it += kDecWarps) {
-        if (it < nseg_items) {
-            const uint64_t d = D[j_lo + it];
-            const int sty = static_cast<int>((d >> 32) & 255u);
-            const uint8_t* seg = ubase + static_cast<int64_t>(d & 0xffffffffull) * 16;
-            const bool tok = (sty == KV2D_TOK || sty == KV2D_BOTH);
+    const int nb_full = (A.S + TB - 1) / TB, nb_tok = (A.r + TB - 1) / TB;
+    int seg = j_lo, blk = 0, item = 0;
+    // walk segments; each warp takes its own items
+    while (seg < j_hi) {
+        const uint64_t d = D[seg];
+        const int sty = static_cast<int>((d >> 32) & 255u);
+        const bool tok = (sty == KV2D_TOK || sty == KV2D_BOTH);
+        const int nblk = tok ? nb_tok : nb_full;
+        // first block of this segment owned by this warp
+        int first = (warp - item) % kDecWarps;
+        if (first < 0) first += kDecWarps;
+        if (first < nblk) {
             const int ntok = tok ? A.r : A.S;
-            const uint8_t* p0 = seg + (tok ? pad16(A.r) : 0);
-            if (sty == KV2D_FULL || sty == KV2D_TOK) {
-                const __half* K = reinterpret_cast<const __half*>(p0);
-                const __half* V = K + static_cast<int64_t>(ntok) * kHeadDim;
-                dense_rows<G>(
-                    st, ntok, [&](int i) { return K + static_cast<int64_t>(i) * kHeadDim; },
-                    [&](int i) { return V + static_cast<int64_t>(i) * kHeadDim; }, qr, ps);
-            } else {
-                const uint8_t* ci = p0;
-                const __half* kv = reinterpret_cast<const __half*>(p0 + pad16(static_cast<int64_t>(ntok) * A.c));
-                const __half* V = reinterpret_cast<const __half*>(
-                    reinterpret_cast<const uint8_t*>(kv) + pad16(static_cast<int64_t>(ntok) * A.c * 2));
-                sparse_rows<G>(st, ntok, A.c, ci, kv, V, q_s, ps);
+            const uint8_t* p0 = ubase + static_cast<int64_t>(d & 0xffffffffull) * 16 + (tok ? pad16(A.r) : 0);
+            for (blk = first; blk < nblk; blk += kDecWarps) {
+                const int t0 = blk * TB;
+                const int n = min(TB, ntok - t0);
+                if (sty == KV2D_FULL || sty == KV2D_TOK) {
+                    const __half* K = reinterpret_cast<const __half*>(p0) + static_cast<int64_t>(t0) * kHeadDim;
+                    const __half* V = reinterpret_cast<const __half*>(p0) + static_cast<int64_t>(ntok + t0) * kHeadDim;
+                    dense_rows<G>(
+                        st, n, [&](int i) { return K + static_cast<int64_t>(i) * kHeadDim; },
+                        [&](int i) { return V + static_cast<int64_t>(i) * kHeadDim; }, qr, ps);
+                } else {
+                    const uint8_t* ci = p0;
+                    const __half* kv = reinterpret_cast<const __half*>(p0 + pad16(static_cast<int64_t>(ntok) * A.c));
+                    const __half* V = reinterpret_cast<const __half*>(
+                        reinterpret_cast<const uint8_t*>(kv) + pad16(static_cast<int64_t>(ntok) * A.c * 2));
+                    sparse_rows<G>(st, n, A.c, ci + static_cast<int64_t>(t0) * A.c,
+                                   kv + static_cast<int64_t>(t0) * A.c,
+                                   V + static_cast<int64_t>(t0) * kHeadDim, q_s, ps);
+                }
             }
-        } else {
-            const int t0 = t_lo + (it - nseg_items) * 16;
-            const int n = min(16, t_hi - t0);
-            uint32_t* status = A.status;
-            const DenseView& dv = A.dv;
+        }
+        item += nblk;
+        ++seg;
+    }
+    {
+        const int ntb = (t_hi - t_lo + TB - 1) / TB;
+        int first = (warp - item) % kDecWarps;
+        if (first < 0) first += kDecWarps;
+        uint32_t* status = A.status;
+        const DenseView& dv = A.dv;
+        for (int tb = first; tb < ntb; tb += kDecWarps) {
+            const int t0 = t_lo + tb * TB;
+            const int n = min(TB, t_hi - t0);
             dense_rows<G>(
                 st, n, [&](int i) { return dense_row(dv, dv.k, b, h, t0 + i, status); },
                 [&](int i) { return dense_row(dv, dv.v, b, h, t0 + i, status); }, qr, ps);
@@ -407,14 +443,16 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(const __grid_consta
     for (int i = tid; i < G * kHeadDim; i += kDecThreads) {
         const int g = i / kHeadDim, x = i % kHeadDim;
         float M = kNegInfF;
+#pragma unroll
         for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, wm[w][g]);
         float O = 0.f, L = 0.f;
         if (M != kNegInfF) {
+#pragma unroll
             for (int w = 0; w < kDecWarps; ++w) {
                 if (wm[w][g] == kNegInfF) continue;
-                const float sc = fast_exp2(wm[w][g] - M);
-                O = fmaf(wo[w][g][x], sc, O);
-                L = fmaf(wl[w][g], sc, L);
+                const float scl = fast_exp2(wm[w][g] - M);
+                O = fmaf(wo[w][g][x], scl, O);
+                L = fmaf(wl[w][g], scl, L);
             }
         }
         myp[g * kRec + 2 + x] = O;
@@ -432,21 +470,29 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(const __grid_consta
 
     // ---- last CTA of the unit: merge the splits in order
     const float* up = A.part + static_cast<int64_t>(u) * A.nsplit * G * kRec;
+    for (int i = tid; i < A.nsplit * G; i += kDecThreads) sc[i / G][i % G] = __ldcg(up + i * kRec);
+    __syncthreads();
+    if (tid < G) {
+        float M = kNegInfF;
+        for (int s2 = 0; s2 < A.nsplit; ++s2) M = fmaxf(M, sc[s2][tid]);
+        float L = 0.f;
+        for (int s2 = 0; s2 < A.nsplit; ++s2) {
+            const float ms = sc[s2][tid];
+            const float scl = (ms == kNegInfF) ? 0.f : fast_exp2(ms - M);
+            sc[s2][tid] = scl;
+            L = fmaf(__ldcg(up + (s2 * G + tid) * kRec + 1), scl, L);
+        }
+        wl[0][tid] = L;
+    }
+    __syncthreads();
     for (int i = tid; i < G * kHeadDim; i += kDecThreads) {
         const int g = i / kHeadDim, x = i % kHeadDim;
-        float M = kNegInfF;
-        for (int s = 0; s < A.nsplit; ++s) M = fmaxf(M, __ldcg(up + (s * G + g) * kRec));
-        float O = 0.f, L = 0.f;
-        if (M != kNegInfF) {
-            for (int s = 0; s < A.nsplit; ++s) {
-                const float* pr = up + (s * G + g) * kRec;
-                const float ms = __ldcg(pr);
-                if (ms == kNegInfF) continue;
-                const float sc = fast_exp2(ms - M);
-                O = fmaf(__ldcg(pr + 2 + x), sc, O);
-                L = fmaf(__ldcg(pr + 1), sc, L);
-            }
+        float O = 0.f;
+        for (int s2 = 0; s2 < A.nsplit; ++s2) {
+            const float scl = sc[s2][g];
+            if (scl != 0.f) O = fmaf(__ldcg(up + (s2 * G + g) * kRec + 2 + x), scl, O);
         }
+        const float L = wl[0][g];
         const float res = (L > 0.f) ? O / L : 0.f;
         A.out[(static_cast<int64_t>(b) * A.Hq + h * G + g) * kHeadDim + x] = __float2half_rn(res);
     }
@@ -456,7 +502,8 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(const __grid_consta
 }  // namespace
 
 int decode_split_count(int units, int64_t max_seq_len, int num_sms) {
-    int ns = (3 * num_sms + units - 1) / units;
+    // two CTAs per SM, one wave
+    int ns = (2 * num_sms) / units;
     const int by_len = static_cast<int>((max_seq_len + 255) / 256);
     ns = min(ns, max(1, by_len));
     return max(1, min(ns, 64));

@@ -37,12 +37,24 @@ struct PackArgs {
 __device__ __forceinline__ void copy_rows(const __half* base, const DenseView& dv, int b, int h,
                                           int t0, const int* toks, int ntok, uint8_t* dst,
                                           uint32_t* status) {
-    for (int idx = threadIdx.x; idx < ntok * 16; idx += blockDim.x) {
-        const int i = idx >> 4, ch = idx & 15;
-        const __half* row = dense_row(dv, base, b, h, t0 + toks[i], status);
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (row) v = *reinterpret_cast<const uint4*>(row + ch * 8);
-        *reinterpret_cast<uint4*>(dst + i * 256 + ch * 16) = v;
+    // 4 independent 16-byte loads in flight per thread before the stores
+    const int n = ntok * 16;
+    for (int i0 = threadIdx.x; i0 < n; i0 += 4 * blockDim.x) {
+        uint4 v[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int idx = i0 + k * blockDim.x;
+            v[k] = make_uint4(0, 0, 0, 0);
+            if (idx < n) {
+                const __half* row = dense_row(dv, base, b, h, t0 + toks[idx >> 4], status);
+                if (row) v[k] = *reinterpret_cast<const uint4*>(row + (idx & 15) * 8);
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int idx = i0 + k * blockDim.x;
+            if (idx < n) *reinterpret_cast<uint4*>(dst + (idx >> 4) * 256 + (idx & 15) * 16) = v[k];
+        }
     }
 }
 

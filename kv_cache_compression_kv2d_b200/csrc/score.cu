@@ -6,15 +6,17 @@
 // Sliding-Window KV Cache Compression", "What carries the argument") scores
 // keys by the attention that all queries of a recent window give them.
 // The kernels here compute, per unit (sequence b, KV head h):
-//   win_stats : a_d = mean_{G*W window rows} |q_d|
 //   pass 1    : lse of every window row over the causal region, from a
 //               tcgen05 product Q_w K^T (M = 128 window rows, N = 128 keys),
 //               split over key ranges -> per-split (max, sum) partials
-//   lse merge : combines the partials in split order
+//   unit stats: combines the partials in split order, and forms
+//               a_d = mean_{G*W window rows} |q_d|
 //   pass 2    : s_t = sum_rows exp(l - lse) from the transposed product
 //               K Q_w^T (M = 128 keys, N = window rows) so that each TMEM lane
 //               owns one key and sums over queries in-thread
-//   chan      : per key: top-c channels of |k_d| a_d and g_t in fp64
+//   chan      : per key: top-c channels of |k_d| a_d and g_t in fp64 (a
+//               packed 16-bit SIMD selection network for c <= 32, a full
+//               32-bit register sort otherwise)
 // Both products take their operands from shared memory written by TMA with
 // the 128-byte swizzle; the fp32 accumulators live in tensor memory.
 #include "kernels.h"
@@ -25,7 +27,7 @@ namespace {
 
 constexpr int kPassThreads = 320;    // 8 epilogue warps, 1 TMA warp, 1 MMA warp
 constexpr int kStage = 128 * 256;    // one K tile: 128 keys x 128 fp16
-constexpr int kP1Stages = 4;
+constexpr int kP1Stages = 2;   // ~99 KB of shared memory: two CTAs per SM
 constexpr uint32_t kNegInf = 0xff800000u;
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
@@ -55,24 +57,6 @@ __device__ __forceinline__ void load_key_tile(uint8_t* dst, const CUtensorMap* k
         tma_load_4d(dst + j * 2048, kmap, bar, 0, row, h, phys);
         tma_load_4d(dst + 16384 + j * 2048, kmap, bar, 64, row, h, phys);
     }
-}
-
-// ------------------------------------------------------------ win_stats
-
-__global__ void win_stats_kernel(const __half* __restrict__ qw, int Hq, int G, int W, int Hkv,
-                                 float* __restrict__ a, float* __restrict__ dbg_a) {
-    const int u = blockIdx.x;
-    const int b = u / Hkv, h = u % Hkv;
-    const int x = threadIdx.x;
-    const int rows = G * W;
-    const __half* base = qw + (static_cast<int64_t>(b) * Hq + static_cast<int64_t>(h) * G) * W *
-                                  kHeadDim;
-    float acc = 0.f;
-    for (int row = 0; row < rows; ++row)
-        acc += fabsf(__half2float(base[static_cast<int64_t>(row) * kHeadDim + x]));
-    float v = acc / static_cast<float>(rows);
-    a[static_cast<int64_t>(u) * kHeadDim + x] = v;
-    if (dbg_a) dbg_a[static_cast<int64_t>(u) * kHeadDim + x] = v;
 }
 
 // --------------------------------------------------------------- pass 1
@@ -258,31 +242,54 @@ __global__ void __launch_bounds__(kPassThreads, 1)
     if (warp == 9) tmem_dealloc(tmem, 256);
 }
 
-// ------------------------------------------------------------ lse merge
+// ------------------------------------------- lse merge and window stats
 
-__global__ void lse_merge_kernel(const float2* __restrict__ part, int nsplit, int GW, int GWpad,
-                                 int Hkv, int Hq, int G, int W, float* __restrict__ lse2,
-                                 float* __restrict__ dbg_lse) {
+// One CTA of 1024 threads per unit: thread rho < G*W (padded) merges the
+// pass-1 partials of window row rho in split order; the block also forms
+// a_d = mean |q_d| over the unit's G*W window rows (row groups of 128 threads,
+// combined in a fixed order).
+__global__ void unit_stats_kernel(const float2* __restrict__ part, int nsplit, int GW, int GWpad,
+                                  int Hkv, int Hq, int G, int W, const __half* __restrict__ qw,
+                                  float* __restrict__ lse2, float* __restrict__ dbg_lse,
+                                  float* __restrict__ a, float* __restrict__ dbg_a) {
     const int u = blockIdx.x;
-    const int rho = threadIdx.x;
-    if (rho >= GWpad) return;
-    float out = __int_as_float(0x7f800000);   // +inf: padded rows weigh nothing
-    if (rho < GW) {
-        const float2* p = part + (static_cast<int64_t>(u) * GWpad + rho) * nsplit;
-        float M = __uint_as_float(kNegInf);
-        for (int s = 0; s < nsplit; ++s) M = fmaxf(M, p[s].x);
-        float L = 0.f;
-        for (int s = 0; s < nsplit; ++s)
-            if (p[s].y > 0.f) L += p[s].y * exp2f(p[s].x - M);
-        out = M + log2f(L);
-        if (dbg_lse) {
-            const int b = u / Hkv, h = u % Hkv;
-            const int g = rho / W, i = rho % W;
-            dbg_lse[(static_cast<int64_t>(b) * Hq + h * G + g) * W + i] =
-                out * 0.69314718055994531f;
+    const int b = u / Hkv, h = u % Hkv;
+    const int tid = threadIdx.x;
+    const int rho = tid;
+    if (rho < GWpad) {
+        float out = __int_as_float(0x7f800000);   // +inf: padded rows weigh nothing
+        if (rho < GW) {
+            const float2* p = part + (static_cast<int64_t>(u) * GWpad + rho) * nsplit;
+            float M = __uint_as_float(kNegInf);
+            for (int s = 0; s < nsplit; ++s) M = fmaxf(M, p[s].x);
+            float L = 0.f;
+            for (int s = 0; s < nsplit; ++s)
+                if (p[s].y > 0.f) L += p[s].y * exp2f(p[s].x - M);
+            out = M + log2f(L);
+            if (dbg_lse) {
+                const int g = rho / W, i = rho % W;
+                dbg_lse[(static_cast<int64_t>(b) * Hq + h * G + g) * W + i] =
+                    out * 0.69314718055994531f;
+            }
         }
+        lse2[static_cast<int64_t>(u) * GWpad + rho] = out;
     }
-    lse2[static_cast<int64_t>(u) * GWpad + rho] = out;
+    __shared__ float acc[8][kHeadDim];
+    const int groups = blockDim.x / kHeadDim;
+    const int grp = tid / kHeadDim, x = tid % kHeadDim;
+    const __half* base = qw + (static_cast<int64_t>(b) * Hq + static_cast<int64_t>(h) * G) * W * kHeadDim;
+    float s = 0.f;
+    for (int row = grp; row < GW; row += groups)
+        s += fabsf(__half2float(base[static_cast<int64_t>(row) * kHeadDim + x]));
+    acc[grp][x] = s;
+    __syncthreads();
+    if (tid < kHeadDim) {
+        float t = 0.f;
+        for (int g2 = 0; g2 < groups; ++g2) t += acc[g2][tid];
+        const float v = t / static_cast<float>(GW);
+        a[static_cast<int64_t>(u) * kHeadDim + tid] = v;
+        if (dbg_a) dbg_a[static_cast<int64_t>(u) * kHeadDim + tid] = v;
+    }
 }
 
 // --------------------------------------------------------------- pass 2
@@ -544,7 +551,7 @@ struct ChanArgs {
 // (trunc(f) desc, x asc).  Let v be the truncated value of the c-th key:
 // channels above v are in, channels below are out, and channels equal to v
 // are ranked exactly by (e desc, x asc) in fp64 when they straddle the cut.
-__global__ void __launch_bounds__(128) chan_kernel(const __grid_constant__ ChanArgs A) {
+__global__ void __launch_bounds__(128) chan_kernel_generic(const __grid_constant__ ChanArgs A) {
     const int u = blockIdx.y;
     const int b = u / A.Hkv, h = u % A.Hkv;
     const int r0 = A.plan.r0[b];
@@ -661,6 +668,235 @@ __global__ void __launch_bounds__(128) chan_kernel(const __grid_constant__ ChanA
     if (A.dbg_g) A.dbg_g[static_cast<int64_t>(u) * A.dbg_stride + t] = gv;
 }
 
+
+// ---- fast path for c <= 32
+//
+// Keys are the top 16 bits of the fp32 product (exponent + 8 mantissa
+// bits; monotone in the exact product), two per register: register i holds
+// channel i in its high half and channel 64 + i in its low half, so every
+// __vmaxu2 / __vminu2 pair is two compare-exchanges.  Sorting registers
+// 0..31 and 32..63 gives four descending 32-lists; max(X_i, Y_{31-i}) and a
+// bitonic merge give the top 32 of channels 0..63 (high halves) and of
+// 64..127 (low halves); one more scalar merge gives the top 32 of all 128,
+// whose (c-1)-th entry v is the c-th largest 16-bit key.  Channels above v
+// are in, below are out; channels equal to v are all in unless they
+// straddle the cut, in which case they are ranked exactly by (e desc, x asc)
+// with the fp64 products.
+
+__device__ __forceinline__ void ce2(uint32_t& a, uint32_t& b) {
+    const uint32_t hi = __vmaxu2(a, b), lo = __vminu2(a, b);
+    a = hi;
+    b = lo;
+}
+
+// One bitonic stage (block size K, distance J) on registers O..O+31, then
+// the next; written as template recursion so that every register index is a
+// compile-time constant.
+template <int O, int K, int J>
+__device__ __forceinline__ void sort32_stage2(uint32_t (&v)[64]) {
+    if constexpr (J > 0) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const int l = i ^ J;
+            if (l > i) {
+                if ((i & K) == 0) ce2(v[O + i], v[O + l]);
+                else ce2(v[O + l], v[O + i]);
+            }
+        }
+        sort32_stage2<O, K, J / 2>(v);
+    } else if constexpr (K < 32) {
+        sort32_stage2<O, K * 2, K>(v);
+    }
+}
+
+template <int O>
+__device__ __forceinline__ void sort32_desc2(uint32_t (&v)[64]) {
+    sort32_stage2<O, 2, 1>(v);
+}
+
+template <int J>
+__device__ __forceinline__ void merge32_desc2(uint32_t (&v)[64]) {
+    if constexpr (J > 0) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const int l = i ^ J;
+            if (l > i) ce2(v[i], v[l]);
+        }
+        merge32_desc2<J / 2>(v);
+    }
+}
+
+template <int J>
+__device__ __forceinline__ void merge32_desc_hi(uint32_t (&v)[64]) {
+    if constexpr (J > 0) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const int l = i ^ J;
+            if (l > i) {
+                const uint32_t hi = max(v[32 + i], v[32 + l]), lo = min(v[32 + i], v[32 + l]);
+                v[32 + i] = hi;
+                v[32 + l] = lo;
+            }
+        }
+        merge32_desc_hi<J / 2>(v);
+    }
+}
+
+// |k_x| of channel x from the row held as 64 half2 registers.
+__device__ __forceinline__ float row_mag(const uint32_t (&row)[64], int x) {
+    const uint32_t w = row[x >> 1];
+    const uint16_t hb = static_cast<uint16_t>((x & 1) ? (w >> 16) : (w & 0xffffu));
+    return fabsf(__half2float(__ushort_as_half(hb)));
+}
+
+// a_x from shared memory through a volatile load, so that the compiler
+// re-reads it where it is used instead of keeping 128 values in registers.
+__device__ __forceinline__ float lds_f32(const float* p) {
+    float v;
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(smem_u32(p)));
+    return v;
+}
+
+// 16-bit key of channel x: bits [30:15] of the fp32 product (monotone).
+__device__ __forceinline__ uint32_t key_bits(float mag, float a) {
+    return __float_as_uint(__fmul_rn(mag, a)) << 1;   // key in the high half
+}
+
+__global__ void __launch_bounds__(128) chan_kernel_c32(const __grid_constant__ ChanArgs A) {
+    const int u = blockIdx.y;
+    const int b = u / A.Hkv, h = u % A.Hkv;
+    const int r0 = A.plan.r0[b];
+    const int ntok = A.plan.nseg[b] * A.S;
+    const int base = blockIdx.x * 128;
+    if (base >= ntok) return;
+    __shared__ float af[128];
+    const int tid = threadIdx.x;
+    af[tid] = A.a[static_cast<int64_t>(u) * kHeadDim + tid];
+    __syncthreads();
+    const int t = base + tid;
+    if (t >= ntok) return;
+    const int c = A.c;
+
+    const __half* src = dense_row(A.dv, A.dv.k, b, h, r0 + t, A.status);
+    auto load_row = [&](uint32_t (&row)[64]) {
+#pragma unroll
+        for (int ch = 0; ch < 16; ++ch) {
+            uint4 q = make_uint4(0, 0, 0, 0);
+            if (src) q = *reinterpret_cast<const uint4*>(src + ch * 8);
+            row[4 * ch] = q.x;
+            row[4 * ch + 1] = q.y;
+            row[4 * ch + 2] = q.z;
+            row[4 * ch + 3] = q.w;
+        }
+    };
+    uint32_t srt[64];
+    {
+        uint32_t row[64];
+        load_row(row);
+#pragma unroll
+        for (int i = 0; i < 64; ++i)
+            srt[i] = __byte_perm(key_bits(row_mag(row, 64 + i), lds_f32(af + 64 + i)),
+                                 key_bits(row_mag(row, i), lds_f32(af + i)), 0x7632);
+    }
+    sort32_desc2<0>(srt);
+    sort32_desc2<32>(srt);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) srt[i] = __vmaxu2(srt[i], srt[63 - i]);
+    merge32_desc2<16>(srt);          // hi halves: top 32 of channels 0..63 (H),
+                                     // lo halves: top 32 of 64..127 (L), descending
+#pragma unroll
+    for (int i = 0; i < 32; ++i) srt[32 + i] = max(srt[i] >> 16, srt[31 - i] & 0xffffu);
+    merge32_desc_hi<16>(srt);        // srt[32..63]: top 32 of all 128, descending
+    // v = c-th largest key = smallest of the first c entries
+    uint32_t v = 0xffffffffu;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v = min(v, (i < c) ? srt[32 + i] : 0xffffffffu);
+    int n_gt = 0;
+    bool maybe = ((srt[31] >> 16) == v) || ((srt[31] & 0xffffu) == v);   // H_31 or L_31 == v
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        n_gt += (srt[32 + i] > v);
+        maybe |= (i >= c) && (srt[32 + i] == v);                           // cut inside top 32
+        maybe |= min(srt[i] >> 16, srt[31 - i] & 0xffffu) == v;            // a merge loser
+    }
+    // Channels with key == v are all in unless more of them exist than the
+    // c - n_gt places left; then rank them exactly by (e desc, x asc).
+    // channel x's magnitude from 16-byte chunk loads of the row (L1 hits)
+    auto chunk = [&](int ch) {
+        uint4 q = make_uint4(0, 0, 0, 0);
+        if (src) q = *reinterpret_cast<const uint4*>(src + ch * 8);
+        return q;
+    };
+    auto chunk_mag = [](const uint4& q, int e) -> float {
+        const uint32_t w = (e >> 1) == 0 ? q.x : (e >> 1) == 1 ? q.y : (e >> 1) == 2 ? q.z : q.w;
+        const uint16_t hb = static_cast<uint16_t>((e & 1) ? (w >> 16) : (w & 0xffffu));
+        return fabsf(__half2float(__ushort_as_half(hb)));
+    };
+    uint32_t m0 = 0xffffffffu, m1 = 0xffffffffu, m2 = 0xffffffffu, m3 = 0xffffffffu;
+    if (maybe) {
+        int cand[128];
+        double ce[128];
+        int nc = 0;
+#pragma unroll 1
+        for (int ch = 0; ch < 16; ++ch) {
+            const uint4 q = chunk(ch);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const int x = ch * 8 + e;
+                const float mag = chunk_mag(q, e);
+                const float ax = lds_f32(af + x);
+                if ((key_bits(mag, ax) >> 16) == v) {
+                    cand[nc] = x;
+                    ce[nc] = __dmul_rn(static_cast<double>(mag), static_cast<double>(ax));
+                    ++nc;
+                }
+            }
+        }
+        const int need = c - n_gt;
+        if (nc > need) {
+            m0 = m1 = m2 = m3 = 0;
+            for (int i = 0; i < nc; ++i) {
+                int rank = 0;
+                for (int j = 0; j < nc; ++j)
+                    rank += (ce[j] > ce[i]) || (ce[j] == ce[i] && cand[j] < cand[i]);
+                if (rank < need) {
+                    const int x = cand[i];
+                    const uint32_t bit = 1u << (x & 31);
+                    const int wsel = x >> 5;
+                    if (wsel == 0) m0 |= bit;
+                    else if (wsel == 1) m1 |= bit;
+                    else if (wsel == 2) m2 |= bit;
+                    else m3 |= bit;
+                }
+            }
+        }
+    }
+    const int64_t slot = static_cast<int64_t>(u) * A.g_stride + t;
+    uint8_t* out = A.cidx + slot * c;
+    int k = 0;
+    double tot = 0.0, drop = 0.0;
+#pragma unroll 1
+    for (int ch = 0; ch < 16; ++ch) {
+        const uint4 q = chunk(ch);
+        const uint32_t mw = (ch < 4) ? m0 : (ch < 8) ? m1 : (ch < 12) ? m2 : m3;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const int x = ch * 8 + e;
+            const float mag = chunk_mag(q, e);
+            const float ax = lds_f32(af + x);
+            const uint32_t kx = key_bits(mag, ax) >> 16;
+            const bool in = (kx > v) || (kx == v && ((mw >> (x & 31)) & 1u));
+            const double ex = __dmul_rn(static_cast<double>(mag), static_cast<double>(ax));
+            tot = __dadd_rn(tot, ex);
+            if (in) out[k++] = static_cast<uint8_t>(x);
+            else drop = __dadd_rn(drop, ex);
+        }
+    }
+    const double gv = tot > 0.0 ? __ddiv_rn(drop, tot) : 0.0;
+    A.g[slot] = gv;
+    if (A.dbg_g) A.dbg_g[static_cast<int64_t>(u) * A.dbg_stride + t] = gv;
+}
+
 }  // namespace
 
 // ------------------------------------------------------------------ host
@@ -676,12 +912,7 @@ int score_pass2_smem_bytes(int gwpad) {
 
 cudaError_t launch_scoring(const ScoreLaunch& L, cudaStream_t stream) {
     const int units = L.batch * L.shp.Hkv;
-    prof_begin(stream, kProfWinStats);
-    win_stats_kernel<<<units, kHeadDim, 0, stream>>>(L.qw, L.shp.Hq, L.shp.G, L.shp.W, L.shp.Hkv,
-                                                      L.a, L.dbg_a);
-    prof_end(stream, kProfWinStats);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
+    cudaError_t e = cudaSuccess;
 
     Pass1Args p1;
     p1.plan = L.plan;
@@ -703,9 +934,9 @@ cudaError_t launch_scoring(const ScoreLaunch& L, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
 
     prof_begin(stream, kProfLseMerge);
-    lse_merge_kernel<<<units, L.shp.GWpad, 0, stream>>>(L.part, L.nsplit1, L.shp.GW, L.shp.GWpad,
-                                                         L.shp.Hkv, L.shp.Hq, L.shp.G, L.shp.W,
-                                                         L.lse2, L.dbg_lse);
+    unit_stats_kernel<<<units, 1024, 0, stream>>>(
+        L.part, L.nsplit1, L.shp.GW, L.shp.GWpad, L.shp.Hkv, L.shp.Hq, L.shp.G, L.shp.W, L.qw,
+        L.lse2, L.dbg_lse, L.a, L.dbg_a);
     prof_end(stream, kProfLseMerge);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
@@ -751,7 +982,8 @@ cudaError_t launch_scoring(const ScoreLaunch& L, cudaStream_t stream) {
     dim3 gc((L.max_nseg * L.shp.S + 127) / 128, units);
     if (gc.x > 0) {
         prof_begin(stream, kProfChan);
-        chan_kernel<<<gc, 128, 0, stream>>>(ca);
+        if (L.shp.c <= 32) chan_kernel_c32<<<gc, 128, 0, stream>>>(ca);
+        else chan_kernel_generic<<<gc, 128, 0, stream>>>(ca);
         prof_end(stream, kProfChan);
     }
     return cudaGetLastError();

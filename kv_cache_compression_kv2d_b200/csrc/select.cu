@@ -220,11 +220,13 @@ __global__ void __launch_bounds__(kBudgetThreads) budget_kernel(const __grid_con
         return;
     }
     __shared__ unsigned long long hist[256];
+    __shared__ unsigned int hcnt[256];
     __shared__ long long red[33];
     __shared__ uint64_t s_phi;
     __shared__ uint32_t s_plo;
     __shared__ long long s_below;
     __shared__ int s_mode;            // 0 all full, 1 all steps, 2 threshold
+    __shared__ int s_unique;
     const uint8_t* H = A.hull + static_cast<int64_t>(u) * A.max_nseg * 8;
     const double* EF = A.eff + static_cast<int64_t>(u) * A.max_nseg * 3;
     const int32_t* DB = A.dbytes + static_cast<int64_t>(u) * A.max_nseg * 3;
@@ -243,49 +245,108 @@ __global__ void __launch_bounds__(kBudgetThreads) budget_kernel(const __grid_con
         s_phi = 0;
         s_plo = 0;
         s_below = 0;
+        s_unique = 0;
     }
     __syncthreads();
     const int mode = s_mode;
-    if (mode == 2) {
-        for (int dp = 0; dp < 12; ++dp) {
-            for (int i = tid; i < 256; i += kBudgetThreads) hist[i] = 0;
-            __syncthreads();
-            const uint64_t phi = s_phi;
-            const uint32_t plo = s_plo;
+    // Weighted radix select of the stopping step: the smallest 96-bit key
+    // (hi = ~bits(eff), lo = 4 * segment + step) whose prefix weight exceeds
+    // rem.  8-bit digits from the top; the search ends early once the chosen
+    // digit bucket holds a single key (that key is the answer).
+    for (int dp = 0; mode == 2 && dp < 12; ++dp) {
+        for (int i = tid; i < 256; i += kBudgetThreads) {
+            hist[i] = 0;
+            hcnt[i] = 0;
+        }
+        __syncthreads();
+        const uint64_t phi = s_phi;
+        const uint32_t plo = s_plo;
+        for (int j = tid; j < nseg; j += kBudgetThreads) {
+            const int nv = H[j * 8];
+            for (int k = 1; k < nv; ++k) {
+                const uint64_t hi = upg_hi(EF[j * 3 + k - 1]);
+                const uint32_t lo = static_cast<uint32_t>(j * 4 + k);
+                bool match;
+                int digit;
+                if (dp < 8) {
+                    const int sh = 64 - 8 * dp;   // bits above the digit
+                    match = (dp == 0) || ((hi >> sh) == (phi >> sh));
+                    digit = static_cast<int>((hi >> (56 - 8 * dp)) & 255u);
+                } else {
+                    const int dl = dp - 8;
+                    const int sh = 32 - 8 * dl;
+                    match = (hi == phi) && (dl == 0 || (lo >> sh) == (plo >> sh));
+                    digit = static_cast<int>((lo >> (24 - 8 * dl)) & 255u);
+                }
+                if (match) {
+                    atomicAdd(&hist[digit], static_cast<unsigned long long>(DB[j * 3 + k - 1]));
+                    atomicAdd(&hcnt[digit], 1u);
+                }
+            }
+        }
+        __syncthreads();
+        if (tid < 32) {
+            // lane l owns buckets 8l .. 8l+7; find the first bucket where the
+            // running weight (below + everything before it + it) exceeds rem
+            const int lane = tid;
+            long long wl = 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) wl += static_cast<long long>(hist[lane * 8 + i]);
+            long long incl = wl;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const long long n = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += n;
+            }
+            long long cum = s_below + (incl - wl);
+            int found = -1;
+            long long before = 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const long long hw = static_cast<long long>(hist[lane * 8 + i]);
+                if (found < 0 && cum + hw > rem) {
+                    found = lane * 8 + i;
+                    before = cum;
+                }
+                cum += hw;
+            }
+            const uint32_t bal = __ballot_sync(0xffffffffu, found >= 0);
+            const int src = bal ? (__ffs(bal) - 1) : 31;
+            const int v = __shfl_sync(0xffffffffu, bal ? found : 255, src);
+            const long long bv = __shfl_sync(0xffffffffu, before, src);
+            if (lane == 0) {
+                s_below = bal ? bv : s_below;
+                if (dp < 8) s_phi |= static_cast<uint64_t>(v) << (56 - 8 * dp);
+                else s_plo |= static_cast<uint32_t>(v) << (24 - 8 * (dp - 8));
+                s_unique = (hcnt[v] == 1u);
+            }
+        }
+        __syncthreads();
+        if (s_unique) {
+            // the bucket holds one key: complete the prefix with its bits
+            const uint64_t phi2 = s_phi;
+            const uint32_t plo2 = s_plo;
             for (int j = tid; j < nseg; j += kBudgetThreads) {
                 const int nv = H[j * 8];
                 for (int k = 1; k < nv; ++k) {
                     const uint64_t hi = upg_hi(EF[j * 3 + k - 1]);
                     const uint32_t lo = static_cast<uint32_t>(j * 4 + k);
                     bool match;
-                    int digit;
                     if (dp < 8) {
-                        const int sh = 64 - 8 * dp;   // bits above the digit
-                        match = (dp == 0) || ((hi >> sh) == (phi >> sh));
-                        digit = static_cast<int>((hi >> (56 - 8 * dp)) & 255u);
+                        const int sh = 56 - 8 * dp;   // bits down to this digit
+                        match = (hi >> sh) == (phi2 >> sh);
                     } else {
-                        const int dl = dp - 8;
-                        const int sh = 32 - 8 * dl;
-                        match = (hi == phi) && (dl == 0 || (lo >> sh) == (plo >> sh));
-                        digit = static_cast<int>((lo >> (24 - 8 * dl)) & 255u);
+                        const int sh = 24 - 8 * (dp - 8);
+                        match = (hi == phi2) && ((lo >> sh) == (plo2 >> sh));
                     }
-                    if (match)
-                        atomicAdd(&hist[digit], static_cast<unsigned long long>(DB[j * 3 + k - 1]));
+                    if (match) {
+                        s_phi = hi;
+                        s_plo = lo;
+                    }
                 }
             }
             __syncthreads();
-            if (tid == 0) {
-                long long cum = s_below;
-                int v = 0;
-                for (; v < 255; ++v) {
-                    if (cum + static_cast<long long>(hist[v]) > rem) break;
-                    cum += static_cast<long long>(hist[v]);
-                }
-                s_below = cum;
-                if (dp < 8) s_phi |= static_cast<uint64_t>(v) << (56 - 8 * dp);
-                else s_plo |= static_cast<uint32_t>(v) << (24 - 8 * (dp - 8));
-            }
-            __syncthreads();
+            break;
         }
     }
     const uint64_t phi = s_phi;

@@ -218,3 +218,19 @@ def test_llama8b_32k_layer_all_units(orc):
     res = parallel_map(lambda bh: H.check_compress_unit(orc, run, bh[0], bh[1]), units)
     assert all(r is not None for r in res)
     _check_decode(orc, run)
+
+
+@pytest.mark.parametrize("keep_channels", [32, 20, 48])
+def test_channel_ties_parity(orc, keep_channels):
+    """Keys rounded to multiples of 0.5 (and a constant row) make many
+    channel products tie exactly at the top-c cut: the selection must still
+    match the oracle bit for bit (ties to the lower channel)."""
+    wl = Workload("ties", 1, 2, 4, 128, 1024, 64, 32, 0.3)
+    batch = synth.generate(wl, seed=21)
+    batch.k[:] = (batch.k.float() * 2).round().div(2).to(torch.float16)
+    batch.k[0, 0, 100] = 1.0
+    batch.qw[:] = (batch.qw.float() * 2).round().div(2).to(torch.float16)
+    run = H.make_run(wl, H.to_device(batch), H.params_for(wl, keep_channels=keep_channels))
+    H.compress(run)
+    _check_all_units(orc, run, independent=False)
+    _check_decode(orc, run)
