@@ -247,7 +247,7 @@ KV2D_API kv2d_status kv2d_decode_attn(const kv2d_params* p, int batch, const kv2
  *   It takes no workspace.  Its split partials and per-unit tickets live in
  *   a fixed 8 MiB array in the library's own device memory, which every GPU
  *   that loads the library holds until the process exits.  Calls whose
- *   scratch would exceed 8 MiB (units x splits x G x (d + 2) x 4 bytes plus
+ *   scratch would exceed 8 MiB (units x splits x G x (d + 4) x 4 bytes plus
  *   a few hundred bytes) return KV2D_ERR_WORKSPACE before launching.
  *   The first call on each device looks up the array's device address with
  *   the CUDA runtime; make that first call outside any stream capture.

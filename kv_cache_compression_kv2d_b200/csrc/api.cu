@@ -166,7 +166,7 @@ DecodeLayout decode_layout(const kv2d_params* p, int batch) {
     Carver c;
     c.take(256);
     L.ticket = c.take(units * 4);
-    L.part = c.take(units * kMaxSplitDec * sh.G * (kHeadDim + 2) * 4);
+    L.part = c.take(units * kMaxSplitDec * sh.G * (kHeadDim + 4) * 4);
     L.total = c.off;
     return L;
 }
@@ -686,7 +686,7 @@ kv2d_status kv2d_decode_attn_noalloc(const kv2d_params* p, int batch, const kv2d
     Carver c;
     c.take(256);                                               // status word
     const size_t ticket_off = c.take(units * 4);
-    const size_t part_off = c.take(units * nsplit * sh.G * (kHeadDim + 2) * 4);
+    const size_t part_off = c.take(units * nsplit * sh.G * (kHeadDim + 4) * 4);
     if (c.off > kNoAllocScratchBytes)
         return fail(KV2D_ERR_WORKSPACE,
                     "decode needs %zu bytes of scratch for %lld units x %d splits; the built-in "

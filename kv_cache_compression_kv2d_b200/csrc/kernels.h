@@ -151,7 +151,7 @@ struct DecodeLaunch {
     const __half* q;
     __half* out;
     int nsplit;
-    float* part;               // [units][nsplit][G][d + 2]
+    float* part;               // [units][nsplit][G][4 + d]: M, L, 0, 0, O[d]
     uint32_t* ticket;          // [units]
     uint32_t* status;
 };

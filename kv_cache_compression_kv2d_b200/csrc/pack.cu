@@ -34,10 +34,10 @@ struct PackArgs {
     uint32_t* status;
 };
 
-__device__ __forceinline__ void copy_rows(const __half* base, const DenseView& dv, int b, int h,
-                                          int t0, const int* toks, int ntok, uint8_t* dst,
-                                          uint32_t* status) {
-    // 4 independent 16-byte loads in flight per thread before the stores
+// Copies ntok whole rows (256 bytes each) into dst; rows[i] points at the
+// i-th source row (nullptr -> zeros).  Four 16-byte loads in flight per
+// thread before the stores.
+__device__ __forceinline__ void copy_rows(const __half* const* rows, int ntok, uint8_t* dst) {
     const int n = ntok * 16;
     for (int i0 = threadIdx.x; i0 < n; i0 += 4 * blockDim.x) {
         uint4 v[4];
@@ -46,7 +46,7 @@ __device__ __forceinline__ void copy_rows(const __half* base, const DenseView& d
             const int idx = i0 + k * blockDim.x;
             v[k] = make_uint4(0, 0, 0, 0);
             if (idx < n) {
-                const __half* row = dense_row(dv, base, b, h, t0 + toks[idx >> 4], status);
+                const __half* row = rows[idx >> 4];
                 if (row) v[k] = *reinterpret_cast<const uint4*>(row + (idx & 15) * 8);
             }
         }
@@ -71,10 +71,16 @@ __global__ void __launch_bounds__(128) pack_kernel(const __grid_constant__ PackA
                    static_cast<int64_t>(d & 0xffffffffull) * 16;
     const int t0 = A.plan.r0[b] + j * S;
     __shared__ int toks[256];
+    __shared__ const __half* krows[256];
+    __shared__ const __half* vrows[256];
     const bool sparse_tok = (st == KV2D_TOK || st == KV2D_BOTH);
     const int ntok = sparse_tok ? r : S;
-    for (int i = threadIdx.x; i < ntok; i += blockDim.x)
-        toks[i] = sparse_tok ? A.tidx[slot * r + i] : i;
+    for (int i = threadIdx.x; i < ntok; i += blockDim.x) {
+        const int tk = sparse_tok ? A.tidx[slot * r + i] : i;
+        toks[i] = tk;
+        krows[i] = dense_row(A.dv, A.dv.k, b, h, t0 + tk, A.status);
+        vrows[i] = dense_row(A.dv, A.dv.v, b, h, t0 + tk, A.status);
+    }
     __syncthreads();
     int64_t o = 0;
     if (sparse_tok) {
@@ -83,7 +89,7 @@ __global__ void __launch_bounds__(128) pack_kernel(const __grid_constant__ PackA
         o = pad16(r);
     }
     if (st == KV2D_FULL || st == KV2D_TOK) {
-        copy_rows(A.dv.k, A.dv, b, h, t0, toks, ntok, out + o, A.status);
+        copy_rows(krows, ntok, out + o);
         o += static_cast<int64_t>(ntok) * 256;
     } else {
         const int n = ntok * c;
@@ -100,14 +106,14 @@ __global__ void __launch_bounds__(128) pack_kernel(const __grid_constant__ PackA
             if (i < n) {
                 const int tk = toks[i / c];
                 const int ch = cbase[static_cast<int64_t>(tk) * c + i % c];
-                const __half* row = dense_row(A.dv, A.dv.k, b, h, t0 + tk, A.status);
+                const __half* row = krows[i / c];
                 if (row) val = __half_as_ushort(row[ch]);
             }
             kv[i] = val;
         }
         o += pad16(2 * n);
     }
-    copy_rows(A.dv.v, A.dv, b, h, t0, toks, ntok, out + o, A.status);
+    copy_rows(vrows, ntok, out + o);
 }
 
 }  // namespace

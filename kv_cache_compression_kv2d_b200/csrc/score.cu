@@ -279,6 +279,7 @@ __global__ void unit_stats_kernel(const float2* __restrict__ part, int nsplit, i
     const int grp = tid / kHeadDim, x = tid % kHeadDim;
     const __half* base = qw + (static_cast<int64_t>(b) * Hq + static_cast<int64_t>(h) * G) * W * kHeadDim;
     float s = 0.f;
+#pragma unroll 8
     for (int row = grp; row < GW; row += groups)
         s += fabsf(__half2float(base[static_cast<int64_t>(row) * kHeadDim + x]));
     acc[grp][x] = s;
@@ -671,29 +672,29 @@ __global__ void __launch_bounds__(128) chan_kernel_generic(const __grid_constant
 
 // ---- fast path for c <= 32
 //
-// Keys are the top 16 bits of the fp32 product (exponent + 8 mantissa
-// bits; monotone in the exact product), two per register: register i holds
-// channel i in its high half and channel 64 + i in its low half, so every
-// __vmaxu2 / __vminu2 pair is two compare-exchanges.  Sorting registers
-// 0..31 and 32..63 gives four descending 32-lists; max(X_i, Y_{31-i}) and a
-// bitonic merge give the top 32 of channels 0..63 (high halves) and of
-// 64..127 (low halves); one more scalar merge gives the top 32 of all 128,
-// whose (c-1)-th entry v is the c-th largest 16-bit key.  Channels above v
-// are in, below are out; channels equal to v are all in unless they
-// straddle the cut, in which case they are ranked exactly by (e desc, x asc)
-// with the fp64 products.
+// Keys are fp16 roundings of the fp32 products |k_x| * a_x (correctly
+// rounded twice, so monotone in the exact product; values below 2^-14 are
+// set to 0), two channels per register: register i holds channel i in its
+// low half and channel 64 + i in its high half, so every __hmax2 / __hmin2
+// pair is two compare-exchanges.  Sorting registers 0..31 and 32..63 gives
+// four descending 32-lists; max(X_i, Y_{31-i}) and a bitonic merge give the
+// top 32 of channels 0..63 (low halves) and of 64..127 (high halves); one
+// more merge gives the top 32 of all 128, whose (c-1)-th entry v is the c-th
+// largest key.  Channels above v are in, below are out; channels equal to v
+// are all in unless they straddle the cut, in which case they are ranked
+// exactly by (e desc, x asc) with the fp64 products.
 
-__device__ __forceinline__ void ce2(uint32_t& a, uint32_t& b) {
-    const uint32_t hi = __vmaxu2(a, b), lo = __vminu2(a, b);
+__device__ __forceinline__ void ce2(__half2& a, __half2& b) {
+    const __half2 hi = __hmax2(a, b), lo = __hmin2(a, b);
     a = hi;
     b = lo;
 }
 
 // One bitonic stage (block size K, distance J) on registers O..O+31, then
-// the next; written as template recursion so that every register index is a
-// compile-time constant.
+// the next; template recursion keeps every register index a compile-time
+// constant.
 template <int O, int K, int J>
-__device__ __forceinline__ void sort32_stage2(uint32_t (&v)[64]) {
+__device__ __forceinline__ void sort32_stage2(__half2 (&v)[64]) {
     if constexpr (J > 0) {
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
@@ -710,12 +711,12 @@ __device__ __forceinline__ void sort32_stage2(uint32_t (&v)[64]) {
 }
 
 template <int O>
-__device__ __forceinline__ void sort32_desc2(uint32_t (&v)[64]) {
+__device__ __forceinline__ void sort32_desc2(__half2 (&v)[64]) {
     sort32_stage2<O, 2, 1>(v);
 }
 
 template <int J>
-__device__ __forceinline__ void merge32_desc2(uint32_t (&v)[64]) {
+__device__ __forceinline__ void merge32_desc2(__half2 (&v)[64]) {
     if constexpr (J > 0) {
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
@@ -727,39 +728,24 @@ __device__ __forceinline__ void merge32_desc2(uint32_t (&v)[64]) {
 }
 
 template <int J>
-__device__ __forceinline__ void merge32_desc_hi(uint32_t (&v)[64]) {
+__device__ __forceinline__ void merge32_desc_f(float (&w)[32]) {
     if constexpr (J > 0) {
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
             const int l = i ^ J;
             if (l > i) {
-                const uint32_t hi = max(v[32 + i], v[32 + l]), lo = min(v[32 + i], v[32 + l]);
-                v[32 + i] = hi;
-                v[32 + l] = lo;
+                const float hi = fmaxf(w[i], w[l]), lo = fminf(w[i], w[l]);
+                w[i] = hi;
+                w[l] = lo;
             }
         }
-        merge32_desc_hi<J / 2>(v);
+        merge32_desc_f<J / 2>(w);
     }
 }
 
-// |k_x| of channel x from the row held as 64 half2 registers.
-__device__ __forceinline__ float row_mag(const uint32_t (&row)[64], int x) {
-    const uint32_t w = row[x >> 1];
-    const uint16_t hb = static_cast<uint16_t>((x & 1) ? (w >> 16) : (w & 0xffffu));
-    return fabsf(__half2float(__ushort_as_half(hb)));
-}
-
-// a_x from shared memory through a volatile load, so that the compiler
-// re-reads it where it is used instead of keeping 128 values in registers.
-__device__ __forceinline__ float lds_f32(const float* p) {
-    float v;
-    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(smem_u32(p)));
-    return v;
-}
-
-// 16-bit key of channel x: bits [30:15] of the fp32 product (monotone).
-__device__ __forceinline__ uint32_t key_bits(float mag, float a) {
-    return __float_as_uint(__fmul_rn(mag, a)) << 1;   // key in the high half
+// fp16 key of an fp32 product: 0 below the fp16 normal range, inf above it.
+__device__ __forceinline__ float key_value(float f) {
+    return f < 6.103515625e-05f ? 0.f : f;
 }
 
 __global__ void __launch_bounds__(128) chan_kernel_c32(const __grid_constant__ ChanArgs A) {
@@ -769,108 +755,118 @@ __global__ void __launch_bounds__(128) chan_kernel_c32(const __grid_constant__ C
     const int ntok = A.plan.nseg[b] * A.S;
     const int base = blockIdx.x * 128;
     if (base >= ntok) return;
-    __shared__ float af[128];
+    __shared__ __align__(16) float af[128];
+    __shared__ double ad[128];
     const int tid = threadIdx.x;
-    af[tid] = A.a[static_cast<int64_t>(u) * kHeadDim + tid];
+    {
+        const float av = A.a[static_cast<int64_t>(u) * kHeadDim + tid];
+        af[tid] = av;
+        ad[tid] = static_cast<double>(av);
+    }
     __syncthreads();
     const int t = base + tid;
     if (t >= ntok) return;
     const int c = A.c;
-
     const __half* src = dense_row(A.dv, A.dv.k, b, h, r0 + t, A.status);
-    auto load_row = [&](uint32_t (&row)[64]) {
-#pragma unroll
-        for (int ch = 0; ch < 16; ++ch) {
-            uint4 q = make_uint4(0, 0, 0, 0);
-            if (src) q = *reinterpret_cast<const uint4*>(src + ch * 8);
-            row[4 * ch] = q.x;
-            row[4 * ch + 1] = q.y;
-            row[4 * ch + 2] = q.z;
-            row[4 * ch + 3] = q.w;
-        }
-    };
-    uint32_t srt[64];
-    {
-        uint32_t row[64];
-        load_row(row);
-#pragma unroll
-        for (int i = 0; i < 64; ++i)
-            srt[i] = __byte_perm(key_bits(row_mag(row, 64 + i), lds_f32(af + 64 + i)),
-                                 key_bits(row_mag(row, i), lds_f32(af + i)), 0x7632);
-    }
-    sort32_desc2<0>(srt);
-    sort32_desc2<32>(srt);
-#pragma unroll
-    for (int i = 0; i < 32; ++i) srt[i] = __vmaxu2(srt[i], srt[63 - i]);
-    merge32_desc2<16>(srt);          // hi halves: top 32 of channels 0..63 (H),
-                                     // lo halves: top 32 of 64..127 (L), descending
-#pragma unroll
-    for (int i = 0; i < 32; ++i) srt[32 + i] = max(srt[i] >> 16, srt[31 - i] & 0xffffu);
-    merge32_desc_hi<16>(srt);        // srt[32..63]: top 32 of all 128, descending
-    // v = c-th largest key = smallest of the first c entries
-    uint32_t v = 0xffffffffu;
-#pragma unroll
-    for (int i = 0; i < 32; ++i) v = min(v, (i < c) ? srt[32 + i] : 0xffffffffu);
-    int n_gt = 0;
-    bool maybe = ((srt[31] >> 16) == v) || ((srt[31] & 0xffffu) == v);   // H_31 or L_31 == v
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-        n_gt += (srt[32 + i] > v);
-        maybe |= (i >= c) && (srt[32 + i] == v);                           // cut inside top 32
-        maybe |= min(srt[i] >> 16, srt[31 - i] & 0xffffu) == v;            // a merge loser
-    }
-    // Channels with key == v are all in unless more of them exist than the
-    // c - n_gt places left; then rank them exactly by (e desc, x asc).
-    // channel x's magnitude from 16-byte chunk loads of the row (L1 hits)
     auto chunk = [&](int ch) {
         uint4 q = make_uint4(0, 0, 0, 0);
         if (src) q = *reinterpret_cast<const uint4*>(src + ch * 8);
         return q;
     };
-    auto chunk_mag = [](const uint4& q, int e) -> float {
-        const uint32_t w = (e >> 1) == 0 ? q.x : (e >> 1) == 1 ? q.y : (e >> 1) == 2 ? q.z : q.w;
-        const uint16_t hb = static_cast<uint16_t>((e & 1) ? (w >> 16) : (w & 0xffffu));
-        return fabsf(__half2float(__ushort_as_half(hb)));
-    };
-    uint32_t m0 = 0xffffffffu, m1 = 0xffffffffu, m2 = 0xffffffffu, m3 = 0xffffffffu;
-    if (maybe) {
-        int cand[128];
-        double ce[128];
-        int nc = 0;
-#pragma unroll 1
-        for (int ch = 0; ch < 16; ++ch) {
-            const uint4 q = chunk(ch);
+
+    // packed keys: key[i] = (k(i), k(64 + i)) as half2
+    __half2 key[64], srt[64];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const int x = ch * 8 + e;
-                const float mag = chunk_mag(q, e);
-                const float ax = lds_f32(af + x);
-                if ((key_bits(mag, ax) >> 16) == v) {
-                    cand[nc] = x;
-                    ce[nc] = __dmul_rn(static_cast<double>(mag), static_cast<double>(ax));
-                    ++nc;
-                }
-            }
-        }
-        const int need = c - n_gt;
-        if (nc > need) {
-            m0 = m1 = m2 = m3 = 0;
-            for (int i = 0; i < nc; ++i) {
-                int rank = 0;
-                for (int j = 0; j < nc; ++j)
-                    rank += (ce[j] > ce[i]) || (ce[j] == ce[i] && cand[j] < cand[i]);
-                if (rank < need) {
-                    const int x = cand[i];
-                    const uint32_t bit = 1u << (x & 31);
-                    const int wsel = x >> 5;
-                    if (wsel == 0) m0 |= bit;
-                    else if (wsel == 1) m1 |= bit;
-                    else if (wsel == 2) m2 |= bit;
-                    else m3 |= bit;
-                }
-            }
+    for (int ch = 0; ch < 8; ++ch) {
+        const uint4 lo4 = chunk(ch), hi4 = chunk(ch + 8);
+        const uint32_t lw[4] = {lo4.x, lo4.y, lo4.z, lo4.w};
+        const uint32_t hw[4] = {hi4.x, hi4.y, hi4.z, hi4.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int x = ch * 8 + 2 * e;               // channels x, x+1 and 64+x, 65+x
+            const float2 ml = __half22float2(__habs2(*reinterpret_cast<const __half2*>(&lw[e])));
+            const float2 mh = __half22float2(__habs2(*reinterpret_cast<const __half2*>(&hw[e])));
+            const float2 al = *reinterpret_cast<const float2*>(af + x);
+            const float2 ah = *reinterpret_cast<const float2*>(af + 64 + x);
+            key[x] = __floats2half2_rn(key_value(__fmul_rn(ml.x, al.x)), key_value(__fmul_rn(mh.x, ah.x)));
+            key[x + 1] = __floats2half2_rn(key_value(__fmul_rn(ml.y, al.y)), key_value(__fmul_rn(mh.y, ah.y)));
+            srt[x] = key[x];
+            srt[x + 1] = key[x + 1];
         }
     }
+    sort32_desc2<0>(srt);
+    sort32_desc2<32>(srt);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) srt[i] = __hmax2(srt[i], srt[63 - i]);
+    merge32_desc2<16>(srt);          // low halves: top 32 of channels 0..63 (L),
+                                     // high halves: top 32 of 64..127 (H), descending
+    float w[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+        w[i] = fmaxf(__low2float(srt[i]), __high2float(srt[31 - i]));
+    merge32_desc_f<16>(w);           // top 32 of all 128, descending
+    float vf = __int_as_float(0x7f800000);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) vf = fminf(vf, (i < c) ? w[i] : __int_as_float(0x7f800000));
+    const __half2 vv = __float2half2_rn(vf);   // vf is a key value: exact in fp16
+
+    // membership masks over channels: gt (key > v) and eq (key == v)
+    uint32_t g0 = 0, g1 = 0, g2 = 0, g3 = 0, q0 = 0, q1 = 0, q2 = 0, q3 = 0;
+#pragma unroll
+    for (int i = 0; i < 64; ++i) {
+        const uint32_t gt = __hgt2_mask(key[i], vv), eq = __heq2_mask(key[i], vv);
+        const uint32_t bit = 1u << (i & 31);
+        // low half: channel i; high half: channel 64 + i
+        if (i < 32) {
+            g0 |= (gt & 1u) ? bit : 0u;
+            q0 |= (eq & 1u) ? bit : 0u;
+            g2 |= (gt >> 31) ? bit : 0u;
+            q2 |= (eq >> 31) ? bit : 0u;
+        } else {
+            g1 |= (gt & 1u) ? bit : 0u;
+            q1 |= (eq & 1u) ? bit : 0u;
+            g3 |= (gt >> 31) ? bit : 0u;
+            q3 |= (eq >> 31) ? bit : 0u;
+        }
+    }
+    const int n_gt = __popc(g0) + __popc(g1) + __popc(g2) + __popc(g3);
+    const int n_eq = __popc(q0) + __popc(q1) + __popc(q2) + __popc(q3);
+    if (n_gt + n_eq > c) {
+        // the channels equal to v straddle the cut: keep the c - n_gt best of
+        // them by the exact product (e desc, x asc)
+        const int need = c - n_gt;
+        uint32_t qm[4] = {q0, q1, q2, q3};
+        uint32_t keep[4] = {0, 0, 0, 0};
+        for (int wi = 0; wi < 4; ++wi) {
+            for (uint32_t m = qm[wi]; m; m &= m - 1) {
+                const int x = wi * 32 + __ffs(m) - 1;
+                const uint4 cx = chunk(x >> 3);
+                const uint32_t wx = (x & 7) < 2 ? cx.x : (x & 7) < 4 ? cx.y : (x & 7) < 6 ? cx.z : cx.w;
+                const float mx = fabsf(__half2float(__ushort_as_half(static_cast<uint16_t>((x & 1) ? (wx >> 16) : (wx & 0xffffu)))));
+                const double ex = __dmul_rn(static_cast<double>(mx), ad[x]);
+                int rank = 0;
+                for (int wj = 0; wj < 4; ++wj) {
+                    for (uint32_t m2 = qm[wj]; m2; m2 &= m2 - 1) {
+                        const int y = wj * 32 + __ffs(m2) - 1;
+                        if (y == x) continue;
+                        const uint4 cy = chunk(y >> 3);
+                        const uint32_t wy = (y & 7) < 2 ? cy.x : (y & 7) < 4 ? cy.y : (y & 7) < 6 ? cy.z : cy.w;
+                        const float my = fabsf(__half2float(__ushort_as_half(static_cast<uint16_t>((y & 1) ? (wy >> 16) : (wy & 0xffffu)))));
+                        const double ey = __dmul_rn(static_cast<double>(my), ad[y]);
+                        rank += (ey > ex) || (ey == ex && y < x);
+                    }
+                }
+                if (rank < need) keep[wi] |= 1u << (x & 31);
+            }
+        }
+        q0 = keep[0];
+        q1 = keep[1];
+        q2 = keep[2];
+        q3 = keep[3];
+    }
+    const uint32_t m0 = g0 | q0, m1 = g1 | q1, m2 = g2 | q2, m3 = g3 | q3;
+
+    // g_t: both fp64 sums ascending in x; selected channels written ascending
     const int64_t slot = static_cast<int64_t>(u) * A.g_stride + t;
     uint8_t* out = A.cidx + slot * c;
     int k = 0;
@@ -879,16 +875,14 @@ __global__ void __launch_bounds__(128) chan_kernel_c32(const __grid_constant__ C
     for (int ch = 0; ch < 16; ++ch) {
         const uint4 q = chunk(ch);
         const uint32_t mw = (ch < 4) ? m0 : (ch < 8) ? m1 : (ch < 12) ? m2 : m3;
+        const uint32_t qw[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
             const int x = ch * 8 + e;
-            const float mag = chunk_mag(q, e);
-            const float ax = lds_f32(af + x);
-            const uint32_t kx = key_bits(mag, ax) >> 16;
-            const bool in = (kx > v) || (kx == v && ((mw >> (x & 31)) & 1u));
-            const double ex = __dmul_rn(static_cast<double>(mag), static_cast<double>(ax));
+            const uint16_t hb = static_cast<uint16_t>((e & 1) ? (qw[e >> 1] >> 16) : (qw[e >> 1] & 0xffffu));
+            const double ex = __dmul_rn(static_cast<double>(fabsf(__half2float(__ushort_as_half(hb)))), ad[x]);
             tot = __dadd_rn(tot, ex);
-            if (in) out[k++] = static_cast<uint8_t>(x);
+            if ((mw >> (x & 31)) & 1u) out[k++] = static_cast<uint8_t>(x);
             else drop = __dadd_rn(drop, ex);
         }
     }

@@ -87,14 +87,15 @@ __global__ void __launch_bounds__(kSegWarps * 32) seg_select_kernel(const __grid
     __syncwarp();
     if (lane != 0) return;
 
+    // three independent sums, each sequential in t (one loop for ILP)
     double etok = 0.0, ech = 0.0, ekept = 0.0;
-    for (int t = 0; t < S; ++t)
-        if (!kept[warp][t]) etok = __dadd_rn(etok, static_cast<double>(ss[warp][t]));
-    for (int t = 0; t < S; ++t)
-        ech = __dadd_rn(ech, __dmul_rn(static_cast<double>(ss[warp][t]), gs[warp][t]));
-    for (int t = 0; t < S; ++t)
-        if (kept[warp][t])
-            ekept = __dadd_rn(ekept, __dmul_rn(static_cast<double>(ss[warp][t]), gs[warp][t]));
+    for (int t = 0; t < S; ++t) {
+        const double sv = static_cast<double>(ss[warp][t]);
+        const double sg = __dmul_rn(sv, gs[warp][t]);
+        ech = __dadd_rn(ech, sg);
+        if (kept[warp][t]) ekept = __dadd_rn(ekept, sg);
+        else etok = __dadd_rn(etok, sv);
+    }
     double E[4];
     E[KV2D_FULL] = 0.0;
     E[KV2D_TOK] = etok;
@@ -210,6 +211,10 @@ __device__ __forceinline__ uint64_t upg_hi(double eff) {
     return ~static_cast<uint64_t>(__double_as_longlong(eff));
 }
 
+// Per-segment hull data cached in shared memory when it fits.
+constexpr int kBudgetCacheSegs = 2048;
+constexpr int kBudgetSmem = kBudgetCacheSegs * (8 + 3 * 8 + 3 * 4);
+
 __global__ void __launch_bounds__(kBudgetThreads) budget_kernel(const __grid_constant__ BudgetArgs A) {
     const int u = blockIdx.x;
     const int b = u / A.Hkv, h = u % A.Hkv;
@@ -230,6 +235,22 @@ __global__ void __launch_bounds__(kBudgetThreads) budget_kernel(const __grid_con
     const uint8_t* H = A.hull + static_cast<int64_t>(u) * A.max_nseg * 8;
     const double* EF = A.eff + static_cast<int64_t>(u) * A.max_nseg * 3;
     const int32_t* DB = A.dbytes + static_cast<int64_t>(u) * A.max_nseg * 3;
+    extern __shared__ __align__(16) uint8_t budget_smem[];
+    if (nseg <= kBudgetCacheSegs) {
+        double* efs = reinterpret_cast<double*>(budget_smem);
+        int32_t* dbs = reinterpret_cast<int32_t*>(efs + 3 * kBudgetCacheSegs);
+        uint8_t* hs = reinterpret_cast<uint8_t*>(dbs + 3 * kBudgetCacheSegs);
+        for (int i = tid; i < nseg * 3; i += kBudgetThreads) {
+            efs[i] = EF[i];
+            dbs[i] = DB[i];
+        }
+        for (int i = tid; i < nseg * 2; i += kBudgetThreads)
+            reinterpret_cast<uint32_t*>(hs)[i] = reinterpret_cast<const uint32_t*>(H)[i];
+        __syncthreads();
+        H = hs;
+        EF = efs;
+        DB = dbs;
+    }
 
     long long base_p = 0, wsum_p = 0;
     for (int j = tid; j < nseg; j += kBudgetThreads) {
@@ -261,26 +282,40 @@ __global__ void __launch_bounds__(kBudgetThreads) budget_kernel(const __grid_con
         __syncthreads();
         const uint64_t phi = s_phi;
         const uint32_t plo = s_plo;
-        for (int j = tid; j < nseg; j += kBudgetThreads) {
-            const int nv = H[j * 8];
-            for (int k = 1; k < nv; ++k) {
-                const uint64_t hi = upg_hi(EF[j * 3 + k - 1]);
-                const uint32_t lo = static_cast<uint32_t>(j * 4 + k);
-                bool match;
-                int digit;
-                if (dp < 8) {
-                    const int sh = 64 - 8 * dp;   // bits above the digit
-                    match = (dp == 0) || ((hi >> sh) == (phi >> sh));
-                    digit = static_cast<int>((hi >> (56 - 8 * dp)) & 255u);
-                } else {
-                    const int dl = dp - 8;
-                    const int sh = 32 - 8 * dl;
-                    match = (hi == phi) && (dl == 0 || (lo >> sh) == (plo >> sh));
-                    digit = static_cast<int>((lo >> (24 - 8 * dl)) & 255u);
+        // all lanes of a warp step through (segment, step) slots together so
+        // that equal digits can be combined into one atomic per warp
+        const int lane = tid & 31;
+        for (int j0 = tid - lane; j0 < nseg; j0 += kBudgetThreads) {
+            const int j = j0 + lane;
+            const int nv = (j < nseg) ? H[j * 8] : 0;
+            for (int k = 1; k < 4; ++k) {
+                int digit = -1;
+                uint32_t w = 0;
+                if (k < nv) {
+                    const uint64_t hi = upg_hi(EF[j * 3 + k - 1]);
+                    const uint32_t lo = static_cast<uint32_t>(j * 4 + k);
+                    bool match;
+                    int dg;
+                    if (dp < 8) {
+                        const int sh = 64 - 8 * dp;   // bits above the digit
+                        match = (dp == 0) || ((hi >> sh) == (phi >> sh));
+                        dg = static_cast<int>((hi >> (56 - 8 * dp)) & 255u);
+                    } else {
+                        const int dl = dp - 8;
+                        const int sh = 32 - 8 * dl;
+                        match = (hi == phi) && (dl == 0 || (lo >> sh) == (plo >> sh));
+                        dg = static_cast<int>((lo >> (24 - 8 * dl)) & 255u);
+                    }
+                    if (match) {
+                        digit = dg;
+                        w = static_cast<uint32_t>(DB[j * 3 + k - 1]);
+                    }
                 }
-                if (match) {
-                    atomicAdd(&hist[digit], static_cast<unsigned long long>(DB[j * 3 + k - 1]));
-                    atomicAdd(&hcnt[digit], 1u);
+                const uint32_t peers = __match_any_sync(0xffffffffu, digit);
+                const uint32_t wsum = __reduce_add_sync(peers, w);
+                if (digit >= 0 && lane == __ffs(peers) - 1) {
+                    atomicAdd(&hist[digit], static_cast<unsigned long long>(wsum));
+                    atomicAdd(&hcnt[digit], static_cast<unsigned>(__popc(peers)));
                 }
             }
         }
@@ -460,7 +495,10 @@ cudaError_t launch_selection(const SelectLaunch& L, cudaStream_t stream) {
     ba.arena_stride = L.arena_stride;
     ba.status = L.status;
     prof_begin(stream, kProfBudget);
-    budget_kernel<<<units, kBudgetThreads, 0, stream>>>(ba);
+    cudaError_t e = cudaFuncSetAttribute(budget_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kBudgetSmem);
+    if (e != cudaSuccess) return e;
+    budget_kernel<<<units, kBudgetThreads, kBudgetSmem, stream>>>(ba);
     prof_end(stream, kProfBudget);
     return cudaGetLastError();
 }
