@@ -231,6 +231,8 @@ KV2D_API kv2d_status kv2d_append(const kv2d_params* p, int batch, const kv2d_den
  *   out               device fp16 [batch][Hq][d].
  *   ws, ws_bytes      kv2d_workspace_bytes(p, DECODE, batch, max_seq_len)
  *                     bytes; split partials and per-unit tickets live here.
+ *                     Zero it once before its first use; every completed
+ *                     call leaves the tickets at zero again.
  * Deterministic: fixed split and merge order. */
 KV2D_API kv2d_status kv2d_decode_attn(const kv2d_params* p, int batch, const kv2d_ccache* cc,
                              const kv2d_dense* kv, const int32_t* seq_len_dev,
@@ -252,7 +254,8 @@ KV2D_API kv2d_status kv2d_decode_attn(const kv2d_params* p, int batch, const kv2
  *   The first call on each device looks up the array's device address with
  *   the CUDA runtime; make that first call outside any stream capture.
  *   All calls on a device share the one array and each leaves its partials
- *   behind; the tickets are cleared at the start of every call.  Calls whose
+ *   behind; the array starts zeroed and every completed call leaves its
+ *   per-unit tickets at zero again.  Calls whose
  *   kernels overlap on the GPU (two streams, or two host threads) race on the
  *   array and give wrong results: serialise them.
  *   status_dev: optional device uint32; device-side faults OR their

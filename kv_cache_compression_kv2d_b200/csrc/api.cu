@@ -123,7 +123,7 @@ constexpr int kMaxSplit1 = 64;
 constexpr int kMaxSplitDec = 64;
 
 struct CompressLayout {
-    size_t a, part, lse2, s, g, cidx, tidx, E, hull, eff, db, strat, ok, total;
+    size_t apart, part, s, g, cidx, tidx, E, hull, eff, db, strat, ok, total;
     int64_t s_stride, g_stride;
     int max_nseg;
 };
@@ -138,9 +138,8 @@ CompressLayout compress_layout(const kv2d_params* p, int batch, int64_t max_regi
     const int64_t ns = std::max(L.max_nseg, 1);
     Carver c;
     c.take(256);   // status header
-    L.a = c.take(units * kHeadDim * 4);
+    L.apart = c.take(units * (sh.GWpad / 128) * kHeadDim * 4);
     L.part = c.take(units * sh.GWpad * kMaxSplit1 * 8);
-    L.lse2 = c.take(units * sh.GWpad * 4);
     L.s = c.take(units * L.s_stride * 4);
     L.g = c.take(units * L.g_stride * 8);
     L.cidx = c.take(units * L.g_stride * sh.c);
@@ -249,9 +248,9 @@ bool g_prof_on = false;
 std::vector<ProfRec> g_prof_open;      // begun, not yet ended (one per stage)
 std::vector<ProfRec> g_prof_done;
 
-const char* const kStageNames[kProfStages] = {"win_stats", "score_pass1", "unit_stats",
-                                              "score_pass2", "chan_topc", "seg_select",
-                                              "budget", "pack", "append", "decode"};
+const char* const kStageNames[kProfStages] = {"score_pass1", "score_pass2", "chan_topc",
+                                              "seg_select",  "budget",      "pack",
+                                              "append",      "decode"};
 
 }  // namespace
 
@@ -493,9 +492,8 @@ kv2d_status kv2d_compress(const kv2d_params* p, int batch, const int32_t* seq_le
         SL.kps2 = static_cast<int>(tiles_per * kKeyTile);
         SL.nsplit2 = static_cast<int>((max_tiles + tiles_per - 1) / tiles_per);
     }
-    SL.a = reinterpret_cast<float*>(w + WL.a);
+    SL.apart = reinterpret_cast<float*>(w + WL.apart);
     SL.part = reinterpret_cast<float2*>(w + WL.part);
-    SL.lse2 = reinterpret_cast<float*>(w + WL.lse2);
     SL.s = reinterpret_cast<float*>(w + WL.s);
     SL.s_stride = WL.s_stride;
     SL.g = reinterpret_cast<double*>(w + WL.g);
@@ -712,7 +710,7 @@ kv2d_status kv2d_decode_attn_noalloc(const kv2d_params* p, int batch, const kv2d
     L.out = static_cast<__half*>(out);
     L.nsplit = nsplit;
     L.part = reinterpret_cast<float*>(w + part_off);
-    L.ticket = reinterpret_cast<uint32_t*>(w + ticket_off);   // zeroed by launch_decode
+    L.ticket = reinterpret_cast<uint32_t*>(w + ticket_off);   // left at zero by every call
     L.status = status_dev ? status_dev : reinterpret_cast<uint32_t*>(w);
     cudaError_t e = launch_decode(L, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return fail(KV2D_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));

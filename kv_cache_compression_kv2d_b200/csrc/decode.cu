@@ -31,6 +31,7 @@ constexpr float kNegInfF = -__builtin_huge_valf();
 // ------------------------------------------------------------------ append
 
 __global__ void append_kernel(const __grid_constant__ AppendLaunch A) {
+    pdl_wait();
     const int b = blockIdx.x;
     __shared__ int ok;
     const int t = A.seq_len[b];
@@ -203,6 +204,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(const __grid_consta
     __shared__ float sc[64][G];
     __shared__ uint64_t dsm[kDescCache];
 
+    pdl_wait();
     if (tid == 0) {
         int T = A.seq_len[b];
         int ce = A.comp_end[b];
@@ -517,7 +519,8 @@ int decode_split_count(int units, int64_t max_seq_len, int num_sms) {
 
 cudaError_t launch_append(const AppendLaunch& L, cudaStream_t stream) {
     prof_begin(stream, kProfAppend);
-    append_kernel<<<L.batch, 256, 0, stream>>>(L);
+    cudaError_t e = launch_k(append_kernel, dim3(L.batch), dim3(256), 0, stream, L);
+    if (e != cudaSuccess) return e;
     prof_end(stream, kProfAppend);
     return cudaGetLastError();
 }
@@ -546,16 +549,16 @@ cudaError_t launch_decode(const DecodeLaunch& L, cudaStream_t stream) {
     a.ticket = L.ticket;
     a.status = L.status;
     const int units = L.batch * L.shp.Hkv;
-    cudaError_t e = cudaMemsetAsync(L.ticket, 0, sizeof(uint32_t) * units, stream);
-    if (e != cudaSuccess) return e;
+    cudaError_t e = cudaSuccess;
     dim3 grid(L.nsplit, units);
     prof_begin(stream, kProfDecode);
     switch (L.shp.G) {
-    case 2: decode_kernel<2><<<grid, kDecThreads, 0, stream>>>(a); break;
-    case 4: decode_kernel<4><<<grid, kDecThreads, 0, stream>>>(a); break;
-    case 8: decode_kernel<8><<<grid, kDecThreads, 0, stream>>>(a); break;
+    case 2: e = launch_k(decode_kernel<2>, grid, dim3(kDecThreads), 0, stream, a); break;
+    case 4: e = launch_k(decode_kernel<4>, grid, dim3(kDecThreads), 0, stream, a); break;
+    case 8: e = launch_k(decode_kernel<8>, grid, dim3(kDecThreads), 0, stream, a); break;
     default: return cudaErrorInvalidValue;
     }
+    if (e != cudaSuccess) return e;
     prof_end(stream, kProfDecode);
     return cudaGetLastError();
 }

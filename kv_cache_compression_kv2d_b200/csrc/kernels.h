@@ -6,15 +6,15 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "common.cuh"
 
 namespace kv2d {
 
 // Kernel stages the optional event profiler tells apart.
 enum ProfStage {
-    kProfWinStats = 0,
-    kProfPass1,
-    kProfLseMerge,
+    kProfPass1 = 0,
     kProfPass2,
     kProfChan,
     kProfSegSelect,
@@ -29,6 +29,25 @@ enum ProfStage {
 // (defined in api.cu; a no-op otherwise).
 void prof_begin(cudaStream_t s, int stage);
 void prof_end(cudaStream_t s, int stage);
+
+// Launches kernel on stream with programmatic stream serialization, so that
+// its launch overlaps the tail of the previous kernel in the stream; every
+// kernel calls pdl_wait() before it reads what earlier work wrote.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                     Args&&... args) {
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg;
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 struct UnitShape {
     int32_t Hkv, Hq, G, W, GW, GWpad;
@@ -49,10 +68,9 @@ struct ScoreLaunch {
     int max_region;            // longest region of the call (tokens)
     int max_nseg;
     // workspace
-    float* a;                  // [units][d]
+    float* apart;              // [units][GWpad / 128][d]
     float2* part;              // [units][GWpad][nsplit1]
     int nsplit1, kps1;
-    float* lse2;               // [units][GWpad]
     float* s;                  // [units][s_stride]
     int64_t s_stride;
     int nsplit2, kps2;

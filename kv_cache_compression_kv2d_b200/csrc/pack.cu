@@ -59,6 +59,7 @@ __device__ __forceinline__ void copy_rows(const __half* const* rows, int ntok, u
 }
 
 __global__ void __launch_bounds__(128) pack_kernel(const __grid_constant__ PackArgs A) {
+    pdl_wait();
     const int j = blockIdx.x, u = blockIdx.y;
     const int b = u / A.Hkv, h = u % A.Hkv;
     if (j >= A.plan.nseg[b] || !A.unit_ok[u]) return;
@@ -140,7 +141,8 @@ cudaError_t launch_pack(const PackLaunch& L, cudaStream_t stream) {
     a.status = L.status;
     dim3 grid(L.max_nseg, L.batch * L.shp.Hkv);
     prof_begin(stream, kProfPack);
-    pack_kernel<<<grid, 128, 0, stream>>>(a);
+    cudaError_t e = launch_k(pack_kernel, grid, dim3(128), 0, stream, a);
+    if (e != cudaSuccess) return e;
     prof_end(stream, kProfPack);
     return cudaGetLastError();
 }

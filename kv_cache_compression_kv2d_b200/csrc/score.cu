@@ -8,13 +8,14 @@
 // The kernels here compute, per unit (sequence b, KV head h):
 //   pass 1    : lse of every window row over the causal region, from a
 //               tcgen05 product Q_w K^T (M = 128 window rows, N = 128 keys),
-//               split over key ranges -> per-split (max, sum) partials
-//   unit stats: combines the partials in split order, and forms
-//               a_d = mean_{G*W window rows} |q_d|
-//   pass 2    : s_t = sum_rows exp(l - lse) from the transposed product
+//               split over key ranges -> per-split (max, sum) partials; the
+//               first split of each row tile also sums |q_d| over its rows
+//   pass 2    : merges the lse partials in split order, then
+//               s_t = sum_rows exp(l - lse) from the transposed product
 //               K Q_w^T (M = 128 keys, N = window rows) so that each TMEM lane
 //               owns one key and sums over queries in-thread
-//   chan      : per key: top-c channels of |k_d| a_d and g_t in fp64 (a
+//   chan      : a_d = (sum of the |q_d| tile sums) / (G*W); per key: top-c
+//               channels of |k_d| a_d and g_t in fp64 (a
 //               packed 16-bit SIMD selection network for c <= 32, a full
 //               32-bit register sort otherwise)
 // Both products take their operands from shared memory written by TMA with
@@ -68,6 +69,7 @@ struct Pass1Args {
     int paged;
     int kps, nsplit;
     float2* part;
+    float* apart;          // [units][mtiles][d]: sum of |q| over the tile's rows
     uint32_t* status;
 };
 
@@ -84,6 +86,7 @@ __global__ void __launch_bounds__(kPassThreads, 1)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     if (nt == 0) {
+        pdl_wait();
         if (tid < 128) {
             int rho = mt * 128 + tid;
             if (rho < GW)
@@ -103,8 +106,8 @@ __global__ void __launch_bounds__(kPassThreads, 1)
     uint64_t* tempty = tfull + 2;
     uint64_t* qbar = tempty + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(qbar + 1);
-    float* xm = reinterpret_cast<float*>(tmem_slot + 4);
-    float* xl = xm + 128;
+    float* xm = reinterpret_cast<float*>(tmem_slot + 4);   // [256]
+    float* xl = xm + 256;
 
     if (tid == 0) {
         for (int i = 0; i < kP1Stages; ++i) {
@@ -126,6 +129,7 @@ __global__ void __launch_bounds__(kPassThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    pdl_wait();
 
     if (warp == 8) {
         if (lane == 0) {
@@ -224,6 +228,25 @@ __global__ void __launch_bounds__(kPassThreads, 1)
             xm[row] = m;
             xl[row] = l;
         }
+        if (sp == 0) {
+            // sum of |q| over this tile's window rows, two threads per
+            // channel (64 rows each), read from the swizzled Q tile once its
+            // TMA load has landed (a warpgroup with no tiles gets here first)
+            mbar_wait(qbar, 0, A.status);
+            const int x = (wg * 128 + row) & 127, half = (wg * 128 + row) >> 7;
+            const int hf = x >> 6, cw = ((x & 63) * 2) >> 4, wb = ((x & 63) * 2) & 15;
+            float acc = 0.f;
+            for (int rr = half * 64; rr < half * 64 + 64; ++rr) {
+                if (mt * 128 + rr >= GW) break;
+                const uint8_t* p = q_s + hf * 16384 + rr * 128 + ((cw ^ (rr & 7)) << 4) + wb;
+                acc += fabsf(__half2float(*reinterpret_cast<const __half*>(p)));
+            }
+            named_bar_sync(3, 256);
+            if (half == 1) xm[128 + x] = acc;     // xm[128..255] is free space
+            named_bar_sync(3, 256);
+            if (half == 0)
+                A.apart[(static_cast<int64_t>(u) * (GWpad / 128) + mt) * kHeadDim + x] = acc + xm[128 + x];
+        }
         named_bar_sync(1, 256);
         if (wg == 0 && rho < GW) {
             const float m1 = xm[row], l1 = xl[row];
@@ -242,57 +265,6 @@ __global__ void __launch_bounds__(kPassThreads, 1)
     if (warp == 9) tmem_dealloc(tmem, 256);
 }
 
-// ------------------------------------------- lse merge and window stats
-
-// One CTA of 1024 threads per unit: thread rho < G*W (padded) merges the
-// pass-1 partials of window row rho in split order; the block also forms
-// a_d = mean |q_d| over the unit's G*W window rows (row groups of 128 threads,
-// combined in a fixed order).
-__global__ void unit_stats_kernel(const float2* __restrict__ part, int nsplit, int GW, int GWpad,
-                                  int Hkv, int Hq, int G, int W, const __half* __restrict__ qw,
-                                  float* __restrict__ lse2, float* __restrict__ dbg_lse,
-                                  float* __restrict__ a, float* __restrict__ dbg_a) {
-    const int u = blockIdx.x;
-    const int b = u / Hkv, h = u % Hkv;
-    const int tid = threadIdx.x;
-    const int rho = tid;
-    if (rho < GWpad) {
-        float out = __int_as_float(0x7f800000);   // +inf: padded rows weigh nothing
-        if (rho < GW) {
-            const float2* p = part + (static_cast<int64_t>(u) * GWpad + rho) * nsplit;
-            float M = __uint_as_float(kNegInf);
-            for (int s = 0; s < nsplit; ++s) M = fmaxf(M, p[s].x);
-            float L = 0.f;
-            for (int s = 0; s < nsplit; ++s)
-                if (p[s].y > 0.f) L += p[s].y * exp2f(p[s].x - M);
-            out = M + log2f(L);
-            if (dbg_lse) {
-                const int g = rho / W, i = rho % W;
-                dbg_lse[(static_cast<int64_t>(b) * Hq + h * G + g) * W + i] =
-                    out * 0.69314718055994531f;
-            }
-        }
-        lse2[static_cast<int64_t>(u) * GWpad + rho] = out;
-    }
-    __shared__ float acc[8][kHeadDim];
-    const int groups = blockDim.x / kHeadDim;
-    const int grp = tid / kHeadDim, x = tid % kHeadDim;
-    const __half* base = qw + (static_cast<int64_t>(b) * Hq + static_cast<int64_t>(h) * G) * W * kHeadDim;
-    float s = 0.f;
-#pragma unroll 8
-    for (int row = grp; row < GW; row += groups)
-        s += fabsf(__half2float(base[static_cast<int64_t>(row) * kHeadDim + x]));
-    acc[grp][x] = s;
-    __syncthreads();
-    if (tid < kHeadDim) {
-        float t = 0.f;
-        for (int g2 = 0; g2 < groups; ++g2) t += acc[g2][tid];
-        const float v = t / static_cast<float>(GW);
-        a[static_cast<int64_t>(u) * kHeadDim + tid] = v;
-        if (dbg_a) dbg_a[static_cast<int64_t>(u) * kHeadDim + tid] = v;
-    }
-}
-
 // --------------------------------------------------------------- pass 2
 
 struct Pass2Args {
@@ -301,7 +273,9 @@ struct Pass2Args {
     DenseView dv;
     int paged;
     int kps, nstages, nqc, Nc;
-    const float* lse2;
+    const float2* part;    // pass-1 partials [units][GWpad][nsplit1]
+    int nsplit1;
+    float* dbg_lse;
     float* s;
     int64_t s_stride;
     float* dbg_s;
@@ -340,10 +314,6 @@ __global__ void __launch_bounds__(kPassThreads, 1)
     uint64_t* qbar = tempty + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(qbar + 1);
 
-    for (int i = tid; i < GWpad; i += kPassThreads) {
-        lse_s[i] = A.lse2[static_cast<int64_t>(u) * GWpad + i];
-        wpos_s[i] = i % W;
-    }
     if (tid == 0) {
         for (int i = 0; i < NS; ++i) {
             mbar_init(&full[i], 1);
@@ -359,6 +329,28 @@ __global__ void __launch_bounds__(kPassThreads, 1)
     if (warp == 9) {
         tmem_alloc(tmem_slot, ncols);
         tmem_relinquish();
+    }
+    pdl_wait();
+    // lse of every window row: merge the pass-1 split partials in split order
+    // (padded rows get +inf so that they weigh nothing)
+    for (int i = tid; i < GWpad; i += kPassThreads) {
+        float out = __int_as_float(0x7f800000);
+        if (i < A.shp.GW) {
+            const float2* p = A.part + (static_cast<int64_t>(u) * GWpad + i) * A.nsplit1;
+            float M = __uint_as_float(kNegInf);
+            for (int s2 = 0; s2 < A.nsplit1; ++s2) M = fmaxf(M, p[s2].x);
+            float L = 0.f;
+            for (int s2 = 0; s2 < A.nsplit1; ++s2)
+                if (p[s2].y > 0.f) L += p[s2].y * exp2f(p[s2].x - M);
+            out = M + log2f(L);
+            if (A.dbg_lse && sp == 0) {
+                const int g = i / W, wi = i % W;
+                A.dbg_lse[(static_cast<int64_t>(b) * A.shp.Hq + h * A.shp.G + g) * W + wi] =
+                    out * 0.69314718055994531f;
+            }
+        }
+        lse_s[i] = out;
+        wpos_s[i] = i % W;
     }
     tc_fence_before();
     __syncthreads();
@@ -531,9 +523,10 @@ __device__ __forceinline__ void sort128_desc(uint32_t (&v)[128]) {
 
 struct ChanArgs {
     SeqPlan plan;
-    int Hkv, S, c;
+    int Hkv, S, c, GW, mtiles;
     DenseView dv;
-    const float* a;
+    const float* apart;    // [units][mtiles][d] partial sums of |q|
+    float* dbg_a;
     double* g;
     uint8_t* cidx;
     int64_t g_stride;
@@ -541,6 +534,16 @@ struct ChanArgs {
     int64_t dbg_stride;
     uint32_t* status;
 };
+
+// a_x = (sum of the row-tile partial sums, in tile order) / (G * W); the
+// first CTA of a unit also writes it to the debug output.
+__device__ __forceinline__ float chan_weight(const ChanArgs& A, int u, int x) {
+    float s = 0.f;
+    for (int mt = 0; mt < A.mtiles; ++mt) s += A.apart[(static_cast<int64_t>(u) * A.mtiles + mt) * kHeadDim + x];
+    const float v = s / static_cast<float>(A.GW);
+    if (A.dbg_a && blockIdx.x == 0) A.dbg_a[static_cast<int64_t>(u) * kHeadDim + x] = v;
+    return v;
+}
 
 // One thread per key.  The block's 128 key rows sit in shared memory with
 // their 16-byte chunks XOR-swizzled by (row & 7), so that 8 consecutive
@@ -553,6 +556,7 @@ struct ChanArgs {
 // channels above v are in, channels below are out, and channels equal to v
 // are ranked exactly by (e desc, x asc) in fp64 when they straddle the cut.
 __global__ void __launch_bounds__(128) chan_kernel_generic(const __grid_constant__ ChanArgs A) {
+    pdl_wait();
     const int u = blockIdx.y;
     const int b = u / A.Hkv, h = u % A.Hkv;
     const int r0 = A.plan.r0[b];
@@ -562,7 +566,7 @@ __global__ void __launch_bounds__(128) chan_kernel_generic(const __grid_constant
     __shared__ __align__(16) uint8_t rows[128 * 256];
     __shared__ float as[128];
     const int tid = threadIdx.x;
-    as[tid] = A.a[static_cast<int64_t>(u) * kHeadDim + tid];
+    as[tid] = chan_weight(A, u, tid);
     for (int idx = tid; idx < 128 * 16; idx += 128) {
         const int rr = idx >> 4, ch = idx & 15;
         uint4 val = make_uint4(0, 0, 0, 0);
@@ -749,6 +753,7 @@ __device__ __forceinline__ float key_value(float f) {
 }
 
 __global__ void __launch_bounds__(128) chan_kernel_c32(const __grid_constant__ ChanArgs A) {
+    pdl_wait();
     const int u = blockIdx.y;
     const int b = u / A.Hkv, h = u % A.Hkv;
     const int r0 = A.plan.r0[b];
@@ -759,7 +764,7 @@ __global__ void __launch_bounds__(128) chan_kernel_c32(const __grid_constant__ C
     __shared__ double ad[128];
     const int tid = threadIdx.x;
     {
-        const float av = A.a[static_cast<int64_t>(u) * kHeadDim + tid];
+        const float av = chan_weight(A, u, tid);
         af[tid] = av;
         ad[tid] = static_cast<double>(av);
     }
@@ -896,7 +901,7 @@ __global__ void __launch_bounds__(128) chan_kernel_c32(const __grid_constant__ C
 // ------------------------------------------------------------------ host
 
 int score_pass1_smem_bytes() {
-    return 1024 + 32768 + kP1Stages * kStage + 256 + 1024;
+    return 1024 + 32768 + kP1Stages * kStage + 256 + 1536;
 }
 
 int score_pass2_smem_bytes(int gwpad) {
@@ -916,22 +921,16 @@ cudaError_t launch_scoring(const ScoreLaunch& L, cudaStream_t stream) {
     p1.kps = L.kps1;
     p1.nsplit = L.nsplit1;
     p1.part = L.part;
+    p1.apart = L.apart;
     p1.status = L.status;
     const int smem1 = score_pass1_smem_bytes();
     e = cudaFuncSetAttribute(score_pass1_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem1);
     if (e != cudaSuccess) return e;
     dim3 g1(L.nsplit1, L.shp.GWpad / 128, units);
     prof_begin(stream, kProfPass1);
-    score_pass1_kernel<<<g1, kPassThreads, smem1, stream>>>(L.qmap, L.kmap, p1);
-    prof_end(stream, kProfPass1);
-    e = cudaGetLastError();
+    e = launch_k(score_pass1_kernel, g1, dim3(kPassThreads), smem1, stream, L.qmap, L.kmap, p1);
     if (e != cudaSuccess) return e;
-
-    prof_begin(stream, kProfLseMerge);
-    unit_stats_kernel<<<units, 1024, 0, stream>>>(
-        L.part, L.nsplit1, L.shp.GW, L.shp.GWpad, L.shp.Hkv, L.shp.Hq, L.shp.G, L.shp.W, L.qw,
-        L.lse2, L.dbg_lse, L.a, L.dbg_a);
-    prof_end(stream, kProfLseMerge);
+    prof_end(stream, kProfPass1);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
 
@@ -944,7 +943,9 @@ cudaError_t launch_scoring(const ScoreLaunch& L, cudaStream_t stream) {
     p2.nstages = L.shp.GWpad <= 256 ? 4 : 2;
     p2.nqc = L.shp.GWpad <= 256 ? 1 : 2;
     p2.Nc = L.shp.GWpad / p2.nqc;
-    p2.lse2 = L.lse2;
+    p2.part = L.part;
+    p2.nsplit1 = L.nsplit1;
+    p2.dbg_lse = L.dbg_lse;
     p2.s = L.s;
     p2.s_stride = L.s_stride;
     p2.dbg_s = L.dbg_s;
@@ -955,7 +956,8 @@ cudaError_t launch_scoring(const ScoreLaunch& L, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     dim3 g2(L.nsplit2, units);
     prof_begin(stream, kProfPass2);
-    score_pass2_kernel<<<g2, kPassThreads, smem2, stream>>>(L.qmap, L.kmap, p2);
+    e = launch_k(score_pass2_kernel, g2, dim3(kPassThreads), smem2, stream, L.qmap, L.kmap, p2);
+    if (e != cudaSuccess) return e;
     prof_end(stream, kProfPass2);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
@@ -966,7 +968,10 @@ cudaError_t launch_scoring(const ScoreLaunch& L, cudaStream_t stream) {
     ca.S = L.shp.S;
     ca.c = L.shp.c;
     ca.dv = L.dv;
-    ca.a = L.a;
+    ca.GW = L.shp.GW;
+    ca.mtiles = L.shp.GWpad / 128;
+    ca.apart = L.apart;
+    ca.dbg_a = L.dbg_a;
     ca.g = L.g;
     ca.cidx = L.cidx;
     ca.g_stride = L.g_stride;
@@ -976,8 +981,9 @@ cudaError_t launch_scoring(const ScoreLaunch& L, cudaStream_t stream) {
     dim3 gc((L.max_nseg * L.shp.S + 127) / 128, units);
     if (gc.x > 0) {
         prof_begin(stream, kProfChan);
-        if (L.shp.c <= 32) chan_kernel_c32<<<gc, 128, 0, stream>>>(ca);
-        else chan_kernel_generic<<<gc, 128, 0, stream>>>(ca);
+        if (L.shp.c <= 32) e = launch_k(chan_kernel_c32, gc, dim3(128), 0, stream, ca);
+        else e = launch_k(chan_kernel_generic, gc, dim3(128), 0, stream, ca);
+        if (e != cudaSuccess) return e;
         prof_end(stream, kProfChan);
     }
     return cudaGetLastError();

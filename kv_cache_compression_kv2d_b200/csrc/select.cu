@@ -47,6 +47,7 @@ struct SegArgs {
 };
 
 __global__ void __launch_bounds__(kSegWarps * 32) seg_select_kernel(const __grid_constant__ SegArgs A) {
+    pdl_wait();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int u = blockIdx.y;
     const int b = u / A.Hkv;
@@ -216,6 +217,7 @@ constexpr int kBudgetCacheSegs = 2048;
 constexpr int kBudgetSmem = kBudgetCacheSegs * (8 + 3 * 8 + 3 * 4);
 
 __global__ void __launch_bounds__(kBudgetThreads) budget_kernel(const __grid_constant__ BudgetArgs A) {
+    pdl_wait();
     const int u = blockIdx.x;
     const int b = u / A.Hkv, h = u % A.Hkv;
     const int nseg = A.plan.nseg[b];
@@ -470,7 +472,8 @@ cudaError_t launch_selection(const SelectLaunch& L, cudaStream_t stream) {
         sa.dbg_seg_stride = L.dbg_seg_stride;
         dim3 grid((L.max_nseg + kSegWarps - 1) / kSegWarps, units);
         prof_begin(stream, kProfSegSelect);
-        seg_select_kernel<<<grid, kSegWarps * 32, 0, stream>>>(sa);
+        cudaError_t e1 = launch_k(seg_select_kernel, grid, dim3(kSegWarps * 32), 0, stream, sa);
+        if (e1 != cudaSuccess) return e1;
         prof_end(stream, kProfSegSelect);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
@@ -498,7 +501,8 @@ cudaError_t launch_selection(const SelectLaunch& L, cudaStream_t stream) {
     cudaError_t e = cudaFuncSetAttribute(budget_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          kBudgetSmem);
     if (e != cudaSuccess) return e;
-    budget_kernel<<<units, kBudgetThreads, kBudgetSmem, stream>>>(ba);
+    e = launch_k(budget_kernel, dim3(units), dim3(kBudgetThreads), kBudgetSmem, stream, ba);
+    if (e != cudaSuccess) return e;
     prof_end(stream, kProfBudget);
     return cudaGetLastError();
 }
