@@ -186,41 +186,58 @@ __global__ void __launch_bounds__(kPassThreads, 1)
             const int t_base = k_lo + i * kKeyTile;
             const uint32_t taddr = tmem + (static_cast<uint32_t>(lg * 32) << 16) + wg * 128;
             const bool whole = (t_base + kKeyTile - 1 <= lim);
-#pragma unroll 1
-            for (int half = 0; half < 2; ++half) {
-                uint32_t ra[32], rb[32];
-                tmem_ld32(taddr + half * 64, ra);
-                tmem_ld32(taddr + half * 64 + 32, rb);
-                tmem_ld_wait();
-                float x[64];
+            // four 32-column chunks; chunk c+1's TMEM load is in flight while
+            // chunk c is processed (online max / sum in the log2 domain)
+            auto proc = [&](const uint32_t (&r)[32], int cc) {
+                float mraw = __uint_as_float(kNegInf);
+                if (whole) {
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    x[j] = __uint_as_float(ra[j]) * c2;
-                    x[32 + j] = __uint_as_float(rb[j]) * c2;
+                    for (int j = 0; j < 32; ++j) mraw = fmaxf(mraw, __uint_as_float(r[j]));
+                } else {
+                    const int t0 = t_base + cc * 32;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        if (t0 + j <= lim) mraw = fmaxf(mraw, __uint_as_float(r[j]));
                 }
-                if (!whole) {
-                    const int t0 = t_base + half * 64;
-#pragma unroll
-                    for (int j = 0; j < 64; ++j)
-                        if (t0 + j > lim) x[j] = __uint_as_float(kNegInf);
-                }
-                float mx = x[0];
-#pragma unroll
-                for (int j = 1; j < 64; ++j) mx = fmaxf(mx, x[j]);
+                if (mraw == __uint_as_float(kNegInf)) return;     // nothing visible here
+                const float mx = mraw * c2;                       // c2 > 0: order kept
                 if (mx > m) {
                     l = (l == 0.f) ? 0.f : l * fast_exp2(m - mx);
                     m = mx;
                 }
-                if (m != __uint_as_float(kNegInf)) {
-                    float acc0 = 0.f, acc1 = 0.f;
+                const float nm = -m;
+                float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+                if (whole) {
 #pragma unroll
-                    for (int j = 0; j < 64; j += 2) {
-                        acc0 += fast_exp2(x[j] - m);
-                        acc1 += fast_exp2(x[j + 1] - m);
+                    for (int j = 0; j < 32; j += 4) {
+                        a0 += fast_exp2(fmaf(__uint_as_float(r[j]), c2, nm));
+                        a1 += fast_exp2(fmaf(__uint_as_float(r[j + 1]), c2, nm));
+                        a2 += fast_exp2(fmaf(__uint_as_float(r[j + 2]), c2, nm));
+                        a3 += fast_exp2(fmaf(__uint_as_float(r[j + 3]), c2, nm));
                     }
-                    l += acc0 + acc1;
+                } else {
+                    const int t0 = t_base + cc * 32;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const float e = fast_exp2(fmaf(__uint_as_float(r[j]), c2, nm));
+                        a0 += (t0 + j <= lim) ? e : 0.f;
+                    }
                 }
-            }
+                l += (a0 + a1) + (a2 + a3);
+            };
+            uint32_t ra[32], rb[32];
+            tmem_ld32(taddr, ra);
+            tmem_ld_wait(ra);
+            tmem_ld32(taddr + 32, rb);
+            proc(ra, 0);
+            tmem_ld_wait(rb);
+            tmem_ld32(taddr + 64, ra);
+            proc(rb, 1);
+            tmem_ld_wait(ra);
+            tmem_ld32(taddr + 96, rb);
+            proc(ra, 2);
+            tmem_ld_wait(rb);
+            proc(rb, 3);
             tc_fence_before();
             mbar_arrive(&tempty[wg]);
         }
@@ -337,11 +354,20 @@ __global__ void __launch_bounds__(kPassThreads, 1)
         float out = __int_as_float(0x7f800000);
         if (i < A.shp.GW) {
             const float2* p = A.part + (static_cast<int64_t>(u) * GWpad + i) * A.nsplit1;
-            float M = __uint_as_float(kNegInf);
-            for (int s2 = 0; s2 < A.nsplit1; ++s2) M = fmaxf(M, p[s2].x);
-            float L = 0.f;
-            for (int s2 = 0; s2 < A.nsplit1; ++s2)
-                if (p[s2].y > 0.f) L += p[s2].y * exp2f(p[s2].x - M);
+            float M = __uint_as_float(kNegInf), L = 0.f;
+            for (int s0 = 0; s0 < A.nsplit1; s0 += 8) {
+                float2 v[8];
+#pragma unroll
+                for (int k2 = 0; k2 < 8; ++k2)
+                    v[k2] = (s0 + k2 < A.nsplit1) ? p[s0 + k2] : make_float2(__uint_as_float(kNegInf), 0.f);
+#pragma unroll
+                for (int k2 = 0; k2 < 8; ++k2) {
+                    if (!(v[k2].y > 0.f)) continue;
+                    const float M2 = fmaxf(M, v[k2].x);
+                    L = L * exp2f(M - M2) + v[k2].y * exp2f(v[k2].x - M2);
+                    M = M2;
+                }
+            }
             out = M + log2f(L);
             if (A.dbg_lse && sp == 0) {
                 const int g = i / W, wi = i % W;
@@ -426,51 +452,44 @@ __global__ void __launch_bounds__(kPassThreads, 1)
             const int col0 = qc * Nc;
             const int need = t - tw;          // row visible iff wpos >= need
             float sacc = 0.f;
-#pragma unroll 1
-            for (int cc = 0; cc < Nc; cc += 64) {
-                uint32_t ra[32], rb[32];
-                tmem_ld32(taddr + cc, ra);
-                const bool two = (cc + 32 < Nc);
-                if (two) tmem_ld32(taddr + cc + 32, rb);
-                tmem_ld_wait();
+            // 32-column chunks, double-buffered: chunk c+1's TMEM load is in
+            // flight while chunk c is summed
+            auto proc = [&](const uint32_t (&r)[32], int cc) {
                 const float4* l4 = reinterpret_cast<const float4*>(lse_s + col0 + cc);
-                float a0 = 0.f, a1 = 0.f;
+                float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
                 if (need <= 0) {
 #pragma unroll
                     for (int j = 0; j < 32; j += 4) {
                         const float4 lz = l4[j >> 2];
-                        a0 += fast_exp2(__uint_as_float(ra[j]) * c2 - lz.x);
-                        a1 += fast_exp2(__uint_as_float(ra[j + 1]) * c2 - lz.y);
-                        a0 += fast_exp2(__uint_as_float(ra[j + 2]) * c2 - lz.z);
-                        a1 += fast_exp2(__uint_as_float(ra[j + 3]) * c2 - lz.w);
-                    }
-                    if (two) {
-#pragma unroll
-                        for (int j = 0; j < 32; j += 4) {
-                            const float4 lz = l4[(32 + j) >> 2];
-                            a0 += fast_exp2(__uint_as_float(rb[j]) * c2 - lz.x);
-                            a1 += fast_exp2(__uint_as_float(rb[j + 1]) * c2 - lz.y);
-                            a0 += fast_exp2(__uint_as_float(rb[j + 2]) * c2 - lz.z);
-                            a1 += fast_exp2(__uint_as_float(rb[j + 3]) * c2 - lz.w);
-                        }
+                        a0 += fast_exp2(fmaf(__uint_as_float(r[j]), c2, -lz.x));
+                        a1 += fast_exp2(fmaf(__uint_as_float(r[j + 1]), c2, -lz.y));
+                        a2 += fast_exp2(fmaf(__uint_as_float(r[j + 2]), c2, -lz.z));
+                        a3 += fast_exp2(fmaf(__uint_as_float(r[j + 3]), c2, -lz.w));
                     }
                 } else {
                     const int* wp = wpos_s + col0 + cc;
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
-                        const float e = fast_exp2(__uint_as_float(ra[j]) * c2 - lse_s[col0 + cc + j]);
+                        const float e = fast_exp2(fmaf(__uint_as_float(r[j]), c2, -lse_s[col0 + cc + j]));
                         a0 += (wp[j] >= need) ? e : 0.f;
                     }
-                    if (two) {
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) {
-                            const float e =
-                                fast_exp2(__uint_as_float(rb[j]) * c2 - lse_s[col0 + cc + 32 + j]);
-                            a1 += (wp[32 + j] >= need) ? e : 0.f;
-                        }
-                    }
                 }
-                sacc += a0 + a1;
+                sacc += (a0 + a1) + (a2 + a3);
+            };
+            uint32_t ra[32], rb[32];
+            const int nch = Nc / 32;          // 4, 6 or 8 chunks (Nc 128..256)
+            tmem_ld32(taddr, ra);
+            tmem_ld_wait(ra);
+#pragma unroll 1
+            for (int ch = 0; ch < nch; ch += 2) {
+                if (ch + 1 < nch) tmem_ld32(taddr + (ch + 1) * 32, rb);
+                proc(ra, ch * 32);
+                if (ch + 1 < nch) {
+                    tmem_ld_wait(rb);
+                    if (ch + 2 < nch) tmem_ld32(taddr + (ch + 2) * 32, ra);
+                    proc(rb, (ch + 1) * 32);
+                    if (ch + 2 < nch) tmem_ld_wait(ra);
+                }
             }
             tc_fence_before();
             if (split_cols) {
