@@ -90,7 +90,10 @@ enum {
     KV2D_DEV_BLOCK_TABLE = 1,   /* a block-table entry was out of range   */
     KV2D_DEV_CAPACITY = 2,      /* an arena would have overflowed          */
     KV2D_DEV_TIMEOUT = 4,       /* a bounded wait gave up                  */
-    KV2D_DEV_SEQ_RANGE = 8      /* a sequence length was out of range      */
+    KV2D_DEV_SEQ_RANGE = 8,     /* a sequence length was out of range      */
+    KV2D_DEV_BAD_MASK = 16      /* a channel keep-mask without exactly c
+                                   bits (an internal invariant; the packed
+                                   indices of that token were truncated)   */
 };
 
 typedef struct kv2d_params {

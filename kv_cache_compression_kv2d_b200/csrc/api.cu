@@ -123,7 +123,7 @@ constexpr int kMaxSplit1 = 64;
 constexpr int kMaxSplitDec = 64;
 
 struct CompressLayout {
-    size_t apart, part, s, g, cidx, tidx, E, hull, eff, db, strat, ok, total;
+    size_t apart, part, s, g, cmask, tidx, E, hull, eff, db, strat, ok, total;
     int64_t s_stride, g_stride;
     int max_nseg;
 };
@@ -142,7 +142,7 @@ CompressLayout compress_layout(const kv2d_params* p, int batch, int64_t max_regi
     L.part = c.take(units * sh.GWpad * kMaxSplit1 * 8);
     L.s = c.take(units * L.s_stride * 4);
     L.g = c.take(units * L.g_stride * 8);
-    L.cidx = c.take(units * L.g_stride * sh.c);
+    L.cmask = c.take(units * L.g_stride * 16);
     L.tidx = c.take(units * ns * sh.r);
     L.E = c.take(units * ns * 4 * 8);
     L.hull = c.take(units * ns * 8);
@@ -497,7 +497,7 @@ kv2d_status kv2d_compress(const kv2d_params* p, int batch, const int32_t* seq_le
     SL.s = reinterpret_cast<float*>(w + WL.s);
     SL.s_stride = WL.s_stride;
     SL.g = reinterpret_cast<double*>(w + WL.g);
-    SL.cidx = w + WL.cidx;
+    SL.cmask = reinterpret_cast<uint4*>(w + WL.cmask);
     SL.g_stride = WL.g_stride;
     SL.status = reinterpret_cast<uint32_t*>(w);
     if (dbg) {
@@ -565,7 +565,7 @@ kv2d_status kv2d_compress(const kv2d_params* p, int batch, const int32_t* seq_le
     PL.max_nseg = max_nseg;
     PL.dv = SL.dv;
     PL.tidx = XL.tidx;
-    PL.cidx = SL.cidx;
+    PL.cmask = SL.cmask;
     PL.g_stride = WL.g_stride;
     PL.strat = XL.strat;
     PL.unit_ok = XL.unit_ok;

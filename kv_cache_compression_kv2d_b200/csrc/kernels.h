@@ -75,7 +75,7 @@ struct ScoreLaunch {
     int64_t s_stride;
     int nsplit2, kps2;
     double* g;                 // [units][g_stride]
-    uint8_t* cidx;             // [units][g_stride][c]
+    uint4* cmask;              // [units][g_stride]: bit x set iff channel x is kept
     int64_t g_stride;
     uint32_t* status;
     // debug
@@ -128,7 +128,7 @@ struct PackLaunch {
     int batch, max_nseg;
     DenseView dv;
     const uint8_t* tidx;
-    const uint8_t* cidx;
+    const uint4* cmask;
     int64_t g_stride;
     const uint8_t* strat;
     const int32_t* unit_ok;

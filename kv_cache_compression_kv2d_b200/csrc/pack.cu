@@ -11,7 +11,9 @@
 //   BOTH : tidx[r] | cidx[r][c] | Kval[r][c] | V[r][d]
 // with Kval[t][j] = K[t][cidx[t][j]], uint8 indices ascending and tidx
 // segment-relative.  One CTA writes one segment: whole K / V rows move as
-// 16-byte vectors, index and Kval sections as consecutive bytes / halves.
+// 16-byte vectors; the channel indices and Kval of a token are expanded from
+// its 128-bit keep mask, one thread per 32-channel word, each word starting
+// at the popcount of the words below it.
 #include "kernels.h"
 
 namespace kv2d {
@@ -23,7 +25,7 @@ struct PackArgs {
     int Hkv, S, r, c, max_nseg;
     DenseView dv;
     const uint8_t* tidx;
-    const uint8_t* cidx;
+    const uint4* cmask;
     int64_t g_stride;
     const uint8_t* strat;
     const int32_t* unit_ok;
@@ -94,24 +96,29 @@ __global__ void __launch_bounds__(128) pack_kernel(const __grid_constant__ PackA
         o += static_cast<int64_t>(ntok) * 256;
     } else {
         const int n = ntok * c;
-        const uint8_t* cbase = A.cidx + (static_cast<int64_t>(u) * A.g_stride + static_cast<int64_t>(j) * S) * c;
-        for (int i = threadIdx.x; i < pad16(n); i += blockDim.x) {
-            uint8_t val = 0;
-            if (i < n) val = cbase[static_cast<int64_t>(toks[i / c]) * c + i % c];
-            out[o + i] = val;
-        }
-        o += pad16(n);
-        uint16_t* kv = reinterpret_cast<uint16_t*>(out + o);
-        for (int i = threadIdx.x; i < pad16(2 * n) / 2; i += blockDim.x) {
-            uint16_t val = 0;
-            if (i < n) {
-                const int tk = toks[i / c];
-                const int ch = cbase[static_cast<int64_t>(tk) * c + i % c];
-                const __half* row = krows[i / c];
-                if (row) val = __half_as_ushort(row[ch]);
+        const uint4* mbase = A.cmask + static_cast<int64_t>(u) * A.g_stride + static_cast<int64_t>(j) * S;
+        uint8_t* ib = out + o;
+        uint16_t* kv = reinterpret_cast<uint16_t*>(out + o + pad16(n));
+        bool bad = false;
+        for (int it = threadIdx.x; it < ntok * 4; it += blockDim.x) {
+            const int i = it >> 2, wd = it & 3;
+            const uint4 m4 = mbase[toks[i]];
+            int k = i * c + (wd > 0 ? __popc(m4.x) : 0) + (wd > 1 ? __popc(m4.y) : 0) +
+                    (wd > 2 ? __popc(m4.z) : 0);
+            bad |= (__popc(m4.x) + __popc(m4.y) + __popc(m4.z) + __popc(m4.w)) != c;
+            const int kend = (i + 1) * c;
+            const __half* row = krows[i];
+            for (uint32_t m = wd == 0 ? m4.x : wd == 1 ? m4.y : wd == 2 ? m4.z : m4.w; m && k < kend; m &= m - 1) {
+                const int x = wd * 32 + __ffs(m) - 1;
+                ib[k] = static_cast<uint8_t>(x);
+                kv[k] = row ? __half_as_ushort(row[x]) : static_cast<uint16_t>(0);
+                ++k;
             }
-            kv[i] = val;
         }
+        if (bad) atomicOr(A.status, KV2D_DEV_BAD_MASK);
+        for (int i = n + threadIdx.x; i < pad16(n); i += blockDim.x) ib[i] = 0;
+        for (int i = n + threadIdx.x; i < pad16(2 * n) / 2; i += blockDim.x) kv[i] = 0;
+        o += pad16(n);
         o += pad16(2 * n);
     }
     copy_rows(vrows, ntok, out + o);
@@ -130,7 +137,7 @@ cudaError_t launch_pack(const PackLaunch& L, cudaStream_t stream) {
     a.max_nseg = L.max_nseg;
     a.dv = L.dv;
     a.tidx = L.tidx;
-    a.cidx = L.cidx;
+    a.cmask = L.cmask;
     a.g_stride = L.g_stride;
     a.strat = L.strat;
     a.unit_ok = L.unit_ok;

@@ -547,7 +547,7 @@ struct ChanArgs {
     const float* apart;    // [units][mtiles][d] partial sums of |q|
     float* dbg_a;
     double* g;
-    uint8_t* cidx;
+    uint4* cmask;          // [units][g_stride]: bit x set iff channel x is kept
     int64_t g_stride;
     double* dbg_g;
     int64_t dbg_stride;
@@ -672,8 +672,6 @@ __global__ void __launch_bounds__(128) chan_kernel_generic(const __grid_constant
         }
     }
     const int64_t slot = static_cast<int64_t>(u) * A.g_stride + t;
-    uint8_t* out = A.cidx + slot * c;
-    int k = 0;
     double tot = 0.0, drop = 0.0;
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
@@ -683,10 +681,10 @@ __global__ void __launch_bounds__(128) chan_kernel_generic(const __grid_constant
             const int x = w * 32 + bit;
             const double e = __dmul_rn(static_cast<double>(elem(x)), static_cast<double>(as[x]));
             tot = __dadd_rn(tot, e);
-            if ((mw >> bit) & 1u) out[k++] = static_cast<uint8_t>(x);
-            else drop = __dadd_rn(drop, e);
+            if (!((mw >> bit) & 1u)) drop = __dadd_rn(drop, e);
         }
     }
+    A.cmask[slot] = make_uint4(m0, m1, m2, m3);
     const double gv = tot > 0.0 ? __ddiv_rn(drop, tot) : 0.0;
     A.g[slot] = gv;
     if (A.dbg_g) A.dbg_g[static_cast<int64_t>(u) * A.dbg_stride + t] = gv;
@@ -695,17 +693,21 @@ __global__ void __launch_bounds__(128) chan_kernel_generic(const __grid_constant
 
 // ---- fast path for c <= 32
 //
-// Keys are fp16 roundings of the fp32 products |k_x| * a_x (correctly
-// rounded twice, so monotone in the exact product; values below 2^-14 are
-// set to 0), two channels per register: register i holds channel i in its
-// low half and channel 64 + i in its high half, so every __hmax2 / __hmin2
-// pair is two compare-exchanges.  Sorting registers 0..31 and 32..63 gives
-// four descending 32-lists; max(X_i, Y_{31-i}) and a bitonic merge give the
-// top 32 of channels 0..63 (low halves) and of 64..127 (high halves); one
-// more merge gives the top 32 of all 128, whose (c-1)-th entry v is the c-th
-// largest key.  Channels above v are in, below are out; channels equal to v
-// are all in unless they straddle the cut, in which case they are ranked
-// exactly by (e desc, x asc) with the fp64 products.
+// Keys are fp16 roundings of the fp32 products |k_x| * a_x.  Both roundings
+// are correct roundings (fp16 conversion, min / max and compare keep
+// subnormals), so a key is a monotone function of the exact product and
+// key_x > key_y implies e_x > e_y.  Register j holds channels 2j (low half)
+// and 2j + 1 (high half), so each __hmax2 / __hmin2 pair is two
+// compare-exchanges and registers 0..31 / 32..63 hold four lists of 32 keys
+// (even and odd channels of 0..63 and of 64..127).  Each list is sorted by
+// Batcher's odd-even merge network (191 compare-exchanges for 32 inputs);
+// max(X_i, Y_{31-i}) of two descending lists is the set of their 32
+// largest, which a bitonic merge sorts again; one more such split gives the
+// 32 largest keys of all 128 and v, the c-th largest.  Channels with key > v
+// are in and those below are out.  When more than c keys are >= v, the keys
+// equal to v straddle the cut and are ranked exactly by (e desc, x asc) with
+// the fp64 products.  The keys stay in shared memory between the sort and
+// the membership pass, so the sort alone holds the registers.
 
 __device__ __forceinline__ void ce2(__half2& a, __half2& b) {
     const __half2 hi = __hmax2(a, b), lo = __hmin2(a, b);
@@ -713,29 +715,26 @@ __device__ __forceinline__ void ce2(__half2& a, __half2& b) {
     b = lo;
 }
 
-// One bitonic stage (block size K, distance J) on registers O..O+31, then
-// the next; template recursion keeps every register index a compile-time
-// constant.
-template <int O, int K, int J>
-__device__ __forceinline__ void sort32_stage2(__half2 (&v)[64]) {
-    if constexpr (J > 0) {
+// One (p, k) stage of Batcher's odd-even merge sort of registers O..O+31
+// into descending order, then the next stage; every register index is a
+// compile-time constant after unrolling.
+template <int O, int P, int K>
+__device__ __forceinline__ void oem32_pass(__half2 (&v)[64]) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            const int l = i ^ J;
-            if (l > i) {
-                if ((i & K) == 0) ce2(v[O + i], v[O + l]);
-                else ce2(v[O + l], v[O + i]);
-            }
+    for (int j = K % P; j + K < 32; j += 2 * K) {
+#pragma unroll
+        for (int i = 0; i < K; ++i) {
+            if (i < 32 - j - K && (i + j) / (2 * P) == (i + j + K) / (2 * P))
+                ce2(v[O + i + j], v[O + i + j + K]);
         }
-        sort32_stage2<O, K, J / 2>(v);
-    } else if constexpr (K < 32) {
-        sort32_stage2<O, K * 2, K>(v);
     }
+    if constexpr (K > 1) oem32_pass<O, P, K / 2>(v);
+    else if constexpr (P < 16) oem32_pass<O, P * 2, P * 2>(v);
 }
 
 template <int O>
 __device__ __forceinline__ void sort32_desc2(__half2 (&v)[64]) {
-    sort32_stage2<O, 2, 1>(v);
+    oem32_pass<O, 1, 1>(v);
 }
 
 template <int J>
@@ -766,9 +765,31 @@ __device__ __forceinline__ void merge32_desc_f(float (&w)[32]) {
     }
 }
 
-// fp16 key of an fp32 product: 0 below the fp16 normal range, inf above it.
-__device__ __forceinline__ float key_value(float f) {
-    return f < 6.103515625e-05f ? 0.f : f;
+// Membership masks of one thread's 128 keys against v: bit x of M[x / 32]
+// is set iff key_x >= v (kStrict: key_x > v).  ks[g][tid] holds the four
+// key registers of channels 8g..8g+7.  A compare yields 0xffff per half;
+// one AND-OR per register moves both flags to spare bit positions, and a
+// final shuffle puts each channel at its own bit.
+template <bool kStrict>
+__device__ __forceinline__ void key_masks(const uint4 (*ks)[128], int tid, __half2 vv, uint32_t (&M)[4]) {
+#pragma unroll
+    for (int wd = 0; wd < 4; ++wd) {
+        uint32_t lo = 0, hi = 0;
+#pragma unroll
+        for (int g4 = 0; g4 < 4; ++g4) {
+            const uint4 q = ks[wd * 4 + g4][tid];
+            const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int s = g4 * 4 + e;        // channels 2s, 2s + 1 of this word
+                const __half2 kk = *reinterpret_cast<const __half2*>(&w[e]);
+                const uint32_t mk = kStrict ? __hgt2_mask(kk, vv) : __hge2_mask(kk, vv);
+                if (s < 8) lo |= mk & ((1u << (2 * s)) | (1u << (2 * s + 17)));
+                else hi |= mk & ((1u << (2 * s - 16)) | (1u << (2 * s + 1)));
+            }
+        }
+        M[wd] = (lo & 0x5555u) | ((lo >> 16) & 0xAAAAu) | ((hi << 16) & 0x55550000u) | (hi & 0xAAAA0000u);
+    }
 }
 
 __global__ void __launch_bounds__(128) chan_kernel_c32(const __grid_constant__ ChanArgs A) {
@@ -780,7 +801,8 @@ __global__ void __launch_bounds__(128) chan_kernel_c32(const __grid_constant__ C
     const int base = blockIdx.x * 128;
     if (base >= ntok) return;
     __shared__ __align__(16) float af[128];
-    __shared__ double ad[128];
+    __shared__ __align__(16) double ad[128];
+    __shared__ uint4 ks[16][128];
     const int tid = threadIdx.x;
     {
         const float av = chan_weight(A, u, tid);
@@ -798,107 +820,94 @@ __global__ void __launch_bounds__(128) chan_kernel_c32(const __grid_constant__ C
         return q;
     };
 
-    // packed keys: key[i] = (k(i), k(64 + i)) as half2
-    __half2 key[64], srt[64];
+    __half2 srt[64];
 #pragma unroll
-    for (int ch = 0; ch < 8; ++ch) {
-        const uint4 lo4 = chunk(ch), hi4 = chunk(ch + 8);
-        const uint32_t lw[4] = {lo4.x, lo4.y, lo4.z, lo4.w};
-        const uint32_t hw[4] = {hi4.x, hi4.y, hi4.z, hi4.w};
+    for (int gi = 0; gi < 16; ++gi) {
+        const uint4 q = chunk(gi);
+        const float4 a0 = *reinterpret_cast<const float4*>(af + 8 * gi);
+        const float4 a1 = *reinterpret_cast<const float4*>(af + 8 * gi + 4);
+        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+        const float al[4] = {a0.x, a0.z, a1.x, a1.z};
+        const float ah[4] = {a0.y, a0.w, a1.y, a1.w};
+        uint32_t kw[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            const int x = ch * 8 + 2 * e;               // channels x, x+1 and 64+x, 65+x
-            const float2 ml = __half22float2(__habs2(*reinterpret_cast<const __half2*>(&lw[e])));
-            const float2 mh = __half22float2(__habs2(*reinterpret_cast<const __half2*>(&hw[e])));
-            const float2 al = *reinterpret_cast<const float2*>(af + x);
-            const float2 ah = *reinterpret_cast<const float2*>(af + 64 + x);
-            key[x] = __floats2half2_rn(key_value(__fmul_rn(ml.x, al.x)), key_value(__fmul_rn(mh.x, ah.x)));
-            key[x + 1] = __floats2half2_rn(key_value(__fmul_rn(ml.y, al.y)), key_value(__fmul_rn(mh.y, ah.y)));
-            srt[x] = key[x];
-            srt[x + 1] = key[x + 1];
+            const float2 m = __half22float2(*reinterpret_cast<const __half2*>(&w[e]));
+            const __half2 kk = __floats2half2_rn(__fmul_rn(fabsf(m.x), al[e]), __fmul_rn(fabsf(m.y), ah[e]));
+            srt[4 * gi + e] = kk;
+            kw[e] = *reinterpret_cast<const uint32_t*>(&kk);
         }
+        ks[gi][tid] = make_uint4(kw[0], kw[1], kw[2], kw[3]);
     }
     sort32_desc2<0>(srt);
     sort32_desc2<32>(srt);
 #pragma unroll
     for (int i = 0; i < 32; ++i) srt[i] = __hmax2(srt[i], srt[63 - i]);
-    merge32_desc2<16>(srt);          // low halves: top 32 of channels 0..63 (L),
-                                     // high halves: top 32 of 64..127 (H), descending
-    float w[32];
+    merge32_desc2<16>(srt);          // low halves: 32 largest even channels (L),
+                                     // high halves: 32 largest odd channels (H), descending
+    float vf;
+    if (c == 32) {
+        // the 32 largest of all are max(L_i, H_{31-i}); with the halves of
+        // register 31-i swapped, one __hmax2 forms the pairs for i and 31-i
+        __half2 mn = __half2half2(__ushort_as_half(0x7c00));   // +inf
 #pragma unroll
-    for (int i = 0; i < 32; ++i)
-        w[i] = fmaxf(__low2float(srt[i]), __high2float(srt[31 - i]));
-    merge32_desc_f<16>(w);           // top 32 of all 128, descending
-    float vf = __int_as_float(0x7f800000);
+        for (int i = 0; i < 16; ++i) mn = __hmin2(mn, __hmax2(srt[i], __lowhigh2highlow(srt[31 - i])));
+        vf = fminf(__low2float(mn), __high2float(mn));
+    } else {
+        float w[32];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) vf = fminf(vf, (i < c) ? w[i] : __int_as_float(0x7f800000));
+        for (int i = 0; i < 32; ++i) w[i] = fmaxf(__low2float(srt[i]), __high2float(srt[31 - i]));
+        merge32_desc_f<16>(w);       // 32 largest of all 128, descending
+        vf = w[0];
+#pragma unroll
+        for (int i = 1; i < 32; ++i) vf = (i < c) ? w[i] : vf;
+    }
     const __half2 vv = __float2half2_rn(vf);   // vf is a key value: exact in fp16
 
-    // membership masks over channels: gt (key > v) and eq (key == v)
-    uint32_t g0 = 0, g1 = 0, g2 = 0, g3 = 0, q0 = 0, q1 = 0, q2 = 0, q3 = 0;
-#pragma unroll
-    for (int i = 0; i < 64; ++i) {
-        const uint32_t gt = __hgt2_mask(key[i], vv), eq = __heq2_mask(key[i], vv);
-        const uint32_t bit = 1u << (i & 31);
-        // low half: channel i; high half: channel 64 + i
-        if (i < 32) {
-            g0 |= (gt & 1u) ? bit : 0u;
-            q0 |= (eq & 1u) ? bit : 0u;
-            g2 |= (gt >> 31) ? bit : 0u;
-            q2 |= (eq >> 31) ? bit : 0u;
-        } else {
-            g1 |= (gt & 1u) ? bit : 0u;
-            q1 |= (eq & 1u) ? bit : 0u;
-            g3 |= (gt >> 31) ? bit : 0u;
-            q3 |= (eq >> 31) ? bit : 0u;
-        }
-    }
-    const int n_gt = __popc(g0) + __popc(g1) + __popc(g2) + __popc(g3);
-    const int n_eq = __popc(q0) + __popc(q1) + __popc(q2) + __popc(q3);
-    if (n_gt + n_eq > c) {
-        // the channels equal to v straddle the cut: keep the c - n_gt best of
+    uint32_t M[4];
+    key_masks<false>(ks, tid, vv, M);
+    const int n_ge = __popc(M[0]) + __popc(M[1]) + __popc(M[2]) + __popc(M[3]);
+    if (n_ge > c) {
+        // the keys equal to v straddle the cut: keep the c - n_gt best of
         // them by the exact product (e desc, x asc)
-        const int need = c - n_gt;
-        uint32_t qm[4] = {q0, q1, q2, q3};
+        uint32_t G[4];
+        key_masks<true>(ks, tid, vv, G);
+        const int need = c - (__popc(G[0]) + __popc(G[1]) + __popc(G[2]) + __popc(G[3]));
+        const uint32_t qm[4] = {M[0] & ~G[0], M[1] & ~G[1], M[2] & ~G[2], M[3] & ~G[3]};
+        auto exact = [&](int x) {
+            const uint4 cx = chunk(x >> 3);
+            const uint32_t wx = (x & 7) < 2 ? cx.x : (x & 7) < 4 ? cx.y : (x & 7) < 6 ? cx.z : cx.w;
+            const float mx = fabsf(__half2float(__ushort_as_half(static_cast<uint16_t>((x & 1) ? (wx >> 16) : (wx & 0xffffu)))));
+            return __dmul_rn(static_cast<double>(mx), ad[x]);
+        };
         uint32_t keep[4] = {0, 0, 0, 0};
         for (int wi = 0; wi < 4; ++wi) {
             for (uint32_t m = qm[wi]; m; m &= m - 1) {
                 const int x = wi * 32 + __ffs(m) - 1;
-                const uint4 cx = chunk(x >> 3);
-                const uint32_t wx = (x & 7) < 2 ? cx.x : (x & 7) < 4 ? cx.y : (x & 7) < 6 ? cx.z : cx.w;
-                const float mx = fabsf(__half2float(__ushort_as_half(static_cast<uint16_t>((x & 1) ? (wx >> 16) : (wx & 0xffffu)))));
-                const double ex = __dmul_rn(static_cast<double>(mx), ad[x]);
+                const double ex = exact(x);
                 int rank = 0;
                 for (int wj = 0; wj < 4; ++wj) {
                     for (uint32_t m2 = qm[wj]; m2; m2 &= m2 - 1) {
                         const int y = wj * 32 + __ffs(m2) - 1;
                         if (y == x) continue;
-                        const uint4 cy = chunk(y >> 3);
-                        const uint32_t wy = (y & 7) < 2 ? cy.x : (y & 7) < 4 ? cy.y : (y & 7) < 6 ? cy.z : cy.w;
-                        const float my = fabsf(__half2float(__ushort_as_half(static_cast<uint16_t>((y & 1) ? (wy >> 16) : (wy & 0xffffu)))));
-                        const double ey = __dmul_rn(static_cast<double>(my), ad[y]);
+                        const double ey = exact(y);
                         rank += (ey > ex) || (ey == ex && y < x);
                     }
                 }
                 if (rank < need) keep[wi] |= 1u << (x & 31);
             }
         }
-        q0 = keep[0];
-        q1 = keep[1];
-        q2 = keep[2];
-        q3 = keep[3];
+#pragma unroll
+        for (int wi = 0; wi < 4; ++wi) M[wi] = G[wi] | keep[wi];
     }
-    const uint32_t m0 = g0 | q0, m1 = g1 | q1, m2 = g2 | q2, m3 = g3 | q3;
 
-    // g_t: both fp64 sums ascending in x; selected channels written ascending
+    // g_t: both fp64 sums ascending in x
     const int64_t slot = static_cast<int64_t>(u) * A.g_stride + t;
-    uint8_t* out = A.cidx + slot * c;
-    int k = 0;
     double tot = 0.0, drop = 0.0;
 #pragma unroll 1
     for (int ch = 0; ch < 16; ++ch) {
         const uint4 q = chunk(ch);
-        const uint32_t mw = (ch < 4) ? m0 : (ch < 8) ? m1 : (ch < 12) ? m2 : m3;
+        const uint32_t mw = (ch < 4) ? M[0] : (ch < 8) ? M[1] : (ch < 12) ? M[2] : M[3];
         const uint32_t qw[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
@@ -906,10 +915,10 @@ __global__ void __launch_bounds__(128) chan_kernel_c32(const __grid_constant__ C
             const uint16_t hb = static_cast<uint16_t>((e & 1) ? (qw[e >> 1] >> 16) : (qw[e >> 1] & 0xffffu));
             const double ex = __dmul_rn(static_cast<double>(fabsf(__half2float(__ushort_as_half(hb)))), ad[x]);
             tot = __dadd_rn(tot, ex);
-            if ((mw >> (x & 31)) & 1u) out[k++] = static_cast<uint8_t>(x);
-            else drop = __dadd_rn(drop, ex);
+            if (!((mw >> (x & 31)) & 1u)) drop = __dadd_rn(drop, ex);
         }
     }
+    A.cmask[slot] = make_uint4(M[0], M[1], M[2], M[3]);
     const double gv = tot > 0.0 ? __ddiv_rn(drop, tot) : 0.0;
     A.g[slot] = gv;
     if (A.dbg_g) A.dbg_g[static_cast<int64_t>(u) * A.dbg_stride + t] = gv;
@@ -992,7 +1001,7 @@ cudaError_t launch_scoring(const ScoreLaunch& L, cudaStream_t stream) {
     ca.apart = L.apart;
     ca.dbg_a = L.dbg_a;
     ca.g = L.g;
-    ca.cidx = L.cidx;
+    ca.cmask = L.cmask;
     ca.g_stride = L.g_stride;
     ca.dbg_g = L.dbg_g;
     ca.dbg_stride = L.dbg_stride;

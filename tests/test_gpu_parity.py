@@ -139,6 +139,19 @@ def test_full_budget_equals_dense_attention(orc):
     assert float((out[0] - ref).abs().max()) <= H.TOL_OUT
 
 
+def test_subnormal_channel_products(orc):
+    """K scaled by 2^-13 (exact in fp16 down to its subnormal grid): the
+    channel products |k_x| a_x then lie on both sides of the smallest normal
+    fp16, so channel selection ranks fp16 subnormal keys too."""
+    wl = CASES["ragged_multi"]
+    run = _run(wl, seed=7)
+    run.batch.k.mul_(2.0 ** -13)
+    H.compress(run)
+    strats = _check_all_units(orc, run)
+    assert len(strats) > 0
+    _check_decode(orc, run)
+
+
 def test_keep_all_channels_is_token_only(orc):
     wl = CASES["ragged_multi"]
     run = _run(wl, keep_channels=128)
