@@ -544,6 +544,7 @@ struct ChanArgs {
     SeqPlan plan;
     int Hkv, S, c, GW, mtiles;
     DenseView dv;
+    int paged;
     const float* apart;    // [units][mtiles][d] partial sums of |q|
     float* dbg_a;
     double* g;
@@ -792,32 +793,74 @@ __device__ __forceinline__ void key_masks(const uint4 (*ks)[128], int tid, __hal
     }
 }
 
-__global__ void __launch_bounds__(128) chan_kernel_c32(const __grid_constant__ ChanArgs A) {
-    pdl_wait();
+// fp64 acc + v unless (m & bit) != 0: one compare into a predicate and one
+// guarded add, so the skipped add costs no select of the 64-bit value.
+__device__ __forceinline__ double dadd_unless(double acc, double v, uint32_t m, uint32_t bit) {
+    asm("{\n\t.reg .pred p;\n\t.reg .b32 t;\n\t"
+        "and.b32 t, %2, %3;\n\t"
+        "setp.eq.u32 p, t, 0;\n\t"
+        "@p add.rn.f64 %0, %0, %1;\n\t}"
+        : "+d"(acc)
+        : "d"(v), "r"(m), "r"(bit));
+    return acc;
+}
+
+constexpr int kChanTile = 0;                  // 128 K rows, two 64-channel halves (SW128)
+constexpr int kChanKeys = kStage;             // uint4 [16][128]: the keys of each thread
+constexpr int kChanAf = kChanKeys + 32768;    // float [128]
+constexpr int kChanAd = kChanAf + 512;        // double [128]
+constexpr int kChanBar = kChanAd + 1024;      // one mbarrier
+constexpr int kChanSmem = 1024 + kChanBar + 16;
+
+// One CTA per 128 tokens of a unit, one thread per token.  The K tile
+// arrives by TMA in the 128-byte-swizzled layout of the scoring passes
+// (row r, 16-byte chunk j of a 64-channel half at r * 128 + ((j ^ (r & 7))
+// << 4)), so the 8 threads of each quarter-warp read 8 different bank
+// groups.  K is never written by the kernels this one follows, so the
+// copy is issued before the wait on them and overlaps their tail.
+__global__ void __launch_bounds__(128) chan_kernel_c32(const __grid_constant__ CUtensorMap kmap,
+                                                       const __grid_constant__ ChanArgs A) {
+    extern __shared__ uint8_t chan_smem_raw[];
+    uint8_t* sm = align1024(chan_smem_raw);
+    uint8_t* tile = sm + kChanTile;
+    uint4 (*ks)[128] = reinterpret_cast<uint4 (*)[128]>(sm + kChanKeys);
+    float* af = reinterpret_cast<float*>(sm + kChanAf);
+    double* ad = reinterpret_cast<double*>(sm + kChanAd);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + kChanBar);
+
     const int u = blockIdx.y;
     const int b = u / A.Hkv, h = u % A.Hkv;
     const int r0 = A.plan.r0[b];
     const int ntok = A.plan.nseg[b] * A.S;
     const int base = blockIdx.x * 128;
     if (base >= ntok) return;
-    __shared__ __align__(16) float af[128];
-    __shared__ __align__(16) double ad[128];
-    __shared__ uint4 ks[16][128];
     const int tid = threadIdx.x;
+    if (tid == 0) {
+        mbar_init(bar, 1);
+        mbar_fence_init();
+        tma_prefetch_desc(&kmap);
+        mbar_expect_tx(bar, kStage);
+        load_key_tile(tile, &kmap, bar, A.dv, A.paged, b, h, r0 + base, r0 + ntok, A.status);
+    }
+    pdl_wait();
     {
         const float av = chan_weight(A, u, tid);
         af[tid] = av;
         ad[tid] = static_cast<double>(av);
     }
     __syncthreads();
+    if (!mbar_wait(bar, 0, A.status)) return;
     const int t = base + tid;
     if (t >= ntok) return;
     const int c = A.c;
-    const __half* src = dense_row(A.dv, A.dv.k, b, h, r0 + t, A.status);
-    auto chunk = [&](int ch) {
-        uint4 q = make_uint4(0, 0, 0, 0);
-        if (src) q = *reinterpret_cast<const uint4*>(src + ch * 8);
-        return q;
+    const uint8_t* myrow = tile + tid * 128;
+    const int sw = tid & 7;
+    auto chunk = [&](int j) {            // channels 8j .. 8j + 7
+        return *reinterpret_cast<const uint4*>(myrow + (j >> 3) * 16384 + (((j & 7) ^ sw) << 4));
+    };
+    auto kabs = [&](int x) {
+        const __half* p = reinterpret_cast<const __half*>(myrow + (x >> 6) * 16384 + ((((x >> 3) & 7) ^ sw) << 4));
+        return fabsf(__half2float(p[x & 7]));
     };
 
     __half2 srt[64];
@@ -874,23 +917,17 @@ __global__ void __launch_bounds__(128) chan_kernel_c32(const __grid_constant__ C
         key_masks<true>(ks, tid, vv, G);
         const int need = c - (__popc(G[0]) + __popc(G[1]) + __popc(G[2]) + __popc(G[3]));
         const uint32_t qm[4] = {M[0] & ~G[0], M[1] & ~G[1], M[2] & ~G[2], M[3] & ~G[3]};
-        auto exact = [&](int x) {
-            const uint4 cx = chunk(x >> 3);
-            const uint32_t wx = (x & 7) < 2 ? cx.x : (x & 7) < 4 ? cx.y : (x & 7) < 6 ? cx.z : cx.w;
-            const float mx = fabsf(__half2float(__ushort_as_half(static_cast<uint16_t>((x & 1) ? (wx >> 16) : (wx & 0xffffu)))));
-            return __dmul_rn(static_cast<double>(mx), ad[x]);
-        };
         uint32_t keep[4] = {0, 0, 0, 0};
         for (int wi = 0; wi < 4; ++wi) {
             for (uint32_t m = qm[wi]; m; m &= m - 1) {
                 const int x = wi * 32 + __ffs(m) - 1;
-                const double ex = exact(x);
+                const double ex = __dmul_rn(static_cast<double>(kabs(x)), ad[x]);
                 int rank = 0;
                 for (int wj = 0; wj < 4; ++wj) {
                     for (uint32_t m2 = qm[wj]; m2; m2 &= m2 - 1) {
                         const int y = wj * 32 + __ffs(m2) - 1;
                         if (y == x) continue;
-                        const double ey = exact(y);
+                        const double ey = __dmul_rn(static_cast<double>(kabs(y)), ad[y]);
                         rank += (ey > ex) || (ey == ex && y < x);
                     }
                 }
@@ -905,17 +942,20 @@ __global__ void __launch_bounds__(128) chan_kernel_c32(const __grid_constant__ C
     const int64_t slot = static_cast<int64_t>(u) * A.g_stride + t;
     double tot = 0.0, drop = 0.0;
 #pragma unroll 1
-    for (int ch = 0; ch < 16; ++ch) {
-        const uint4 q = chunk(ch);
-        const uint32_t mw = (ch < 4) ? M[0] : (ch < 8) ? M[1] : (ch < 12) ? M[2] : M[3];
+    for (int j = 0; j < 16; ++j) {
+        const uint4 q = chunk(j);
+        const uint32_t mw = ((j < 4) ? M[0] : (j < 8) ? M[1] : (j < 12) ? M[2] : M[3]) >> ((j & 3) * 8);
         const uint32_t qw[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            const int x = ch * 8 + e;
-            const uint16_t hb = static_cast<uint16_t>((e & 1) ? (qw[e >> 1] >> 16) : (qw[e >> 1] & 0xffffu));
-            const double ex = __dmul_rn(static_cast<double>(fabsf(__half2float(__ushort_as_half(hb)))), ad[x]);
-            tot = __dadd_rn(tot, ex);
-            if (!((mw >> (x & 31)) & 1u)) drop = __dadd_rn(drop, ex);
+        for (int e = 0; e < 4; ++e) {
+            const float2 f2 = __half22float2(*reinterpret_cast<const __half2*>(&qw[e]));
+            const double2 a2 = *reinterpret_cast<const double2*>(ad + 8 * j + 2 * e);
+            const double e0 = __dmul_rn(fabs(static_cast<double>(f2.x)), a2.x);
+            const double e1 = __dmul_rn(fabs(static_cast<double>(f2.y)), a2.y);
+            tot = __dadd_rn(tot, e0);
+            drop = dadd_unless(drop, e0, mw, 1u << (2 * e));
+            tot = __dadd_rn(tot, e1);
+            drop = dadd_unless(drop, e1, mw, 2u << (2 * e));
         }
     }
     A.cmask[slot] = make_uint4(M[0], M[1], M[2], M[3]);
@@ -996,6 +1036,7 @@ cudaError_t launch_scoring(const ScoreLaunch& L, cudaStream_t stream) {
     ca.S = L.shp.S;
     ca.c = L.shp.c;
     ca.dv = L.dv;
+    ca.paged = L.paged;
     ca.GW = L.shp.GW;
     ca.mtiles = L.shp.GWpad / 128;
     ca.apart = L.apart;
@@ -1009,8 +1050,12 @@ cudaError_t launch_scoring(const ScoreLaunch& L, cudaStream_t stream) {
     dim3 gc((L.max_nseg * L.shp.S + 127) / 128, units);
     if (gc.x > 0) {
         prof_begin(stream, kProfChan);
-        if (L.shp.c <= 32) e = launch_k(chan_kernel_c32, gc, dim3(128), 0, stream, ca);
-        else e = launch_k(chan_kernel_generic, gc, dim3(128), 0, stream, ca);
+        if (L.shp.c <= 32) {
+            e = cudaFuncSetAttribute(chan_kernel_c32, cudaFuncAttributeMaxDynamicSharedMemorySize, kChanSmem);
+            if (e == cudaSuccess) e = launch_k(chan_kernel_c32, gc, dim3(128), kChanSmem, stream, L.kmap, ca);
+        } else {
+            e = launch_k(chan_kernel_generic, gc, dim3(128), 0, stream, ca);
+        }
         if (e != cudaSuccess) return e;
         prof_end(stream, kProfChan);
     }
