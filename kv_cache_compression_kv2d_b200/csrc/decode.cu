@@ -10,11 +10,14 @@
 //     byte range evenly over nsplit CTAs (a CTA takes the segments whose
 //     first byte falls in its range, found by binary search on the
 //     descriptors, and the tail tokens likewise);
-//   - each warp takes 16-token blocks and runs q.k and p.v on the tensor
-//     cores (mma.sync m16n8k16, fp16 in, fp32 accumulate; the G heads are
-//     the rows of the 16-row tile); key and value fragments come straight
-//     from global memory with 16-byte loads; CH / BOTH keys are first
-//     scattered into a dense 16 x 128 tile in shared memory;
+//   - each warp takes every 8th 16-token block of its CTA's range and runs
+//     q.k and p.v on the tensor cores (mma.sync m16n8k16, fp16 in, fp32
+//     accumulate; the G heads are the rows of the 16-row tile);
+//   - every lane copies the exact 16-byte fragments it will read into its
+//     own shared-memory slots with cp.async, three blocks ahead, so a warp
+//     always has two blocks in flight while it computes a third and every
+//     fragment read is conflict-free; CH / BOTH keys are scattered from
+//     their (index, value) pairs into the key slots of the same stage;
 //   - scores meet an online softmax per head in the log2 domain; warps, then
 //     CTAs, merge their (max, sum, output) partials in a fixed order, the
 //     last CTA of a unit (atomic ticket) writing the fp16 output.
@@ -24,8 +27,11 @@ namespace kv2d {
 
 namespace {
 
-constexpr int kDecWarps = 4;
+constexpr int kDecWarps = 8;
 constexpr int kDecThreads = kDecWarps * 32;
+constexpr int kDecStages = 3;                       // blocks in flight per warp
+constexpr int kDecSlotBytes = 16 * 32 * 16;         // 16 slots x 32 lanes x 16 bytes
+constexpr int kDecSmem = kDecWarps * kDecStages * kDecSlotBytes;
 constexpr float kNegInfF = -__builtin_huge_valf();
 
 // ------------------------------------------------------------------ append
@@ -114,18 +120,35 @@ __device__ __forceinline__ uint4 ld_nc16(const void* p) {
     return *reinterpret_cast<const uint4*>(p);
 }
 
-// One 16-token block.  kw[nt][i]: this lane's key window of row nt*8 + g
-// (chunk i of [32t, 32t+32)); vw[k][i]: value window of row {2t, 2t+1,
-// 2t+8, 2t+9}[k], chunk i of [16g, 16g+16).  ntok valid tokens.
+// m16n8k8: rows 0..7 of A (the heads), k = 8 tokens.
+__device__ __forceinline__ void mma16808(float& d0, float& d1, uint32_t a0, uint32_t b0) {
+    float x2, x3;   // rows 8..15 of the tile: never used
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5}, {%6}, "
+        "{%7, %8, %9, %10};"
+        : "=f"(d0), "=f"(d1), "=f"(x2), "=f"(x3)
+        : "r"(a0), "r"(0u), "r"(b0), "f"(d0), "f"(d1), "f"(0.f), "f"(0.f));
+    (void)x2;
+    (void)x3;
+}
+
+// One 16-token block made of two halves of 8 token rows: rows 0..7 hold
+// nlo valid tokens, rows 8..15 hold nhi (a half is a slice of one segment,
+// or a whole segment of at most 8 tokens).  kw[nt][i]: this lane's key
+// window of row nt*8 + g (chunk i of [32t, 32t+32)); vw[k][i]: value window
+// of row {2t, 2t+1, 2t+8, 2t+9}[k], chunk i of [16g, 16g+16).
+//
+// The running max moves only when a block max exceeds it by more than 8 (in
+// log2 units), so the fp16 numerators stay <= 2^8 and most blocks skip the
+// rescale of O; every partial carries the max it was scaled by.
 __device__ __forceinline__ void mma_block(MmaState& st, const uint32_t (&qa)[8][2], const uint4 (&kw)[2][4],
-                                          const uint4 (&vw)[4][2], int ntok, float c2) {
+                                          const uint4 (&vw)[4][2], int nlo, int nhi, float c2) {
     const int lane = threadIdx.x & 31;
     const int t = lane & 3;
-    float sacc[2][2];
+    float sacc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
-        sacc[nt][0] = 0.f;
-        sacc[nt][1] = 0.f;
+        if (nt == 1 && nhi == 0) break;
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
             const uint4& w = kw[nt][ks >> 1];
@@ -141,15 +164,15 @@ __device__ __forceinline__ void mma_block(MmaState& st, const uint32_t (&qa)[8][
     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-            const int tok = nt * 8 + 2 * t + e;
-            ok[nt * 2 + e] = tok < ntok;
+            ok[nt * 2 + e] = (2 * t + e) < (nt ? nhi : nlo);
             x[nt * 2 + e] = ok[nt * 2 + e] ? sacc[nt][e] * c2 : kNegInfF;
         }
     float bm = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
     bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 1));
     bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 2));
-    const float mn = fmaxf(st.m, bm);
-    const float alpha = (st.m == mn) ? 1.f : fast_exp2(st.m - mn);   // st.m = -inf -> 0
+    const bool move = bm > st.m + 8.f;               // st.m = -inf: any finite bm moves
+    const float mn = move ? bm : st.m;
+    const float alpha = move ? ((st.m == kNegInfF) ? 0.f : fast_exp2(st.m - mn)) : 1.f;
     st.m = mn;
     float p[4];
 #pragma unroll
@@ -166,63 +189,62 @@ __device__ __forceinline__ void mma_block(MmaState& st, const uint32_t (&qa)[8][
     const __half2 pb = __floats2half2_rn(p[2], p[3]);
     const uint32_t a0 = *reinterpret_cast<const uint32_t*>(&pa);
     const uint32_t a2 = *reinterpret_cast<const uint32_t*>(&pb);
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-        // element j of the windows: chunk j / 8, 32-bit word (j % 8) / 2
+    auto bfrag = [&](int j, int k0) {
+        // element j of the windows of rows k0, k0 + 1: chunk j / 8, word (j % 8) / 2
         const int ci = j >> 3, wi = (j & 7) >> 1;
         const uint32_t sel = (j & 1) ? 0x7632u : 0x5410u;
         auto word = [&](const uint4& q4) {
             return wi == 0 ? q4.x : wi == 1 ? q4.y : wi == 2 ? q4.z : q4.w;
         };
-        const uint32_t b0 = __byte_perm(word(vw[0][ci]), word(vw[1][ci]), sel);
-        const uint32_t b1 = __byte_perm(word(vw[2][ci]), word(vw[3][ci]), sel);
-        mma16816(st.o[j][0], st.o[j][1], a0, a2, b0, b1);
+        return __byte_perm(word(vw[k0][ci]), word(vw[k0 + 1][ci]), sel);
+    };
+    if (nhi > 0) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) mma16816(st.o[j][0], st.o[j][1], a0, a2, bfrag(j, 0), bfrag(j, 2));
+    } else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) mma16808(st.o[j][0], st.o[j][1], a0, bfrag(j, 0));
     }
 }
 
-// Position of channel chunk c (16 bytes) of row r in a warp's 16 x 128 key
-// tile, XOR-swizzled so that the fragment loads of 8 lanes hit 8 different
-// bank groups.
-__device__ __forceinline__ int tile_chunk(int r, int c) {
-    return c ^ (((c >> 3) & 1) << 1) ^ (r & 1);
+// 16-byte asynchronous copy global -> shared; src_bytes 0 writes zeros and
+// reads nothing.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+                 : "memory");
 }
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// A 16-token block of one warp.  kind: 0 none, 1 dense rows (FULL / TOK
+// segment or tail), 2 channel-sparse keys (CH / BOTH).
+struct DecBlock {
+    int kind, nlo, nhi;
+    const uint8_t* ci;      // sparse: the block's index bytes
+    const __half* kv;       // sparse: the block's key values
+};
+
+constexpr int kDescPerThread = 4;   // descriptors each thread loads in the prologue
 
 template <int G>
-__global__ void __launch_bounds__(kDecThreads) decode_kernel(const __grid_constant__ DecodeArgs A) {
+__global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_constant__ DecodeArgs A) {
+    extern __shared__ __align__(16) uint8_t dec_smem[];
     const int sp = blockIdx.x, u = blockIdx.y;
     const int b = u / A.Hkv, h = u % A.Hkv;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, t = lane & 3;
     __shared__ float wm[kDecWarps][G], wl[kDecWarps][G];
-    // per-warp 16 x 128 key tiles; reused for the warp partials at the end
-    __shared__ __align__(16) uint8_t ktile[kDecWarps][16 * 256];
-    static_assert(sizeof(float) * kDecWarps * G * kHeadDim <= sizeof(ktile), "partials fit");
-    float (*wo)[G][kHeadDim] = reinterpret_cast<float (*)[G][kHeadDim]>(&ktile[0][0]);
-    __shared__ long long hdr[4];
-    __shared__ int cnt[2];
+    __shared__ int wcnt[kDecWarps][2];
+    __shared__ int item_ctr;
     __shared__ int is_last;
-    __shared__ float sc[64][G];
     __shared__ uint64_t dsm[kDescCache];
+    // the warp partials reuse the stage buffers once every warp is done
+    static_assert(sizeof(float) * kDecWarps * G * kHeadDim <= kDecSmem, "partials fit");
+    static_assert(kDescPerThread * kDecThreads <= kDescCache, "prologue descriptors fit the cache");
+    float (*wo)[G][kHeadDim] = reinterpret_cast<float (*)[G][kHeadDim]>(dec_smem);
 
     pdl_wait();
-    if (tid == 0) {
-        int T = A.seq_len[b];
-        int ce = A.comp_end[b];
-        const int64_t U = A.used_bytes[u];
-        const int cap = A.dv.block_table ? A.dv.max_blocks * A.dv.block_size : A.dv.capacity;
-        if (T < 0 || T > cap || ce < 0 || ce > T) {
-            set_status(A.status, KV2D_DEV_SEQ_RANGE);
-            T = max(0, min(T, cap));
-            ce = max(0, min(ce, T));
-        }
-        const int64_t Wt = U + static_cast<int64_t>(T - ce) * kTailBytes;
-        hdr[0] = Wt * sp / A.nsplit;
-        hdr[1] = Wt * (sp + 1) / A.nsplit;
-        hdr[2] = U;
-        hdr[3] = (static_cast<long long>(ce) << 32) | static_cast<unsigned>(T - ce);
-        cnt[0] = 0;
-        cnt[1] = 0;
-    }
     // q fragments (rows g < G): halves [32t, 32t + 32) of head g, step ks at 4ks
     uint32_t qa[8][2];
     {
@@ -240,14 +262,42 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(const __grid_consta
             qa[ks][1] = (ks & 1) ? w.w : w.y;
         }
     }
-    __syncthreads();
-    const int64_t lo = hdr[0], hi = hdr[1], U = hdr[2];
-    const int ce = static_cast<int>(hdr[3] >> 32), ntail = static_cast<int>(hdr[3] & 0xffffffff);
-    const int nsg = A.n_segs[u];
+    // ---- one round trip: q, the unit's lengths and its first descriptors
     const uint64_t* D = A.desc + static_cast<int64_t>(u) * A.max_segs;
+    int T = A.seq_len[b], ce = A.comp_end[b];
+    const int64_t U = A.used_bytes[u];
+    int nsg = A.n_segs[u];
+    uint64_t dreg[kDescPerThread];
+#pragma unroll
+    for (int k = 0; k < kDescPerThread; ++k) {
+        const int j = tid + k * kDecThreads;
+        dreg[k] = (j < A.max_segs) ? D[j] : 0ull;
+    }
+    {
+        const int cap = A.dv.block_table ? A.dv.max_blocks * A.dv.block_size : A.dv.capacity;
+        if (T < 0 || T > cap || ce < 0 || ce > T || nsg < 0 || nsg > A.max_segs) {
+            if (tid == 0) set_status(A.status, KV2D_DEV_SEQ_RANGE);
+            T = max(0, min(T, cap));
+            ce = max(0, min(ce, T));
+            nsg = max(0, min(nsg, A.max_segs));
+        }
+    }
+    const int ntail = T - ce;
+    const int64_t Wt = U + static_cast<int64_t>(ntail) * kTailBytes;
+    const int64_t lo = Wt * sp / A.nsplit, hi = Wt * (sp + 1) / A.nsplit;
+    // segments whose first byte lies in [lo, hi)
     {
         int c_lo = 0, c_hi = 0;
-        for (int j = tid; j < nsg; j += kDecThreads) {
+#pragma unroll
+        for (int k = 0; k < kDescPerThread; ++k) {
+            const int j = tid + k * kDecThreads;
+            if (j < nsg) {
+                const int64_t off = static_cast<int64_t>(dreg[k] & 0xffffffffull) * 16;
+                c_lo += off < lo;
+                c_hi += off < hi;
+            }
+        }
+        for (int j = tid + kDescPerThread * kDecThreads; j < nsg; j += kDecThreads) {
             const int64_t off = static_cast<int64_t>(D[j] & 0xffffffffull) * 16;
             c_lo += off < lo;
             c_hi += off < hi;
@@ -258,22 +308,36 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(const __grid_consta
             c_hi += __shfl_xor_sync(0xffffffffu, c_hi, o);
         }
         if (lane == 0) {
-            atomicAdd(&cnt[0], c_lo);
-            atomicAdd(&cnt[1], c_hi);
+            wcnt[warp][0] = c_lo;
+            wcnt[warp][1] = c_hi;
         }
+        if (tid == 0) item_ctr = 0;
     }
     __syncthreads();
-    const int j_lo = cnt[0], j_hi = cnt[1];
+    int j_lo = 0, j_hi = 0;
+#pragma unroll
+    for (int w = 0; w < kDecWarps; ++w) {
+        j_lo += wcnt[w][0];
+        j_hi += wcnt[w][1];
+    }
     const bool cached = (j_hi - j_lo) <= kDescCache;
-    if (cached)
-        for (int j = j_lo + tid; j < j_hi; j += kDecThreads) dsm[j - j_lo] = D[j];
-    __syncthreads();
+    if (cached) {
+#pragma unroll
+        for (int k = 0; k < kDescPerThread; ++k) {
+            const int j = tid + k * kDecThreads;
+            if (j >= j_lo && j < j_hi) dsm[j - j_lo] = dreg[k];
+        }
+        for (int j = max(j_lo, kDescPerThread * kDecThreads) + tid; j < j_hi; j += kDecThreads) dsm[j - j_lo] = D[j];
+    }
     auto tail_at_or_after = [&](int64_t x) -> int {
         if (x <= U) return 0;
         const int64_t i = (x - U + kTailBytes - 1) / kTailBytes;
         return static_cast<int>(i < ntail ? i : static_cast<int64_t>(ntail));
     };
     const int t_lo = ce + tail_at_or_after(lo), t_hi = ce + tail_at_or_after(hi);
+    const int ntb = (t_hi - t_lo + 15) >> 4;
+
+    __syncthreads();
 
     MmaState st;
     st.m = kNegInfF;
@@ -284,128 +348,255 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(const __grid_consta
         st.o[j][1] = 0.f;
     }
     const float c2 = A.c2;
+    const int S = A.S, r = A.r, c = A.c;
     const uint8_t* ubase = A.arena + static_cast<int64_t>(u) * A.arena_stride;
-    uint8_t* tile = ktile[warp];
-    const uint4 zero4 = make_uint4(0, 0, 0, 0);
-
-    // dense rows: Kr(i) / Vr(i) point at row i of the block (nullptr -> zeros)
-    auto dense_block = [&](auto Kr, auto Vr, int n) {
-        uint4 kw[2][4], vw[4][2];
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-            const int r = nt * 8 + g;
-            const __half* kp = (r < n) ? Kr(r) : nullptr;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) kw[nt][i] = kp ? ld_nc16(kp + 32 * t + 8 * i) : zero4;
-        }
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const int r = 2 * t + (k & 1) + 8 * (k >> 1);
-            const __half* vp = (r < n) ? Vr(r) : nullptr;
-#pragma unroll
-            for (int i = 0; i < 2; ++i) vw[k][i] = vp ? ld_nc16(vp + 16 * g + 8 * i) : zero4;
-        }
-        mma_block(st, qa, kw, vw, n, c2);
+    const uint32_t wbase = smem_u32(dec_smem) + warp * (kDecStages * kDecSlotBytes);
+    auto slot = [&](int stage, int cidx, int ln) -> uint32_t {
+        return wbase + stage * kDecSlotBytes + (cidx * 32 + ln) * 16;
+    };
+    auto lds16 = [&](uint32_t a) {
+        uint4 v;
+        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                     : "r"(a));
+        return v;
+    };
+    auto desc = [&](int j) -> uint64_t { return cached ? dsm[j - j_lo] : D[j]; };
+    auto seg_ntok = [&](uint64_t d) {
+        const int sty = static_cast<int>((d >> 32) & 255u);
+        return (sty == KV2D_TOK || sty == KV2D_BOTH) ? r : S;
+    };
+    auto seg_dense = [&](uint64_t d) {
+        const int sty = static_cast<int>((d >> 32) & 255u);
+        return sty == KV2D_FULL || sty == KV2D_TOK;
+    };
+    // first K row of a dense segment (its V rows follow its ntok K rows)
+    auto seg_k = [&](uint64_t d) {
+        const int sty = static_cast<int>((d >> 32) & 255u);
+        return reinterpret_cast<const __half*>(ubase + static_cast<int64_t>(d & 0xffffffffull) * 16 +
+                                               (sty == KV2D_TOK ? pad16(r) : 0));
     };
 
-    // ---- work items: (segment, block of 16 tokens), then tail blocks;
-    // item i goes to warp i % kDecWarps
-    int seg = j_lo, item = 0;
-    while (seg < j_hi) {
-        const uint64_t d = cached ? dsm[seg - j_lo] : D[seg];
-        const int sty = static_cast<int>((d >> 32) & 255u);
-        const bool tok = (sty == KV2D_TOK || sty == KV2D_BOTH);
-        const int ntok = tok ? A.r : A.S;
-        const int nblk = (ntok + 15) >> 4;
-        int first = (warp - item) % kDecWarps;
-        if (first < 0) first += kDecWarps;
-        if (first < nblk) {
-            const uint8_t* p0 = ubase + static_cast<int64_t>(d & 0xffffffffull) * 16 + (tok ? pad16(A.r) : 0);
-            for (int blk = first; blk < nblk; blk += kDecWarps) {
-                const int t0 = blk * 16;
-                const int n = min(16, ntok - t0);
-                if (sty == KV2D_FULL || sty == KV2D_TOK) {
-                    const __half* K = reinterpret_cast<const __half*>(p0) + static_cast<int64_t>(t0) * kHeadDim;
-                    const __half* V = reinterpret_cast<const __half*>(p0) + static_cast<int64_t>(ntok + t0) * kHeadDim;
-                    dense_block([&](int i) { return K + static_cast<int64_t>(i) * kHeadDim; },
-                                [&](int i) { return V + static_cast<int64_t>(i) * kHeadDim; }, n);
+    // ---- the CTA's items, in order: a dense segment of at most 8 tokens
+    // pairs with the next one if that is one too (one item, a segment per
+    // half); other segments give one item per 16 tokens; then the dense
+    // tail in 16-token items.  Warps take the next item from a shared
+    // counter when they issue its copies, so they finish together.
+    int g_seg = j_lo, g_base = 0;
+    auto next_block = [&](int stage) -> DecBlock {
+        DecBlock bk{0, 0, 0, nullptr, nullptr};
+        int g_idx = 0;
+        if (lane == 0) g_idx = atomicAdd(&item_ctr, 1);
+        g_idx = __shfl_sync(0xffffffffu, g_idx, 0);
+        const __half* kh[2] = {nullptr, nullptr};   // first K row of each half
+        const __half* vh[2] = {nullptr, nullptr};   // first V row of each half
+        int nh[2] = {0, 0};
+        bool tail = false;
+        uint64_t d = 0;
+        int nitems = 0, t0 = 0;
+        bool pair = false;
+        while (g_seg < j_hi) {
+            d = desc(g_seg);
+            const int ntok = seg_ntok(d);
+            pair = false;
+            if (seg_dense(d) && ntok <= 8) {
+                nitems = 1;
+                if (g_seg + 1 < j_hi) {
+                    const uint64_t d2 = desc(g_seg + 1);
+                    pair = seg_dense(d2) && seg_ntok(d2) <= 8;
+                }
+            } else {
+                nitems = (ntok + 15) >> 4;
+            }
+            if (g_idx < g_base + nitems) break;
+            g_base += nitems;
+            g_seg += pair ? 2 : 1;
+        }
+        if (g_seg < j_hi) {
+            const int ntok = seg_ntok(d);
+            t0 = (g_idx - g_base) * 16;
+            if (seg_dense(d)) {
+                bk.kind = 1;
+                const __half* K = seg_k(d);
+                const __half* V = K + static_cast<int64_t>(ntok) * kHeadDim;
+                if (ntok <= 8) {
+                    kh[0] = K;
+                    vh[0] = V;
+                    nh[0] = ntok;
+                    if (pair) {
+                        const uint64_t d2 = desc(g_seg + 1);
+                        const int n2 = seg_ntok(d2);
+                        kh[1] = seg_k(d2);
+                        vh[1] = kh[1] + static_cast<int64_t>(n2) * kHeadDim;
+                        nh[1] = n2;
+                    }
                 } else {
-                    const int c = A.c;
-                    const uint8_t* ci = p0 + static_cast<int64_t>(t0) * c;
-                    const __half* kv = reinterpret_cast<const __half*>(p0 + pad16(static_cast<int64_t>(ntok) * c)) +
-                                       static_cast<int64_t>(t0) * c;
-                    const __half* V = reinterpret_cast<const __half*>(
-                                          p0 + pad16(static_cast<int64_t>(ntok) * c) +
-                                          pad16(static_cast<int64_t>(ntok) * c * 2)) +
-                                      static_cast<int64_t>(t0) * kHeadDim;
-                    // dense 16 x 128 key tile in shared memory: zero, scatter
 #pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        reinterpret_cast<uint4*>(tile)[lane + 32 * i] = zero4;
-                    __syncwarp();
-                    // 16 (index, value) pairs per lane from three 16-byte loads
-                    // (the pair arrays start 16-byte aligned; a read past the
-                    // last pair stays inside the segment's later sections)
-                    const int np = n * c;
-                    for (int e0 = lane * 16; e0 < np; e0 += 32 * 16) {
-                        const uint4 iw = ld_nc16(ci + e0);
-                        const uint4 va = ld_nc16(kv + e0), vb = ld_nc16(kv + e0 + 8);
-                        const uint32_t iws[4] = {iw.x, iw.y, iw.z, iw.w};
-                        const uint32_t vws[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
-                        int r = e0 / c, col = e0 - r * c;
-#pragma unroll
-                        for (int k = 0; k < 16; ++k) {
-                            if (e0 + k < np) {
-                                const int ch = (iws[k >> 2] >> (8 * (k & 3))) & 0xff;
-                                const uint16_t hv = static_cast<uint16_t>(vws[k >> 1] >> (16 * (k & 1)));
-                                *reinterpret_cast<uint16_t*>(tile + r * 256 + tile_chunk(r, ch >> 3) * 16 + (ch & 7) * 2) = hv;
-                            }
-                            if (++col == c) {
-                                col = 0;
-                                ++r;
-                            }
-                        }
+                    for (int hh = 0; hh < 2; ++hh) {
+                        kh[hh] = K + static_cast<int64_t>(t0 + 8 * hh) * kHeadDim;
+                        vh[hh] = V + static_cast<int64_t>(t0 + 8 * hh) * kHeadDim;
+                        nh[hh] = max(0, min(8, ntok - t0 - 8 * hh));
                     }
-                    __syncwarp();
-                    uint4 kw[2][4], vw[4][2];
+                }
+            } else {
+                bk.kind = 2;
+                const bool tok = ((d >> 32) & 255u) == KV2D_BOTH;
+                const uint8_t* p0 = ubase + static_cast<int64_t>(d & 0xffffffffull) * 16 + (tok ? pad16(r) : 0);
+                bk.ci = p0 + static_cast<int64_t>(t0) * c;
+                bk.kv = reinterpret_cast<const __half*>(p0 + pad16(static_cast<int64_t>(ntok) * c)) +
+                        static_cast<int64_t>(t0) * c;
+                const __half* V = reinterpret_cast<const __half*>(p0 + pad16(static_cast<int64_t>(ntok) * c) +
+                                                                  pad16(static_cast<int64_t>(ntok) * c * 2)) +
+                                  static_cast<int64_t>(t0) * kHeadDim;
 #pragma unroll
-                    for (int nt = 0; nt < 2; ++nt) {
-                        const int r = nt * 8 + g;
-#pragma unroll
-                        for (int i = 0; i < 4; ++i)
-                            kw[nt][i] = *reinterpret_cast<const uint4*>(tile + r * 256 + tile_chunk(r, 4 * t + i) * 16);
-                    }
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const int r = 2 * t + (k & 1) + 8 * (k >> 1);
-#pragma unroll
-                        for (int i = 0; i < 2; ++i)
-                            vw[k][i] = (r < n) ? ld_nc16(V + static_cast<int64_t>(r) * kHeadDim + 16 * g + 8 * i) : zero4;
-                    }
-                    __syncwarp();
-                    mma_block(st, qa, kw, vw, n, c2);
+                for (int hh = 0; hh < 2; ++hh) {
+                    vh[hh] = V + static_cast<int64_t>(8 * hh) * kHeadDim;
+                    nh[hh] = max(0, min(8, ntok - t0 - 8 * hh));
                 }
             }
+        } else {
+            const int tb = g_idx - g_base;
+            if (tb < ntb) {
+                bk.kind = 1;
+                tail = true;
+                t0 = t_lo + tb * 16;
+                nh[0] = max(0, min(8, t_hi - t0));
+                nh[1] = max(0, min(8, t_hi - t0 - 8));
+            }
         }
-        item += nblk;
-        ++seg;
-    }
+        bk.nlo = nh[0];
+        bk.nhi = nh[1];
+        // Copies.  Warp instruction q moves block rows R = 2q and 2q + 1
+        // (512 contiguous source bytes when both rows sit in one segment):
+        // lane l takes row R = 2q + (l >> 4), 16-byte chunk j = l & 15, and
+        // writes it where its reader finds it: key row R chunk j is read by
+        // lane 4 (R & 7) + (j >> 2) as key slot (R >> 3) * 4 + (j & 3);
+        // value row R chunk j by lane 4 (j >> 1) + ((R & 7) >> 1) as value
+        // slot 8 + 2k + (j & 1), k = 2 (R >> 3) + (R & 1), at lane position
+        // XOR ((2k + (j & 1)) & 3) so that the 32 stores of one instruction
+        // spread over all bank groups.  Sparse keys stage their (index,
+        // value) pairs in key slots 0..2 instead.
+        const void* nul = A.q;       // any valid address: nothing is read
+        const int jj = lane & 15;
+        auto copy_row = [&](int stage_, int q, const __half* krow, const __half* vrow) {
+            const int R = 2 * q + (lane >> 4);
+            const int hh = R >> 3, rr = R & 7;
+            if (bk.kind == 1)
+                cp_async16(slot(stage_, hh * 4 + (jj & 3), 4 * rr + (jj >> 2)), krow ? krow + 8 * jj : nul,
+                           krow ? 16u : 0u);
+            const int k = 2 * hh + (R & 1), vs = 2 * k + (jj & 1);
+            cp_async16(slot(stage_, 8 + vs, (4 * (jj >> 1) + (rr >> 1)) ^ (vs & 3)), vrow ? vrow + 8 * jj : nul,
+                       vrow ? 16u : 0u);
+        };
+        if (bk.kind != 0 && !tail) {
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const int R = 2 * q + (lane >> 4);
+                const int hh = R >> 3, rr = R & 7;
+                const bool v = rr < nh[hh];
+                const __half* krow = (v && bk.kind == 1) ? kh[hh] + static_cast<int64_t>(rr) * kHeadDim : nullptr;
+                const __half* vrow = v ? vh[hh] + static_cast<int64_t>(rr) * kHeadDim : nullptr;
+                copy_row(stage, q, krow, vrow);
+            }
+        } else if (bk.kind != 0) {
+            // dense tail: rows come from the dense view (paged or not)
+#pragma unroll 1
+            for (int q = 0; q < 8; ++q) {
+                const int R = 2 * q + (lane >> 4);
+                const bool v = (R & 7) < nh[R >> 3];
+                const __half* krow = v ? dense_row(A.dv, A.dv.k, b, h, t0 + R, A.status) : nullptr;
+                const __half* vrow = v ? dense_row(A.dv, A.dv.v, b, h, t0 + R, A.status) : nullptr;
+                copy_row(stage, q, krow, vrow);
+            }
+        }
+        if (bk.kind == 2 && c <= 32) {
+            const int e0 = lane * 16;
+            const bool v = e0 < (bk.nlo + bk.nhi) * c;
+            cp_async16(slot(stage, 0, lane), v ? static_cast<const void*>(bk.ci + e0) : nul, v ? 16u : 0u);
+            cp_async16(slot(stage, 1, lane), v ? static_cast<const void*>(bk.kv + e0) : nul, v ? 16u : 0u);
+            cp_async16(slot(stage, 2, lane), v ? static_cast<const void*>(bk.kv + e0 + 8) : nul, v ? 16u : 0u);
+        }
+        cp_async_commit();
+        return bk;
+    };
+
+    auto compute = [&](const DecBlock& bk, int stage) {
+        if (bk.kind == 2) {
+            // zero the 16 x 128 key tile (key slots 0..7), then scatter the
+            // block's n * c pairs into it; 16 pairs per lane and round
+            const int np = (bk.nlo + bk.nhi) * c;
+            uint4 iw = make_uint4(0, 0, 0, 0), va = iw, vb = iw;
+            if (c <= 32) {
+                iw = lds16(slot(stage, 0, lane));
+                va = lds16(slot(stage, 1, lane));
+                vb = lds16(slot(stage, 2, lane));
+            }
+            __syncwarp();
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(slot(stage, i, lane)), "r"(0u)
+                             : "memory");
+            __syncwarp();
+            for (int e0 = lane * 16; e0 < np; e0 += 32 * 16) {
+                if (c > 32) {
+                    iw = ld_nc16(bk.ci + e0);
+                    va = ld_nc16(bk.kv + e0);
+                    vb = ld_nc16(bk.kv + e0 + 8);
+                }
+                const uint32_t iws[4] = {iw.x, iw.y, iw.z, iw.w};
+                const uint32_t vws[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
+                int rr = e0 / c, col = e0 - rr * c;
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    if (e0 + k < np) {
+                        // indices are < 128; the mask keeps a corrupt byte inside the tile
+                        const int ch = (iws[k >> 2] >> (8 * (k & 3))) & 0x7f;
+                        const uint16_t hv = static_cast<uint16_t>(vws[k >> 1] >> (16 * (k & 1)));
+                        const int j = ch >> 3;
+                        const uint32_t a = slot(stage, (rr >> 3) * 4 + (j & 3), 4 * (rr & 7) + (j >> 2)) + (ch & 7) * 2;
+                        asm volatile("st.shared.u16 [%0], %1;" ::"r"(a), "h"(hv) : "memory");
+                    }
+                    if (++col == c) {
+                        col = 0;
+                        ++rr;
+                    }
+                }
+            }
+            __syncwarp();
+        }
+        uint4 kw[2][4], vw[4][2];
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) kw[nt][i] = lds16(slot(stage, nt * 4 + i, lane));
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+#pragma unroll
+            for (int i = 0; i < 2; ++i) vw[k][i] = lds16(slot(stage, 8 + 2 * k + i, lane ^ ((2 * k + i) & 3)));
+        mma_block(st, qa, kw, vw, bk.nlo, bk.nhi, c2);
+        __syncwarp();    // the stage is refilled next: every lane is done with it
+    };
+
     {
-        const int ntb = (t_hi - t_lo + 15) >> 4;
-        int first = (warp - item) % kDecWarps;
-        if (first < 0) first += kDecWarps;
-        uint32_t* status = A.status;
-        const DenseView& dv = A.dv;
-        for (int tb = first; tb < ntb; tb += kDecWarps) {
-            const int t0 = t_lo + tb * 16;
-            const int n = min(16, t_hi - t0);
-            dense_block([&](int i) -> const __half* { return dense_row(dv, dv.k, b, h, t0 + i, status); },
-                        [&](int i) -> const __half* { return dense_row(dv, dv.v, b, h, t0 + i, status); }, n);
+        // iterations -2 and -1 only issue; block k is issued at iteration
+        // k - 2 and computed at iteration k (one call site each keeps the
+        // loop body small enough for the instruction cache)
+        DecBlock f0{0, 0, 0, nullptr, nullptr}, f1 = f0;
+        for (int k = -2;; ++k) {
+            const DecBlock f2 = next_block((k + 2) % kDecStages);
+            if (k >= 0) {
+                if (f0.kind == 0) break;
+                cp_async_wait<2>();
+                compute(f0, k % kDecStages);
+            }
+            f0 = f1;
+            f1 = f2;
         }
+        cp_async_wait<0>();
     }
 
     // ---- warp partials -> shared memory (lanes with g < G hold real rows)
-    __syncthreads();   // every warp is done with its key tile
+    __syncthreads();   // every warp is done with its stage buffers
     float l = st.lp;
     l += __shfl_xor_sync(0xffffffffu, l, 1);
     l += __shfl_xor_sync(0xffffffffu, l, 2);
@@ -453,56 +644,58 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(const __grid_consta
     if (!is_last) return;
     __threadfence();
 
-    // ---- last CTA of the unit: merge the splits in order
-    const float* up = A.part + static_cast<int64_t>(u) * A.nsplit * G * kRec;
-    for (int i = tid; i < A.nsplit * G; i += kDecThreads) sc[i / G][i % G] = __ldcg(up + i * kRec);
-    __syncthreads();
-    if (tid < G) {
-        float M = kNegInfF;
-        for (int s2 = 0; s2 < A.nsplit; ++s2) M = fmaxf(M, sc[s2][tid]);
-        for (int s2 = 0; s2 < A.nsplit; ++s2) {
-            const float ms = sc[s2][tid];
-            sc[s2][tid] = (ms == kNegInfF) ? 0.f : fast_exp2(ms - M);
-        }
-    }
-    __syncthreads();
-    if (tid < G) {
-        float L = 0.f;
-        for (int s2 = 0; s2 < A.nsplit; ++s2)
-            L = fmaf(__ldcg(up + (s2 * G + tid) * kRec + 1), sc[s2][tid], L);
-        wl[0][tid] = L;
-    }
-    // a thread merges 4 consecutive channels of one head; up to 16 splits'
-    // 16-byte records are loaded before they are summed in split order
-    for (int i = tid; i < G * (kHeadDim / 4); i += kDecThreads) {
-        const int gg = i / (kHeadDim / 4), x4 = (i % (kHeadDim / 4)) * 4;
+    // ---- last CTA of the unit: merge the splits in order.  A thread owns
+    // 4 channels of one head and loads (M, L, O) of up to kMergeChunk splits
+    // at once; chunks merge online.
+    if (tid < G * (kHeadDim / 4)) {
+        constexpr int kMergeChunk = 20;
+        const int gg = tid / (kHeadDim / 4), x4 = (tid % (kHeadDim / 4)) * 4;
+        const float* up = A.part + static_cast<int64_t>(u) * A.nsplit * G * kRec + gg * kRec;
+        float Mrun = kNegInfF, Lrun = 0.f;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int s0 = 0; s0 < A.nsplit; s0 += 16) {
-            float4 v16[16];
+        for (int s0 = 0; s0 < A.nsplit; s0 += kMergeChunk) {
+            float2 ml[kMergeChunk];
+            float4 ov[kMergeChunk];
 #pragma unroll
-            for (int k = 0; k < 16; ++k)
-                v16[k] = (s0 + k < A.nsplit)
-                             ? __ldcg(reinterpret_cast<const float4*>(up + ((s0 + k) * G + gg) * kRec + 4 + x4))
-                             : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-            for (int k = 0; k < 16; ++k) {
-                if (s0 + k >= A.nsplit) break;
-                const float scl = sc[s0 + k][gg];
-                acc.x = fmaf(v16[k].x, scl, acc.x);
-                acc.y = fmaf(v16[k].y, scl, acc.y);
-                acc.z = fmaf(v16[k].z, scl, acc.z);
-                acc.w = fmaf(v16[k].w, scl, acc.w);
+            for (int k = 0; k < kMergeChunk; ++k) {
+                if (s0 + k < A.nsplit) {
+                    const float* rec = up + static_cast<int64_t>(s0 + k) * G * kRec;
+                    ml[k] = __ldcg(reinterpret_cast<const float2*>(rec));
+                    ov[k] = __ldcg(reinterpret_cast<const float4*>(rec + 4 + x4));
+                } else {
+                    ml[k] = make_float2(kNegInfF, 0.f);
+                    ov[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+                }
             }
+            float Mc = Mrun;
+#pragma unroll
+            for (int k = 0; k < kMergeChunk; ++k) Mc = fmaxf(Mc, ml[k].x);
+            if (Mc == kNegInfF) continue;
+            const float r = (Mrun == kNegInfF) ? 0.f : fast_exp2(Mrun - Mc);
+            Lrun *= r;
+            acc.x *= r;
+            acc.y *= r;
+            acc.z *= r;
+            acc.w *= r;
+#pragma unroll
+            for (int k = 0; k < kMergeChunk; ++k) {
+                if (ml[k].x == kNegInfF) continue;
+                const float scl = fast_exp2(ml[k].x - Mc);
+                Lrun = fmaf(ml[k].y, scl, Lrun);
+                acc.x = fmaf(ov[k].x, scl, acc.x);
+                acc.y = fmaf(ov[k].y, scl, acc.y);
+                acc.z = fmaf(ov[k].z, scl, acc.z);
+                acc.w = fmaf(ov[k].w, scl, acc.w);
+            }
+            Mrun = Mc;
         }
-        reinterpret_cast<float4*>(ktile)[(gg * kHeadDim + x4) / 4] = acc;
-    }
-    __syncthreads();
-    for (int i = tid; i < G * kHeadDim; i += kDecThreads) {
-        const int gg = i / kHeadDim, x = i % kHeadDim;
-        const float L = wl[0][gg];
-        const float O = reinterpret_cast<const float*>(ktile)[gg * kHeadDim + x];
-        const float res = (L > 0.f) ? O / L : 0.f;
-        A.out[(static_cast<int64_t>(b) * A.Hq + h * G + gg) * kHeadDim + x] = __float2half_rn(res);
+        const float inv = (Lrun > 0.f) ? 1.f / Lrun : 0.f;
+        __half2 h01 = __floats2half2_rn(acc.x * inv, acc.y * inv);
+        __half2 h23 = __floats2half2_rn(acc.z * inv, acc.w * inv);
+        uint2 pk;
+        pk.x = *reinterpret_cast<const uint32_t*>(&h01);
+        pk.y = *reinterpret_cast<const uint32_t*>(&h23);
+        *reinterpret_cast<uint2*>(A.out + (static_cast<int64_t>(b) * A.Hq + h * G + gg) * kHeadDim + x4) = pk;
     }
     if (tid == 0) A.ticket[u] = 0;
 }
@@ -510,8 +703,8 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(const __grid_consta
 }  // namespace
 
 int decode_split_count(int units, int64_t max_seq_len, int num_sms) {
-    // two CTAs per SM, one wave
-    int ns = (2 * num_sms) / units;
+    // one 8-warp CTA per SM, one wave
+    int ns = num_sms / units;
     const int by_len = static_cast<int>((max_seq_len + 255) / 256);
     ns = min(ns, max(1, by_len));
     return max(1, min(ns, 64));
@@ -551,11 +744,16 @@ cudaError_t launch_decode(const DecodeLaunch& L, cudaStream_t stream) {
     const int units = L.batch * L.shp.Hkv;
     cudaError_t e = cudaSuccess;
     dim3 grid(L.nsplit, units);
+    auto launch_dec = [&](auto kern) {
+        cudaError_t r = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmem);
+        if (r != cudaSuccess) return r;
+        return launch_k(kern, grid, dim3(kDecThreads), kDecSmem, stream, a);
+    };
     prof_begin(stream, kProfDecode);
     switch (L.shp.G) {
-    case 2: e = launch_k(decode_kernel<2>, grid, dim3(kDecThreads), 0, stream, a); break;
-    case 4: e = launch_k(decode_kernel<4>, grid, dim3(kDecThreads), 0, stream, a); break;
-    case 8: e = launch_k(decode_kernel<8>, grid, dim3(kDecThreads), 0, stream, a); break;
+    case 2: e = launch_dec(decode_kernel<2>); break;
+    case 4: e = launch_dec(decode_kernel<4>); break;
+    case 8: e = launch_dec(decode_kernel<8>); break;
     default: return cudaErrorInvalidValue;
     }
     if (e != cudaSuccess) return e;
