@@ -13,11 +13,12 @@
 //   - each warp takes every 8th 16-token block of its CTA's range and runs
 //     q.k and p.v on the tensor cores (mma.sync m16n8k16, fp16 in, fp32
 //     accumulate; the G heads are the rows of the 16-row tile);
-//   - every lane copies the exact 16-byte fragments it will read into its
-//     own shared-memory slots with cp.async, three blocks ahead, so a warp
-//     always has two blocks in flight while it computes a third and every
-//     fragment read is conflict-free; CH / BOTH keys are scattered from
-//     their (index, value) pairs into the key slots of the same stage;
+//   - lane 0 of each warp has the TMA unit copy the key and value rows of
+//     its blocks into a three-stage shared-memory ring (one bulk copy per
+//     contiguous run of rows, completion on a per-stage mbarrier), so a warp
+//     has two blocks in flight while it computes a third; CH / BOTH keys are
+//     scattered from their (index, value) pairs into a dense key tile;
+//   - segments of at most 8 tokens pair up, one per half of a 16-row block;
 //   - scores meet an online softmax per head in the log2 domain; warps, then
 //     CTAs, merge their (max, sum, output) partials in a fixed order, the
 //     last CTA of a unit (atomic ticket) writing the fp16 output.
@@ -30,7 +31,13 @@ namespace {
 constexpr int kDecWarps = 8;
 constexpr int kDecThreads = kDecWarps * 32;
 constexpr int kDecStages = 3;                       // blocks in flight per warp
-constexpr int kDecSlotBytes = 16 * 32 * 16;         // 16 slots x 32 lanes x 16 bytes
+// A stage holds one block: 16 key rows back to back (a half of a block is
+// one contiguous copy; a quarter-warp's key reads meet 2 rows per bank group),
+// then 16 value rows at a 272-byte stride (each row its own copy; a
+// quarter-warp's value reads hit 8 different bank groups).
+constexpr int kDecKStride = 256, kDecVStride = 272;
+constexpr int kDecKBytes = 16 * kDecKStride;
+constexpr int kDecSlotBytes = kDecKBytes + 15 * kDecVStride + 256;
 constexpr int kDecSmem = kDecWarps * kDecStages * kDecSlotBytes;
 constexpr float kNegInfF = -__builtin_huge_valf();
 
@@ -82,7 +89,7 @@ struct DecodeArgs {
 };
 
 constexpr int64_t kTailBytes = 2 * kHeadDim * 2;   // K + V row of one dense token
-constexpr int kDescCache = 1024;                   // descriptors staged per CTA
+constexpr int kDescCache = 512;                    // descriptors staged per CTA
 
 // ------------------------------------------------------ tensor-core decode
 //
@@ -91,11 +98,11 @@ constexpr int kDescCache = 1024;                   // descriptors staged per CTA
 //   S[16 x 16] = Q[16 x 128] K^T   (rows = the G query heads, zero-padded)
 //   O[16 x 128] += P[16 x 16] V    (P = softmax numerators in fp16)
 // Lane (g = lane / 4, t = lane % 4).  The q.k contraction runs over d in a
-// fixed permuted order: mma k-index 2t+e of step ks <-> d = 32t + 4ks + e
-// and 2t+8+e <-> d = 32t + 4ks + 2 + e, so a lane's key data for all eight
-// steps is the contiguous window [32t, 32t + 32) of a row.  In p.v the
-// output column n of n-tile j stands for d = 16n + j, so a lane's value data
-// is the window [16g, 16g + 16) of rows 2t, 2t+1, 2t+8, 2t+9.
+// fixed permuted order: mma k-index 2t+e of step ks <-> d = 8 (4 (ks / 2) +
+// t) + 4 (ks % 2) + e and 2t+8+e <-> the same + 2, so a lane's key data is
+// the 16-byte chunks t, t+4, t+8, t+12 of a row.  In p.v the output column n
+// of n-tile j stands for d = 8n + 64 (j / 8) + j % 8, so a lane's value data
+// is chunks g and g+8 of rows 2t, 2t+1, 2t+8, 2t+9.
 
 __device__ __forceinline__ void mma16816(float& d0, float& d1, uint32_t a0, uint32_t a2, uint32_t b0,
                                          uint32_t b1) {
@@ -113,7 +120,7 @@ __device__ __forceinline__ void mma16816(float& d0, float& d1, uint32_t a0, uint
 struct MmaState {
     float m;          // running max of this lane's head row (log2 domain)
     float lp;         // this lane's share of the row's softmax sum
-    float o[16][2];   // O[g][d = 32t + 16e + j] at o[j][e]
+    float o[16][2];   // O[g][d = 8 (2t + e) + 64 (j / 8) + j % 8] at o[j][e]
 };
 
 __device__ __forceinline__ uint4 ld_nc16(const void* p) {
@@ -134,9 +141,9 @@ __device__ __forceinline__ void mma16808(float& d0, float& d1, uint32_t a0, uint
 
 // One 16-token block made of two halves of 8 token rows: rows 0..7 hold
 // nlo valid tokens, rows 8..15 hold nhi (a half is a slice of one segment,
-// or a whole segment of at most 8 tokens).  kw[nt][i]: this lane's key
-// window of row nt*8 + g (chunk i of [32t, 32t+32)); vw[k][i]: value window
-// of row {2t, 2t+1, 2t+8, 2t+9}[k], chunk i of [16g, 16g+16).
+// or a whole segment of at most 8 tokens).  kw[nt][i]: chunk 4i + t of key
+// row nt*8 + g; vw[k][i]: chunk g + 8i of value row {2t, 2t+1, 2t+8,
+// 2t+9}[k].
 //
 // The running max moves only when a block max exceeds it by more than 8 (in
 // log2 units), so the fp16 numerators stay <= 2^8 and most blocks skip the
@@ -207,15 +214,14 @@ __device__ __forceinline__ void mma_block(MmaState& st, const uint32_t (&qa)[8][
     }
 }
 
-// 16-byte asynchronous copy global -> shared; src_bytes 0 writes zeros and
-// reads nothing.
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+// Contiguous global -> shared copy by the TMA unit (no tensor map, no
+// multicast); 16-byte aligned addresses, size a multiple of 16; completion
+// counted in bytes on the mbarrier.
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "l"(src), "r"(bytes), "r"(bar)
                  : "memory");
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 // A 16-token block of one warp.  kind: 0 none, 1 dense rows (FULL / TOK
 // segment or tail), 2 channel-sparse keys (CH / BOTH).
@@ -225,7 +231,7 @@ struct DecBlock {
     const __half* kv;       // sparse: the block's key values
 };
 
-constexpr int kDescPerThread = 4;   // descriptors each thread loads in the prologue
+constexpr int kDescPerThread = 2;   // descriptors each thread loads in the prologue
 
 template <int G>
 __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_constant__ DecodeArgs A) {
@@ -237,6 +243,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
     __shared__ float wm[kDecWarps][G], wl[kDecWarps][G];
     __shared__ int wcnt[kDecWarps][2];
     __shared__ int item_ctr;
+    __shared__ __align__(8) uint64_t sbar[kDecWarps][kDecStages];
     __shared__ int is_last;
     __shared__ uint64_t dsm[kDescCache];
     // the warp partials reuse the stage buffers once every warp is done
@@ -245,15 +252,15 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
     float (*wo)[G][kHeadDim] = reinterpret_cast<float (*)[G][kHeadDim]>(dec_smem);
 
     pdl_wait();
-    // q fragments (rows g < G): halves [32t, 32t + 32) of head g, step ks at 4ks
+    // q fragments (rows g < G): chunk 4 (ks / 2) + t of head g, words of step ks
     uint32_t qa[8][2];
     {
         uint4 qw[4] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0),
                        make_uint4(0, 0, 0, 0)};
         if (g < G) {
-            const __half* qrow = A.q + (static_cast<int64_t>(b) * A.Hq + h * G + g) * kHeadDim + 32 * t;
+            const __half* qrow = A.q + (static_cast<int64_t>(b) * A.Hq + h * G + g) * kHeadDim;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) qw[i] = ld_nc16(qrow + 8 * i);
+            for (int i = 0; i < 4; ++i) qw[i] = ld_nc16(qrow + 8 * (4 * i + t));
         }
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
@@ -312,6 +319,13 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
             wcnt[warp][1] = c_hi;
         }
         if (tid == 0) item_ctr = 0;
+        if (tid < kDecWarps * kDecStages) {
+            mbar_init(&sbar[tid / kDecStages][tid % kDecStages], 1);
+            mbar_fence_init();
+        }
+        // value rows past a block's last token must hold finite numbers
+        for (int i = tid; i < kDecSmem / 16; i += kDecThreads)
+            reinterpret_cast<uint4*>(dec_smem)[i] = make_uint4(0, 0, 0, 0);
     }
     __syncthreads();
     int j_lo = 0, j_hi = 0;
@@ -351,9 +365,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
     const int S = A.S, r = A.r, c = A.c;
     const uint8_t* ubase = A.arena + static_cast<int64_t>(u) * A.arena_stride;
     const uint32_t wbase = smem_u32(dec_smem) + warp * (kDecStages * kDecSlotBytes);
-    auto slot = [&](int stage, int cidx, int ln) -> uint32_t {
-        return wbase + stage * kDecSlotBytes + (cidx * 32 + ln) * 16;
-    };
+    // stage s of this warp: key rows at kreg(s), value rows at kreg(s) +
+    // kDecKBytes; sparse keys stage their pairs in the key region (index
+    // bytes, then values from byte 512) before they are scattered
+    auto kreg = [&](int stage) -> uint32_t { return wbase + stage * kDecSlotBytes; };
+    const uint32_t bar0 = smem_u32(&sbar[warp][0]);
     auto lds16 = [&](uint32_t a) {
         uint4 v;
         asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
@@ -466,75 +482,70 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
         }
         bk.nlo = nh[0];
         bk.nhi = nh[1];
-        // Copies.  Warp instruction q moves block rows R = 2q and 2q + 1
-        // (512 contiguous source bytes when both rows sit in one segment):
-        // lane l takes row R = 2q + (l >> 4), 16-byte chunk j = l & 15, and
-        // writes it where its reader finds it: key row R chunk j is read by
-        // lane 4 (R & 7) + (j >> 2) as key slot (R >> 3) * 4 + (j & 3);
-        // value row R chunk j by lane 4 (j >> 1) + ((R & 7) >> 1) as value
-        // slot 8 + 2k + (j & 1), k = 2 (R >> 3) + (R & 1), at lane position
-        // XOR ((2k + (j & 1)) & 3) so that the 32 stores of one instruction
-        // spread over all bank groups.  Sparse keys stage their (index,
-        // value) pairs in key slots 0..2 instead.
-        const void* nul = A.q;       // any valid address: nothing is read
-        const int jj = lane & 15;
-        auto copy_row = [&](int stage_, int q, const __half* krow, const __half* vrow) {
-            const int R = 2 * q + (lane >> 4);
-            const int hh = R >> 3, rr = R & 7;
-            if (bk.kind == 1)
-                cp_async16(slot(stage_, hh * 4 + (jj & 3), 4 * rr + (jj >> 2)), krow ? krow + 8 * jj : nul,
-                           krow ? 16u : 0u);
-            const int k = 2 * hh + (R & 1), vs = 2 * k + (jj & 1);
-            cp_async16(slot(stage_, 8 + vs, (4 * (jj >> 1) + (rr >> 1)) ^ (vs & 3)), vrow ? vrow + 8 * jj : nul,
-                       vrow ? 16u : 0u);
-        };
-        if (bk.kind != 0 && !tail) {
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                const int R = 2 * q + (lane >> 4);
-                const int hh = R >> 3, rr = R & 7;
-                const bool v = rr < nh[hh];
-                const __half* krow = (v && bk.kind == 1) ? kh[hh] + static_cast<int64_t>(rr) * kHeadDim : nullptr;
-                const __half* vrow = v ? vh[hh] + static_cast<int64_t>(rr) * kHeadDim : nullptr;
-                copy_row(stage, q, krow, vrow);
+        // Copies by the TMA unit: lane 0 copies the key rows of each half of
+        // a segment block in one piece (or a sparse block's two pair
+        // sections); lane l < 16 copies value row l to its padded place; in
+        // the dense tail lane 16 + l copies key row l.
+        if (bk.kind != 0) {
+            const uint32_t K0 = kreg(stage), V0 = K0 + kDecKBytes, bar = bar0 + stage * 8;
+            const int R = lane & 15, rr = R & 7;
+            const bool hi = R >= 8;
+            const int nrow = hi ? nh[1] : nh[0];
+            const __half* row = nullptr;
+            const bool krow_lane = lane >= 16;
+            if (rr < nrow) {
+                if (tail) {
+                    row = dense_row(A.dv, krow_lane ? A.dv.k : A.dv.v, b, h, t0 + R, A.status);
+                } else if (!krow_lane) {
+                    row = (hi ? vh[1] : vh[0]) + static_cast<int64_t>(rr) * kHeadDim;
+                }
             }
-        } else if (bk.kind != 0) {
-            // dense tail: rows come from the dense view (paged or not)
-#pragma unroll 1
-            for (int q = 0; q < 8; ++q) {
-                const int R = 2 * q + (lane >> 4);
-                const bool v = (R & 7) < nh[R >> 3];
-                const __half* krow = v ? dense_row(A.dv, A.dv.k, b, h, t0 + R, A.status) : nullptr;
-                const __half* vrow = v ? dense_row(A.dv, A.dv.v, b, h, t0 + R, A.status) : nullptr;
-                copy_row(stage, q, krow, vrow);
+            const uint32_t nrows = __popc(__ballot_sync(0xffffffffu, row != nullptr));
+            if (lane == 0) {
+                uint32_t bytes = nrows * 256;
+                const bool kbulk = !tail && bk.kind == 1;
+                int npb = 0, nkb = 0;
+                if (kbulk) bytes += (nh[0] + nh[1]) * 256;
+                if (bk.kind == 2 && c <= 32) {
+                    npb = pad16((bk.nlo + bk.nhi) * c);
+                    nkb = pad16(2 * (bk.nlo + bk.nhi) * c);
+                    bytes += npb + nkb;
+                }
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                mbar_expect_tx(&sbar[warp][stage], bytes);
+                if (kbulk) {
+                    if (nh[0]) bulk_g2s(K0, kh[0], nh[0] * 256, bar);
+                    if (nh[1]) bulk_g2s(K0 + 2048, kh[1], nh[1] * 256, bar);
+                }
+                if (npb) {
+                    bulk_g2s(K0, bk.ci, npb, bar);
+                    bulk_g2s(K0 + 512, bk.kv, nkb, bar);
+                }
             }
+            __syncwarp();
+            if (row) bulk_g2s(krow_lane ? K0 + R * kDecKStride : V0 + R * kDecVStride, row, 256, bar);
         }
-        if (bk.kind == 2 && c <= 32) {
-            const int e0 = lane * 16;
-            const bool v = e0 < (bk.nlo + bk.nhi) * c;
-            cp_async16(slot(stage, 0, lane), v ? static_cast<const void*>(bk.ci + e0) : nul, v ? 16u : 0u);
-            cp_async16(slot(stage, 1, lane), v ? static_cast<const void*>(bk.kv + e0) : nul, v ? 16u : 0u);
-            cp_async16(slot(stage, 2, lane), v ? static_cast<const void*>(bk.kv + e0 + 8) : nul, v ? 16u : 0u);
-        }
-        cp_async_commit();
         return bk;
     };
 
     auto compute = [&](const DecBlock& bk, int stage) {
+        const uint32_t K0 = kreg(stage), V0 = K0 + kDecKBytes;
         if (bk.kind == 2) {
-            // zero the 16 x 128 key tile (key slots 0..7), then scatter the
-            // block's n * c pairs into it; 16 pairs per lane and round
+            // the 16 x 128 key tile: zero it, then scatter the block's n * c
+            // pairs into it; 16 pairs per lane and round
             const int np = (bk.nlo + bk.nhi) * c;
             uint4 iw = make_uint4(0, 0, 0, 0), va = iw, vb = iw;
-            if (c <= 32) {
-                iw = lds16(slot(stage, 0, lane));
-                va = lds16(slot(stage, 1, lane));
-                vb = lds16(slot(stage, 2, lane));
+            if (c <= 32 && lane * 16 < np) {
+                iw = lds16(K0 + lane * 16);
+                va = lds16(K0 + 512 + lane * 32);
+                vb = lds16(K0 + 512 + lane * 32 + 16);
             }
             __syncwarp();
 #pragma unroll
             for (int i = 0; i < 8; ++i)
-                asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(slot(stage, i, lane)), "r"(0u)
+                asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(K0 + (2 * i + (lane >> 4)) * kDecKStride +
+                                                                             (lane & 15) * 16),
+                             "r"(0u)
                              : "memory");
             __syncwarp();
             for (int e0 = lane * 16; e0 < np; e0 += 32 * 16) {
@@ -552,9 +563,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
                         // indices are < 128; the mask keeps a corrupt byte inside the tile
                         const int ch = (iws[k >> 2] >> (8 * (k & 3))) & 0x7f;
                         const uint16_t hv = static_cast<uint16_t>(vws[k >> 1] >> (16 * (k & 1)));
-                        const int j = ch >> 3;
-                        const uint32_t a = slot(stage, (rr >> 3) * 4 + (j & 3), 4 * (rr & 7) + (j >> 2)) + (ch & 7) * 2;
-                        asm volatile("st.shared.u16 [%0], %1;" ::"r"(a), "h"(hv) : "memory");
+                        asm volatile("st.shared.u16 [%0], %1;" ::"r"(K0 + rr * kDecKStride + ch * 2), "h"(hv) : "memory");
                     }
                     if (++col == c) {
                         col = 0;
@@ -568,31 +577,31 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-            for (int i = 0; i < 4; ++i) kw[nt][i] = lds16(slot(stage, nt * 4 + i, lane));
+            for (int i = 0; i < 4; ++i) kw[nt][i] = lds16(K0 + (nt * 8 + g) * kDecKStride + (4 * i + t) * 16);
 #pragma unroll
         for (int k = 0; k < 4; ++k)
 #pragma unroll
-            for (int i = 0; i < 2; ++i) vw[k][i] = lds16(slot(stage, 8 + 2 * k + i, lane ^ ((2 * k + i) & 3)));
+            for (int i = 0; i < 2; ++i)
+                vw[k][i] = lds16(V0 + (2 * t + (k & 1) + 8 * (k >> 1)) * kDecVStride + (g + 8 * i) * 16);
         mma_block(st, qa, kw, vw, bk.nlo, bk.nhi, c2);
         __syncwarp();    // the stage is refilled next: every lane is done with it
     };
 
     {
         // iterations -2 and -1 only issue; block k is issued at iteration
-        // k - 2 and computed at iteration k (one call site each keeps the
-        // loop body small enough for the instruction cache)
+        // k - 2 into stage k % 3 and computed at iteration k, after the
+        // stage's barrier completes its (k / 3)-th phase
         DecBlock f0{0, 0, 0, nullptr, nullptr}, f1 = f0;
         for (int k = -2;; ++k) {
             const DecBlock f2 = next_block((k + 2) % kDecStages);
             if (k >= 0) {
                 if (f0.kind == 0) break;
-                cp_async_wait<2>();
+                if (!mbar_wait(&sbar[warp][k % kDecStages], (k / kDecStages) & 1, A.status)) break;
                 compute(f0, k % kDecStages);
             }
             f0 = f1;
             f1 = f2;
         }
-        cp_async_wait<0>();
     }
 
     // ---- warp partials -> shared memory (lanes with g < G hold real rows)
@@ -607,8 +616,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
         }
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
-            wo[warp][g][32 * t + j] = st.o[j][0];
-            wo[warp][g][32 * t + 16 + j] = st.o[j][1];
+            wo[warp][g][16 * t + 64 * (j >> 3) + (j & 7)] = st.o[j][0];
+            wo[warp][g][16 * t + 8 + 64 * (j >> 3) + (j & 7)] = st.o[j][1];
         }
     }
     __syncthreads();
