@@ -36,11 +36,13 @@ struct PackArgs {
     uint32_t* status;
 };
 
-// Copies ntok whole rows (256 bytes each) into dst; rows[i] points at the
-// i-th source row (nullptr -> zeros).  Four 16-byte loads in flight per
-// thread before the stores.
-__device__ __forceinline__ void copy_rows(const __half* const* rows, int ntok, uint8_t* dst) {
-    const int n = ntok * 16;
+// Copies whole rows (256 bytes each): chunk c < nk * 16 is chunk c % 16 of
+// key row c / 16 (rows kr, destination kdst); the next nv * 16 chunks are
+// the value rows (vr, vdst).  A null row reads as zeros.  Four 16-byte loads
+// are in flight per thread before their stores.
+__device__ __forceinline__ void copy_rows2(const __half* const* kr, int nk, uint8_t* kdst,
+                                           const __half* const* vr, int nv, uint8_t* vdst) {
+    const int n = (nk + nv) * 16;
     for (int i0 = threadIdx.x; i0 < n; i0 += 4 * blockDim.x) {
         uint4 v[4];
 #pragma unroll
@@ -48,14 +50,20 @@ __device__ __forceinline__ void copy_rows(const __half* const* rows, int ntok, u
             const int idx = i0 + k * blockDim.x;
             v[k] = make_uint4(0, 0, 0, 0);
             if (idx < n) {
-                const __half* row = rows[idx >> 4];
-                if (row) v[k] = *reinterpret_cast<const uint4*>(row + (idx & 15) * 8);
+                const bool isk = idx < nk * 16;
+                const int c = isk ? idx : idx - nk * 16;
+                const __half* row = isk ? kr[c >> 4] : vr[c >> 4];
+                if (row) v[k] = *reinterpret_cast<const uint4*>(row + (c & 15) * 8);
             }
         }
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
             const int idx = i0 + k * blockDim.x;
-            if (idx < n) *reinterpret_cast<uint4*>(dst + (idx >> 4) * 256 + (idx & 15) * 16) = v[k];
+            if (idx < n) {
+                const bool isk = idx < nk * 16;
+                const int c = isk ? idx : idx - nk * 16;
+                *reinterpret_cast<uint4*>((isk ? kdst : vdst) + (c >> 4) * 256 + (c & 15) * 16) = v[k];
+            }
         }
     }
 }
@@ -64,12 +72,17 @@ __global__ void __launch_bounds__(128) pack_kernel(const __grid_constant__ PackA
     pdl_wait();
     const int j = blockIdx.x, u = blockIdx.y;
     const int b = u / A.Hkv, h = u % A.Hkv;
-    if (j >= A.plan.nseg[b] || !A.unit_ok[u]) return;
+    if (j >= A.plan.nseg[b]) return;
     const int S = A.S, r = A.r, c = A.c;
     const int64_t slot = static_cast<int64_t>(u) * A.max_nseg + j;
-    const int st = A.strat[slot];
     const int segbase = A.plan.r0[b] / S;
+    // one round trip: the unit flag, the strategy, the descriptor and (on
+    // speculation) this thread's token index
+    const int ok = A.unit_ok[u];
+    const int st = A.strat[slot];
     const uint64_t d = A.desc[static_cast<int64_t>(u) * A.max_segs + segbase + j];
+    const int tk0 = (static_cast<int>(threadIdx.x) < r) ? A.tidx[slot * r + threadIdx.x] : 0;
+    if (!ok) return;
     uint8_t* out = A.arena + static_cast<int64_t>(u) * A.arena_stride +
                    static_cast<int64_t>(d & 0xffffffffull) * 16;
     const int t0 = A.plan.r0[b] + j * S;
@@ -79,7 +92,7 @@ __global__ void __launch_bounds__(128) pack_kernel(const __grid_constant__ PackA
     const bool sparse_tok = (st == KV2D_TOK || st == KV2D_BOTH);
     const int ntok = sparse_tok ? r : S;
     for (int i = threadIdx.x; i < ntok; i += blockDim.x) {
-        const int tk = sparse_tok ? A.tidx[slot * r + i] : i;
+        const int tk = sparse_tok ? (i == static_cast<int>(threadIdx.x) ? tk0 : A.tidx[slot * r + i]) : i;
         toks[i] = tk;
         krows[i] = dense_row(A.dv, A.dv.k, b, h, t0 + tk, A.status);
         vrows[i] = dense_row(A.dv, A.dv.v, b, h, t0 + tk, A.status);
@@ -92,9 +105,11 @@ __global__ void __launch_bounds__(128) pack_kernel(const __grid_constant__ PackA
         o = pad16(r);
     }
     if (st == KV2D_FULL || st == KV2D_TOK) {
-        copy_rows(krows, ntok, out + o);
-        o += static_cast<int64_t>(ntok) * 256;
-    } else {
+        // K rows then V rows, copied in one pass
+        copy_rows2(krows, ntok, out + o, vrows, ntok, out + o + static_cast<int64_t>(ntok) * 256);
+        return;
+    }
+    {
         const int n = ntok * c;
         const uint4* mbase = A.cmask + static_cast<int64_t>(u) * A.g_stride + static_cast<int64_t>(j) * S;
         uint8_t* ib = out + o;
@@ -118,10 +133,9 @@ __global__ void __launch_bounds__(128) pack_kernel(const __grid_constant__ PackA
         if (bad) atomicOr(A.status, KV2D_DEV_BAD_MASK);
         for (int i = n + threadIdx.x; i < pad16(n); i += blockDim.x) ib[i] = 0;
         for (int i = n + threadIdx.x; i < pad16(2 * n) / 2; i += blockDim.x) kv[i] = 0;
-        o += pad16(n);
-        o += pad16(2 * n);
+        o += pad16(n) + pad16(2 * n);
     }
-    copy_rows(vrows, ntok, out + o);
+    copy_rows2(nullptr, 0, nullptr, vrows, ntok, out + o);
 }
 
 }  // namespace

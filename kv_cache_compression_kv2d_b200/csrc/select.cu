@@ -65,25 +65,27 @@ __global__ void __launch_bounds__(kSegWarps * 32) seg_select_kernel(const __grid
     __syncwarp();
     const int64_t slot = static_cast<int64_t>(u) * A.max_nseg + j;
     int before = 0;
-    for (int tb = 0; tb < S; tb += 32) {
-        const int t = tb + lane;
-        bool kp = false;
-        if (t < S) {
-            const float v = ss[warp][t];
-            int rank = 0;
-            for (int t2 = 0; t2 < S; ++t2) {
-                const float v2 = ss[warp][t2];
-                rank += (v2 > v) || (v2 == v && t2 < t);
-            }
-            kp = rank < r;
-            kept[warp][t] = kp ? 1 : 0;
+    for (int tb = 0; tb < S; tb += 64) {
+        // two tokens per lane and pass: t = tb + lane and tb + 32 + lane
+        const int ta = tb + lane, tc = tb + 32 + lane;
+        const float va = (ta < S) ? ss[warp][ta] : 0.f;
+        const float vc = (tc < S) ? ss[warp][tc] : 0.f;
+        int ra = 0, rc = 0;
+        for (int t2 = 0; t2 < S; ++t2) {
+            const float v2 = ss[warp][t2];
+            ra += (v2 > va) || (v2 == va && t2 < ta);
+            rc += (v2 > vc) || (v2 == vc && t2 < tc);
         }
-        const uint32_t bal = __ballot_sync(0xffffffffu, kp);
-        if (kp) {
-            const int pos = before + __popc(bal & ((1u << lane) - 1u));
-            A.tidx[slot * r + pos] = static_cast<uint8_t>(t);
-        }
-        before += __popc(bal);
+        const bool ka = ta < S && ra < r, kc = tc < S && rc < r;
+        if (ta < S) kept[warp][ta] = ka ? 1 : 0;
+        if (tc < S) kept[warp][tc] = kc ? 1 : 0;
+        const uint32_t lt = (1u << lane) - 1u;
+        const uint32_t ba = __ballot_sync(0xffffffffu, ka);
+        if (ka) A.tidx[slot * r + before + __popc(ba & lt)] = static_cast<uint8_t>(ta);
+        before += __popc(ba);
+        const uint32_t bc = __ballot_sync(0xffffffffu, kc);
+        if (kc) A.tidx[slot * r + before + __popc(bc & lt)] = static_cast<uint8_t>(tc);
+        before += __popc(bc);
     }
     __syncwarp();
     if (lane != 0) return;
