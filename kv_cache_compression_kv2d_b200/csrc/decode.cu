@@ -242,7 +242,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
     const int g = lane >> 2, t = lane & 3;
     __shared__ float wm[kDecWarps][G], wl[kDecWarps][G];
     __shared__ int wcnt[kDecWarps][2];
-    __shared__ int item_ctr;
     __shared__ __align__(8) uint64_t sbar[kDecWarps][kDecStages];
     __shared__ int is_last;
     __shared__ uint64_t dsm[kDescCache];
@@ -318,7 +317,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
             wcnt[warp][0] = c_lo;
             wcnt[warp][1] = c_hi;
         }
-        if (tid == 0) item_ctr = 0;
         if (tid < kDecWarps * kDecStages) {
             mbar_init(&sbar[tid / kDecStages][tid % kDecStages], 1);
             mbar_fence_init();
@@ -396,14 +394,13 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
     // ---- the CTA's items, in order: a dense segment of at most 8 tokens
     // pairs with the next one if that is one too (one item, a segment per
     // half); other segments give one item per 16 tokens; then the dense
-    // tail in 16-token items.  Warps take the next item from a shared
-    // counter when they issue its copies, so they finish together.
-    int g_seg = j_lo, g_base = 0;
+    // tail in 16-token items.  Item i belongs to warp i % kDecWarps, so the
+    // order of every sum is fixed and the output is deterministic.
+    int g_seg = j_lo, g_base = 0, g_next = warp;
     auto next_block = [&](int stage) -> DecBlock {
         DecBlock bk{0, 0, 0, nullptr, nullptr};
-        int g_idx = 0;
-        if (lane == 0) g_idx = atomicAdd(&item_ctr, 1);
-        g_idx = __shfl_sync(0xffffffffu, g_idx, 0);
+        const int g_idx = g_next;
+        g_next += kDecWarps;
         const __half* kh[2] = {nullptr, nullptr};   // first K row of each half
         const __half* vh[2] = {nullptr, nullptr};   // first V row of each half
         int nh[2] = {0, 0};

@@ -767,15 +767,15 @@ __device__ __forceinline__ void merge32_desc_f(float (&w)[32]) {
 }
 
 // Membership masks of one thread's 128 keys against v: bit x of M[x / 32]
-// is set iff key_x >= v (kStrict: key_x > v).  ks[g][tid] holds the four
-// key registers of channels 8g..8g+7.  A compare yields 0xffff per half;
-// one AND-OR per register moves both flags to spare bit positions, and a
-// final shuffle puts each channel at its own bit.
-template <bool kStrict>
-__device__ __forceinline__ void key_masks(const uint4 (*ks)[128], int tid, __half2 vv, uint32_t (&M)[4]) {
+// is set iff key_x >= v, of Gt iff key_x > v.  ks[g][tid] holds the four key
+// registers of channels 8g..8g+7.  A compare yields 0xffff per half; one
+// AND-OR per register moves both flags to spare bit positions, and a final
+// shuffle puts each channel at its own bit.
+__device__ __forceinline__ void key_masks(const uint4 (*ks)[128], int tid, __half2 vv, uint32_t (&M)[4],
+                                          uint32_t (&Gt)[4]) {
 #pragma unroll
     for (int wd = 0; wd < 4; ++wd) {
-        uint32_t lo = 0, hi = 0;
+        uint32_t lo = 0, hi = 0, glo = 0, ghi = 0;
 #pragma unroll
         for (int g4 = 0; g4 < 4; ++g4) {
             const uint4 q = ks[wd * 4 + g4][tid];
@@ -784,12 +784,20 @@ __device__ __forceinline__ void key_masks(const uint4 (*ks)[128], int tid, __hal
             for (int e = 0; e < 4; ++e) {
                 const int s = g4 * 4 + e;        // channels 2s, 2s + 1 of this word
                 const __half2 kk = *reinterpret_cast<const __half2*>(&w[e]);
-                const uint32_t mk = kStrict ? __hgt2_mask(kk, vv) : __hge2_mask(kk, vv);
-                if (s < 8) lo |= mk & ((1u << (2 * s)) | (1u << (2 * s + 17)));
-                else hi |= mk & ((1u << (2 * s - 16)) | (1u << (2 * s + 1)));
+                const uint32_t mk = __hge2_mask(kk, vv), gk = __hgt2_mask(kk, vv);
+                if (s < 8) {
+                    const uint32_t bits = (1u << (2 * s)) | (1u << (2 * s + 17));
+                    lo |= mk & bits;
+                    glo |= gk & bits;
+                } else {
+                    const uint32_t bits = (1u << (2 * s - 16)) | (1u << (2 * s + 1));
+                    hi |= mk & bits;
+                    ghi |= gk & bits;
+                }
             }
         }
         M[wd] = (lo & 0x5555u) | ((lo >> 16) & 0xAAAAu) | ((hi << 16) & 0x55550000u) | (hi & 0xAAAA0000u);
+        Gt[wd] = (glo & 0x5555u) | ((glo >> 16) & 0xAAAAu) | ((ghi << 16) & 0x55550000u) | (ghi & 0xAAAA0000u);
     }
 }
 
@@ -907,14 +915,12 @@ __global__ void __launch_bounds__(128) chan_kernel_c32(const __grid_constant__ C
     }
     const __half2 vv = __float2half2_rn(vf);   // vf is a key value: exact in fp16
 
-    uint32_t M[4];
-    key_masks<false>(ks, tid, vv, M);
+    uint32_t M[4], G[4];
+    key_masks(ks, tid, vv, M, G);
     const int n_ge = __popc(M[0]) + __popc(M[1]) + __popc(M[2]) + __popc(M[3]);
     if (n_ge > c) {
         // the keys equal to v straddle the cut: keep the c - n_gt best of
         // them by the exact product (e desc, x asc)
-        uint32_t G[4];
-        key_masks<true>(ks, tid, vv, G);
         const int need = c - (__popc(G[0]) + __popc(G[1]) + __popc(G[2]) + __popc(G[3]));
         const uint32_t qm[4] = {M[0] & ~G[0], M[1] & ~G[1], M[2] & ~G[2], M[3] & ~G[3]};
         uint32_t keep[4] = {0, 0, 0, 0};
@@ -948,10 +954,10 @@ __global__ void __launch_bounds__(128) chan_kernel_c32(const __grid_constant__ C
         const uint32_t qw[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            const float2 f2 = __half22float2(*reinterpret_cast<const __half2*>(&qw[e]));
+            const float2 f2 = __half22float2(__habs2(*reinterpret_cast<const __half2*>(&qw[e])));
             const double2 a2 = *reinterpret_cast<const double2*>(ad + 8 * j + 2 * e);
-            const double e0 = __dmul_rn(fabs(static_cast<double>(f2.x)), a2.x);
-            const double e1 = __dmul_rn(fabs(static_cast<double>(f2.y)), a2.y);
+            const double e0 = __dmul_rn(static_cast<double>(f2.x), a2.x);
+            const double e1 = __dmul_rn(static_cast<double>(f2.y), a2.y);
             tot = __dadd_rn(tot, e0);
             drop = dadd_unless(drop, e0, mw, 1u << (2 * e));
             tot = __dadd_rn(tot, e1);
