@@ -38,6 +38,33 @@ SMI_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.act
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
 
+def profiled_traffic(kernel, workload):
+    """DRAM bytes (read + write) per launch of `kernel` on `workload` from the
+    committed ncu summary profiles/<kernel>_<workload>.md, or None when there
+    is none or the kernel's source file has changed since the capture (the
+    summary records the SHA-256 of the source it was measured with)."""
+    import hashlib
+    root = os.path.dirname(os.path.abspath(__file__))
+    path = os.path.join(root, "profiles", f"{kernel}_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    fields = {}
+    with open(path) as f:
+        for line in f:
+            if ":" in line and line.split(":", 1)[0] in ("traffic_bytes_per_launch", "kernel_source",
+                                                        "kernel_source_sha256"):
+                k, v = line.split(":", 1)
+                fields[k] = v.strip()
+    try:
+        with open(os.path.join(root, fields["kernel_source"]), "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()
+        if sha != fields["kernel_source_sha256"]:
+            return None
+        return int(fields["traffic_bytes_per_launch"])
+    except (KeyError, OSError, ValueError):
+        return None
+
+
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -380,7 +407,8 @@ def main():
     work = {
         "score_pass1": ("tensor", flops_pass),
         "score_pass2": ("tensor", 2.0 * wl.num_q_heads * wl.window * seg_tokens * wl.head_dim),
-        "chan_topc": ("hbm", kv_seg_bytes + seg_tokens * wl.num_kv_heads * (wl.c + 8)),
+        # K rows in; a 16-byte keep mask and the fp64 g_t out per token
+        "chan_topc": ("hbm", kv_seg_bytes + seg_tokens * wl.num_kv_heads * (16 + 8)),
         "pack": ("hbm", 2 * sum(used)),   # gathers about as many bytes as it writes
         "decode": ("hbm", dec_bytes),
     }
@@ -395,12 +423,13 @@ def main():
     if kind == "tensor":
         achieved = amount / avg_s / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": tf_burst, "unit": "TFLOP/s",
-                "frac": achieved / tf_burst, "traffic": None,
+                "frac": achieved / tf_burst, "traffic": profiled_traffic(dominant, wl.name),
                 "kernel": dominant, "peak_source": f"{src} bf16 burst (fp16 runs at the bf16 rate)"}
     else:
         achieved = amount / avg_s / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                "frac": achieved / hbm, "traffic": None, "kernel": dominant,
+                "frac": achieved / hbm, "traffic": profiled_traffic(dominant, wl.name),
+                "kernel": dominant,
                 "peak_source": f"{src} HBM copy"}
     gpu_launches = sum(v_["launches"] for v_ in kernels.values())
 
