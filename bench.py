@@ -38,6 +38,29 @@ SMI_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.act
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
 
+def rank_seed(seed, rank):
+    """Seed of a rank's batch: every rank draws its own independent batch
+    (weak scaling: per-GPU work is fixed as the number of ranks grows)."""
+    return seed + 1000 * rank
+
+
+def max_over_ranks(x, dist, device):
+    """The largest x over all ranks (a job takes as long as its slowest
+    rank); x itself without a process group."""
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(bytes_per_rank, world, ms_per_step):
+    """Whole-job GB/s: the bytes all ranks processed over the slowest rank's
+    time per step."""
+    return bytes_per_rank * world / (ms_per_step * 1e-3) / 1e9
+
+
 def profiled_traffic(kernel, workload):
     """DRAM bytes (read + write) per launch of `kernel` on `workload` from the
     committed ncu summary profiles/<kernel>_<workload>.md, or None when there
@@ -264,7 +287,7 @@ def main():
 
     wl = synth.WORKLOADS[args.workload]
     dev = torch.device("cuda", local)
-    host = synth.generate(wl, seed=args.seed + 1000 * rank, device="cpu", extra_capacity=16)
+    host = synth.generate(wl, seed=rank_seed(args.seed, rank), device="cpu", extra_capacity=16)
     lens = [int(x) for x in host.seq_len]
     k = host.k.to(dev)
     v = host.v.to(dev)
@@ -381,14 +404,10 @@ def main():
         torch.cuda.synchronize(dev)
     assert B.kv2d_read_status(ws_c, stream) == 0 and B.kv2d_read_status(ws_d, stream) == 0
 
-    total_ms = sum(step_ms)
-    if dist is not None:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), dist, dev)
     ms_step = total_ms / args.steps
     nbytes = dense_bytes(wl, lens)
-    value = nbytes * world / (ms_step * 1e-3) / 1e9
+    value = job_throughput(nbytes, world, ms_step)
 
     # ---- algorithmic work per launch
     hbm, tf_burst, tf_sust, src = peaks()
@@ -465,13 +484,8 @@ def main():
             if i >= max(3, args.warmup):
                 evs.append((a, b_))
         torch.cuda.synchronize(dev)
-        e_ms = sum(a.elapsed_time(b_) for a, b_ in evs)
-        if dist is not None:
-            t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
-        e_ms /= args.steps
-        e2e = {"value": nbytes * world / (e_ms * 1e-3) / 1e9, "unit": UNIT,
+        e_ms = max_over_ranks(sum(a.elapsed_time(b_) for a, b_ in evs), dist, dev) / args.steps
+        e2e = {"value": job_throughput(nbytes, world, e_ms), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms}
 
     cpu = None
