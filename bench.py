@@ -312,9 +312,7 @@ def main():
     stream = torch.cuda.current_stream(dev)
 
     def reset():
-        cc.n_segs.zero_()
-        cc.used_bytes.zero_()
-        cc.comp_end.zero_()
+        cc.reset()
         seq.copy_(seq0)
 
     def compress():

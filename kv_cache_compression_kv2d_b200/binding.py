@@ -248,12 +248,22 @@ class CompressedCache:
         self.max_segs = max(1, max_tokens // p.segment_len)
         self.arena = torch.zeros(units * self.arena_stride, dtype=torch.uint8, device=device)
         self.desc = torch.zeros((units, self.max_segs), dtype=torch.int64, device=device)
-        self.n_segs = torch.zeros(units, dtype=torch.int32, device=device)
-        self.used_bytes = torch.zeros(units, dtype=torch.int64, device=device)
-        self.comp_end = torch.zeros(batch, dtype=torch.int32, device=device)
+        # bookkeeping in one buffer: used_bytes (int64), then n_segs and
+        # comp_end (int32), so that reset() is a single fill
+        n32 = units + batch
+        self.book = torch.zeros(units + (n32 + 1) // 2, dtype=torch.int64, device=device)
+        self.used_bytes = self.book[:units]
+        book32 = self.book[units:].view(torch.int32)
+        self.n_segs = book32[:units]
+        self.comp_end = book32[units:units + batch]
         self.struct = kv2d_ccache(_ptr(self.arena), self.arena_stride, _ptr(self.desc),
                                   self.max_segs, _ptr(self.n_segs), _ptr(self.used_bytes),
                                   _ptr(self.comp_end))
+
+    def reset(self):
+        """Forget every compressed segment (the arena bytes are left as they
+        are; descriptors past n_segs are never read)."""
+        self.book.zero_()
 
 
 def workspace(nbytes: int, device="cuda") -> torch.Tensor:
