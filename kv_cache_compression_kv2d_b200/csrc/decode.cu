@@ -31,13 +31,13 @@ namespace {
 constexpr int kDecWarps = 8;
 constexpr int kDecThreads = kDecWarps * 32;
 constexpr int kDecStages = 3;                       // blocks in flight per warp
-// A stage holds one block: 16 key rows back to back (a half of a block is
-// one contiguous copy; a quarter-warp's key reads meet 2 rows per bank group),
-// then 16 value rows at a 272-byte stride (each row its own copy; a
-// quarter-warp's value reads hit 8 different bank groups).
-constexpr int kDecKStride = 256, kDecVStride = 272;
+// A stage holds one block: 16 key rows, then 16 value rows, back to back, so
+// that each half of a segment block arrives in two bulk copies (the TMA unit
+// is bound by its copy count when rows come one by one).  A quarter-warp's
+// key reads meet 2 rows per bank group and its value reads 4.
+constexpr int kDecKStride = 256, kDecVStride = 256;
 constexpr int kDecKBytes = 16 * kDecKStride;
-constexpr int kDecSlotBytes = kDecKBytes + 15 * kDecVStride + 256;
+constexpr int kDecSlotBytes = kDecKBytes + 16 * kDecVStride;
 constexpr int kDecSmem = kDecWarps * kDecStages * kDecSlotBytes;
 constexpr float kNegInfF = -__builtin_huge_valf();
 
@@ -479,48 +479,49 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
         }
         bk.nlo = nh[0];
         bk.nhi = nh[1];
-        // Copies by the TMA unit: lane 0 copies the key rows of each half of
-        // a segment block in one piece (or a sparse block's two pair
-        // sections); lane l < 16 copies value row l to its padded place; in
-        // the dense tail lane 16 + l copies key row l.
+        // Copies by the TMA unit.  Segment blocks: lane 0 copies the key rows
+        // and the value rows of each half in one piece each (or a sparse
+        // block's two pair sections and its value rows); the dense tail, whose
+        // rows need not be contiguous, is copied row by row (lane l < 16: value
+        // row l, lane 16 + l: key row l).
         if (bk.kind != 0) {
             const uint32_t K0 = kreg(stage), V0 = K0 + kDecKBytes, bar = bar0 + stage * 8;
-            const int R = lane & 15, rr = R & 7;
-            const bool hi = R >= 8;
-            const int nrow = hi ? nh[1] : nh[0];
-            const __half* row = nullptr;
-            const bool krow_lane = lane >= 16;
-            if (rr < nrow) {
-                if (tail) {
-                    row = dense_row(A.dv, krow_lane ? A.dv.k : A.dv.v, b, h, t0 + R, A.status);
-                } else if (!krow_lane) {
-                    row = (hi ? vh[1] : vh[0]) + static_cast<int64_t>(rr) * kHeadDim;
+            if (!tail) {
+                if (lane == 0) {
+                    uint32_t bytes = (nh[0] + nh[1]) * 256 * (bk.kind == 1 ? 2 : 1);
+                    int npb = 0, nkb = 0;
+                    if (bk.kind == 2 && c <= 32) {
+                        npb = pad16((bk.nlo + bk.nhi) * c);
+                        nkb = pad16(2 * (bk.nlo + bk.nhi) * c);
+                        bytes += npb + nkb;
+                    }
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    mbar_expect_tx(&sbar[warp][stage], bytes);
+                    for (int hh = 0; hh < 2; ++hh) {
+                        if (nh[hh] == 0) continue;
+                        if (bk.kind == 1) bulk_g2s(K0 + hh * 2048, kh[hh], nh[hh] * 256, bar);
+                        bulk_g2s(V0 + hh * 2048, vh[hh], nh[hh] * 256, bar);
+                    }
+                    if (npb) {
+                        bulk_g2s(K0, bk.ci, npb, bar);
+                        bulk_g2s(K0 + 512, bk.kv, nkb, bar);
+                    }
                 }
+            } else {
+                const int R = lane & 15, rr = R & 7;
+                const bool krow_lane = lane >= 16;
+                const int nrow = (R >= 8) ? nh[1] : nh[0];
+                const __half* row = (rr < nrow)
+                                        ? dense_row(A.dv, krow_lane ? A.dv.k : A.dv.v, b, h, t0 + R, A.status)
+                                        : nullptr;
+                const uint32_t nrows = __popc(__ballot_sync(0xffffffffu, row != nullptr));
+                if (lane == 0) {
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    mbar_expect_tx(&sbar[warp][stage], nrows * 256);
+                }
+                __syncwarp();
+                if (row) bulk_g2s(krow_lane ? K0 + R * kDecKStride : V0 + R * kDecVStride, row, 256, bar);
             }
-            const uint32_t nrows = __popc(__ballot_sync(0xffffffffu, row != nullptr));
-            if (lane == 0) {
-                uint32_t bytes = nrows * 256;
-                const bool kbulk = !tail && bk.kind == 1;
-                int npb = 0, nkb = 0;
-                if (kbulk) bytes += (nh[0] + nh[1]) * 256;
-                if (bk.kind == 2 && c <= 32) {
-                    npb = pad16((bk.nlo + bk.nhi) * c);
-                    nkb = pad16(2 * (bk.nlo + bk.nhi) * c);
-                    bytes += npb + nkb;
-                }
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                mbar_expect_tx(&sbar[warp][stage], bytes);
-                if (kbulk) {
-                    if (nh[0]) bulk_g2s(K0, kh[0], nh[0] * 256, bar);
-                    if (nh[1]) bulk_g2s(K0 + 2048, kh[1], nh[1] * 256, bar);
-                }
-                if (npb) {
-                    bulk_g2s(K0, bk.ci, npb, bar);
-                    bulk_g2s(K0 + 512, bk.kv, nkb, bar);
-                }
-            }
-            __syncwarp();
-            if (row) bulk_g2s(krow_lane ? K0 + R * kDecKStride : V0 + R * kDecVStride, row, 256, bar);
         }
         return bk;
     };
