@@ -30,14 +30,16 @@ namespace {
 
 constexpr int kDecWarps = 8;
 constexpr int kDecThreads = kDecWarps * 32;
-constexpr int kDecStages = 3;                       // blocks in flight per warp
-// A stage holds one block: 16 key rows, then 16 value rows, back to back, so
-// that each half of a segment block arrives in two bulk copies (the TMA unit
-// is bound by its copy count when rows come one by one).  A quarter-warp's
-// key reads meet 2 rows per bank group and its value reads 4.
+constexpr int kDecStages = 6;                       // stages per warp: 5 blocks in flight
+// A stage holds one block of up to 8 tokens: 8 key rows, then 8 value rows,
+// back to back, so that a segment block arrives in two bulk copies.  Short
+// blocks keep many stages in flight: the copy latency under load is several
+// microseconds, so the bytes a warp has in flight set its rate.  A
+// quarter-warp's key reads meet 2 rows per bank group and its value reads 4.
+constexpr int kDecRows = 8;
 constexpr int kDecKStride = 256, kDecVStride = 256;
-constexpr int kDecKBytes = 16 * kDecKStride;
-constexpr int kDecSlotBytes = kDecKBytes + 16 * kDecVStride;
+constexpr int kDecKBytes = kDecRows * kDecKStride;
+constexpr int kDecSlotBytes = kDecKBytes + kDecRows * kDecVStride;
 constexpr int kDecSmem = kDecWarps * kDecStages * kDecSlotBytes;
 constexpr float kNegInfF = -__builtin_huge_valf();
 
@@ -347,7 +349,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
         return static_cast<int>(i < ntail ? i : static_cast<int64_t>(ntail));
     };
     const int t_lo = ce + tail_at_or_after(lo), t_hi = ce + tail_at_or_after(hi);
-    const int ntb = (t_hi - t_lo + 15) >> 4;
+    const int ntb = (t_hi - t_lo + kDecRows - 1) / kDecRows;
 
     __syncthreads();
 
@@ -391,66 +393,36 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
                                                (sty == KV2D_TOK ? pad16(r) : 0));
     };
 
-    // ---- the CTA's items, in order: a dense segment of at most 8 tokens
-    // pairs with the next one if that is one too (one item, a segment per
-    // half); other segments give one item per 16 tokens; then the dense
-    // tail in 16-token items.  Item i belongs to warp i % kDecWarps, so the
-    // order of every sum is fixed and the output is deterministic.
+    // ---- the CTA's items, in order: every segment in blocks of up to 8
+    // tokens, then the dense tail in blocks of 8.  Item i belongs to warp
+    // i % kDecWarps, so the order of every sum is fixed and the output is
+    // deterministic.
     int g_seg = j_lo, g_base = 0, g_next = warp;
     auto next_block = [&](int stage) -> DecBlock {
         DecBlock bk{0, 0, 0, nullptr, nullptr};
         const int g_idx = g_next;
         g_next += kDecWarps;
-        const __half* kh[2] = {nullptr, nullptr};   // first K row of each half
-        const __half* vh[2] = {nullptr, nullptr};   // first V row of each half
-        int nh[2] = {0, 0};
+        const __half* kh = nullptr;   // first K row of the block
+        const __half* vh = nullptr;   // first V row of the block
+        int n = 0;
         bool tail = false;
         uint64_t d = 0;
-        int nitems = 0, t0 = 0;
-        bool pair = false;
+        int t0 = 0;
         while (g_seg < j_hi) {
             d = desc(g_seg);
-            const int ntok = seg_ntok(d);
-            pair = false;
-            if (seg_dense(d) && ntok <= 8) {
-                nitems = 1;
-                if (g_seg + 1 < j_hi) {
-                    const uint64_t d2 = desc(g_seg + 1);
-                    pair = seg_dense(d2) && seg_ntok(d2) <= 8;
-                }
-            } else {
-                nitems = (ntok + 15) >> 4;
-            }
+            const int nitems = (seg_ntok(d) + kDecRows - 1) / kDecRows;
             if (g_idx < g_base + nitems) break;
             g_base += nitems;
-            g_seg += pair ? 2 : 1;
+            ++g_seg;
         }
         if (g_seg < j_hi) {
             const int ntok = seg_ntok(d);
-            t0 = (g_idx - g_base) * 16;
+            t0 = (g_idx - g_base) * kDecRows;
+            n = min(kDecRows, ntok - t0);
             if (seg_dense(d)) {
                 bk.kind = 1;
-                const __half* K = seg_k(d);
-                const __half* V = K + static_cast<int64_t>(ntok) * kHeadDim;
-                if (ntok <= 8) {
-                    kh[0] = K;
-                    vh[0] = V;
-                    nh[0] = ntok;
-                    if (pair) {
-                        const uint64_t d2 = desc(g_seg + 1);
-                        const int n2 = seg_ntok(d2);
-                        kh[1] = seg_k(d2);
-                        vh[1] = kh[1] + static_cast<int64_t>(n2) * kHeadDim;
-                        nh[1] = n2;
-                    }
-                } else {
-#pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        kh[hh] = K + static_cast<int64_t>(t0 + 8 * hh) * kHeadDim;
-                        vh[hh] = V + static_cast<int64_t>(t0 + 8 * hh) * kHeadDim;
-                        nh[hh] = max(0, min(8, ntok - t0 - 8 * hh));
-                    }
-                }
+                kh = seg_k(d) + static_cast<int64_t>(t0) * kHeadDim;
+                vh = seg_k(d) + static_cast<int64_t>(ntok + t0) * kHeadDim;
             } else {
                 bk.kind = 2;
                 const bool tok = ((d >> 32) & 255u) == KV2D_BOTH;
@@ -458,62 +430,51 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
                 bk.ci = p0 + static_cast<int64_t>(t0) * c;
                 bk.kv = reinterpret_cast<const __half*>(p0 + pad16(static_cast<int64_t>(ntok) * c)) +
                         static_cast<int64_t>(t0) * c;
-                const __half* V = reinterpret_cast<const __half*>(p0 + pad16(static_cast<int64_t>(ntok) * c) +
-                                                                  pad16(static_cast<int64_t>(ntok) * c * 2)) +
-                                  static_cast<int64_t>(t0) * kHeadDim;
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    vh[hh] = V + static_cast<int64_t>(8 * hh) * kHeadDim;
-                    nh[hh] = max(0, min(8, ntok - t0 - 8 * hh));
-                }
+                vh = reinterpret_cast<const __half*>(p0 + pad16(static_cast<int64_t>(ntok) * c) +
+                                                     pad16(static_cast<int64_t>(ntok) * c * 2)) +
+                     static_cast<int64_t>(t0) * kHeadDim;
             }
         } else {
             const int tb = g_idx - g_base;
             if (tb < ntb) {
                 bk.kind = 1;
                 tail = true;
-                t0 = t_lo + tb * 16;
-                nh[0] = max(0, min(8, t_hi - t0));
-                nh[1] = max(0, min(8, t_hi - t0 - 8));
+                t0 = t_lo + tb * kDecRows;
+                n = min(kDecRows, t_hi - t0);
             }
         }
-        bk.nlo = nh[0];
-        bk.nhi = nh[1];
-        // Copies by the TMA unit.  Segment blocks: lane 0 copies the key rows
-        // and the value rows of each half in one piece each (or a sparse
-        // block's two pair sections and its value rows); the dense tail, whose
-        // rows need not be contiguous, is copied row by row (lane l < 16: value
-        // row l, lane 16 + l: key row l).
+        bk.nlo = n;
+        bk.nhi = 0;
+        // Copies by the TMA unit.  Segment blocks: lane 0 copies the block's
+        // key rows and value rows in one piece each (or a sparse block's two
+        // pair sections and its value rows); the dense tail, whose rows need
+        // not be contiguous, is copied row by row (lane l < 8: value row l,
+        // lane 16 + l: key row l).
         if (bk.kind != 0) {
             const uint32_t K0 = kreg(stage), V0 = K0 + kDecKBytes, bar = bar0 + stage * 8;
             if (!tail) {
                 if (lane == 0) {
-                    uint32_t bytes = (nh[0] + nh[1]) * 256 * (bk.kind == 1 ? 2 : 1);
+                    uint32_t bytes = n * 256 * (bk.kind == 1 ? 2 : 1);
                     int npb = 0, nkb = 0;
                     if (bk.kind == 2 && c <= 32) {
-                        npb = pad16((bk.nlo + bk.nhi) * c);
-                        nkb = pad16(2 * (bk.nlo + bk.nhi) * c);
+                        npb = pad16(n * c);
+                        nkb = pad16(2 * n * c);
                         bytes += npb + nkb;
                     }
                     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                     mbar_expect_tx(&sbar[warp][stage], bytes);
-                    for (int hh = 0; hh < 2; ++hh) {
-                        if (nh[hh] == 0) continue;
-                        if (bk.kind == 1) bulk_g2s(K0 + hh * 2048, kh[hh], nh[hh] * 256, bar);
-                        bulk_g2s(V0 + hh * 2048, vh[hh], nh[hh] * 256, bar);
-                    }
+                    if (bk.kind == 1) bulk_g2s(K0, kh, n * 256, bar);
+                    bulk_g2s(V0, vh, n * 256, bar);
                     if (npb) {
                         bulk_g2s(K0, bk.ci, npb, bar);
                         bulk_g2s(K0 + 512, bk.kv, nkb, bar);
                     }
                 }
             } else {
-                const int R = lane & 15, rr = R & 7;
+                const int R = lane & 15;
                 const bool krow_lane = lane >= 16;
-                const int nrow = (R >= 8) ? nh[1] : nh[0];
-                const __half* row = (rr < nrow)
-                                        ? dense_row(A.dv, krow_lane ? A.dv.k : A.dv.v, b, h, t0 + R, A.status)
-                                        : nullptr;
+                const __half* row = (R < n) ? dense_row(A.dv, krow_lane ? A.dv.k : A.dv.v, b, h, t0 + R, A.status)
+                                            : nullptr;
                 const uint32_t nrows = __popc(__ballot_sync(0xffffffffu, row != nullptr));
                 if (lane == 0) {
                     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -540,7 +501,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
             }
             __syncwarp();
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
+            for (int i = 0; i < kDecRows / 2; ++i)
                 asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(K0 + (2 * i + (lane >> 4)) * kDecKStride +
                                                                              (lane & 15) * 16),
                              "r"(0u)
@@ -571,34 +532,45 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
             }
             __syncwarp();
         }
+        // 8-token blocks: key rows g and value rows 2t, 2t+1 only (the second
+        // half of the 16-row MMA tile stays zero)
+        const uint4 z4 = make_uint4(0, 0, 0, 0);
         uint4 kw[2][4], vw[4][2];
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
+        for (int i = 0; i < 4; ++i) {
+            kw[0][i] = lds16(K0 + g * kDecKStride + (4 * i + t) * 16);
+            kw[1][i] = z4;
+        }
 #pragma unroll
-            for (int i = 0; i < 4; ++i) kw[nt][i] = lds16(K0 + (nt * 8 + g) * kDecKStride + (4 * i + t) * 16);
+        for (int k = 0; k < 2; ++k)
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
-#pragma unroll
-            for (int i = 0; i < 2; ++i)
-                vw[k][i] = lds16(V0 + (2 * t + (k & 1) + 8 * (k >> 1)) * kDecVStride + (g + 8 * i) * 16);
-        mma_block(st, qa, kw, vw, bk.nlo, bk.nhi, c2);
+            for (int i = 0; i < 2; ++i) {
+                vw[k][i] = lds16(V0 + (2 * t + k) * kDecVStride + (g + 8 * i) * 16);
+                vw[k + 2][i] = z4;
+            }
+        mma_block(st, qa, kw, vw, bk.nlo, 0, c2);
         __syncwarp();    // the stage is refilled next: every lane is done with it
     };
 
     {
-        // iterations -2 and -1 only issue; block k is issued at iteration
-        // k - 2 into stage k % 3 and computed at iteration k, after the
-        // stage's barrier completes its (k / 3)-th phase
-        DecBlock f0{0, 0, 0, nullptr, nullptr}, f1 = f0;
-        for (int k = -2;; ++k) {
-            const DecBlock f2 = next_block((k + 2) % kDecStages);
+        // the first kDecStages - 1 iterations only issue; block k is issued at
+        // iteration k - (kDecStages - 1) into stage k % kDecStages and
+        // computed at iteration k, after the stage's barrier completes its
+        // (k / kDecStages)-th phase; f[j] holds block k + j
+        constexpr int kAhead = kDecStages - 1;
+        DecBlock f[kAhead];
+#pragma unroll
+        for (int j = 0; j < kAhead; ++j) f[j] = DecBlock{0, 0, 0, nullptr, nullptr};
+        for (int k = -kAhead;; ++k) {
+            const DecBlock nb = next_block((k + kAhead) % kDecStages);
             if (k >= 0) {
-                if (f0.kind == 0) break;
+                if (f[0].kind == 0) break;
                 if (!mbar_wait(&sbar[warp][k % kDecStages], (k / kDecStages) & 1, A.status)) break;
-                compute(f0, k % kDecStages);
+                compute(f[0], k % kDecStages);
             }
-            f0 = f1;
-            f1 = f2;
+#pragma unroll
+            for (int j = 0; j + 1 < kAhead; ++j) f[j] = f[j + 1];
+            f[kAhead - 1] = nb;
         }
     }
 

@@ -145,3 +145,25 @@ def test_decode_and_append_host_checks(L):
     dp = B.kv2d_dense(1 << 20, 2 << 20, 0, 0, 0, 0, 1 << 21, 8, 16, 100)
     assert lib.kv2d_append(C.byref(p), 1, C.byref(dp), 1 << 23, 1 << 23, 1 << 22, 9 << 20, 256,
                            None) == 1
+
+
+def test_cache_bookkeeping_views_and_reset(L):
+    """n_segs, used_bytes and comp_end live in one buffer: writing one never
+    touches another, and reset() clears all three with one fill."""
+    import torch
+    p = B.params(128, 32, 8, 64, 64, 8, 32, 0.2)
+    cc = B.CompressedCache(p, 3, 4096, device="cpu")
+    assert cc.n_segs.dtype == torch.int32 and cc.n_segs.numel() == 24
+    assert cc.used_bytes.dtype == torch.int64 and cc.used_bytes.numel() == 24
+    assert cc.comp_end.dtype == torch.int32 and cc.comp_end.numel() == 3
+    cc.used_bytes.copy_(torch.arange(24, dtype=torch.int64) + (1 << 40))
+    cc.n_segs.copy_(torch.arange(24, dtype=torch.int32) + 7)
+    cc.comp_end.copy_(torch.tensor([64, 128, 192], dtype=torch.int32))
+    assert torch.equal(cc.used_bytes, torch.arange(24, dtype=torch.int64) + (1 << 40))
+    assert torch.equal(cc.n_segs, torch.arange(24, dtype=torch.int32) + 7)
+    assert cc.comp_end.tolist() == [64, 128, 192]
+    ptrs = [cc.used_bytes.data_ptr(), cc.n_segs.data_ptr(), cc.comp_end.data_ptr()]
+    assert all(x % 4 == 0 for x in ptrs) and ptrs[0] % 8 == 0
+    cc.reset()
+    assert int(cc.used_bytes.abs().sum()) == 0
+    assert int(cc.n_segs.abs().sum()) == 0 and int(cc.comp_end.abs().sum()) == 0
