@@ -21,7 +21,8 @@ def L():
 
 
 def test_exports_match_header(L):
-    hdr = open(os.path.join(ROOT, "include", "kv2d.h")).read()
+    with open(os.path.join(ROOT, "include", "kv2d.h")) as f:
+        hdr = f.read()
     declared = re.findall(r"KV2D_API\s+[\w\s\*]+?\b(kv2d_\w+)\s*\(", hdr)
     assert len(declared) >= 9
     assert sorted(declared) == sorted(B.EXPORTS)

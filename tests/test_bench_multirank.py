@@ -37,7 +37,7 @@ def _rank_main(rank, world, port, out):
 
 def test_two_gloo_ranks_take_the_max_and_draw_distinct_batches():
     world = 2
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:
         out = m.dict()
         mp.start_processes(_rank_main, args=(world, _free_port(), out), nprocs=world,
                            start_method="spawn", join=True)
