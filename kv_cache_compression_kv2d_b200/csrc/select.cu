@@ -26,7 +26,7 @@ namespace kv2d {
 
 namespace {
 
-constexpr int kSegWarps = 8;
+constexpr int kSegWarps = 32;   // segments per CTA (one warp each, then one lane each)
 
 struct SegArgs {
     SeqPlan plan;
@@ -46,59 +46,89 @@ struct SegArgs {
     int32_t dbg_seg_stride;
 };
 
+// Shared memory of one CTA: per segment (row) the fp32 s_t, the fp64 s_t g_t
+// and the kept flags, rows padded by one element so that lane-per-segment
+// reads spread over the banks; then the three sums per segment.
+__host__ __device__ constexpr int seg_row(int S) { return S + 1; }
+inline int seg_smem_bytes(int S) {
+    return kSegWarps * seg_row(S) * (8 + 4 + 1) + 3 * kSegWarps * 8 + 16;
+}
+
+// Phase 1, one warp per segment: R_j by rank counting (two tokens per lane
+// and pass), tidx, kept flags, and the products s_t g_t.  Phase 2, one lane
+// per segment: E_CH (warp 0), the kept part of E_BOTH (warp 1) and E_TOK
+// (warp 2), each summed sequentially in ascending t.  Phase 3, one lane per
+// segment: the error proxies and the lower hull.
 __global__ void __launch_bounds__(kSegWarps * 32) seg_select_kernel(const __grid_constant__ SegArgs A) {
     pdl_wait();
+    extern __shared__ __align__(16) uint8_t seg_smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int u = blockIdx.y;
     const int b = u / A.Hkv;
-    const int j = blockIdx.x * kSegWarps + warp;
-    if (j >= A.plan.nseg[b]) return;
-    __shared__ float ss[kSegWarps][256];
-    __shared__ double gs[kSegWarps][256];
-    __shared__ uint8_t kept[kSegWarps][256];
-    const int S = A.S, r = A.r;
-    const int64_t t0 = static_cast<int64_t>(j) * S;
-    for (int t = lane; t < S; t += 32) {
-        ss[warp][t] = A.s[static_cast<int64_t>(u) * A.s_stride + t0 + t];
-        gs[warp][t] = A.g[static_cast<int64_t>(u) * A.g_stride + t0 + t];
-    }
-    __syncwarp();
-    const int64_t slot = static_cast<int64_t>(u) * A.max_nseg + j;
-    int before = 0;
-    for (int tb = 0; tb < S; tb += 64) {
-        // two tokens per lane and pass: t = tb + lane and tb + 32 + lane
-        const int ta = tb + lane, tc = tb + 32 + lane;
-        const float va = (ta < S) ? ss[warp][ta] : 0.f;
-        const float vc = (tc < S) ? ss[warp][tc] : 0.f;
-        int ra = 0, rc = 0;
-        for (int t2 = 0; t2 < S; ++t2) {
-            const float v2 = ss[warp][t2];
-            ra += (v2 > va) || (v2 == va && t2 < ta);
-            rc += (v2 > vc) || (v2 == vc && t2 < tc);
-        }
-        const bool ka = ta < S && ra < r, kc = tc < S && rc < r;
-        if (ta < S) kept[warp][ta] = ka ? 1 : 0;
-        if (tc < S) kept[warp][tc] = kc ? 1 : 0;
-        const uint32_t lt = (1u << lane) - 1u;
-        const uint32_t ba = __ballot_sync(0xffffffffu, ka);
-        if (ka) A.tidx[slot * r + before + __popc(ba & lt)] = static_cast<uint8_t>(ta);
-        before += __popc(ba);
-        const uint32_t bc = __ballot_sync(0xffffffffu, kc);
-        if (kc) A.tidx[slot * r + before + __popc(bc & lt)] = static_cast<uint8_t>(tc);
-        before += __popc(bc);
-    }
-    __syncwarp();
-    if (lane != 0) return;
+    const int nseg = A.plan.nseg[b];
+    const int jb = blockIdx.x * kSegWarps;
+    if (jb >= nseg) return;
+    const int S = A.S, r = A.r, RW = seg_row(S);
+    double* sgs = reinterpret_cast<double*>(seg_smem);                      // [32][RW]
+    double* sums = sgs + kSegWarps * RW;                                    // [3][32]
+    float* ss = reinterpret_cast<float*>(sums + 3 * kSegWarps);             // [32][RW]
+    uint8_t* kept = reinterpret_cast<uint8_t*>(ss + kSegWarps * RW);        // [32][RW]
 
-    // three independent sums, each sequential in t (one loop for ILP)
-    double etok = 0.0, ech = 0.0, ekept = 0.0;
-    for (int t = 0; t < S; ++t) {
-        const double sv = static_cast<double>(ss[warp][t]);
-        const double sg = __dmul_rn(sv, gs[warp][t]);
-        ech = __dadd_rn(ech, sg);
-        if (kept[warp][t]) ekept = __dadd_rn(ekept, sg);
-        else etok = __dadd_rn(etok, sv);
+    const int j = jb + warp;
+    if (j < nseg) {
+        const int64_t t0 = static_cast<int64_t>(j) * S;
+        float* srow = ss + warp * RW;
+        for (int t = lane; t < S; t += 32) {
+            const float sv = A.s[static_cast<int64_t>(u) * A.s_stride + t0 + t];
+            srow[t] = sv;
+            sgs[warp * RW + t] = __dmul_rn(static_cast<double>(sv), A.g[static_cast<int64_t>(u) * A.g_stride + t0 + t]);
+        }
+        __syncwarp();
+        const int64_t slot = static_cast<int64_t>(u) * A.max_nseg + j;
+        int before = 0;
+        for (int tb = 0; tb < S; tb += 64) {
+            // two tokens per lane and pass: t = tb + lane and tb + 32 + lane
+            const int ta = tb + lane, tc = tb + 32 + lane;
+            const float va = (ta < S) ? srow[ta] : 0.f;
+            const float vc = (tc < S) ? srow[tc] : 0.f;
+            int ra = 0, rc = 0;
+            for (int t2 = 0; t2 < S; ++t2) {
+                const float v2 = srow[t2];
+                ra += (v2 > va) || (v2 == va && t2 < ta);
+                rc += (v2 > vc) || (v2 == vc && t2 < tc);
+            }
+            const bool ka = ta < S && ra < r, kc = tc < S && rc < r;
+            if (ta < S) kept[warp * RW + ta] = ka ? 1 : 0;
+            if (tc < S) kept[warp * RW + tc] = kc ? 1 : 0;
+            const uint32_t lt = (1u << lane) - 1u;
+            const uint32_t ba = __ballot_sync(0xffffffffu, ka);
+            if (ka) A.tidx[slot * r + before + __popc(ba & lt)] = static_cast<uint8_t>(ta);
+            before += __popc(ba);
+            const uint32_t bc = __ballot_sync(0xffffffffu, kc);
+            if (kc) A.tidx[slot * r + before + __popc(bc & lt)] = static_cast<uint8_t>(tc);
+            before += __popc(bc);
+        }
     }
+    __syncthreads();
+    if (warp < 3 && jb + lane < nseg) {
+        // lane <-> segment jb + lane; the fp64 sums in ascending t
+        double acc = 0.0;
+        const double* grow = sgs + lane * RW;
+        const float* srow = ss + lane * RW;
+        const uint8_t* krow = kept + lane * RW;
+        for (int t = 0; t < S; ++t) {
+            const bool kp = krow[t] != 0;
+            if (warp == 0) acc = __dadd_rn(acc, grow[t]);
+            else if (warp == 1) { if (kp) acc = __dadd_rn(acc, grow[t]); }
+            else if (!kp) acc = __dadd_rn(acc, static_cast<double>(srow[t]));
+        }
+        sums[warp * kSegWarps + lane] = acc;
+    }
+    __syncthreads();
+    if (warp != 0 || jb + lane >= nseg) return;
+    const int js = jb + lane;
+    const int64_t slot = static_cast<int64_t>(u) * A.max_nseg + js;
+    const double ech = sums[lane], ekept = sums[kSegWarps + lane], etok = sums[2 * kSegWarps + lane];
     double E[4];
     E[KV2D_FULL] = 0.0;
     E[KV2D_TOK] = etok;
@@ -107,7 +137,7 @@ __global__ void __launch_bounds__(kSegWarps * 32) seg_select_kernel(const __grid
     for (int k = 0; k < 4; ++k) A.E[slot * 4 + k] = E[k];
     if (A.dbg_E)
         for (int k = 0; k < 4; ++k)
-            A.dbg_E[(static_cast<int64_t>(u) * A.dbg_seg_stride + j) * 4 + k] = E[k];
+            A.dbg_E[(static_cast<int64_t>(u) * A.dbg_seg_stride + js) * 4 + k] = E[k];
 
     // lower convex hull over (bytes, E), options visited by (bytes, id)
     int hv[4];
@@ -473,8 +503,11 @@ cudaError_t launch_selection(const SelectLaunch& L, cudaStream_t stream) {
         sa.dbg_E = L.dbg_E;
         sa.dbg_seg_stride = L.dbg_seg_stride;
         dim3 grid((L.max_nseg + kSegWarps - 1) / kSegWarps, units);
+        const int sm_bytes = seg_smem_bytes(sa.S);
+        cudaError_t e0 = cudaFuncSetAttribute(seg_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, sm_bytes);
+        if (e0 != cudaSuccess) return e0;
         prof_begin(stream, kProfSegSelect);
-        cudaError_t e1 = launch_k(seg_select_kernel, grid, dim3(kSegWarps * 32), 0, stream, sa);
+        cudaError_t e1 = launch_k(seg_select_kernel, grid, dim3(kSegWarps * 32), sm_bytes, stream, sa);
         if (e1 != cudaSuccess) return e1;
         prof_end(stream, kProfSegSelect);
         cudaError_t e = cudaGetLastError();
