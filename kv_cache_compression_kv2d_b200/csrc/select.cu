@@ -26,7 +26,8 @@ namespace kv2d {
 
 namespace {
 
-constexpr int kSegWarps = 32;   // segments per CTA (one warp each, then one lane each)
+constexpr int kSegWarps = 32;   // segments per CTA (one warp each, then one lane each; <= 32)
+static_assert(kSegWarps <= 32, "phases 2 and 3 give each segment one lane of a warp");
 
 struct SegArgs {
     SeqPlan plan;
@@ -110,7 +111,7 @@ __global__ void __launch_bounds__(kSegWarps * 32) seg_select_kernel(const __grid
         }
     }
     __syncthreads();
-    if (warp < 3 && jb + lane < nseg) {
+    if (warp < 3 && lane < kSegWarps && jb + lane < nseg) {
         // lane <-> segment jb + lane; the fp64 sums in ascending t
         double acc = 0.0;
         const double* grow = sgs + lane * RW;
@@ -125,7 +126,7 @@ __global__ void __launch_bounds__(kSegWarps * 32) seg_select_kernel(const __grid
         sums[warp * kSegWarps + lane] = acc;
     }
     __syncthreads();
-    if (warp != 0 || jb + lane >= nseg) return;
+    if (warp != 0 || lane >= kSegWarps || jb + lane >= nseg) return;
     const int js = jb + lane;
     const int64_t slot = static_cast<int64_t>(u) * A.max_nseg + js;
     const double ech = sums[lane], ekept = sums[kSegWarps + lane], etok = sums[2 * kSegWarps + lane];
