@@ -225,6 +225,26 @@ __device__ __forceinline__ float fast_exp2(float x) {
     return y;
 }
 
+// 2^x on the FMA pipe (for x <= 0; below -126 the result is ~0): Cody-Waite
+// range reduction x = n + f with n = round(x) by the 1.5 * 2^23 shifter and
+// f in [-1/2, 1/2], then 2^f by a degree-5 polynomial whose coefficients were
+// fitted to minimise the relative error on that interval (max 2.2e-7 with
+// fp32 Horner steps), and n added to the exponent bits.  Used for part of
+// the exponentials of the scoring epilogues so that the MUFU pipe is not the
+// only one busy.
+__device__ __forceinline__ float exp2_fma(float x) {
+    x = fmaxf(x, -126.f);
+    const float t = x + 12582912.f;
+    const float f = x - (t - 12582912.f);
+    float p = 1.327646780e-03f;
+    p = fmaf(p, f, 9.675540961e-03f);
+    p = fmaf(p, f, 5.550713465e-02f);
+    p = fmaf(p, f, 2.402212024e-01f);
+    p = fmaf(p, f, 6.931469440e-01f);
+    p = fmaf(p, f, 1.000000119e+00f);
+    return __int_as_float(__float_as_int(p) + ((__float_as_int(t) - 0x4B400000) << 23));
+}
+
 // Programmatic dependent launch: wait until the grids this one depends on
 // have completed and their writes are visible (a no-op without a dependency).
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }

@@ -464,7 +464,7 @@ __global__ void __launch_bounds__(kPassThreads, 1)
                         a0 += fast_exp2(fmaf(__uint_as_float(r[j]), c2, -lz.x));
                         a1 += fast_exp2(fmaf(__uint_as_float(r[j + 1]), c2, -lz.y));
                         a2 += fast_exp2(fmaf(__uint_as_float(r[j + 2]), c2, -lz.z));
-                        a3 += fast_exp2(fmaf(__uint_as_float(r[j + 3]), c2, -lz.w));
+                        a3 += exp2_fma(fmaf(__uint_as_float(r[j + 3]), c2, -lz.w));
                     }
                 } else {
                     const int* wp = wpos_s + col0 + cc;
