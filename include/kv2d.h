@@ -233,10 +233,12 @@ KV2D_API kv2d_status kv2d_append(const kv2d_params* p, int batch, const kv2d_den
  *   q                 device fp16 [batch][Hq][d].
  *   out               device fp16 [batch][Hq][d].
  *   ws, ws_bytes      kv2d_workspace_bytes(p, DECODE, batch, max_seq_len)
- *                     bytes; split partials and per-unit tickets live here.
+ *                     bytes; per-CTA partials and per-unit tickets live
+ *                     here.
  *                     Zero it once before its first use; every completed
  *                     call leaves the tickets at zero again.
- * Deterministic: fixed split and merge order. */
+ * Deterministic: the batch's bytes are cut into one share per CTA (a
+ * function of the data and the SM count only); fixed merge order. */
 KV2D_API kv2d_status kv2d_decode_attn(const kv2d_params* p, int batch, const kv2d_ccache* cc,
                              const kv2d_dense* kv, const int32_t* seq_len_dev,
                              int32_t max_seq_len_host, const void* q, void* out, void* ws,
@@ -249,11 +251,12 @@ KV2D_API kv2d_status kv2d_decode_attn(const kv2d_params* p, int batch, const kv2
  * cudaMalloc because that call can synchronise the device in the middle of a
  * latency-critical loop.  There is no counterpart on the pages; it is an
  * interface convenience only.
- *   It takes no workspace.  Its split partials and per-unit tickets live in
- *   a fixed 8 MiB array in the library's own device memory, which every GPU
- *   that loads the library holds until the process exits.  Calls whose
- *   scratch would exceed 8 MiB (units x splits x G x (d + 4) x 4 bytes plus
- *   a few hundred bytes) return KV2D_ERR_WORKSPACE before launching.
+ *   It takes no workspace.  Its per-CTA partials and per-unit tickets live
+ *   in a fixed 8 MiB array in the library's own device memory, which every
+ *   GPU that loads the library holds until the process exits.  Calls whose
+ *   scratch would exceed 8 MiB ((units + CTAs) x G x (d + 4) x 4 bytes plus
+ *   4 bytes per unit and 256 bytes; CTAs <= the SM count) return
+ *   KV2D_ERR_WORKSPACE before launching.
  *   The first call on each device looks up the array's device address with
  *   the CUDA runtime; make that first call outside any stream capture.
  *   All calls on a device share the one array and each leaves its partials

@@ -120,7 +120,6 @@ struct Carver {
 };
 
 constexpr int kMaxSplit1 = 64;
-constexpr int kMaxSplitDec = 64;
 
 struct CompressLayout {
     size_t apart, part, s, g, cmask, tidx, E, hull, eff, db, strat, ok, total;
@@ -165,7 +164,7 @@ DecodeLayout decode_layout(const kv2d_params* p, int batch) {
     Carver c;
     c.take(256);
     L.ticket = c.take(units * 4);
-    L.part = c.take(units * kMaxSplitDec * sh.G * (kHeadDim + 4) * 4);
+    L.part = c.take((units + kMaxDecCtas) * sh.G * (kHeadDim + 4) * 4);
     L.total = c.off;
     return L;
 }
@@ -647,7 +646,7 @@ kv2d_status kv2d_decode_attn(const kv2d_params* p, int batch, const kv2d_ccache*
     L.seq_len = seq_len_dev;
     L.q = static_cast<const __half*>(q);
     L.out = static_cast<__half*>(out);
-    L.nsplit = std::min(kMaxSplitDec, decode_split_count(batch * sh.Hkv, max_seq_len_host, num_sms()));
+    L.nctas = decode_cta_count(batch * sh.Hkv, max_seq_len_host, num_sms(), &L.kps);
     L.part = reinterpret_cast<float*>(w + WL.part);
     L.ticket = reinterpret_cast<uint32_t*>(w + WL.ticket);
     L.status = reinterpret_cast<uint32_t*>(w);
@@ -679,17 +678,17 @@ kv2d_status kv2d_decode_attn_noalloc(const kv2d_params* p, int batch, const kv2d
     if (max_seq_len_host < 0 || max_seq_len_host > dense_capacity(kv))
         return fail(KV2D_ERR_INVALID_ARG, "max_seq_len %d outside [0, capacity]", max_seq_len_host);
     const int64_t units = static_cast<int64_t>(batch) * sh.Hkv;
-    const int nsplit =
-        std::min(kMaxSplitDec, decode_split_count(static_cast<int>(units), max_seq_len_host, num_sms()));
+    int kps = 0;
+    const int nctas = decode_cta_count(static_cast<int>(units), max_seq_len_host, num_sms(), &kps);
     Carver c;
     c.take(256);                                               // status word
     const size_t ticket_off = c.take(units * 4);
-    const size_t part_off = c.take(units * nsplit * sh.G * (kHeadDim + 4) * 4);
+    const size_t part_off = c.take((units + nctas) * sh.G * (kHeadDim + 4) * 4);
     if (c.off > kNoAllocScratchBytes)
         return fail(KV2D_ERR_WORKSPACE,
-                    "decode needs %zu bytes of scratch for %lld units x %d splits; the built-in "
+                    "decode needs %zu bytes of scratch for %lld units on %d CTAs; the built-in "
                     "scratch holds %zu bytes",
-                    c.off, static_cast<long long>(units), nsplit, kNoAllocScratchBytes);
+                    c.off, static_cast<long long>(units), nctas, kNoAllocScratchBytes);
     void* scratch = nullptr;
     if ((st = noalloc_scratch(&scratch)) != KV2D_OK) return st;
     uint8_t* w = static_cast<uint8_t*>(scratch);
@@ -708,7 +707,8 @@ kv2d_status kv2d_decode_attn_noalloc(const kv2d_params* p, int batch, const kv2d
     L.seq_len = seq_len_dev;
     L.q = static_cast<const __half*>(q);
     L.out = static_cast<__half*>(out);
-    L.nsplit = nsplit;
+    L.nctas = nctas;
+    L.kps = kps;
     L.part = reinterpret_cast<float*>(w + part_off);
     L.ticket = reinterpret_cast<uint32_t*>(w + ticket_off);   // left at zero by every call
     L.status = status_dev ? status_dev : reinterpret_cast<uint32_t*>(w);

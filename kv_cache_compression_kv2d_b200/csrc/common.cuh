@@ -88,6 +88,12 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32
 
 // ---------------------------------------------------------------- TMA
 
+// Orders this thread's earlier shared-memory accesses (generic proxy) before
+// later accesses by the copy engine (async proxy) to the same bytes.
+__device__ __forceinline__ void fence_proxy_async() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // 2-D / 4-D tiled bulk tensor load into this CTA's shared memory, completion
 // counted in bytes on an mbarrier.  No multicast.
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar,

@@ -5,37 +5,44 @@
 // Compression", Sec. 5.3 PackedAttention and Fig. 6 packed sparse attention)
 // runs decode attention directly on the compressed segments.  Here one unit
 // (sequence b, KV head h) serves its G query heads from every byte it loads:
-//   - the unit's work is its packed arena plus its dense tail
-//     [comp_end, seq_len), 512 bytes per dense token; the kernel splits that
-//     byte range evenly over nsplit CTAs (a CTA takes the segments whose
-//     first byte falls in its range, found by binary search on the
-//     descriptors, and the tail tokens likewise);
-//   - each warp takes every 8th 16-token block of its CTA's range and runs
-//     q.k and p.v on the tensor cores (mma.sync m16n8k16, fp16 in, fp32
-//     accumulate; the G heads are the rows of the 16-row tile);
-//   - lane 0 of each warp has the TMA unit copy the key and value rows of
-//     its blocks into a three-stage shared-memory ring (one bulk copy per
-//     contiguous run of rows, completion on a per-stage mbarrier), so a warp
-//     has two blocks in flight while it computes a third; CH / BOTH keys are
-//     scattered from their (index, value) pairs into a dense key tile;
-//   - segments of at most 8 tokens pair up, one per half of a 16-row block;
+//   - a unit's work is its packed arena plus its dense tail
+//     [comp_end, seq_len), 512 bytes per dense token; the units' byte
+//     ranges, laid end to end over the batch, are cut into one equal share
+//     per CTA (one CTA per SM), so every SM reads the same number of bytes
+//     whatever the units' lengths; a CTA takes the segments whose first
+//     byte falls in its share (counted on the descriptors) and the tail
+//     tokens likewise, one unit after another when its share spans several;
+//   - the CTA's range is cut into blocks of at most 8 tokens (a segment of
+//     at most 8 tokens is one block); with W warps, warp w takes blocks w,
+//     w + W, ... and runs q.k and p.v on the tensor cores (mma.sync
+//     m16n8k16 / m16n8k8, fp16 in, fp32 accumulate; the G heads are the
+//     rows of the tile);
+//   - lane 0 of each warp has the TMA unit copy the bytes of its blocks
+//     into a four-stage shared-memory ring (one bulk copy per contiguous
+//     run, completion on a per-stage mbarrier), so a warp has three blocks
+//     in flight while it computes a fourth; CH / BOTH keys are scattered
+//     from their (index, value) pairs into a dense key tile;
+//   - the per-block work is a chain of dependent steps (copy wait, q.k,
+//     softmax shuffles, p.v), so the CTA runs 12 warps, three per
+//     scheduler, to overlap the chains;
 //   - scores meet an online softmax per head in the log2 domain; warps, then
-//     CTAs, merge their (max, sum, output) partials in a fixed order, the
-//     last CTA of a unit (atomic ticket) writing the fp16 output.
+//     the CTAs holding pieces of a unit, merge their (max, sum, output)
+//     partials in a fixed order, the last CTA of a unit (atomic ticket)
+//     writing the fp16 output.
 #include "kernels.h"
 
 namespace kv2d {
 
 namespace {
 
-constexpr int kDecWarps = 8;
+constexpr int kDecWarps = 12;
 constexpr int kDecThreads = kDecWarps * 32;
-constexpr int kDecStages = 6;                       // stages per warp: 5 blocks in flight
+constexpr int kDecStages = 4;                       // stages per warp: 3 blocks in flight
 // A stage holds one block of up to 8 tokens: 8 key rows, then 8 value rows,
-// back to back, so that a segment block arrives in two bulk copies.  Short
-// blocks keep many stages in flight: the copy latency under load is several
-// microseconds, so the bytes a warp has in flight set its rate.  A
-// quarter-warp's key reads meet 2 rows per bank group and its value reads 4.
+// back to back.  Short blocks keep many stages in flight (12 warps x 3 x
+// 4 KB per SM): the copy latency under load is microseconds, so the bytes in
+// flight set the rate.  A quarter-warp's key reads meet 2 rows per bank
+// group and its value reads 4.
 constexpr int kDecRows = 8;
 constexpr int kDecKStride = 256, kDecVStride = 256;
 constexpr int kDecKBytes = kDecRows * kDecKStride;
@@ -84,14 +91,50 @@ struct DecodeArgs {
     const int32_t* seq_len;
     const __half* q;
     __half* out;
-    int nsplit;
+    int units;
+    int kps;          // > 0: unit c / kps, piece c % kps of kps equal ones; 0: batch-wide shares
     float* part;
     uint32_t* ticket;
     uint32_t* status;
 };
 
 constexpr int64_t kTailBytes = 2 * kHeadDim * 2;   // K + V row of one dense token
-constexpr int kDescCache = 512;                    // descriptors staged per CTA
+
+// The lengths of one unit, clamped into range (a value out of range sets
+// KV2D_DEV_SEQ_RANGE when report is set): dense length T, compression end
+// ce, segment count nsg, packed bytes U.
+struct UnitLens {
+    int T, ce, nsg;
+    int64_t U;
+};
+
+__device__ __forceinline__ UnitLens unit_lens(const DecodeArgs& A, int u, bool report) {
+    const int b = u / A.Hkv;
+    UnitLens L;
+    L.T = A.seq_len[b];
+    L.ce = A.comp_end[b];
+    L.nsg = A.n_segs[u];
+    L.U = A.used_bytes[u];
+    const int cap = A.dv.block_table ? A.dv.max_blocks * A.dv.block_size : A.dv.capacity;
+    if (L.T < 0 || L.T > cap || L.ce < 0 || L.ce > L.T || L.nsg < 0 || L.nsg > A.max_segs || L.U < 0 ||
+        L.U > A.arena_stride) {
+        if (report) set_status(A.status, KV2D_DEV_SEQ_RANGE);
+        L.T = max(0, min(L.T, cap));
+        L.ce = max(0, min(L.ce, L.T));
+        L.nsg = max(0, min(L.nsg, A.max_segs));
+        L.U = max(static_cast<int64_t>(0), min(L.U, A.arena_stride));
+    }
+    return L;
+}
+
+// A unit's length in the batch-wide byte range the CTAs share: one byte that
+// stands for the unit itself (so that every unit, even an empty one, has a
+// CTA that writes its output), then its packed bytes, then 512 bytes per
+// dense tail token.
+__device__ __forceinline__ int64_t unit_span(const UnitLens& L) {
+    return 1 + L.U + static_cast<int64_t>(L.T - L.ce) * kTailBytes;
+}
+constexpr int kDescCache = 2048;                   // descriptors staged per CTA (a 128K-token unit at S = 64)
 
 // ------------------------------------------------------ tensor-core decode
 //
@@ -225,25 +268,30 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
                  : "memory");
 }
 
-// A 16-token block of one warp.  kind: 0 none, 1 dense rows (FULL / TOK
-// segment or tail), 2 channel-sparse keys (CH / BOTH).
+// A block of up to 8 tokens of one warp.  kind & 3: 0 none, 1 dense rows
+// (FULL / TOK segment or tail), 2 channel-sparse keys (CH / BOTH); kind & 4:
+// the block is a whole segment whose sections are contiguous in the arena
+// and arrive in one copy (dense: key rows, then value rows right after
+// them; sparse: index bytes and key values end where the value rows start).
+constexpr int kBlkOne = 4;
 struct DecBlock {
     int kind, nlo, nhi;
     const uint8_t* ci;      // sparse: the block's index bytes
     const __half* kv;       // sparse: the block's key values
 };
 
-constexpr int kDescPerThread = 2;   // descriptors each thread loads in the prologue
+constexpr int kDescPerThread = kDescCache / kDecThreads;   // descriptors each thread loads in the prologue
 
 template <int G>
 __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_constant__ DecodeArgs A) {
     extern __shared__ __align__(16) uint8_t dec_smem[];
-    const int sp = blockIdx.x, u = blockIdx.y;
-    const int b = u / A.Hkv, h = u % A.Hkv;
+    const int cta = blockIdx.x, ncta = gridDim.x;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, t = lane & 3;
     __shared__ float wm[kDecWarps][G], wl[kDecWarps][G];
     __shared__ int wcnt[kDecWarps][2];
+    __shared__ long long wsum[kDecWarps];
+    __shared__ long long s_part[3];   // first unit, its start, last unit
     __shared__ __align__(8) uint64_t sbar[kDecWarps][kDecStages];
     __shared__ int is_last;
     __shared__ uint64_t dsm[kDescCache];
@@ -253,6 +301,105 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
     float (*wo)[G][kHeadDim] = reinterpret_cast<float (*)[G][kHeadDim]>(dec_smem);
 
     pdl_wait();
+    // ---- the batch-wide partition: the units' spans laid end to end, CTA c
+    // takes bytes [lo_c, lo_{c+1}) with lo_c = floor(Wtot c / n) and works
+    // on every unit from the one holding byte lo_c to the one holding byte
+    // max(lo_c, lo_{c+1} - 1) (a "piece" of each); a segment or tail token
+    // belongs to the CTA that holds its first byte.  A CTA whose range is
+    // empty (fewer bytes than CTAs) still takes the unit holding lo_c, with
+    // no work, so that the pieces of a unit are consecutive CTAs.
+    const int units = A.units, kps = A.kps;
+    long long Wtot = 0, GL = 0, GH = 0;
+    if (kps == 0) {
+        long long mine = 0;
+        for (int u = tid; u < units; u += kDecThreads) mine += unit_span(unit_lens(A, u, false));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mine += __shfl_xor_sync(0xffffffffu, mine, o);
+        if (lane == 0) wsum[warp] = mine;
+        __syncthreads();
+#pragma unroll
+        for (int w = 0; w < kDecWarps; ++w) Wtot += wsum[w];
+        GL = Wtot * cta / ncta;
+        GH = Wtot * (cta + 1) / ncta;
+        const long long Gend = GH > GL ? GH - 1 : GL;   // the last byte the CTA looks at
+        long long base = 0;   // span of the units before the chunk
+        for (int c0 = 0; c0 < units && base <= Gend; c0 += kDecThreads) {
+            const int u = c0 + tid;
+            const long long w = (u < units) ? unit_span(unit_lens(A, u, false)) : 0;
+            long long x = w;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const long long y = __shfl_up_sync(0xffffffffu, x, o);
+                if (lane >= o) x += y;
+            }
+            __syncthreads();   // wsum is free again
+            if (lane == 31) wsum[warp] = x;
+            __syncthreads();
+            long long before = base, chunk = 0;
+#pragma unroll
+            for (int w2 = 0; w2 < kDecWarps; ++w2) {
+                if (w2 < warp) before += wsum[w2];
+                chunk += wsum[w2];
+            }
+            const long long incl = before + x, excl = incl - w;
+            if (u < units && excl <= GL && GL < incl) {
+                s_part[0] = u;
+                s_part[1] = excl;
+            }
+            if (u < units && excl <= Gend && Gend < incl) s_part[2] = u;
+            base += chunk;
+        }
+    } else if (tid == 0) {
+        // few units: kps CTAs each, so that no CTA pays a second piece's
+        // fixed costs (lengths, descriptors, merges)
+        s_part[0] = s_part[2] = cta / kps;
+        s_part[1] = 0;
+    }
+    if (tid < kDecWarps * kDecStages) {
+        mbar_init(&sbar[tid / kDecStages][tid % kDecStages], 1);
+        mbar_fence_init();
+    }
+    // value rows past a block's last token must hold finite numbers; the
+    // copy engine writes these buffers next
+    for (int i = tid; i < kDecSmem / 16; i += kDecThreads)
+        reinterpret_cast<uint4*>(dec_smem)[i] = make_uint4(0, 0, 0, 0);
+    fence_proxy_async();
+    __syncthreads();
+    const int u_first = static_cast<int>(s_part[0]), u_last = static_cast<int>(s_part[2]);
+    long long P = s_part[1];   // start of the current unit's span
+    // the last CTA c with lo_c <= x, and the first CTA c with lo_c >= x
+    auto cta_at = [&](long long x) { return static_cast<int>(((x + 1) * ncta - 1) / Wtot); };
+    auto cta_from = [&](long long x) { return static_cast<int>((x * ncta + Wtot - 1) / Wtot); };
+
+    const float c2 = A.c2;
+    const int S = A.S, r = A.r, c = A.c;
+    const uint32_t wbase = smem_u32(dec_smem) + warp * (kDecStages * kDecSlotBytes);
+    // stage s of this warp: key rows at kreg(s), value rows at kreg(s) +
+    // kDecKBytes (see DecBlock for the one-copy layouts)
+    auto kreg = [&](int stage) -> uint32_t { return wbase + stage * kDecSlotBytes; };
+    const uint32_t bar0 = smem_u32(&sbar[warp][0]);
+    auto lds16 = [&](uint32_t a) {
+        uint4 v;
+        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                     : "r"(a));
+        return v;
+    };
+    auto seg_ntok = [&](uint64_t d) {
+        const int sty = static_cast<int>((d >> 32) & 255u);
+        return (sty == KV2D_TOK || sty == KV2D_BOTH) ? r : S;
+    };
+    auto seg_dense = [&](uint64_t d) {
+        const int sty = static_cast<int>((d >> 32) & 255u);
+        return sty == KV2D_FULL || sty == KV2D_TOK;
+    };
+    // blocks this warp has consumed so far: block k of the warp uses stage
+    // k % kDecStages and that stage's (k / kDecStages)-th barrier phase
+    int kbase = 0;
+    bool dead = false;   // a copy wait gave up: no more copies from this warp
+
+    for (int u = u_first; u <= u_last; ++u) {
+    const int b = u / A.Hkv, h = u % A.Hkv;
     // q fragments (rows g < G): chunk 4 (ks / 2) + t of head g, words of step ks
     uint32_t qa[8][2];
     {
@@ -272,27 +419,36 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
     }
     // ---- one round trip: q, the unit's lengths and its first descriptors
     const uint64_t* D = A.desc + static_cast<int64_t>(u) * A.max_segs;
-    int T = A.seq_len[b], ce = A.comp_end[b];
-    const int64_t U = A.used_bytes[u];
-    int nsg = A.n_segs[u];
+    const UnitLens Ln = unit_lens(A, u, tid == 0);
+    const int T = Ln.T, ce = Ln.ce, nsg = Ln.nsg;
+    const int64_t U = Ln.U;
     uint64_t dreg[kDescPerThread];
 #pragma unroll
     for (int k = 0; k < kDescPerThread; ++k) {
         const int j = tid + k * kDecThreads;
         dreg[k] = (j < A.max_segs) ? D[j] : 0ull;
     }
-    {
-        const int cap = A.dv.block_table ? A.dv.max_blocks * A.dv.block_size : A.dv.capacity;
-        if (T < 0 || T > cap || ce < 0 || ce > T || nsg < 0 || nsg > A.max_segs) {
-            if (tid == 0) set_status(A.status, KV2D_DEV_SEQ_RANGE);
-            T = max(0, min(T, cap));
-            ce = max(0, min(ce, T));
-            nsg = max(0, min(nsg, A.max_segs));
-        }
-    }
     const int ntail = T - ce;
-    const int64_t Wt = U + static_cast<int64_t>(ntail) * kTailBytes;
-    const int64_t lo = Wt * sp / A.nsplit, hi = Wt * (sp + 1) / A.nsplit;
+    // this CTA's piece of the unit, as offsets into its packed bytes and
+    // tail (byte x of the unit is byte P + 1 + x of the batch-wide range)
+    const long long span = unit_span(Ln);
+    int64_t lo, hi;
+    int first, last;   // the pieces of the unit are CTAs first .. last
+    if (kps > 0) {
+        const int sp = cta - u * kps;
+        lo = span * sp / kps - 1;
+        hi = span * (sp + 1) / kps - 1;
+        first = u * kps;
+        last = first + kps - 1;
+    } else {
+        lo = GL - P - 1;
+        hi = GH - P - 1;
+        // first: the first CTA whose last byte (first byte when it has none)
+        // reaches P
+        first = min(cta_from(P), cta_from(P + 1) - 1);
+        last = cta_at(P + span - 1);
+        P += span;
+    }
     // segments whose first byte lies in [lo, hi)
     {
         int c_lo = 0, c_hi = 0;
@@ -319,13 +475,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
             wcnt[warp][0] = c_lo;
             wcnt[warp][1] = c_hi;
         }
-        if (tid < kDecWarps * kDecStages) {
-            mbar_init(&sbar[tid / kDecStages][tid % kDecStages], 1);
-            mbar_fence_init();
-        }
-        // value rows past a block's last token must hold finite numbers
-        for (int i = tid; i < kDecSmem / 16; i += kDecThreads)
-            reinterpret_cast<uint4*>(dec_smem)[i] = make_uint4(0, 0, 0, 0);
     }
     __syncthreads();
     int j_lo = 0, j_hi = 0;
@@ -361,31 +510,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
         st.o[j][0] = 0.f;
         st.o[j][1] = 0.f;
     }
-    const float c2 = A.c2;
-    const int S = A.S, r = A.r, c = A.c;
     const uint8_t* ubase = A.arena + static_cast<int64_t>(u) * A.arena_stride;
-    const uint32_t wbase = smem_u32(dec_smem) + warp * (kDecStages * kDecSlotBytes);
-    // stage s of this warp: key rows at kreg(s), value rows at kreg(s) +
-    // kDecKBytes; sparse keys stage their pairs in the key region (index
-    // bytes, then values from byte 512) before they are scattered
-    auto kreg = [&](int stage) -> uint32_t { return wbase + stage * kDecSlotBytes; };
-    const uint32_t bar0 = smem_u32(&sbar[warp][0]);
-    auto lds16 = [&](uint32_t a) {
-        uint4 v;
-        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                     : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                     : "r"(a));
-        return v;
-    };
     auto desc = [&](int j) -> uint64_t { return cached ? dsm[j - j_lo] : D[j]; };
-    auto seg_ntok = [&](uint64_t d) {
-        const int sty = static_cast<int>((d >> 32) & 255u);
-        return (sty == KV2D_TOK || sty == KV2D_BOTH) ? r : S;
-    };
-    auto seg_dense = [&](uint64_t d) {
-        const int sty = static_cast<int>((d >> 32) & 255u);
-        return sty == KV2D_FULL || sty == KV2D_TOK;
-    };
     // first K row of a dense segment (its V rows follow its ntok K rows)
     auto seg_k = [&](uint64_t d) {
         const int sty = static_cast<int>((d >> 32) & 255u);
@@ -396,8 +522,29 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
     // ---- the CTA's items, in order: every segment in blocks of up to 8
     // tokens, then the dense tail in blocks of 8.  Item i belongs to warp
     // i % kDecWarps, so the order of every sum is fixed and the output is
-    // deterministic.
-    int g_seg = j_lo, g_base = 0, g_next = warp;
+    // deterministic.  A warp finds the segment of an item in a window of 32
+    // consecutive segments it holds one per lane (descriptor and inclusive
+    // prefix of item counts): one ballot instead of a walk over the
+    // segments in between.
+    int w_j0 = j_lo;          // first segment of the window
+    uint64_t w_d = 0;         // lane l: descriptor of segment w_j0 + l
+    int w_pre = 0;            // lane l: items of segments w_j0 .. w_j0 + l
+    int w_base = 0;           // items of the segments before the window
+    int w_tot = 0;            // items of the window
+    auto load_window = [&]() {
+        const int j = w_j0 + lane;
+        w_d = (j < j_hi) ? desc(j) : 0ull;
+        int n = (j < j_hi) ? (seg_ntok(w_d) + kDecRows - 1) / kDecRows : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, n, o);
+            if (lane >= o) n += y;
+        }
+        w_pre = n;
+        w_tot = __shfl_sync(0xffffffffu, n, 31);
+    };
+    if (w_j0 < j_hi) load_window();
+    int g_next = warp;
     auto next_block = [&](int stage) -> DecBlock {
         DecBlock bk{0, 0, 0, nullptr, nullptr};
         const int g_idx = g_next;
@@ -408,23 +555,27 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
         bool tail = false;
         uint64_t d = 0;
         int t0 = 0;
-        while (g_seg < j_hi) {
-            d = desc(g_seg);
-            const int nitems = (seg_ntok(d) + kDecRows - 1) / kDecRows;
-            if (g_idx < g_base + nitems) break;
-            g_base += nitems;
-            ++g_seg;
+        while (w_j0 < j_hi && g_idx >= w_base + w_tot) {
+            w_base += w_tot;
+            w_tot = 0;
+            w_j0 += 32;
+            if (w_j0 < j_hi) load_window();
         }
-        if (g_seg < j_hi) {
+        if (w_j0 < j_hi) {
+            const int rel = g_idx - w_base;
+            const int L = __ffs(__ballot_sync(0xffffffffu, w_pre > rel)) - 1;
+            d = __shfl_sync(0xffffffffu, w_d, L);
+            const int pre = __shfl_sync(0xffffffffu, w_pre, L);
             const int ntok = seg_ntok(d);
-            t0 = (g_idx - g_base) * kDecRows;
+            t0 = (rel - (pre - (ntok + kDecRows - 1) / kDecRows)) * kDecRows;
             n = min(kDecRows, ntok - t0);
+            const int one = (ntok <= kDecRows) ? kBlkOne : 0;
             if (seg_dense(d)) {
-                bk.kind = 1;
+                bk.kind = 1 | one;
                 kh = seg_k(d) + static_cast<int64_t>(t0) * kHeadDim;
                 vh = seg_k(d) + static_cast<int64_t>(ntok + t0) * kHeadDim;
             } else {
-                bk.kind = 2;
+                bk.kind = 2 | (c <= 32 ? one : 0);
                 const bool tok = ((d >> 32) & 255u) == KV2D_BOTH;
                 const uint8_t* p0 = ubase + static_cast<int64_t>(d & 0xffffffffull) * 16 + (tok ? pad16(r) : 0);
                 bk.ci = p0 + static_cast<int64_t>(t0) * c;
@@ -435,7 +586,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
                      static_cast<int64_t>(t0) * kHeadDim;
             }
         } else {
-            const int tb = g_idx - g_base;
+            const int tb = g_idx - w_base;
             if (tb < ntb) {
                 bk.kind = 1;
                 tail = true;
@@ -454,20 +605,25 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
             const uint32_t K0 = kreg(stage), V0 = K0 + kDecKBytes, bar = bar0 + stage * 8;
             if (!tail) {
                 if (lane == 0) {
-                    uint32_t bytes = n * 256 * (bk.kind == 1 ? 2 : 1);
+                    const int kd = bk.kind & 3;
                     int npb = 0, nkb = 0;
-                    if (bk.kind == 2 && c <= 32) {
+                    if (kd == 2 && c <= 32) {
                         npb = pad16(n * c);
                         nkb = pad16(2 * n * c);
-                        bytes += npb + nkb;
                     }
-                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    const uint32_t bytes = n * 256 * (kd == 1 ? 2 : 1) + npb + nkb;
                     mbar_expect_tx(&sbar[warp][stage], bytes);
-                    if (bk.kind == 1) bulk_g2s(K0, kh, n * 256, bar);
-                    bulk_g2s(V0, vh, n * 256, bar);
-                    if (npb) {
-                        bulk_g2s(K0, bk.ci, npb, bar);
-                        bulk_g2s(K0 + 512, bk.kv, nkb, bar);
+                    if (bk.kind == (1 | kBlkOne)) {
+                        bulk_g2s(K0, kh, bytes, bar);
+                    } else if (bk.kind == (2 | kBlkOne)) {
+                        bulk_g2s(V0 - npb - nkb, bk.ci, bytes, bar);
+                    } else {
+                        if (kd == 1) bulk_g2s(K0, kh, n * 256, bar);
+                        bulk_g2s(V0, vh, n * 256, bar);
+                        if (npb) {
+                            bulk_g2s(K0, bk.ci, npb, bar);
+                            bulk_g2s(K0 + 512, bk.kv, nkb, bar);
+                        }
                     }
                 }
             } else {
@@ -476,10 +632,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
                 const __half* row = (R < n) ? dense_row(A.dv, krow_lane ? A.dv.k : A.dv.v, b, h, t0 + R, A.status)
                                             : nullptr;
                 const uint32_t nrows = __popc(__ballot_sync(0xffffffffu, row != nullptr));
-                if (lane == 0) {
-                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                    mbar_expect_tx(&sbar[warp][stage], nrows * 256);
-                }
+                if (lane == 0) mbar_expect_tx(&sbar[warp][stage], nrows * 256);
                 __syncwarp();
                 if (row) bulk_g2s(krow_lane ? K0 + R * kDecKStride : V0 + R * kDecVStride, row, 256, bar);
             }
@@ -488,16 +641,22 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
     };
 
     auto compute = [&](const DecBlock& bk, int stage) {
-        const uint32_t K0 = kreg(stage), V0 = K0 + kDecKBytes;
-        if (bk.kind == 2) {
-            // the 16 x 128 key tile: zero it, then scatter the block's n * c
+        const int kd = bk.kind & 3;
+        const bool one = bk.kind & kBlkOne;
+        const uint32_t K0 = kreg(stage);
+        const uint32_t V0 = K0 + ((one && kd == 1) ? bk.nlo * 256 : kDecKBytes);
+        if (kd == 2) {
+            // the 8 x 128 key tile: zero it, then scatter the block's n * c
             // pairs into it; 16 pairs per lane and round
-            const int np = (bk.nlo + bk.nhi) * c;
+            const int np = bk.nlo * c;
             uint4 iw = make_uint4(0, 0, 0, 0), va = iw, vb = iw;
             if (c <= 32 && lane * 16 < np) {
-                iw = lds16(K0 + lane * 16);
-                va = lds16(K0 + 512 + lane * 32);
-                vb = lds16(K0 + 512 + lane * 32 + 16);
+                const uint32_t nkb = one ? pad16(2 * np) : 0;
+                const uint32_t P0 = one ? V0 - nkb - pad16(np) : K0;
+                const uint32_t Q0 = one ? V0 - nkb : K0 + 512;
+                iw = lds16(P0 + lane * 16);
+                va = lds16(Q0 + lane * 32);
+                vb = lds16(Q0 + lane * 32 + 16);
             }
             __syncwarp();
 #pragma unroll
@@ -549,7 +708,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
                 vw[k + 2][i] = z4;
             }
         mma_block(st, qa, kw, vw, bk.nlo, 0, c2);
-        __syncwarp();    // the stage is refilled next: every lane is done with it
+        // the stage is refilled next by the copy engine: after a scatter
+        // (plain stores into the key rows) every writer orders its stores
+        // before those copies; plain reads need no fence
+        if (kd == 2) fence_proxy_async();
+        __syncwarp();
     };
 
     {
@@ -561,11 +724,17 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
         DecBlock f[kAhead];
 #pragma unroll
         for (int j = 0; j < kAhead; ++j) f[j] = DecBlock{0, 0, 0, nullptr, nullptr};
-        for (int k = -kAhead;; ++k) {
+        for (int k = kbase - kAhead; !dead; ++k) {
             const DecBlock nb = next_block((k + kAhead) % kDecStages);
-            if (k >= 0) {
-                if (f[0].kind == 0) break;
-                if (!mbar_wait(&sbar[warp][k % kDecStages], (k / kDecStages) & 1, A.status)) break;
+            if (k >= kbase) {
+                if (f[0].kind == 0) {
+                    kbase = k;   // every block after it is empty too: no copy in flight
+                    break;
+                }
+                if (!mbar_wait(&sbar[warp][k % kDecStages], (k / kDecStages) & 1, A.status)) {
+                    dead = true;
+                    break;
+                }
                 compute(f[0], k % kDecStages);
             }
 #pragma unroll
@@ -592,9 +761,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
     }
     __syncthreads();
 
-    // ---- CTA partial: part[u][sp][g] = {M, L, 0, 0, O[d]} (16-byte aligned O)
+    // ---- CTA partial: part[cta + u][g] = {M, L, 0, 0, O[d]} (16-byte
+    // aligned O).  cta + u is unique: both grow along the batch-wide range,
+    // so the pieces of unit u sit at first + u .. last + u, in order.
     constexpr int kRec = kHeadDim + 4;
-    float* myp = A.part + (static_cast<int64_t>(u) * A.nsplit + sp) * G * kRec;
+    float* myp = A.part + (static_cast<int64_t>(cta) + u) * G * kRec;
     for (int i = tid; i < G * kHeadDim; i += kDecThreads) {
         const int gg = i / kHeadDim, x = i % kHeadDim;
         float M = kNegInfF;
@@ -618,26 +789,27 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
     }
     __threadfence();
     __syncthreads();
-    if (tid == 0) is_last = (atomicAdd(&A.ticket[u], 1u) == static_cast<uint32_t>(A.nsplit - 1));
+    const int npieces = last - first + 1;
+    if (tid == 0) is_last = (atomicAdd(&A.ticket[u], 1u) == static_cast<uint32_t>(npieces - 1));
     __syncthreads();
-    if (!is_last) return;
+    if (is_last) {
     __threadfence();
 
-    // ---- last CTA of the unit: merge the splits in order.  A thread owns
-    // 4 channels of one head and loads (M, L, O) of up to kMergeChunk splits
+    // ---- last CTA of the unit: merge the pieces in order.  A thread owns
+    // 4 channels of one head and loads (M, L, O) of up to kMergeChunk pieces
     // at once; chunks merge online.
     if (tid < G * (kHeadDim / 4)) {
         constexpr int kMergeChunk = 20;
         const int gg = tid / (kHeadDim / 4), x4 = (tid % (kHeadDim / 4)) * 4;
-        const float* up = A.part + static_cast<int64_t>(u) * A.nsplit * G * kRec + gg * kRec;
+        const float* up = A.part + (static_cast<int64_t>(first) + u) * G * kRec + gg * kRec;
         float Mrun = kNegInfF, Lrun = 0.f;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int s0 = 0; s0 < A.nsplit; s0 += kMergeChunk) {
+        for (int s0 = 0; s0 < npieces; s0 += kMergeChunk) {
             float2 ml[kMergeChunk];
             float4 ov[kMergeChunk];
 #pragma unroll
             for (int k = 0; k < kMergeChunk; ++k) {
-                if (s0 + k < A.nsplit) {
+                if (s0 + k < npieces) {
                     const float* rec = up + static_cast<int64_t>(s0 + k) * G * kRec;
                     ml[k] = __ldcg(reinterpret_cast<const float2*>(rec));
                     ov[k] = __ldcg(reinterpret_cast<const float4*>(rec + 4 + x4));
@@ -677,16 +849,33 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
         *reinterpret_cast<uint2*>(A.out + (static_cast<int64_t>(b) * A.Hq + h * G + gg) * kHeadDim + x4) = pk;
     }
     if (tid == 0) A.ticket[u] = 0;
+    }   // is_last
+
+    // ---- the next piece's copies land where the warp partials were: put
+    // finite numbers back
+    __syncthreads();
+    for (int i = tid; i < static_cast<int>(sizeof(float) * kDecWarps * G * kHeadDim / 16); i += kDecThreads)
+        reinterpret_cast<uint4*>(dec_smem)[i] = make_uint4(0, 0, 0, 0);
+    fence_proxy_async();
+    __syncthreads();
+    }   // pieces
 }
 
 }  // namespace
 
-int decode_split_count(int units, int64_t max_seq_len, int num_sms) {
-    // one 8-warp CTA per SM, one wave
-    int ns = num_sms / units;
-    const int by_len = static_cast<int>((max_seq_len + 255) / 256);
-    ns = min(ns, max(1, by_len));
-    return max(1, min(ns, 64));
+int decode_cta_count(int units, int64_t max_seq_len, int num_sms, int* kps) {
+    // one CTA per SM, one wave; a unit of L tokens is cut into at most
+    // min(64, L / 256) pieces.  With at least two SMs per unit every unit
+    // gets the same number of CTAs; otherwise the batch's bytes are shared
+    // out evenly.
+    const int sms = std::min(num_sms, kMaxDecCtas);
+    const int64_t by_len = std::max<int64_t>(1, std::min<int64_t>(64, (max_seq_len + 255) / 256));
+    if (2 * static_cast<int64_t>(units) <= sms) {
+        *kps = static_cast<int>(std::min<int64_t>(sms / units, by_len));
+        return units * *kps;
+    }
+    *kps = 0;
+    return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(sms, units * by_len)));
 }
 
 cudaError_t launch_append(const AppendLaunch& L, cudaStream_t stream) {
@@ -716,13 +905,13 @@ cudaError_t launch_decode(const DecodeLaunch& L, cudaStream_t stream) {
     a.seq_len = L.seq_len;
     a.q = L.q;
     a.out = L.out;
-    a.nsplit = L.nsplit;
+    a.units = L.batch * L.shp.Hkv;
+    a.kps = L.kps;
     a.part = L.part;
     a.ticket = L.ticket;
     a.status = L.status;
-    const int units = L.batch * L.shp.Hkv;
     cudaError_t e = cudaSuccess;
-    dim3 grid(L.nsplit, units);
+    dim3 grid(L.nctas);
     auto launch_dec = [&](auto kern) {
         cudaError_t r = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmem);
         if (r != cudaSuccess) return r;

@@ -168,12 +168,14 @@ struct DecodeLaunch {
     const int32_t* seq_len;
     const __half* q;
     __half* out;
-    int nsplit;
-    float* part;               // [units][nsplit][G][4 + d]: M, L, 0, 0, O[d]
+    int nctas;                 // grid size, at most kMaxDecCtas
+    int kps;                   // CTAs per unit, or 0: batch-wide byte shares
+    float* part;               // [nctas + units][G][4 + d]: M, L, 0, 0, O[d]
     uint32_t* ticket;          // [units]
     uint32_t* status;
 };
+constexpr int kMaxDecCtas = 512;
 cudaError_t launch_decode(const DecodeLaunch& L, cudaStream_t stream);
-int decode_split_count(int units, int64_t max_seq_len, int num_sms);
+int decode_cta_count(int units, int64_t max_seq_len, int num_sms, int* kps);
 
 }  // namespace kv2d
