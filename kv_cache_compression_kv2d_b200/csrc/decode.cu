@@ -197,17 +197,25 @@ __device__ __forceinline__ void mma_block(MmaState& st, const uint32_t (&qa)[8][
                                           const uint4 (&vw)[4][2], int nlo, int nhi, float c2) {
     const int lane = threadIdx.x & 31;
     const int t = lane & 3;
+    // two accumulation chains per tile (even and odd k-steps) halve the
+    // dependent MMA latency
     float sacc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
         if (nt == 1 && nhi == 0) break;
+        float odd0 = 0.f, odd1 = 0.f;
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
             const uint4& w = kw[nt][ks >> 1];
             const uint32_t b0 = (ks & 1) ? w.z : w.x;
             const uint32_t b1 = (ks & 1) ? w.w : w.y;
-            mma16816(sacc[nt][0], sacc[nt][1], qa[ks][0], qa[ks][1], b0, b1);
+            if (ks & 1)
+                mma16816(odd0, odd1, qa[ks][0], qa[ks][1], b0, b1);
+            else
+                mma16816(sacc[nt][0], sacc[nt][1], qa[ks][0], qa[ks][1], b0, b1);
         }
+        sacc[nt][0] += odd0;
+        sacc[nt][1] += odd1;
     }
     // scores of tokens nt*8 + 2t + e, online softmax over the head row
     float x[4];
@@ -275,9 +283,9 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
 // them; sparse: index bytes and key values end where the value rows start).
 constexpr int kBlkOne = 4;
 struct DecBlock {
-    int kind, nlo, nhi;
+    int kind, nlo;
     const uint8_t* ci;      // sparse: the block's index bytes
-    const __half* kv;       // sparse: the block's key values
+    int dkv;                // sparse: its key values start at ci + dkv
 };
 
 constexpr int kDescPerThread = kDescCache / kDecThreads;   // descriptors each thread loads in the prologue
@@ -373,6 +381,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
 
     const float c2 = A.c2;
     const int S = A.S, r = A.r, c = A.c;
+    const bool c8 = c <= 32 && (c & 7) == 0;       // the sparse fast path
+    const int row8 = c8 ? (lane * 8) / c : 0;      // its key row for this lane
     const uint32_t wbase = smem_u32(dec_smem) + warp * (kDecStages * kDecSlotBytes);
     // stage s of this warp: key rows at kreg(s), value rows at kreg(s) +
     // kDecKBytes (see DecBlock for the one-copy layouts)
@@ -546,11 +556,12 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
     if (w_j0 < j_hi) load_window();
     int g_next = warp;
     auto next_block = [&](int stage) -> DecBlock {
-        DecBlock bk{0, 0, 0, nullptr, nullptr};
+        DecBlock bk{0, 0, nullptr, 0};
         const int g_idx = g_next;
         g_next += kDecWarps;
         const __half* kh = nullptr;   // first K row of the block
         const __half* vh = nullptr;   // first V row of the block
+        const __half* kv = nullptr;   // sparse: first key value of the block
         int n = 0;
         bool tail = false;
         uint64_t d = 0;
@@ -579,8 +590,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
                 const bool tok = ((d >> 32) & 255u) == KV2D_BOTH;
                 const uint8_t* p0 = ubase + static_cast<int64_t>(d & 0xffffffffull) * 16 + (tok ? pad16(r) : 0);
                 bk.ci = p0 + static_cast<int64_t>(t0) * c;
-                bk.kv = reinterpret_cast<const __half*>(p0 + pad16(static_cast<int64_t>(ntok) * c)) +
-                        static_cast<int64_t>(t0) * c;
+                kv = reinterpret_cast<const __half*>(p0 + pad16(static_cast<int64_t>(ntok) * c)) +
+                     static_cast<int64_t>(t0) * c;
+                bk.dkv = static_cast<int>(reinterpret_cast<const uint8_t*>(kv) - bk.ci);
                 vh = reinterpret_cast<const __half*>(p0 + pad16(static_cast<int64_t>(ntok) * c) +
                                                      pad16(static_cast<int64_t>(ntok) * c * 2)) +
                      static_cast<int64_t>(t0) * kHeadDim;
@@ -595,7 +607,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
             }
         }
         bk.nlo = n;
-        bk.nhi = 0;
         // Copies by the TMA unit.  Segment blocks: lane 0 copies the block's
         // key rows and value rows in one piece each (or a sparse block's two
         // pair sections and its value rows); the dense tail, whose rows need
@@ -622,7 +633,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
                         bulk_g2s(V0, vh, n * 256, bar);
                         if (npb) {
                             bulk_g2s(K0, bk.ci, npb, bar);
-                            bulk_g2s(K0 + 512, bk.kv, nkb, bar);
+                            bulk_g2s(K0 + 512, kv, nkb, bar);
                         }
                     }
                 }
@@ -645,7 +656,41 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
         const bool one = bk.kind & kBlkOne;
         const uint32_t K0 = kreg(stage);
         const uint32_t V0 = K0 + ((one && kd == 1) ? bk.nlo * 256 : kDecKBytes);
-        if (kd == 2) {
+        if (kd == 2 && c8) {
+            // c <= 32, a multiple of 8: lane l takes pairs 8l .. 8l + 7, all
+            // in key row 8l / c; zero the 8 x 128 key tile, then scatter
+            const int np = bk.nlo * c;
+            const bool act = lane * 8 < np;
+            uint2 iw = make_uint2(0, 0);
+            uint4 va = make_uint4(0, 0, 0, 0);
+            if (act) {
+                const uint32_t nkb = one ? pad16(2 * np) : 0;
+                const uint32_t P0 = one ? V0 - nkb - pad16(np) : K0;
+                const uint32_t Q0 = one ? V0 - nkb : K0 + 512;
+                asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(iw.x), "=r"(iw.y) : "r"(P0 + lane * 8));
+                va = lds16(Q0 + lane * 16);
+            }
+            __syncwarp();
+#pragma unroll
+            for (int i = 0; i < kDecRows / 2; ++i)
+                asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(K0 + (2 * i + (lane >> 4)) * kDecKStride +
+                                                                             (lane & 15) * 16),
+                             "r"(0u)
+                             : "memory");
+            __syncwarp();
+            if (act) {
+                const uint32_t row = K0 + row8 * kDecKStride;
+                const uint32_t vws[4] = {va.x, va.y, va.z, va.w};
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    // indices are < 128; the mask keeps a corrupt byte inside the tile
+                    const int ch = (((k < 4) ? iw.x : iw.y) >> (8 * (k & 3))) & 0x7f;
+                    const uint16_t hv = static_cast<uint16_t>(vws[k >> 1] >> (16 * (k & 1)));
+                    asm volatile("st.shared.u16 [%0], %1;" ::"r"(row + ch * 2), "h"(hv) : "memory");
+                }
+            }
+            __syncwarp();
+        } else if (kd == 2) {
             // the 8 x 128 key tile: zero it, then scatter the block's n * c
             // pairs into it; 16 pairs per lane and round
             const int np = bk.nlo * c;
@@ -669,8 +714,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
             for (int e0 = lane * 16; e0 < np; e0 += 32 * 16) {
                 if (c > 32) {
                     iw = ld_nc16(bk.ci + e0);
-                    va = ld_nc16(bk.kv + e0);
-                    vb = ld_nc16(bk.kv + e0 + 8);
+                    const __half* kv = reinterpret_cast<const __half*>(bk.ci + bk.dkv);
+                    va = ld_nc16(kv + e0);
+                    vb = ld_nc16(kv + e0 + 8);
                 }
                 const uint32_t iws[4] = {iw.x, iw.y, iw.z, iw.w};
                 const uint32_t vws[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
@@ -723,7 +769,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
         constexpr int kAhead = kDecStages - 1;
         DecBlock f[kAhead];
 #pragma unroll
-        for (int j = 0; j < kAhead; ++j) f[j] = DecBlock{0, 0, 0, nullptr, nullptr};
+        for (int j = 0; j < kAhead; ++j) f[j] = DecBlock{0, 0, nullptr, 0};
         for (int k = kbase - kAhead; !dead; ++k) {
             const DecBlock nb = next_block((k + kAhead) % kDecStages);
             if (k >= kbase) {
