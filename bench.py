@@ -98,6 +98,8 @@ def parse_args():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-decode-large", action="store_true",
+                    help="skip the decode-only measurement on the batch-16 x 128K cache")
     return ap.parse_args()
 
 
@@ -259,6 +261,51 @@ def cpu_baseline(wl, batch_host, p_gpu, budget_s=30.0):
 
 
 # ------------------------------------------------------------------- kv2d
+
+
+def decode_batch16_128k(B, synth, torch, dev, stream, hbm, steps):
+    """Decode alone over the batch-16 x 128K cache (8 KV heads, four-class
+    segment mix, budget 15 %): 1.29 GB of packed bytes, larger than L2, a size
+    at which decode is bound by HBM rather than by its fixed phases."""
+    wl = synth.WORKLOADS["llama3_8b_b16_128k_mix"]
+    bt = synth.generate(wl, seed=0, device=dev, extra_capacity=16)
+    lens = [int(x) for x in bt.seq_len]
+    scale = float(torch.tensor(1.0 / wl.head_dim ** 0.5, dtype=torch.float32))
+    p = B.params(wl.head_dim, wl.num_q_heads, wl.num_kv_heads, wl.segment_len, wl.window, wl.r,
+                 wl.c, wl.budget, scale)
+    dv = B.dense(bt.k, bt.v)
+    cc = B.CompressedCache(p, wl.batch, bt.capacity, device=dev)
+    ws_c = B.workspace(B.kv2d_workspace_bytes(p, B.OP_COMPRESS, wl.batch, max(lens)), dev)
+    ws_d = B.workspace(B.kv2d_workspace_bytes(p, B.OP_DECODE, wl.batch, bt.capacity), dev)
+    B.kv2d_compress(p, wl.batch, lens, [0] * wl.batch, dv, bt.qw, cc.struct, ws_c, stream=stream)
+    seq = torch.tensor(lens, dtype=torch.int32, device=dev)
+    out = torch.empty((wl.batch, wl.num_q_heads, wl.head_dim), dtype=torch.float16, device=dev)
+
+    def decode():
+        B.kv2d_decode_attn(p, wl.batch, cc.struct, dv, seq, bt.capacity, bt.q, out, ws_d, stream=stream)
+
+    for _ in range(3):
+        decode()
+    evs = []
+    for _ in range(steps):
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        decode()
+        b_.record(stream)
+        evs.append((a, b_))
+    torch.cuda.synchronize(dev)
+    assert B.kv2d_read_status(ws_c, stream) == 0 and B.kv2d_read_status(ws_d, stream) == 0
+    us = 1e3 * statistics.mean(a.elapsed_time(b_) for a, b_ in evs)
+    ce = cc.comp_end.cpu().tolist()
+    tail = sum((lens[b] - ce[b]) * wl.num_kv_heads for b in range(wl.batch))
+    nbytes = (int(cc.used_bytes.sum()) + 8 * int(cc.n_segs.sum()) + tail * wl.head_dim * 4 +
+              2 * wl.batch * wl.num_q_heads * wl.head_dim * 2)
+    del bt, dv, cc, ws_c, ws_d, out
+    torch.cuda.empty_cache()
+    gbs = nbytes / (us * 1e-6) / 1e9
+    return {"workload": wl.name, "us_per_call": us, "bytes_per_call": nbytes, "hbm_gbs": gbs,
+            "hbm_frac": gbs / hbm, "calls": steps,
+            "l2": "no flush: 1.29 GB of packed bytes per call > L2"}
 
 
 def main():
@@ -486,6 +533,10 @@ def main():
         e2e = {"value": job_throughput(nbytes, world, e_ms), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms}
 
+    dec_large = None
+    if world == 1 and not args.no_decode_large:
+        dec_large = decode_batch16_128k(B, synth, torch, dev, stream, hbm, max(args.steps, 5))
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(wl, host, p)
@@ -510,6 +561,7 @@ def main():
                    "hbm_gbs": dec_bytes / (dec_us * 1e-6) / 1e9,
                    "hbm_frac": dec_bytes / (dec_us * 1e-6) / 1e9 / hbm},
         "compress": {"us": comp_us, "gbs": nbytes / (comp_us * 1e-6) / 1e9},
+        "decode_batch16_128k": dec_large,
         "kernels": kernels,
         "kernels_note": "per-launch CUDA-event times from a profiled repeat of the K timed steps",
         "roofline": roof,

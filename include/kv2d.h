@@ -288,6 +288,14 @@ KV2D_API kv2d_status kv2d_profile_enable(int on);
 KV2D_API int kv2d_profile_read(double* ms, int64_t* launches, int max_stages);
 KV2D_API const char* kv2d_profile_stage_name(int stage);
 
+/* Testing aid: caps the number of blocks (8-token slices of segments) the
+ * decode kernel tables per chunk of a CTA's share (cap in [32, 4096]; 0
+ * restores the default 4096), so that small inputs reach the path that
+ * handles shares larger than one chunk.  Affects later decode calls of the
+ * process; results do not depend on it.  KV2D_ERR_INVALID_ARG outside the
+ * range. */
+KV2D_API kv2d_status kv2d_set_decode_table_cap(int cap);
+
 /* Human-readable reason of the calling thread's last non-OK status. */
 KV2D_API const char* kv2d_last_error(void);
 

@@ -54,7 +54,7 @@ class kv2d_debug(C.Structure):
 
 EXPORTS = ["kv2d_segment_bytes", "kv2d_arena_bytes", "kv2d_workspace_bytes", "kv2d_compress",
            "kv2d_append", "kv2d_decode_attn", "kv2d_read_status", "kv2d_last_error",
-           "kv2d_version", "kv2d_profile_enable", "kv2d_profile_read",
+           "kv2d_version", "kv2d_profile_enable", "kv2d_profile_read", "kv2d_set_decode_table_cap",
            "kv2d_profile_stage_name", "kv2d_decode_attn_noalloc"]
 
 _lib = None
@@ -95,6 +95,8 @@ def lib():
         L.kv2d_last_error.restype = C.c_char_p
         L.kv2d_version.argtypes = []
         L.kv2d_version.restype = C.c_char_p
+        L.kv2d_set_decode_table_cap.argtypes = [C.c_int]
+        L.kv2d_set_decode_table_cap.restype = C.c_int
         L.kv2d_profile_enable.argtypes = [C.c_int]
         L.kv2d_profile_enable.restype = C.c_int
         L.kv2d_profile_read.argtypes = [P(C.c_double), P(C.c_int64), C.c_int]
@@ -200,6 +202,12 @@ def kv2d_decode_attn(p, batch, cc, dense_view, seq_len_dev, max_seq_len_host, q,
                                 _ptr(ws), ws.numel() if hasattr(ws, "numel") else 0,
                                 _stream(stream))
     return _check(rc) if check else rc
+
+
+def kv2d_set_decode_table_cap(cap: int) -> None:
+    """Testing aid: blocks per chunk of the decode kernel's block table
+    (0 restores the default)."""
+    _check(lib().kv2d_set_decode_table_cap(int(cap)))
 
 
 def kv2d_profile_enable(on: bool) -> int:

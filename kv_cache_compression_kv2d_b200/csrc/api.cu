@@ -7,6 +7,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -168,6 +169,9 @@ DecodeLayout decode_layout(const kv2d_params* p, int batch) {
     L.total = c.off;
     return L;
 }
+
+// blocks per chunk of the decode kernel's block table (kv2d_set_decode_table_cap)
+std::atomic<int> g_dec_table_cap{kDecTableMax};
 
 int num_sms() {
     int dev = 0, n = 148;
@@ -647,6 +651,7 @@ kv2d_status kv2d_decode_attn(const kv2d_params* p, int batch, const kv2d_ccache*
     L.q = static_cast<const __half*>(q);
     L.out = static_cast<__half*>(out);
     L.nctas = decode_cta_count(batch * sh.Hkv, max_seq_len_host, num_sms(), &L.kps);
+    L.tbl_cap = g_dec_table_cap.load();
     L.part = reinterpret_cast<float*>(w + WL.part);
     L.ticket = reinterpret_cast<uint32_t*>(w + WL.ticket);
     L.status = reinterpret_cast<uint32_t*>(w);
@@ -709,6 +714,7 @@ kv2d_status kv2d_decode_attn_noalloc(const kv2d_params* p, int batch, const kv2d
     L.out = static_cast<__half*>(out);
     L.nctas = nctas;
     L.kps = kps;
+    L.tbl_cap = g_dec_table_cap.load();
     L.part = reinterpret_cast<float*>(w + part_off);
     L.ticket = reinterpret_cast<uint32_t*>(w + ticket_off);   // left at zero by every call
     L.status = status_dev ? status_dev : reinterpret_cast<uint32_t*>(w);
@@ -733,6 +739,13 @@ kv2d_status kv2d_read_status(void* ws, void* stream, uint32_t* bits) {
 const char* kv2d_last_error(void) { return g_err.c_str(); }
 
 const char* kv2d_version(void) { return "kv2d 0.1.0 (sm_100a)"; }
+
+kv2d_status kv2d_set_decode_table_cap(int cap) {
+    if (cap != 0 && (cap < 32 || cap > kDecTableMax))
+        return fail(KV2D_ERR_INVALID_ARG, "decode table cap %d not 0 or in [32, %d]", cap, kDecTableMax);
+    g_dec_table_cap.store(cap == 0 ? kDecTableMax : cap);
+    return ok();
+}
 
 kv2d_status kv2d_profile_enable(int on) {
     std::lock_guard<std::mutex> lk(g_prof_mu);

@@ -93,6 +93,7 @@ struct DecodeArgs {
     __half* out;
     int units;
     int kps;          // > 0: unit c / kps, piece c % kps of kps equal ones; 0: batch-wide shares
+    int tbl_cap;      // blocks per table chunk (<= kTbl; >= 32, the most blocks of a segment)
     float* part;
     uint32_t* ticket;
     uint32_t* status;
@@ -134,7 +135,8 @@ __device__ __forceinline__ UnitLens unit_lens(const DecodeArgs& A, int u, bool r
 __device__ __forceinline__ int64_t unit_span(const UnitLens& L) {
     return 1 + L.U + static_cast<int64_t>(L.T - L.ce) * kTailBytes;
 }
-constexpr int kDescCache = 2048;                   // descriptors staged per CTA (a 128K-token unit at S = 64)
+constexpr int kDescRegs = 2048;                    // descriptors the counting pass holds in registers
+constexpr int kTbl = kDecTableMax;                 // blocks in the block table (one chunk of a piece)
 
 // ------------------------------------------------------ tensor-core decode
 //
@@ -288,7 +290,7 @@ struct DecBlock {
     int dkv;                // sparse: its key values start at ci + dkv
 };
 
-constexpr int kDescPerThread = kDescCache / kDecThreads;   // descriptors each thread loads in the prologue
+constexpr int kDescPerThread = kDescRegs / kDecThreads;   // descriptors each thread loads in the prologue
 
 template <int G>
 __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_constant__ DecodeArgs A) {
@@ -302,10 +304,12 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
     __shared__ long long s_part[3];   // first unit, its start, last unit
     __shared__ __align__(8) uint64_t sbar[kDecWarps][kDecStages];
     __shared__ int is_last;
-    __shared__ uint64_t dsm[kDescCache];
+    // block table: entry i = descriptor of the segment holding block i of
+    // the chunk, with the block's first token (segment-relative) in bits 40..55
+    __shared__ uint64_t tbl[kTbl];
     // the warp partials reuse the stage buffers once every warp is done
     static_assert(sizeof(float) * kDecWarps * G * kHeadDim <= kDecSmem, "partials fit");
-    static_assert(kDescPerThread * kDecThreads <= kDescCache, "prologue descriptors fit the cache");
+
     float (*wo)[G][kHeadDim] = reinterpret_cast<float (*)[G][kHeadDim]>(dec_smem);
 
     pdl_wait();
@@ -493,15 +497,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
         j_lo += wcnt[w][0];
         j_hi += wcnt[w][1];
     }
-    const bool cached = (j_hi - j_lo) <= kDescCache;
-    if (cached) {
-#pragma unroll
-        for (int k = 0; k < kDescPerThread; ++k) {
-            const int j = tid + k * kDecThreads;
-            if (j >= j_lo && j < j_hi) dsm[j - j_lo] = dreg[k];
-        }
-        for (int j = max(j_lo, kDescPerThread * kDecThreads) + tid; j < j_hi; j += kDecThreads) dsm[j - j_lo] = D[j];
-    }
     auto tail_at_or_after = [&](int64_t x) -> int {
         if (x <= U) return 0;
         const int64_t i = (x - U + kTailBytes - 1) / kTailBytes;
@@ -509,8 +504,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
     };
     const int t_lo = ce + tail_at_or_after(lo), t_hi = ce + tail_at_or_after(hi);
     const int ntb = (t_hi - t_lo + kDecRows - 1) / kDecRows;
-
-    __syncthreads();
 
     MmaState st;
     st.m = kNegInfF;
@@ -521,7 +514,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
         st.o[j][1] = 0.f;
     }
     const uint8_t* ubase = A.arena + static_cast<int64_t>(u) * A.arena_stride;
-    auto desc = [&](int j) -> uint64_t { return cached ? dsm[j - j_lo] : D[j]; };
     // first K row of a dense segment (its V rows follow its ntok K rows)
     auto seg_k = [&](uint64_t d) {
         const int sty = static_cast<int>((d >> 32) & 255u);
@@ -530,30 +522,56 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
     };
 
     // ---- the CTA's items, in order: every segment in blocks of up to 8
-    // tokens, then the dense tail in blocks of 8.  Item i belongs to warp
-    // i % kDecWarps, so the order of every sum is fixed and the output is
-    // deterministic.  A warp finds the segment of an item in a window of 32
-    // consecutive segments it holds one per lane (descriptor and inclusive
-    // prefix of item counts): one ballot instead of a walk over the
-    // segments in between.
-    int w_j0 = j_lo;          // first segment of the window
-    uint64_t w_d = 0;         // lane l: descriptor of segment w_j0 + l
-    int w_pre = 0;            // lane l: items of segments w_j0 .. w_j0 + l
-    int w_base = 0;           // items of the segments before the window
-    int w_tot = 0;            // items of the window
-    auto load_window = [&]() {
-        const int j = w_j0 + lane;
-        w_d = (j < j_hi) ? desc(j) : 0ull;
-        int n = (j < j_hi) ? (seg_ntok(w_d) + kDecRows - 1) / kDecRows : 0;
+    // tokens, then the dense tail in blocks of 8.  Item i of a chunk belongs
+    // to warp i % kDecWarps, so the order of every sum is fixed and the
+    // output is deterministic.  The segments go through the block table in
+    // chunks of whole segments (one chunk unless a piece has more than kTbl
+    // blocks); a warp finds its block with one shared-memory load.
+    int seg_next = j_lo;   // first segment not tabled yet
+    for (bool last_chunk = false; !last_chunk;) {
+    int n_tab = 0;         // blocks in the table
+    {
+        __shared__ int s_cut[2];
+        if (tid == 0) s_cut[0] = -1;
+        for (int c0 = seg_next; c0 < j_hi; c0 += kDecThreads) {
+            const int j = c0 + tid;
+            const uint64_t d = (j < j_hi) ? D[j] : 0ull;
+            const int nit = (j < j_hi) ? (seg_ntok(d) + kDecRows - 1) / kDecRows : 0;
+            int x = nit;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, n, o);
-            if (lane >= o) n += y;
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, x, o);
+                if (lane >= o) x += y;
+            }
+            __syncthreads();   // wcnt is free
+            if (lane == 31) wcnt[warp][0] = x;
+            __syncthreads();
+            int pos = n_tab + x - nit, tot = 0;
+#pragma unroll
+            for (int w2 = 0; w2 < kDecWarps; ++w2) {
+                if (w2 < warp) pos += wcnt[w2][0];
+                tot += wcnt[w2][0];
+            }
+            if (j < j_hi) {
+                if (pos + nit <= A.tbl_cap) {
+                    for (int q = 0; q < nit; ++q) tbl[pos + q] = d | (static_cast<uint64_t>(q * kDecRows) << 40);
+                } else if (pos <= A.tbl_cap) {   // the first segment that does not fit
+                    s_cut[0] = pos;
+                    s_cut[1] = j;
+                }
+            }
+            __syncthreads();
+            if (s_cut[0] >= 0) {
+                n_tab = s_cut[0];
+                seg_next = s_cut[1];
+                break;
+            }
+            n_tab += tot;
+            seg_next = min(c0 + kDecThreads, j_hi);
         }
-        w_pre = n;
-        w_tot = __shfl_sync(0xffffffffu, n, 31);
-    };
-    if (w_j0 < j_hi) load_window();
+        last_chunk = seg_next >= j_hi;
+        __syncthreads();   // the table is complete
+    }
     int g_next = warp;
     auto next_block = [&](int stage) -> DecBlock {
         DecBlock bk{0, 0, nullptr, 0};
@@ -566,19 +584,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
         bool tail = false;
         uint64_t d = 0;
         int t0 = 0;
-        while (w_j0 < j_hi && g_idx >= w_base + w_tot) {
-            w_base += w_tot;
-            w_tot = 0;
-            w_j0 += 32;
-            if (w_j0 < j_hi) load_window();
-        }
-        if (w_j0 < j_hi) {
-            const int rel = g_idx - w_base;
-            const int L = __ffs(__ballot_sync(0xffffffffu, w_pre > rel)) - 1;
-            d = __shfl_sync(0xffffffffu, w_d, L);
-            const int pre = __shfl_sync(0xffffffffu, w_pre, L);
+        if (g_idx < n_tab) {
+            d = tbl[g_idx];
+            t0 = static_cast<int>((d >> 40) & 0xffffu);
+            d &= 0xffffffffffull;
             const int ntok = seg_ntok(d);
-            t0 = (rel - (pre - (ntok + kDecRows - 1) / kDecRows)) * kDecRows;
             n = min(kDecRows, ntok - t0);
             const int one = (ntok <= kDecRows) ? kBlkOne : 0;
             if (seg_dense(d)) {
@@ -597,8 +607,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
                                                      pad16(static_cast<int64_t>(ntok) * c * 2)) +
                      static_cast<int64_t>(t0) * kHeadDim;
             }
-        } else {
-            const int tb = g_idx - w_base;
+        } else if (last_chunk) {
+            const int tb = g_idx - n_tab;
             if (tb < ntb) {
                 bk.kind = 1;
                 tail = true;
@@ -788,6 +798,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
             f[kAhead - 1] = nb;
         }
     }
+    if (!last_chunk) __syncthreads();   // every warp is done with the table
+    }   // chunks
 
     // ---- warp partials -> shared memory (lanes with g < G hold real rows)
     __syncthreads();   // every warp is done with its stage buffers
@@ -953,6 +965,7 @@ cudaError_t launch_decode(const DecodeLaunch& L, cudaStream_t stream) {
     a.out = L.out;
     a.units = L.batch * L.shp.Hkv;
     a.kps = L.kps;
+    a.tbl_cap = min(max(L.tbl_cap, 32), kTbl);
     a.part = L.part;
     a.ticket = L.ticket;
     a.status = L.status;

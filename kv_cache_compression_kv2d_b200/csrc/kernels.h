@@ -170,11 +170,13 @@ struct DecodeLaunch {
     __half* out;
     int nctas;                 // grid size, at most kMaxDecCtas
     int kps;                   // CTAs per unit, or 0: batch-wide byte shares
+    int tbl_cap;               // blocks per block-table chunk, in [32, kDecTableMax]
     float* part;               // [nctas + units][G][4 + d]: M, L, 0, 0, O[d]
     uint32_t* ticket;          // [units]
     uint32_t* status;
 };
 constexpr int kMaxDecCtas = 512;
+constexpr int kDecTableMax = 4096;
 cudaError_t launch_decode(const DecodeLaunch& L, cudaStream_t stream);
 int decode_cta_count(int units, int64_t max_seq_len, int num_sms, int* kps);
 

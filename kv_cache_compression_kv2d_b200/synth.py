@@ -76,6 +76,10 @@ WORKLOADS = {
     # same layer, batch 16 x 128K, budget 15%, all four strategies, 256 steps.
     "llama3_8b_b16_128k_mix": Workload("llama3_8b_b16_128k_mix", 16, 8, 4, 128, 131072, 64, 64,
                                        0.15, segment_mix=True, decode_steps=256),
+    # the same batch at 16K tokens per sequence (1.1 GB dense K/V, 160 MB
+    # packed): a size that a full hardware-counter capture of decode can hold
+    "llama3_8b_b16_16k_mix": Workload("llama3_8b_b16_16k_mix", 16, 8, 4, 128, 16384, 64, 64,
+                                      0.15, segment_mix=True),
     # same layer, batch 1, 1M tokens, S=W=128, budget 10%, 0.1% planted.
     "llama3_8b_1m": Workload("llama3_8b_1m", 1, 8, 4, 128, 1 << 20, 128, 128, 0.10,
                              planted_frac=0.001, planted_layout="stratified"),

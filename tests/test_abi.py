@@ -168,3 +168,12 @@ def test_cache_bookkeeping_views_and_reset(L):
     cc.reset()
     assert int(cc.used_bytes.abs().sum()) == 0
     assert int(cc.n_segs.abs().sum()) == 0 and int(cc.comp_end.abs().sum()) == 0
+
+
+def test_decode_table_cap_range(L):
+    # host-only setter: 0 (default) or [32, 4096]
+    for bad in (31, 4097, -1):
+        with pytest.raises(B.Kv2dError):
+            B.kv2d_set_decode_table_cap(bad)
+    for good in (32, 4096, 0):
+        B.kv2d_set_decode_table_cap(good)

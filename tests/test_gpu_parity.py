@@ -247,3 +247,20 @@ def test_channel_ties_parity(orc, keep_channels):
     H.compress(run)
     _check_all_units(orc, run, independent=False)
     _check_decode(orc, run)
+
+
+@pytest.mark.parametrize("cap", [32, 41])
+def test_decode_block_table_in_chunks(orc, cap):
+    """With more units than half the SMs the batch's bytes are shared out
+    over the CTAs, and each CTA tables its blocks in chunks of whole
+    segments; a cap of 32 or 41 blocks per chunk makes every share take
+    several chunks (a 64-token segment is 8 blocks, so 41 leaves a remainder),
+    with the dense tail after the last chunk."""
+    wl = Workload("chunks", 40, 2, 4, 128, 1601, 64, 64, 0.15, ragged_min=900, segment_mix=True)
+    run = _run(wl, seed=5)
+    H.compress(run)
+    B.kv2d_set_decode_table_cap(cap)
+    try:
+        _check_decode(orc, run)
+    finally:
+        B.kv2d_set_decode_table_cap(0)
