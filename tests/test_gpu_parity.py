@@ -264,3 +264,31 @@ def test_decode_block_table_in_chunks(orc, cap):
         _check_decode(orc, run)
     finally:
         B.kv2d_set_decode_table_cap(0)
+
+
+def test_decode_in_cuda_graph(orc):
+    """kv2d_decode_attn is capturable in a CUDA graph (no host sync, fixed
+    grid from the host maxima, tickets back at zero after every call): three
+    captured calls replayed give the direct call's output bit for bit."""
+    wl = CASES["ragged_multi"]
+    run = _run(wl, seed=2)
+    H.compress(run)
+    q = run.batch.q
+    ref = H.gpu_decode(run, q)
+    p = run.p
+    ws = B.workspace(B.kv2d_workspace_bytes(p, B.OP_DECODE, wl.batch, run.batch.capacity))
+    out = torch.full_like(ref, float("nan"))
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=s):
+        for _ in range(3):
+            B.kv2d_decode_attn(p, wl.batch, run.cc.struct, run.dv, run.seq_len, run.batch.capacity,
+                               q, out, ws, stream=s)
+    torch.cuda.current_stream().wait_stream(s)
+    for _ in range(2):
+        out.fill_(float("nan"))
+        graph.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out, ref)
+    assert B.kv2d_read_status(ws) == 0
