@@ -140,16 +140,18 @@ constexpr int kTbl = kDecTableMax;                 // blocks in the block table 
 
 // ------------------------------------------------------ tensor-core decode
 //
-// Per warp, blocks of 16 tokens go through two m16n8k16 products (fp16 in,
-// fp32 accumulate):
-//   S[16 x 16] = Q[16 x 128] K^T   (rows = the G query heads, zero-padded)
-//   O[16 x 128] += P[16 x 16] V    (P = softmax numerators in fp16)
-// Lane (g = lane / 4, t = lane % 4).  The q.k contraction runs over d in a
-// fixed permuted order: mma k-index 2t+e of step ks <-> d = 8 (4 (ks / 2) +
-// t) + 4 (ks % 2) + e and 2t+8+e <-> the same + 2, so a lane's key data is
-// the 16-byte chunks t, t+4, t+8, t+12 of a row.  In p.v the output column n
-// of n-tile j stands for d = 8n + 64 (j / 8) + j % 8, so a lane's value data
-// is chunks g and g+8 of rows 2t, 2t+1, 2t+8, 2t+9.
+// Per warp, a block of up to 8 tokens goes through two mma.sync products
+// (fp16 in, fp32 accumulate), lane (g = lane / 4, t = lane % 4):
+//   S[16 x 8]  = Q[16 x 128] K^T      m16n8k16 x 8 (rows = the G query heads,
+//                                     zero-padded; columns = the 8 tokens)
+//   O^T[128 x 8] += V^T[128 x 8] P^T  m16n8k8 x 8 (rows = d, columns = the
+//                                     heads; P^T is S's fragment as it lies)
+// The q.k contraction runs over d in a fixed permuted order: mma k-index
+// 2t+e of step ks <-> d = 8 (4 (ks / 2) + t) + 4 (ks % 2) + e and 2t+8+e <->
+// the same + 2, so a lane's key data is the 16-byte chunks t, t+4, t+8, t+12
+// of key row g.  In p.v, row g of tile i stands for d = 8g + i and row g + 8
+// for d = 64 + 8g + i, so a lane's value data is chunks g and g + 8 of value
+// rows 2t and 2t + 1, and its accumulators hold heads 2t and 2t + 1.
 
 __device__ __forceinline__ void mma16816(float& d0, float& d1, uint32_t a0, uint32_t a2, uint32_t b0,
                                          uint32_t b1) {
@@ -164,109 +166,90 @@ __device__ __forceinline__ void mma16816(float& d0, float& d1, uint32_t a0, uint
     (void)x3;
 }
 
+// m16n8k8, all four accumulators live: D[16 x 8] += A[16 x 8] B[8 x 8].
+__device__ __forceinline__ void mma16808(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t b0) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5}, {%6}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(b0));
+}
+
 struct MmaState {
-    float m;          // running max of this lane's head row (log2 domain)
-    float lp;         // this lane's share of the row's softmax sum
-    float o[16][2];   // O[g][d = 8 (2t + e) + 64 (j / 8) + j % 8] at o[j][e]
+    float m;          // running max of this lane's head row g (log2 domain)
+    float lp;         // this lane's share of that row's softmax sum
+    float o[8][4];    // O[head 2t + (e & 1)][d = 8g + i + 64 (e >> 1)] at o[i][e]
 };
 
 __device__ __forceinline__ uint4 ld_nc16(const void* p) {
     return *reinterpret_cast<const uint4*>(p);
 }
 
-// m16n8k8: rows 0..7 of A (the heads), k = 8 tokens.
-__device__ __forceinline__ void mma16808(float& d0, float& d1, uint32_t a0, uint32_t b0) {
-    float x2, x3;   // rows 8..15 of the tile: never used
-    asm volatile(
-        "mma.sync.aligned.m16n8k8.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5}, {%6}, "
-        "{%7, %8, %9, %10};"
-        : "=f"(d0), "=f"(d1), "=f"(x2), "=f"(x3)
-        : "r"(a0), "r"(0u), "r"(b0), "f"(d0), "f"(d1), "f"(0.f), "f"(0.f));
-    (void)x2;
-    (void)x3;
-}
-
-// One 16-token block made of two halves of 8 token rows: rows 0..7 hold
-// nlo valid tokens, rows 8..15 hold nhi (a half is a slice of one segment,
-// or a whole segment of at most 8 tokens).  kw[nt][i]: chunk 4i + t of key
-// row nt*8 + g; vw[k][i]: chunk g + 8i of value row {2t, 2t+1, 2t+8,
-// 2t+9}[k].
+// One block of up to 8 token rows, n of them valid.  kw[i]: chunk 4i + t of
+// key row g; vw[k][i]: chunk g + 8i of value row 2t + k.
 //
 // The running max moves only when a block max exceeds it by more than 8 (in
 // log2 units), so the fp16 numerators stay <= 2^8 and most blocks skip the
 // rescale of O; every partial carries the max it was scaled by.
-__device__ __forceinline__ void mma_block(MmaState& st, const uint32_t (&qa)[8][2], const uint4 (&kw)[2][4],
-                                          const uint4 (&vw)[4][2], int nlo, int nhi, float c2) {
+__device__ __forceinline__ void mma_block(MmaState& st, const uint32_t (&qa)[8][2], const uint4 (&kw)[4],
+                                          const uint4 (&vw)[2][2], int n, float c2) {
     const int lane = threadIdx.x & 31;
     const int t = lane & 3;
-    // two accumulation chains per tile (even and odd k-steps) halve the
-    // dependent MMA latency
-    float sacc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+    // two accumulation chains (even and odd k-steps) halve the dependent
+    // MMA latency
+    float s0 = 0.f, s1 = 0.f, u0 = 0.f, u1 = 0.f;
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-        if (nt == 1 && nhi == 0) break;
-        float odd0 = 0.f, odd1 = 0.f;
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-            const uint4& w = kw[nt][ks >> 1];
-            const uint32_t b0 = (ks & 1) ? w.z : w.x;
-            const uint32_t b1 = (ks & 1) ? w.w : w.y;
-            if (ks & 1)
-                mma16816(odd0, odd1, qa[ks][0], qa[ks][1], b0, b1);
-            else
-                mma16816(sacc[nt][0], sacc[nt][1], qa[ks][0], qa[ks][1], b0, b1);
-        }
-        sacc[nt][0] += odd0;
-        sacc[nt][1] += odd1;
+    for (int ks = 0; ks < 8; ++ks) {
+        const uint4& w = kw[ks >> 1];
+        const uint32_t b0 = (ks & 1) ? w.z : w.x;
+        const uint32_t b1 = (ks & 1) ? w.w : w.y;
+        if (ks & 1)
+            mma16816(u0, u1, qa[ks][0], qa[ks][1], b0, b1);
+        else
+            mma16816(s0, s1, qa[ks][0], qa[ks][1], b0, b1);
     }
-    // scores of tokens nt*8 + 2t + e, online softmax over the head row
-    float x[4];
-    bool ok[4];
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            ok[nt * 2 + e] = (2 * t + e) < (nt ? nhi : nlo);
-            x[nt * 2 + e] = ok[nt * 2 + e] ? sacc[nt][e] * c2 : kNegInfF;
-        }
-    float bm = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+    s0 += u0;
+    s1 += u1;
+    // scores of tokens 2t, 2t + 1 of head row g, online softmax over the row
+    const bool ok0 = 2 * t < n, ok1 = 2 * t + 1 < n;
+    const float x0 = ok0 ? s0 * c2 : kNegInfF;
+    const float x1 = ok1 ? s1 * c2 : kNegInfF;
+    float bm = fmaxf(x0, x1);
     bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 1));
     bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 2));
     const bool move = bm > st.m + 8.f;               // st.m = -inf: any finite bm moves
     const float mn = move ? bm : st.m;
     const float alpha = move ? ((st.m == kNegInfF) ? 0.f : fast_exp2(st.m - mn)) : 1.f;
     st.m = mn;
-    float p[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) p[i] = ok[i] ? fast_exp2(x[i] - mn) : 0.f;
-    st.lp = st.lp * alpha + ((p[0] + p[1]) + (p[2] + p[3]));
+    const float p0 = ok0 ? fast_exp2(x0 - mn) : 0.f;
+    const float p1 = ok1 ? fast_exp2(x1 - mn) : 0.f;
+    st.lp = st.lp * alpha + (p0 + p1);
     if (__any_sync(0xffffffffu, alpha != 1.f)) {
+        // this lane's accumulators belong to heads 2t and 2t + 1, whose
+        // factors sit in lanes 4 (2t) and 4 (2t + 1)
+        const float a_lo = __shfl_sync(0xffffffffu, alpha, 8 * t);
+        const float a_hi = __shfl_sync(0xffffffffu, alpha, 8 * t + 4);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            st.o[j][0] *= alpha;
-            st.o[j][1] *= alpha;
+        for (int i = 0; i < 8; ++i) {
+            st.o[i][0] *= a_lo;
+            st.o[i][1] *= a_hi;
+            st.o[i][2] *= a_lo;
+            st.o[i][3] *= a_hi;
         }
     }
-    const __half2 pa = __floats2half2_rn(p[0], p[1]);
-    const __half2 pb = __floats2half2_rn(p[2], p[3]);
-    const uint32_t a0 = *reinterpret_cast<const uint32_t*>(&pa);
-    const uint32_t a2 = *reinterpret_cast<const uint32_t*>(&pb);
-    auto bfrag = [&](int j, int k0) {
-        // element j of the windows of rows k0, k0 + 1: chunk j / 8, word (j % 8) / 2
-        const int ci = j >> 3, wi = (j & 7) >> 1;
-        const uint32_t sel = (j & 1) ? 0x7632u : 0x5410u;
+    const __half2 pp = __floats2half2_rn(p0, p1);
+    const uint32_t b0 = *reinterpret_cast<const uint32_t*>(&pp);
+    // element i of chunk window ci of value rows 2t, 2t + 1, packed in pairs
+    auto afrag = [&](int i, int ci) {
+        const int wi = i >> 1;
+        const uint32_t sel = (i & 1) ? 0x7632u : 0x5410u;
         auto word = [&](const uint4& q4) {
             return wi == 0 ? q4.x : wi == 1 ? q4.y : wi == 2 ? q4.z : q4.w;
         };
-        return __byte_perm(word(vw[k0][ci]), word(vw[k0 + 1][ci]), sel);
+        return __byte_perm(word(vw[0][ci]), word(vw[1][ci]), sel);
     };
-    if (nhi > 0) {
 #pragma unroll
-        for (int j = 0; j < 16; ++j) mma16816(st.o[j][0], st.o[j][1], a0, a2, bfrag(j, 0), bfrag(j, 2));
-    } else {
-#pragma unroll
-        for (int j = 0; j < 16; ++j) mma16808(st.o[j][0], st.o[j][1], a0, bfrag(j, 0));
-    }
+    for (int i = 0; i < 8; ++i) mma16808(st.o[i], afrag(i, 0), afrag(i, 1), b0);
 }
 
 // Contiguous global -> shared copy by the TMA unit (no tensor map, no
@@ -509,10 +492,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
     st.m = kNegInfF;
     st.lp = 0.f;
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-        st.o[j][0] = 0.f;
-        st.o[j][1] = 0.f;
-    }
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) st.o[i][e] = 0.f;
     const uint8_t* ubase = A.arena + static_cast<int64_t>(u) * A.arena_stride;
     // first K row of a dense segment (its V rows follow its ntok K rows)
     auto seg_k = [&](uint64_t d) {
@@ -747,23 +729,15 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
             }
             __syncwarp();
         }
-        // 8-token blocks: key rows g and value rows 2t, 2t+1 only (the second
-        // half of the 16-row MMA tile stays zero)
-        const uint4 z4 = make_uint4(0, 0, 0, 0);
-        uint4 kw[2][4], vw[4][2];
+        // key row g, value rows 2t and 2t + 1
+        uint4 kw[4], vw[2][2];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            kw[0][i] = lds16(K0 + g * kDecKStride + (4 * i + t) * 16);
-            kw[1][i] = z4;
-        }
+        for (int i = 0; i < 4; ++i) kw[i] = lds16(K0 + g * kDecKStride + (4 * i + t) * 16);
 #pragma unroll
         for (int k = 0; k < 2; ++k)
 #pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                vw[k][i] = lds16(V0 + (2 * t + k) * kDecVStride + (g + 8 * i) * 16);
-                vw[k + 2][i] = z4;
-            }
-        mma_block(st, qa, kw, vw, bk.nlo, 0, c2);
+            for (int i = 0; i < 2; ++i) vw[k][i] = lds16(V0 + (2 * t + k) * kDecVStride + (g + 8 * i) * 16);
+        mma_block(st, qa, kw, vw, bk.nlo, c2);
         // the stage is refilled next by the copy engine: after a scatter
         // (plain stores into the key rows) every writer orders its stores
         // before those copies; plain reads need no fence
@@ -806,15 +780,20 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
     float l = st.lp;
     l += __shfl_xor_sync(0xffffffffu, l, 1);
     l += __shfl_xor_sync(0xffffffffu, l, 2);
-    if (g < G) {
-        if (t == 0) {
-            wm[warp][g] = st.m;
-            wl[warp][g] = l;
-        }
+    if (g < G && t == 0) {
+        wm[warp][g] = st.m;
+        wl[warp][g] = l;
+    }
+    // lane (g, t) holds heads 2t, 2t + 1 at d = 8g + i and 64 + 8g + i
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            wo[warp][g][16 * t + 64 * (j >> 3) + (j & 7)] = st.o[j][0];
-            wo[warp][g][16 * t + 8 + 64 * (j >> 3) + (j & 7)] = st.o[j][1];
+    for (int e = 0; e < 2; ++e) {
+        const int hh = 2 * t + e;
+        if (hh < G) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                wo[warp][hh][8 * g + i] = st.o[i][e];
+                wo[warp][hh][64 + 8 * g + i] = st.o[i][2 + e];
+            }
         }
     }
     __syncthreads();
