@@ -515,10 +515,23 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
     {
         __shared__ int s_cut[2];
         if (tid == 0) s_cut[0] = -1;
-        for (int c0 = seg_next; c0 < j_hi; c0 += kDecThreads) {
+        // chunks of kDecThreads segments aligned like the counting pass, so
+        // that the descriptors it left in registers serve again
+        for (int c0 = seg_next / kDecThreads * kDecThreads; c0 < j_hi; c0 += kDecThreads) {
             const int j = c0 + tid;
-            const uint64_t d = (j < j_hi) ? D[j] : 0ull;
-            const int nit = (j < j_hi) ? (seg_ntok(d) + kDecRows - 1) / kDecRows : 0;
+            const bool in = j >= seg_next && j < j_hi;
+            uint64_t d = 0;
+            if (in) {
+                const int kk = c0 / kDecThreads;
+                if (kk < kDescPerThread) {
+#pragma unroll
+                    for (int k = 0; k < kDescPerThread; ++k)
+                        if (k == kk) d = dreg[k];
+                } else {
+                    d = D[j];
+                }
+            }
+            const int nit = in ? (seg_ntok(d) + kDecRows - 1) / kDecRows : 0;
             int x = nit;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
@@ -534,7 +547,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
                 if (w2 < warp) pos += wcnt[w2][0];
                 tot += wcnt[w2][0];
             }
-            if (j < j_hi) {
+            if (in) {
                 if (pos + nit <= A.tbl_cap) {
                     for (int q = 0; q < nit; ++q) tbl[pos + q] = d | (static_cast<uint64_t>(q * kDecRows) << 40);
                 } else if (pos <= A.tbl_cap) {   // the first segment that does not fit
