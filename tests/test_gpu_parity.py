@@ -292,3 +292,47 @@ def test_decode_in_cuda_graph(orc):
         torch.cuda.synchronize()
         assert torch.equal(out, ref)
     assert B.kv2d_read_status(ws) == 0
+
+
+def _tail_only_decode(lengths, group=4, hkv=2, d=128):
+    """Decode over dense tails only (nothing compressed): sequence b holds
+    lengths[b] tokens.  Returns (out, k, v, q) on the device."""
+    batch = len(lengths)
+    cap = 300   # > 256: two CTAs per unit allowed, so 80 units ask for all 148
+    g = torch.Generator(device="cuda").manual_seed(17)
+    k = torch.randn((batch, hkv, cap, d), generator=g, device="cuda").to(torch.float16)
+    v = torch.randn((batch, hkv, cap, d), generator=g, device="cuda").to(torch.float16)
+    q = torch.randn((batch, hkv * group, d), generator=g, device="cuda").to(torch.float16)
+    p = B.params(d, hkv * group, hkv, 64, 32, 8, 32, 0.25, float(np.float32(1.0 / np.sqrt(d))))
+    cc = B.CompressedCache(p, batch, cap)
+    seq = torch.tensor(lengths, dtype=torch.int32, device="cuda")
+    out = torch.full((batch, hkv * group, d), float("nan"), dtype=torch.float16, device="cuda")
+    ws = B.workspace(B.kv2d_workspace_bytes(p, B.OP_DECODE, batch, cap))
+    B.kv2d_decode_attn(p, batch, cc.struct, B.dense(k, v), seq, cap, q, out, ws)
+    torch.cuda.synchronize()
+    assert B.kv2d_read_status(ws) == 0
+    return out, k, v, q
+
+
+def test_decode_empty_batch_leaves_ctas_without_bytes(orc):
+    """80 units with no token at all: the batch-wide range holds 80 bytes
+    (one per unit) for 148 CTAs, so most CTAs get an empty share; each unit
+    still gets exactly one writer, and a unit without tokens decodes to 0."""
+    out, _, _, _ = _tail_only_decode([0] * 40)
+    assert torch.equal(out, torch.zeros_like(out))
+
+
+def test_decode_one_token_over_many_empty_pieces(orc):
+    """One sequence with a single dense token among 39 empty ones: its two
+    units span ~70 CTAs each, all but one with no token, and the merge of
+    those pieces must give that token's value row exactly (softmax weight 1)."""
+    lengths = [0] * 39 + [1]
+    out, _, v, _ = _tail_only_decode(lengths)
+    G = 4
+    for b in range(40):
+        for h in range(2):
+            got = out[b, h * G:(h + 1) * G]
+            if lengths[b] == 0:
+                assert torch.equal(got, torch.zeros_like(got))
+            else:
+                assert torch.equal(got, v[b, h, 0].expand(G, -1))
