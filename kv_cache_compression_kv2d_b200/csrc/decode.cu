@@ -612,11 +612,12 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
             }
         }
         bk.nlo = n;
-        // Copies by the TMA unit.  Segment blocks: lane 0 copies the block's
-        // key rows and value rows in one piece each (or a sparse block's two
-        // pair sections and its value rows); the dense tail, whose rows need
-        // not be contiguous, is copied row by row (lane l < 8: value row l,
-        // lane 16 + l: key row l).
+        // Copies by the TMA unit.  Segment blocks: lane 0 copies a whole
+        // short segment in one piece, else the block's key rows and value
+        // rows (or a sparse block's two pair sections and its value rows) in
+        // one piece each; the dense tail, whose rows need not be contiguous,
+        // is copied row by row (lane l < 8: value row l, lane 16 + l: key
+        // row l).
         if (bk.kind != 0) {
             const uint32_t K0 = kreg(stage), V0 = K0 + kDecKBytes, bar = bar0 + stage * 8;
             if (!tail) {
