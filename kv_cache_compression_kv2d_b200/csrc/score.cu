@@ -801,15 +801,18 @@ __device__ __forceinline__ void key_masks(const uint4 (*ks)[128], int tid, __hal
     }
 }
 
-// fp64 acc + v unless (m & bit) != 0: one compare into a predicate and one
-// guarded add, so the skipped add costs no select of the 64-bit value.
-__device__ __forceinline__ double dadd_unless(double acc, double v, uint32_t m, uint32_t bit) {
+// fp64 acc + x * y unless (m & bit) != 0, as one fused multiply-add: the
+// callers' products are exact in fp64 (an fp16 magnitude times an fp32
+// weight: 11 x 24 significant bits), so rounding x * y + acc once equals
+// adding the exact product with one rounding.  One compare into a predicate
+// and one guarded instruction, so the skipped add costs no 64-bit select.
+__device__ __forceinline__ double dfma_unless(double acc, double x, double y, uint32_t m, uint32_t bit) {
     asm("{\n\t.reg .pred p;\n\t.reg .b32 t;\n\t"
-        "and.b32 t, %2, %3;\n\t"
+        "and.b32 t, %3, %4;\n\t"
         "setp.eq.u32 p, t, 0;\n\t"
-        "@p add.rn.f64 %0, %0, %1;\n\t}"
+        "@p fma.rn.f64 %0, %1, %2, %0;\n\t}"
         : "+d"(acc)
-        : "d"(v), "r"(m), "r"(bit));
+        : "d"(x), "d"(y), "r"(m), "r"(bit));
     return acc;
 }
 
@@ -956,12 +959,13 @@ __global__ void __launch_bounds__(128) chan_kernel_c32(const __grid_constant__ C
         for (int e = 0; e < 4; ++e) {
             const float2 f2 = __half22float2(__habs2(*reinterpret_cast<const __half2*>(&qw[e])));
             const double2 a2 = *reinterpret_cast<const double2*>(ad + 8 * j + 2 * e);
-            const double e0 = __dmul_rn(static_cast<double>(f2.x), a2.x);
-            const double e1 = __dmul_rn(static_cast<double>(f2.y), a2.y);
-            tot = __dadd_rn(tot, e0);
-            drop = dadd_unless(drop, e0, mw, 1u << (2 * e));
-            tot = __dadd_rn(tot, e1);
-            drop = dadd_unless(drop, e1, mw, 2u << (2 * e));
+            // e = |k| a_x is exact in fp64, so each fused multiply-add
+            // rounds exactly as adding e does
+            const double k0 = static_cast<double>(f2.x), k1 = static_cast<double>(f2.y);
+            tot = __fma_rn(k0, a2.x, tot);
+            drop = dfma_unless(drop, k0, a2.x, mw, 1u << (2 * e));
+            tot = __fma_rn(k1, a2.y, tot);
+            drop = dfma_unless(drop, k1, a2.y, mw, 2u << (2 * e));
         }
     }
     A.cmask[slot] = make_uint4(M[0], M[1], M[2], M[3]);
