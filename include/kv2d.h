@@ -40,8 +40,10 @@
  * Memory.  Every buffer is allocated and owned by the caller; the library
  * never allocates device memory, never synchronises a stream inside
  * kv2d_compress / kv2d_append / kv2d_decode_attn, and keeps no state between
- * calls except a thread-local error string.  All device work is enqueued on
- * the caller's stream.  fp16 means IEEE binary16.
+ * calls except a thread-local error string and two process-wide switches of
+ * its aids (kv2d_profile_enable, kv2d_set_decode_table_cap); the fixed
+ * scratch of kv2d_decode_attn_noalloc is described with that call.  All
+ * device work is enqueued on the caller's stream.  fp16 means IEEE binary16.
  *
  * Errors.  Every entry point validates its arguments on the host before it
  * launches anything and returns a kv2d_status; kv2d_last_error() gives the
