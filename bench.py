@@ -2,16 +2,20 @@
 """Benchmark of the kv2d hot path on synthetic long-context inputs.
 
 One step = one pass of the whole path over one batch: kv2d_compress of the
-prompt (window statistics, scoring passes, channel top-c, segment selection,
+prompts (window statistics, scoring passes, channel top-c, segment selection,
 budget, packing), kv2d_append of one new token per (sequence, KV head), and
 kv2d_decode_attn of every query head over the compressed cache plus its dense
 tail.  The compressed-cache bookkeeping is reset at the start of each step so
-every step compresses the full prompt again.
+every step compresses the full prompts again.
 
-Default workload: one Llama-3-8B-shaped attention layer (32 query / 8 KV
-heads, d = 128), batch 1, 32K-token context in fp16, segment 64, window 64,
-budget 20%.  Inputs are resident in HBM (K + V = 134 MB > the 126 MB L2) and
-L2 is flushed between timed steps by writing a 256 MB buffer.
+Default workload (the largest single-GPU configuration): one
+Llama-3-8B-shaped attention layer (32 query / 8 KV heads, d = 128), batch 16
+x 128K-token contexts in fp16, segment 64, window 64, budget 15 %, segment
+classes mixed so that all four strategies occur.  The dense K + V is 8.6 GB,
+far larger than the 126 MB L2, and L2 is also flushed between timed steps.
+The other configurations (the 32K layer, the 1M-token layer, the ragged
+paged batch of 32 with a periodic re-compression) are timed as extra keys:
+compress alone and decode alone.
 
 Prints ONE JSON line (rank 0).  Multi-GPU: one process per GPU (torchrun);
 each rank compresses and decodes its own independent batch (weak scaling, no
@@ -32,10 +36,12 @@ sys.path.insert(0, ROOT)
 
 METRIC = "decode-attn us/step & HBM GB/s over compressed KV; kv2d_compress GB/s"
 UNIT = "GB/s"
-DEFAULT_WORKLOAD = "llama3_8b_32k"
+DEFAULT_WORKLOAD = "llama3_8b_b16_128k_mix"
+EXTRA_WORKLOADS = ("llama3_8b_32k", "llama3_8b_1m", "ragged32_paged")
 SMI_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+VALUE_IS = "dense KV bytes (K+V of the prompts) per step / step time"
 
 
 def rank_seed(seed, rank):
@@ -61,31 +67,36 @@ def job_throughput(bytes_per_rank, world, ms_per_step):
     return bytes_per_rank * world / (ms_per_step * 1e-3) / 1e9
 
 
-def profiled_traffic(kernel, workload):
-    """DRAM bytes (read + write) per launch of `kernel` on `workload` from the
-    committed ncu summary profiles/<kernel>_<workload>.md, or None when there
-    is none or the kernel's source file has changed since the capture (the
-    summary records the SHA-256 of the source it was measured with)."""
+def profiled_traffic(kernel, tokens):
+    """DRAM bytes (read + write) of one launch of `kernel` over `tokens`
+    tokens, from the committed ncu summary profiles/<kernel>_*.md whose
+    `kernel_source_sha256` still matches the kernel's source file: the
+    captured launch's traffic scaled by tokens (the kernels' traffic grows in
+    proportion to the tokens they read).  None when no current summary
+    exists.  Returns (bytes, note)."""
+    import glob
     import hashlib
-    root = os.path.dirname(os.path.abspath(__file__))
-    path = os.path.join(root, "profiles", f"{kernel}_{workload}.md")
-    if not os.path.exists(path):
-        return None
-    fields = {}
-    with open(path) as f:
-        for line in f:
-            if ":" in line and line.split(":", 1)[0] in ("traffic_bytes_per_launch", "kernel_source",
-                                                        "kernel_source_sha256"):
-                k, v = line.split(":", 1)
-                fields[k] = v.strip()
-    try:
-        with open(os.path.join(root, fields["kernel_source"]), "rb") as f:
-            sha = hashlib.sha256(f.read()).hexdigest()
-        if sha != fields["kernel_source_sha256"]:
-            return None
-        return int(fields["traffic_bytes_per_launch"])
-    except (KeyError, OSError, ValueError):
-        return None
+    for path in sorted(glob.glob(os.path.join(ROOT, "profiles", f"{kernel}_*.md"))):
+        fields = {}
+        with open(path) as f:
+            for line in f:
+                if ":" in line:
+                    k, v = line.split(":", 1)
+                    if k in ("traffic_bytes_per_launch", "tokens_per_launch", "kernel_source",
+                             "kernel_source_sha256", "workload"):
+                        fields[k] = v.strip()
+        try:
+            with open(os.path.join(ROOT, fields["kernel_source"]), "rb") as f:
+                sha = hashlib.sha256(f.read()).hexdigest()
+            if sha != fields["kernel_source_sha256"]:
+                continue
+            per = int(fields["traffic_bytes_per_launch"]) / int(fields["tokens_per_launch"])
+            note = (f"ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch on "
+                    f"{fields.get('workload', '?')} ({os.path.basename(path)}), scaled by tokens")
+            return per * tokens, note
+        except (KeyError, OSError, ValueError, ZeroDivisionError):
+            continue
+    return None, "no ncu summary of the current kernel source"
 
 
 def parse_args():
@@ -100,8 +111,8 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true",
                     help="skip the CUDA-graph decode timing and the budget-1 decode")
-    ap.add_argument("--no-decode-large", action="store_true",
-                    help="skip the decode-only measurement on the batch-16 x 128K cache")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the compress / decode timings of the other configurations")
     return ap.parse_args()
 
 
@@ -117,6 +128,25 @@ def peaks():
 
 def dense_bytes(wl, lens):
     return sum(int(T) for T in lens) * wl.num_kv_heads * wl.head_dim * 2 * 2
+
+
+def config_of(wl, lens, world):
+    """The workload's description, shared by both arms of the benchmark."""
+    return {"workload": wl.name, "global_batch": wl.batch * world, "seq_len": max(int(x) for x in lens),
+            "num_q_heads": wl.num_q_heads, "num_kv_heads": wl.num_kv_heads,
+            "head_dim": wl.head_dim, "segment_len": wl.segment_len, "window": wl.window,
+            "budget": wl.budget, "segment_mix": wl.segment_mix,
+            "parallelism": f"dp{world}" if world > 1 else "single GPU",
+            "l2": "flushed between steps (256 MB write); inputs larger than L2",
+            "value_is": VALUE_IS}
+
+
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            return next((l.split(":", 1)[1].strip() for l in f if l.startswith("model name")), None)
+    except OSError:
+        return None
 
 
 # ------------------------------------------------------------------ clocks
@@ -170,150 +200,265 @@ class ClockSampler:
                 "sm_max_mhz": mx or None, "reasons": sorted(reasons), "samples": len(sm)}
 
 
+# ------------------------------------------------------- CPU oracle sample
+
+
+def cpu_sample_units(wl, seed, n):
+    """The seeded sample of (sequence, KV head) units the oracle is timed on
+    (both arms use the same sample)."""
+    import numpy as np
+    units = wl.batch * wl.num_kv_heads
+    rng = np.random.default_rng(seed + 424242)
+    pick = sorted(rng.choice(units, size=min(n, units), replace=False).tolist())
+    return [(u // wl.num_kv_heads, u % wl.num_kv_heads) for u in pick]
+
+
+def cpu_sample_size():
+    """Units in the CPU sample: one per host core, at most 16 (about 10 s of
+    oracle work per unit of a 128K-token sequence)."""
+    return max(1, min(os.cpu_count() or 1, 16))
+
+
+def host_units(batch, wl, units):
+    """fp16 host copies of the sampled units' prompt rows, window queries and
+    decode queries (inputs of the oracle)."""
+    out = []
+    G = wl.group
+    from kv_cache_compression_kv2d_b200 import synth
+    for b, h in units:
+        T = int(batch.seq_len[b])
+        k, v = synth.dense_rows(batch, b, h, 0, T)
+        out.append(dict(T=T, K=k.cpu().numpy(), V=v.cpu().numpy(),
+                        qw=batch.qw[b, h * G:(h + 1) * G].reshape(-1, wl.head_dim).cpu().numpy(),
+                        q=batch.q[b, h * G:(h + 1) * G].cpu().numpy()))
+    return out
+
+
+def oracle_unit_phases(O, p, x):
+    """The oracle over one unit, step by step with a clock around each phase:
+    scoring (window statistics, lse and s_t), selection (channel top-c and
+    g_t, top-r and error proxies per segment, hulls and the budget walk),
+    packing (every segment's bytes) and decode (attention of the G heads over
+    the packed segments and the dense tail).  Returns the phases' seconds."""
+    import numpy as np
+    pc = time.perf_counter
+    T, S = x["T"], p.S
+    nseg = T // S
+    t0 = pc()
+    Kd = x["K"].astype(np.float64)
+    qw = x["qw"].astype(np.float64)
+    a = O.win_stats(p, qw)
+    _, s = O.score(p, T, 0, Kd, qw)
+    t1 = pc()
+    cidx, g = O.channel(p, Kd[:nseg * S], a)
+    tidx = np.zeros((nseg, p.r), np.uint8)
+    E = np.zeros((nseg, 4))
+    for j in range(nseg):
+        tidx[j] = O.topr(p, s[j * S:(j + 1) * S])
+        E[j] = O.segment_errors(p, s[j * S:(j + 1) * S], g[j * S:(j + 1) * S], tidx[j])
+    st, strat, used = O.budget(p, E)
+    assert st == 0
+    t2 = pc()
+    parts, offs, off = [], np.zeros(nseg, np.int64), 0
+    for j in range(nseg):
+        rows = slice(j * S, (j + 1) * S)
+        seg = O.pack_segment(p, int(strat[j]), x["K"][rows], x["V"][rows], tidx[j], cidx[rows])
+        offs[j] = off
+        off += seg.size
+        parts.append(seg)
+    arena = np.concatenate(parts) if parts else np.zeros(0, np.uint8)
+    t3 = pc()
+    O.decode_unit(p, arena, offs, strat, x["K"][nseg * S:], x["V"][nseg * S:], x["q"])
+    t4 = pc()
+    return {"scoring": t1 - t0, "selection": t2 - t1, "packing": t3 - t2, "decode": t4 - t3}
+
+
+def oracle_sample(wl, xs, scale):
+    """The oracle on the sample, one unit per host thread (units are
+    independent).  Returns (wall seconds, per-phase thread seconds, dense
+    bytes of the sample)."""
+    import numpy as np
+    from oracle import oracle as O
+    O.build()
+    p = O.params(wl.head_dim, wl.group, wl.segment_len, wl.window, wl.r, wl.c,
+                 float(np.float32(wl.budget)), float(np.float32(scale)))
+    t0 = time.perf_counter()
+    res = O.parallel_map(lambda x: oracle_unit_phases(O, p, x), xs, threads=len(xs))
+    wall = time.perf_counter() - t0
+    phases = {k: sum(r[k] for r in res) for k in res[0]}
+    nbytes = sum(x["T"] for x in xs) * wl.head_dim * 4
+    return wall, phases, nbytes
+
+
+def cpu_record(wl, units, xs, wall, phases, nbytes):
+    total_units = wl.batch * wl.num_kv_heads
+    tot = sum(phases.values())
+    return {"value": nbytes / wall / 1e9, "unit": UNIT, "cores": len(xs), "kind": "oracle",
+            "cpu_model": cpu_model(), "host_cores": os.cpu_count(),
+            "sample": (f"{len(xs)} of {total_units} (sequence, KV head) units of {wl.name} "
+                       f"(seeded: {units}), each compress of its whole prompt + one decode, one "
+                       f"unit per thread, in {wall:.1f} s"),
+            "extrapolated_step_s": wall * total_units / len(xs),
+            "extrapolation": "linear in the unit count (units are independent): "
+                             "sample wall time x all units / sampled units",
+            "phase_thread_s": phases,
+            "phase_share": {k: v / tot for k, v in phases.items()}}
+
+
 # --------------------------------------------------------------- reference
 
 
 def run_reference(args, rank):
     """The reference arm: the fp64 CPU oracle, as it stands, on host cores,
-    each step a bounded sample of the workload (units in parallel threads)."""
+    each step the same bounded sample of the workload as the kv2d arm's
+    cpu_baseline (the same units on the same number of threads)."""
     if rank != 0:
         return
-    import numpy as np
     import torch
     from kv_cache_compression_kv2d_b200 import synth
-    from oracle import oracle as O
-    O.build()
     wl = synth.WORKLOADS[args.workload]
-    lens = synth.lengths(wl, args.seed)
-    ncpu = os.cpu_count() or 1
-    threads = max(1, min(ncpu, 2))
-    batch = synth.generate(wl.with_(batch=1, seq_len=int(lens[0]), ragged_min=0,
-                                    num_kv_heads=threads), seed=args.seed)
-    p = O.params(wl.head_dim, wl.group, wl.segment_len, wl.window, wl.r, wl.c,
-                 float(np.float32(wl.budget)), float(np.float32(1 / np.sqrt(wl.head_dim))))
-    T = int(batch.seq_len[0])
-    G = wl.group
-
-    def unit(h):
-        K = batch.k[0, h, :T].numpy()
-        V = batch.v[0, h, :T].numpy()
-        qw = batch.qw[0, h * G:(h + 1) * G].reshape(-1, wl.head_dim).numpy()
-        res = O.compress_unit(p, T, 0, K, V, qw)
-        nc = res["nseg"] * wl.segment_len
-        O.decode_unit(p, res["arena"], res["offs"], res["strat"], K[nc:], V[nc:],
-                      batch.q[0, h * G:(h + 1) * G].numpy())
-
-    times = []
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    batch = synth.generate(wl, seed=rank_seed(args.seed, 0), device=dev, extra_capacity=16)
+    lens = [int(x) for x in batch.seq_len]
+    units = cpu_sample_units(wl, args.seed, cpu_sample_size())
+    xs = host_units(batch, wl, units)
+    del batch
+    if dev == "cuda":
+        torch.cuda.empty_cache()
+    scale = float(torch.tensor(1.0 / wl.head_dim ** 0.5, dtype=torch.float32))
+    walls, last = [], None
     for i in range(args.warmup + args.steps):
-        t0 = time.perf_counter()
-        O.parallel_map(unit, list(range(threads)), threads=threads)
-        dt = time.perf_counter() - t0
+        wall, phases, nbytes = oracle_sample(wl, xs, scale)
         if i >= args.warmup:
-            times.append(dt)
-    sample_bytes = T * threads * wl.head_dim * 4
-    ms = 1e3 * statistics.mean(times)
-    value = sample_bytes / (ms * 1e-3) / 1e9
-    sample = (f"{threads} of {wl.batch * wl.num_kv_heads} (sequence, KV head) units of "
-              f"{wl.name}: compress of {T} tokens + one decode each, per step")
+            walls.append(wall)
+            last = (wall, phases, nbytes)
+    ms = 1e3 * statistics.mean(walls)
+    value = last[2] / (ms * 1e-3) / 1e9
+    cpu = cpu_record(wl, units, xs, ms * 1e-3, last[1], last[2])
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic",
-            "config": {"workload": wl.name, "global_batch": wl.batch, "seq_len": T,
-                       "parallelism": "host threads", "l2": "n/a (CPU)"},
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
-                             "sample": sample},
+            "data": "synthetic", "config": config_of(wl, lens, world),
+            "cpu_baseline": cpu,
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
-
-
-def cpu_baseline(wl, batch_host, p_gpu, budget_s=30.0):
-    """The oracle as it stands, on the host cores, over a bounded sample of
-    units of the same workload (one thread per unit)."""
-    import numpy as np
-    from oracle import oracle as O
-    O.build()
-    ncpu = os.cpu_count() or 1
-    units = [(b, h) for b in range(wl.batch) for h in range(wl.num_kv_heads)]
-    n = max(1, min(len(units), ncpu))
-    units = units[:n]
-    p = O.params(wl.head_dim, wl.group, wl.segment_len, wl.window, wl.r, wl.c,
-                 float(np.float32(wl.budget)), float(np.float32(p_gpu.scale)))
-    G = wl.group
-
-    def unit(bh):
-        b, h = bh
-        T = int(batch_host.seq_len[b])
-        K = batch_host.k[b, h, :T].numpy()
-        V = batch_host.v[b, h, :T].numpy()
-        qw = batch_host.qw[b, h * G:(h + 1) * G].reshape(-1, wl.head_dim).numpy()
-        res = O.compress_unit(p, T, 0, K, V, qw)
-        nc = res["nseg"] * wl.segment_len
-        O.decode_unit(p, res["arena"], res["offs"], res["strat"], K[nc:], V[nc:],
-                      batch_host.q[b, h * G:(h + 1) * G].numpy())
-        return T
-
-    t0 = time.perf_counter()
-    toks = O.parallel_map(unit, units, threads=n)
-    dt = time.perf_counter() - t0
-    nbytes = sum(toks) * wl.head_dim * 4
-    model = None
-    try:
-        with open("/proc/cpuinfo") as f:
-            model = next((l.split(":", 1)[1].strip() for l in f if l.startswith("model name")), None)
-    except OSError:
-        pass
-    return {"value": nbytes / dt / 1e9, "unit": UNIT, "cores": n, "kind": "oracle", "cpu_model": model,
-            "sample": f"{n} of {wl.batch * wl.num_kv_heads} (sequence, KV head) units "
-                      f"(compress + one decode each) in {dt:.1f} s"}
 
 
 # ------------------------------------------------------------------- kv2d
 
 
-def decode_batch16_128k(B, synth, torch, dev, stream, hbm, steps):
-    """Decode alone over the batch-16 x 128K cache (8 KV heads, four-class
-    segment mix, budget 15 %): 1.29 GB of packed bytes, larger than L2, a size
-    at which decode is bound by HBM rather than by its fixed phases."""
-    wl = synth.WORKLOADS["llama3_8b_b16_128k_mix"]
-    bt = synth.generate(wl, seed=0, device=dev, extra_capacity=16)
+def decode_bytes(wl, cc, seq):
+    """Algorithmic bytes of one decode call: the packed payload used, the
+    descriptors, the dense tail's K and V rows, q and out."""
+    used = int(cc.used_bytes.sum())
+    nsegs = int(cc.n_segs.sum())
+    ce = cc.comp_end.cpu().tolist()
+    sq = seq.cpu().tolist()
+    tail = sum((sq[b] - ce[b]) * wl.num_kv_heads for b in range(wl.batch))
+    return used + 8 * nsegs + tail * wl.head_dim * 4 + 2 * wl.batch * wl.num_q_heads * wl.head_dim * 2
+
+
+def compress_alg_bytes(wl, lens, used):
+    """Algorithmic bytes of kv2d_compress: K and V of the region read once,
+    the window queries, the packed bytes written, and s (4 B) and g (8 B)
+    per segment token."""
+    seg_tokens = sum((T // wl.segment_len) * wl.segment_len for T in lens)
+    return (dense_bytes(wl, lens) + wl.batch * wl.num_q_heads * wl.window * wl.head_dim * 2 + used +
+            seg_tokens * wl.num_kv_heads * 12)
+
+
+def event_pair(torch):
+    return torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+
+def timed(torch, stream, fn, n, before=None, flush=None):
+    """Mean CUDA-event milliseconds of fn() over n calls on stream, each call
+    preceded (outside the events) by before() and an L2 flush."""
+    evs = []
+    for _ in range(n):
+        if before is not None:
+            before()
+        if flush is not None:
+            flush.zero_()
+        a, b = event_pair(torch)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        evs.append((a, b))
+    torch.cuda.synchronize()
+    return statistics.mean(a.elapsed_time(b) for a, b in evs)
+
+
+def measure_extra(name, B, synth, torch, dev, stream, flush, hbm, n):
+    """Compress alone and decode alone on another configuration (L2 flushed
+    before each call); for the ragged paged batch also one periodic
+    re-compression of the trailing region after 128 appended tokens."""
+    wl = synth.WORKLOADS[name]
+    extra = wl.recompress_every + 16 if wl.recompress_every else 16
+    bt = synth.generate(wl, seed=0, device=dev, extra_capacity=extra)
     lens = [int(x) for x in bt.seq_len]
     scale = float(torch.tensor(1.0 / wl.head_dim ** 0.5, dtype=torch.float32))
     p = B.params(wl.head_dim, wl.num_q_heads, wl.num_kv_heads, wl.segment_len, wl.window, wl.r,
                  wl.c, wl.budget, scale)
-    dv = B.dense(bt.k, bt.v)
-    cc = B.CompressedCache(p, wl.batch, bt.capacity, device=dev)
+    paged = bt.block_table is not None
+    dv = B.dense(bt.k, bt.v, bt.block_table, wl.block_size) if paged else B.dense(bt.k, bt.v)
+    cap = bt.capacity
+    cc = B.CompressedCache(p, wl.batch, cap, device=dev)
     ws_c = B.workspace(B.kv2d_workspace_bytes(p, B.OP_COMPRESS, wl.batch, max(lens)), dev)
-    ws_d = B.workspace(B.kv2d_workspace_bytes(p, B.OP_DECODE, wl.batch, bt.capacity), dev)
-    B.kv2d_compress(p, wl.batch, lens, [0] * wl.batch, dv, bt.qw, cc.struct, ws_c, stream=stream)
+    ws_d = B.workspace(B.kv2d_workspace_bytes(p, B.OP_DECODE, wl.batch, cap), dev)
+    zeros = [0] * wl.batch
     seq = torch.tensor(lens, dtype=torch.int32, device=dev)
     out = torch.empty((wl.batch, wl.num_q_heads, wl.head_dim), dtype=torch.float16, device=dev)
 
+    def compress():
+        B.kv2d_compress(p, wl.batch, lens, zeros, dv, bt.qw, cc.struct, ws_c, stream=stream)
+
     def decode():
-        B.kv2d_decode_attn(p, wl.batch, cc.struct, dv, seq, bt.capacity, bt.q, out, ws_d, stream=stream)
+        B.kv2d_decode_attn(p, wl.batch, cc.struct, dv, seq, cap, bt.q, out, ws_d, stream=stream)
 
     for _ in range(3):
-        decode()
-    evs = []
-    for _ in range(steps):
-        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        decode()
-        b_.record(stream)
-        evs.append((a, b_))
-    torch.cuda.synchronize(dev)
+        cc.reset()
+        compress()
+    comp_ms = timed(torch, stream, compress, n, before=cc.reset, flush=flush)
+    cc.reset()
+    compress()
+    decode()
+    dec_ms = timed(torch, stream, decode, n, flush=flush)
     assert B.kv2d_read_status(ws_c, stream) == 0 and B.kv2d_read_status(ws_d, stream) == 0
-    us = 1e3 * statistics.mean(a.elapsed_time(b_) for a, b_ in evs)
-    ce = cc.comp_end.cpu().tolist()
-    tail = sum((lens[b] - ce[b]) * wl.num_kv_heads for b in range(wl.batch))
-    nbytes = (int(cc.used_bytes.sum()) + 8 * int(cc.n_segs.sum()) + tail * wl.head_dim * 4 +
-              2 * wl.batch * wl.num_q_heads * wl.head_dim * 2)
+    used = int(cc.used_bytes.sum())
+    dbytes = decode_bytes(wl, cc, seq)
+    calg = compress_alg_bytes(wl, lens, used)
+    rec = {"compress": {"us": 1e3 * comp_ms, "gbs": dense_bytes(wl, lens) / (comp_ms * 1e-3) / 1e9,
+                        "alg_bytes": calg, "hbm_frac": calg / (comp_ms * 1e-3) / 1e9 / hbm},
+           "decode": {"us_per_call": 1e3 * dec_ms, "bytes_per_call": dbytes,
+                      "hbm_gbs": dbytes / (dec_ms * 1e-3) / 1e9,
+                      "hbm_frac": dbytes / (dec_ms * 1e-3) / 1e9 / hbm},
+           "dense_bytes": dense_bytes(wl, lens), "calls": n, "l2": "flushed before each call"}
+    if wl.recompress_every:
+        # 128 decode steps of appends, then the periodic compression of the
+        # complete segments of [comp_end, seq_len); the cache bookkeeping is
+        # put back before each timed repeat so every repeat does the same work
+        ws_a = B.workspace(256, dev)
+        for step in range(wl.recompress_every):
+            kn, vn, _ = synth.decode_tokens(wl, step, device=dev, mu=bt.mu)
+            B.kv2d_append(p, wl.batch, dv, kn, vn, seq, ws_a, stream=stream)
+        torch.cuda.synchronize()
+        seq_h = seq.cpu().tolist()
+        ce_h = cc.comp_end.cpu().tolist()
+        saved = cc.book.clone()
+
+        def recompress():
+            B.kv2d_compress(p, wl.batch, seq_h, ce_h, dv, bt.qw, cc.struct, ws_c, stream=stream)
+
+        re_ms = timed(torch, stream, recompress, n, before=lambda: cc.book.copy_(saved), flush=flush)
+        region = sum(seq_h[b] - ce_h[b] for b in range(wl.batch))
+        assert B.kv2d_read_status(ws_c, stream) == 0 and B.kv2d_read_status(ws_a, stream) == 0
+        rec["recompress"] = {"us": 1e3 * re_ms, "region_tokens_per_sequence_mean": region / wl.batch,
+                             "note": "compression of [comp_end, seq_len) after 128 appended tokens"}
     del bt, dv, cc, ws_c, ws_d, out
     torch.cuda.empty_cache()
-    gbs = nbytes / (us * 1e-6) / 1e9
-    return {"workload": wl.name, "us_per_call": us, "bytes_per_call": nbytes, "hbm_gbs": gbs,
-            "hbm_frac": gbs / hbm, "calls": steps,
-            "l2": "no flush: 1.29 GB of packed bytes per call > L2"}
+    return rec
 
 
 def main():
@@ -342,29 +487,27 @@ def main():
 
     wl = synth.WORKLOADS[args.workload]
     dev = torch.device("cuda", local)
-    host = synth.generate(wl, seed=rank_seed(args.seed, rank), device="cpu", extra_capacity=16)
-    lens = [int(x) for x in host.seq_len]
-    k = host.k.to(dev)
-    v = host.v.to(dev)
-    qw = host.qw.to(dev)
-    q = host.q.to(dev)
-    bt = host.block_table.to(dev) if host.block_table is not None else None
+    stream = torch.cuda.current_stream(dev)
+    # inputs are drawn on the device (seeded); host copies serve the
+    # end-to-end timing and the CPU baseline
+    bat = synth.generate(wl, seed=rank_seed(args.seed, rank), device=dev, extra_capacity=16)
+    lens = [int(x) for x in bat.seq_len]
+    k, v, qw, q, bt = bat.k, bat.v, bat.qw, bat.q, bat.block_table
     scale = float(torch.tensor(1.0 / wl.head_dim ** 0.5, dtype=torch.float32))
     p = B.params(wl.head_dim, wl.num_q_heads, wl.num_kv_heads, wl.segment_len, wl.window, wl.r,
                  wl.c, wl.budget, scale)
     dv = B.dense(k, v, bt, wl.block_size) if bt is not None else B.dense(k, v)
-    cap = host.capacity
+    cap = bat.capacity
     cc = B.CompressedCache(p, wl.batch, cap, device=dev)
     ws_c = B.workspace(B.kv2d_workspace_bytes(p, B.OP_COMPRESS, wl.batch, max(lens)), dev)
     ws_d = B.workspace(B.kv2d_workspace_bytes(p, B.OP_DECODE, wl.batch, cap), dev)
     ws_a = B.workspace(256, dev)
-    kn, vn, _ = synth.decode_tokens(wl, 0, seed=args.seed, device=dev, mu=host.mu.to(dev))
+    kn, vn, _ = synth.decode_tokens(wl, 0, seed=args.seed, device=dev, mu=bat.mu)
     out = torch.empty((wl.batch, wl.num_q_heads, wl.head_dim), dtype=torch.float16, device=dev)
     seq0 = torch.tensor(lens, dtype=torch.int32, device=dev)
     seq = seq0.clone()
     zeros_ce = [0] * wl.batch
     flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=dev)   # 256 MB > L2
-    stream = torch.cuda.current_stream(dev)
 
     def reset():
         cc.reset()
@@ -409,8 +552,7 @@ def main():
         assert B.kv2d_read_status(ws_c, stream) == 0 and B.kv2d_read_status(ws_d, stream) == 0
 
         # ---- timed region: exactly K steps, L2 flushed between steps
-        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(args.steps)]
+        ev = [event_pair(torch) for _ in range(args.steps)]
         barrier()
         for i in range(args.steps):
             flush.zero_()
@@ -433,30 +575,14 @@ def main():
         prof = B.kv2d_profile_read()
 
         # ---- decode alone and compress alone (L2 flushed before each)
-        dec_ms, comp_ms = [], []
-        for i in range(args.steps):
-            flush.zero_()
-            a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            decode()
-            b_.record(stream)
-            dec_ms.append((a, b_))
-        for i in range(args.steps):
-            reset()
-            flush.zero_()
-            a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            compress()
-            b_.record(stream)
-            comp_ms.append((a, b_))
-        torch.cuda.synchronize(dev)
-        dec_ms = [a.elapsed_time(b_) for a, b_ in dec_ms]
-        comp_ms = [a.elapsed_time(b_) for a, b_ in comp_ms]
+        dec_ms = timed(torch, stream, decode, args.steps, flush=flush)
+        comp_ms = timed(torch, stream, compress, args.steps, before=reset, flush=flush)
 
         # ---- 100 back-to-back decodes captured in one CUDA graph (launch
-        # overhead amortised; the 32K cache then stays in L2 between calls)
+        # overhead amortised)
         graph_us = None
         if not args.no_graph:
+            step()
             try:
                 g_stream = torch.cuda.Stream(dev)
                 g_stream.wait_stream(stream)
@@ -468,7 +594,7 @@ def main():
                 stream.wait_stream(g_stream)
                 graph.replay()
                 torch.cuda.synchronize(dev)
-                a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a, b_ = event_pair(torch)
                 a.record(stream)
                 for _ in range(5):
                     graph.replay()
@@ -479,7 +605,7 @@ def main():
             except RuntimeError as exc:   # reported, not fatal: the step numbers stand
                 graph_us = f"capture failed: {exc}"[:200]
 
-        # ---- the same prompt compressed at budget 1 (every segment FULL):
+        # ---- the same prompts compressed at budget 1 (every segment FULL):
         # decode over the uncompressed cache, for the speedup of the packed one
         dense_dec_us = None
         if not args.no_graph:
@@ -487,18 +613,14 @@ def main():
                           wl.r, wl.c, 1.0, scale)
             cc1 = B.CompressedCache(p1, wl.batch, cap, device=dev)
             B.kv2d_compress(p1, wl.batch, lens, zeros_ce, dv, qw, cc1.struct, ws_c, stream=stream)
-            ev1 = []
-            for i in range(args.steps + 3):
-                flush.zero_()
-                a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                a.record(stream)
+
+            def decode1():
                 B.kv2d_decode_attn(p1, wl.batch, cc1.struct, dv, seq, cap, q, out, ws_d, stream=stream)
-                b_.record(stream)
-                if i >= 3:
-                    ev1.append((a, b_))
-            torch.cuda.synchronize(dev)
-            dense_dec_us = 1e3 * statistics.mean(a.elapsed_time(b_) for a, b_ in ev1)
+
+            decode1()
+            dense_dec_us = 1e3 * timed(torch, stream, decode1, args.steps, flush=flush)
             del cc1
+            torch.cuda.empty_cache()
         # leave the cache in its post-step state for the byte accounting
         step()
         torch.cuda.synchronize(dev)
@@ -511,45 +633,44 @@ def main():
 
     # ---- algorithmic work per launch
     hbm, tf_burst, tf_sust, src = peaks()
-    used = cc.used_bytes.cpu().tolist()
-    nsegs = cc.n_segs.cpu().tolist()
-    ce = cc.comp_end.cpu().tolist()
-    seq_after = seq.cpu().tolist()
-    tail_tokens = sum((seq_after[b] - ce[b]) * wl.num_kv_heads for b in range(wl.batch))
-    dec_bytes = (sum(used) + 8 * sum(nsegs) + tail_tokens * wl.head_dim * 4 +
-                 2 * wl.batch * wl.num_q_heads * wl.head_dim * 2)
-    dec_us = 1e3 * statistics.mean(dec_ms)
-    comp_us = 1e3 * statistics.mean(comp_ms)
+    used = int(cc.used_bytes.sum())
+    dec_bytes = decode_bytes(wl, cc, seq)
+    dec_us = 1e3 * dec_ms
+    comp_us = 1e3 * comp_ms
     flops_pass = 2.0 * wl.num_q_heads * wl.window * sum(lens) * wl.head_dim
     seg_tokens = sum((T // wl.segment_len) * wl.segment_len for T in lens)
     kv_seg_bytes = seg_tokens * wl.num_kv_heads * wl.head_dim * 2
+    chan_tokens = seg_tokens * wl.num_kv_heads
     work = {
-        "score_pass1": ("tensor", flops_pass),
-        "score_pass2": ("tensor", 2.0 * wl.num_q_heads * wl.window * seg_tokens * wl.head_dim),
+        "score_pass1": ("tensor", flops_pass, sum(lens) * wl.num_kv_heads),
+        "score_pass2": ("tensor", 2.0 * wl.num_q_heads * wl.window * seg_tokens * wl.head_dim,
+                        chan_tokens),
         # K rows in; a 16-byte keep mask and the fp64 g_t out per token
-        "chan_topc": ("hbm", kv_seg_bytes + seg_tokens * wl.num_kv_heads * (16 + 8)),
-        "pack": ("hbm", 2 * sum(used)),   # gathers about as many bytes as it writes
-        "decode": ("hbm", dec_bytes),
+        "chan_topc": ("hbm", kv_seg_bytes + chan_tokens * (16 + 8), chan_tokens),
+        "pack": ("hbm", 2 * used, chan_tokens),   # gathers about as many bytes as it writes
+        "decode": ("hbm", dec_bytes, None),
     }
     kernels = {}
+    tot_prof = sum(t for t, _ in prof.values())
     for name, (tot, n) in prof.items():
         if n:
-            kernels[name] = {"launches": n, "avg_us": 1e3 * tot / n,
-                             "share": tot / max(sum(t for t, _ in prof.values()), 1e-12)}
+            kernels[name] = {"launches": n, "avg_us": 1e3 * tot / n, "share": tot / max(tot_prof, 1e-12)}
     dominant = max(kernels, key=lambda k_: kernels[k_]["avg_us"] * kernels[k_]["launches"])
-    kind, amount = work.get(dominant, ("hbm", 0.0))
+    kind, amount, toks = work.get(dominant, ("hbm", 0.0, None))
     avg_s = kernels[dominant]["avg_us"] * 1e-6
+    traffic, traffic_note = profiled_traffic(dominant, toks) if toks else (None, "not captured")
     if kind == "tensor":
         achieved = amount / avg_s / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": tf_burst, "unit": "TFLOP/s",
-                "frac": achieved / tf_burst, "traffic": profiled_traffic(dominant, wl.name),
-                "kernel": dominant, "peak_source": f"{src} bf16 burst (fp16 runs at the bf16 rate)"}
+                "frac": achieved / tf_burst, "traffic": traffic, "kernel": dominant,
+                "peak_source": f"{src} bf16 burst (fp16 runs at the bf16 rate)"}
     else:
         achieved = amount / avg_s / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                "frac": achieved / hbm, "traffic": profiled_traffic(dominant, wl.name),
-                "kernel": dominant,
+                "frac": achieved / hbm, "traffic": traffic, "kernel": dominant,
                 "peak_source": f"{src} HBM copy"}
+    roof["algorithmic_per_launch"] = amount
+    roof["traffic_source"] = traffic_note
     gpu_launches = sum(v_["launches"] for v_ in kernels.values())
     # the scoring contraction, both passes (executed MMA flops = algorithmic)
     scoring = None
@@ -557,29 +678,25 @@ def main():
         t12 = (kernels["score_pass1"]["avg_us"] + kernels["score_pass2"]["avg_us"]) * 1e-6
         sflops = flops_pass + work["score_pass2"][1]
         scoring = {"tflops": sflops / t12 / 1e12, "frac": sflops / t12 / 1e12 / tf_burst,
-                   "peak": tf_burst, "peak_source": f"{src} bf16 burst"}
-    # compress, algorithmic bytes: K and V of the region read once, the window
-    # queries, the packed bytes written, and s (4 B) and g (8 B) per token
-    comp_alg = (nbytes + wl.batch * wl.num_q_heads * wl.window * wl.head_dim * 2 + sum(used) +
-                seg_tokens * wl.num_kv_heads * 12)
+                   "peak": tf_burst, "peak_source": f"{src} bf16 burst",
+                   "pass1_tflops": flops_pass / (kernels["score_pass1"]["avg_us"] * 1e-6) / 1e12,
+                   "pass2_tflops": work["score_pass2"][1] / (kernels["score_pass2"]["avg_us"] * 1e-6) / 1e12}
+    comp_alg = compress_alg_bytes(wl, lens, used)
 
     # ---- end to end through the public API with host buffers
     e2e = None
     if not args.no_e2e:
-        hk = host.k.pin_memory()
-        hv = host.v.pin_memory()
-        hqw = host.qw.pin_memory()
-        hq = host.q.pin_memory()
+        hk, hv, hqw, hq = (t.cpu().pin_memory() for t in (k, v, qw, q))
         hkn, hvn = kn.cpu().pin_memory(), vn.cpu().pin_memory()
         hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
         h2d = sum(t.numel() * t.element_size() for t in (hk, hv, hqw, hq, hkn, hvn))
         if bt is not None:
-            hbt = host.block_table.pin_memory()
+            hbt = bt.cpu().pin_memory()
             h2d += hbt.numel() * 4
         d2h = hout.numel() * hout.element_size()
         evs = []
         for i in range(max(3, args.warmup) + args.steps):
-            a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a, b_ = event_pair(torch)
             a.record(stream)
             k.copy_(hk, non_blocking=True)
             v.copy_(hv, non_blocking=True)
@@ -598,14 +715,25 @@ def main():
         e_ms = max_over_ranks(sum(a.elapsed_time(b_) for a, b_ in evs), dist, dev) / args.steps
         e2e = {"value": job_throughput(nbytes, world, e_ms), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms}
-
-    dec_large = None
-    if world == 1 and not args.no_decode_large:
-        dec_large = decode_batch16_128k(B, synth, torch, dev, stream, hbm, max(args.steps, 5))
+        del hk, hv, hqw, hq
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(wl, host, p)
+        units = cpu_sample_units(wl, args.seed, cpu_sample_size())
+        xs = host_units(bat, wl, units)
+        wall, phases, nb = oracle_sample(wl, xs, scale)
+        cpu = cpu_record(wl, units, xs, wall, phases, nb)
+        del xs
+
+    extras = None
+    if world == 1 and not args.no_extras:
+        del bat, k, v, qw, q, cc, ws_c, dv
+        torch.cuda.empty_cache()
+        extras = {}
+        for name in EXTRA_WORKLOADS:
+            if name != wl.name:
+                extras[name] = measure_extra(name, B, synth, torch, dev, stream, flush, hbm,
+                                             max(args.steps, 5))
 
     if dist is not None:
         dist.barrier()
@@ -616,25 +744,19 @@ def main():
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
-        "config": {"workload": wl.name, "global_batch": wl.batch * world, "seq_len": max(lens),
-                   "num_q_heads": wl.num_q_heads, "num_kv_heads": wl.num_kv_heads,
-                   "head_dim": wl.head_dim, "segment_len": wl.segment_len,
-                   "window": wl.window, "budget": wl.budget,
-                   "parallelism": f"dp{world}" if world > 1 else "single GPU",
-                   "l2": "flushed between steps (256 MB write); inputs 134 MB > L2",
-                   "value_is": "dense KV bytes (K+V of the prompt) per step / step time"},
+        "config": config_of(wl, lens, world),
         "decode": {"us_per_step": dec_us, "bytes_per_step": dec_bytes,
                    "hbm_gbs": dec_bytes / (dec_us * 1e-6) / 1e9,
                    "hbm_frac": dec_bytes / (dec_us * 1e-6) / 1e9 / hbm,
                    "hbm_frac_of_8tbs_nominal": dec_bytes / (dec_us * 1e-6) / 1e9 / 8000.0,
                    "graph_us_per_call": graph_us,
-                   "graph_note": "100 back-to-back calls in one CUDA graph; the cache stays in L2",
+                   "graph_note": "100 back-to-back calls in one CUDA graph, no flush between them",
                    "budget1_us": dense_dec_us,
                    "speedup_vs_budget1": (dense_dec_us / dec_us) if dense_dec_us else None},
         "compress": {"us": comp_us, "gbs": nbytes / (comp_us * 1e-6) / 1e9,
                      "alg_bytes": comp_alg, "hbm_frac": comp_alg / (comp_us * 1e-6) / 1e9 / hbm},
         "scoring": scoring,
-        "decode_batch16_128k": dec_large,
+        "extras": extras,
         "kernels": kernels,
         "kernels_note": "per-launch CUDA-event times from a profiled repeat of the K timed steps",
         "roofline": roof,

@@ -240,7 +240,9 @@ KV2D_API kv2d_status kv2d_append(const kv2d_params* p, int batch, const kv2d_den
  *                     Zero it once before its first use; every completed
  *                     call leaves the tickets at zero again.
  * Deterministic: the batch's bytes are cut into one share per CTA (a
- * function of the data and the SM count only); fixed merge order. */
+ * function of the data and the SM count only); fixed merge order.
+ * If a call sets KV2D_DEV_TIMEOUT (a copy into shared memory never
+ * completed), its outputs are undefined. */
 KV2D_API kv2d_status kv2d_decode_attn(const kv2d_params* p, int batch, const kv2d_ccache* cc,
                              const kv2d_dense* kv, const int32_t* seq_len_dev,
                              int32_t max_seq_len_host, const void* q, void* out, void* ws,
@@ -255,19 +257,23 @@ KV2D_API kv2d_status kv2d_decode_attn(const kv2d_params* p, int batch, const kv2
  * interface convenience only.
  *   It takes no workspace.  Its per-CTA partials and per-unit tickets live
  *   in a fixed 8 MiB array in the library's own device memory, which every
- *   GPU that loads the library holds until the process exits.  Calls whose
- *   scratch would exceed 8 MiB ((units + CTAs) x G x (d + 4) x 4 bytes plus
- *   4 bytes per unit and 256 bytes; CTAs <= the SM count) return
+ *   GPU that loads the library holds until the process exits.  The scratch
+ *   a call needs is three regions, each rounded up to a multiple of 256
+ *   bytes: 256 bytes, 4 bytes per unit, and (units + CTAs) x G x (d + 4) x 4
+ *   bytes (CTAs <= the SM count); calls needing more than 8 MiB return
  *   KV2D_ERR_WORKSPACE before launching.
  *   The first call on each device looks up the array's device address with
- *   the CUDA runtime; make that first call outside any stream capture.
+ *   the CUDA runtime (and makes the device's primary context current); make
+ *   that first call outside any stream capture.  The address is kept per
+ *   device together with the id of the context it belongs to, and looked up
+ *   again when that context has changed (after cudaDeviceReset).
  *   All calls on a device share the one array and each leaves its partials
  *   behind; the array starts zeroed and every completed call leaves its
  *   per-unit tickets at zero again.  Calls whose
  *   kernels overlap on the GPU (two streams, or two host threads) race on the
  *   array and give wrong results: serialise them.
  *   status_dev: optional device uint32; device-side faults OR their
- *   KV2D_DEV_* bits into it (NULL: they are not reported).
+ *   KV2D_DEV_* bits into it.  NULL: faults are not recorded anywhere.
  * Other arguments, layouts and errors as kv2d_decode_attn.  Allocates no
  * memory: no cudaMalloc / cudaFree and no allocating library call. */
 KV2D_API kv2d_status kv2d_decode_attn_noalloc(const kv2d_params* p, int batch,

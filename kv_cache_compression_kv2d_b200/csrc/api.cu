@@ -294,8 +294,29 @@ namespace {
 constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;   // 8 MiB per GPU
 constexpr int kNoAllocMaxDevices = 64;
 
+// Per device: the id of the context the address was looked up in, and the
+// address.  A device reset (cudaDeviceReset) ends that context and the
+// module is loaded again, possibly elsewhere, in a new one; context ids are
+// never reused within a process, so a changed id means the lookup is redone.
+struct NoAllocSlot {
+    unsigned long long ctx_id;
+    void* ptr;
+};
 std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+NoAllocSlot g_noalloc[kNoAllocMaxDevices] = {};
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+template <typename Fn>
+Fn driver_fn(const char* name) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint(name, &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+        return reinterpret_cast<Fn>(ptr);
+    return nullptr;
+}
 
 }  // namespace
 
@@ -303,24 +324,37 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 
 namespace {
 
-// Device address of the scratch array on the current device, resolved on
-// the first call per device.
+// Device address of the scratch array in the current device's current
+// context, looked up on the first call per device (and again after the
+// context changed).
 kv2d_status noalloc_scratch(void** out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return fail(KV2D_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
     if (dev < 0 || dev >= kNoAllocMaxDevices)
         return fail(KV2D_ERR_UNSUPPORTED, "device ordinal %d beyond %d", dev, kNoAllocMaxDevices);
+    static const CtxGetCurrentFn get_ctx = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+    static const CtxGetIdFn get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+    if (!get_ctx || !get_id) return fail(KV2D_ERR_CUDA, "the driver's context queries are unavailable");
+    auto current_id = [&](unsigned long long* id) {
+        CUcontext ctx = nullptr;
+        return get_ctx(&ctx) == CUDA_SUCCESS && ctx && get_id(ctx, id) == CUDA_SUCCESS;
+    };
     std::lock_guard<std::mutex> lk(g_noalloc_mu);
-    if (!g_noalloc_ptr[dev]) {
+    NoAllocSlot& slot = g_noalloc[dev];
+    unsigned long long id = 0;
+    if (!slot.ptr || !current_id(&id) || slot.ctx_id != id) {
+        // the lookup also makes the device's primary context current
         void* ptr = nullptr;
         e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
         if (e != cudaSuccess || !ptr)
             return fail(KV2D_ERR_CUDA, "cudaGetSymbolAddress of the decode scratch: %s",
                         cudaGetErrorString(e));
-        g_noalloc_ptr[dev] = ptr;
+        if (!current_id(&id)) return fail(KV2D_ERR_CUDA, "cannot identify the current CUDA context");
+        slot.ctx_id = id;
+        slot.ptr = ptr;
     }
-    *out = g_noalloc_ptr[dev];
+    *out = slot.ptr;
     return KV2D_OK;
 }
 
@@ -717,7 +751,7 @@ kv2d_status kv2d_decode_attn_noalloc(const kv2d_params* p, int batch, const kv2d
     L.tbl_cap = g_dec_table_cap.load();
     L.part = reinterpret_cast<float*>(w + part_off);
     L.ticket = reinterpret_cast<uint32_t*>(w + ticket_off);   // left at zero by every call
-    L.status = status_dev ? status_dev : reinterpret_cast<uint32_t*>(w);
+    L.status = status_dev;   // NULL: device faults are not recorded anywhere
     cudaError_t e = launch_decode(L, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return fail(KV2D_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
     return ok();

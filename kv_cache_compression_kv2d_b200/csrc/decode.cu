@@ -776,6 +776,16 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
                     break;
                 }
                 if (!mbar_wait(&sbar[warp][k % kDecStages], (k / kDecStages) & 1, A.status)) {
+                    // give the copies this warp has in flight (blocks k + 1
+                    // .. k + kAhead) one more bounded wait each before the
+                    // stage buffers are reused; the outputs are undefined
+                    // from here on (the status bit says so)
+#pragma unroll
+                    for (int j = 1; j <= kAhead; ++j) {
+                        const DecBlock& fb = (j < kAhead) ? f[j] : nb;
+                        if (fb.kind != 0)
+                            mbar_wait(&sbar[warp][(k + j) % kDecStages], ((k + j) / kDecStages) & 1, A.status);
+                    }
                     dead = true;
                     break;
                 }

@@ -71,7 +71,7 @@ def make_run(wl, batch_dev, p, max_tokens=None):
     return GpuRun(wl, batch_dev, p, cc, dv, seq, [0] * B_, {}, ws)
 
 
-def compress(run: GpuRun, seq_host=None):
+def compress(run: GpuRun, seq_host=None, expect_bits=0):
     wl, p = run.wl, run.p
     Bn = wl.batch
     seq_host = [int(x) for x in (seq_host if seq_host is not None else run.seq_len.cpu().tolist())]
@@ -94,7 +94,7 @@ def compress(run: GpuRun, seq_host=None):
     B.kv2d_compress(p, Bn, seq_host, ce_before, run.dv, run.batch.qw, run.cc.struct, run.ws, d)
     torch.cuda.synchronize()
     bits = B.kv2d_read_status(run.ws)
-    assert bits == 0, f"device status bits {bits:#x}"
+    assert bits == expect_bits, f"device status bits {bits:#x}, expected {expect_bits:#x}"
     run.dbg = dict(dbg, ce_before=ce_before, seq_host=seq_host)
     run.comp_end_host = [ce_before[b] + (regions[b] // wl.segment_len) * wl.segment_len
                          for b in range(Bn)]
@@ -111,9 +111,90 @@ def unit_qw(run: GpuRun, b: int, h: int):
     return run.batch.qw[b, h * G:(h + 1) * G].reshape(G * W, d).cpu().numpy()
 
 
+def oracle_scores(orc, run: GpuRun, b: int, h: int, threads=None):
+    """The oracle's own a_d, lse and s_t of unit (b, h) for the latest
+    compress() call, scored one query head at a time on host threads: head
+    g's W window rows are an independent single-head problem over the same
+    keys (its rows' lse values are those of the full call, and s_t is the
+    sum over heads of each head's share).  Returns (a, lse[G*W], s[n])."""
+    wl, p = run.wl, run.p
+    po = oracle_params(orc, p)
+    T = run.dbg["seq_host"][b]
+    r0 = run.dbg["ce_before"][b]
+    G, W, d = wl.group, wl.window, wl.head_dim
+    K16, _ = unit_inputs(run, b, h, r0, T)
+    Kd = K16.astype(np.float64)
+    qw = unit_qw(run, b, h).astype(np.float64)
+    po1 = orc.params(d, 1, p.segment_len, W, p.keep_tokens, p.keep_channels,
+                     float(np.float32(p.budget)), float(np.float32(p.scale)))
+    parts = orc.parallel_map(lambda g: orc.score(po1, T, r0, Kd, qw[g * W:(g + 1) * W]),
+                             list(range(G)), threads=threads)
+    lse = np.concatenate([lp for lp, _ in parts])
+    s = np.zeros(T - r0)
+    for _, sp in parts:
+        s += sp
+    return orc.win_stats(po, qw), lse, s
+
+
+def check_scores(run: GpuRun, b: int, h: int, scores):
+    """a_d, lse and s_t of unit (b, h) against the oracle's (a, lse, s)."""
+    wl = run.wl
+    a_ref, lse_ref, s_ref = scores
+    u = b * wl.num_kv_heads + h
+    n = run.dbg["seq_host"][b] - run.dbg["ce_before"][b]
+    nS = (n // wl.segment_len) * wl.segment_len
+    a_gpu = run.dbg["a"][u].double().cpu().numpy()
+    s_gpu = run.dbg["s"][u, :nS].double().cpu().numpy()
+    lse_gpu = run.dbg["lse"][b, h * wl.group:(h + 1) * wl.group].reshape(-1).double().cpu().numpy()
+    assert np.max(np.abs(a_gpu - a_ref) / np.maximum(np.abs(a_ref), 1e-30)) < 1e-5
+    assert np.max(np.abs(lse_gpu - lse_ref) / np.maximum(1.0, np.abs(lse_ref))) < TOL_REL, \
+        f"lse mismatch {np.max(np.abs(lse_gpu - lse_ref))}"
+    s_seg = s_ref[:nS]
+    floor = 1e-6 * np.max(s_seg)
+    err = np.abs(s_gpu - s_seg) / np.maximum(np.abs(s_seg), floor)
+    assert np.max(err) < TOL_REL, f"s mismatch {np.max(err)} at {np.argmax(err)}"
+    return float(np.max(err))
+
+
+def end_to_end_unit(orc, run: GpuRun, b: int, h: int, scores, q: torch.Tensor):
+    """The fully independent end-to-end oracle for unit (b, h): the oracle's
+    own a_d and s_t (scores), its own selection and packing of the region of
+    the latest compress() call, and its decode of q over that arena plus the
+    unit's dense tail.  Returns (strategy agreement with the GPU as
+    (agreeing, total), max abs difference between the GPU's decode output
+    (out, fp16 [B][Hq][d] on the host) and the oracle's)."""
+    wl, p = run.wl, run.p
+    po = oracle_params(orc, p)
+    a_ref, _, s_ref = scores
+    T = run.dbg["seq_host"][b]
+    r0 = run.dbg["ce_before"][b]
+    S = wl.segment_len
+    u = b * wl.num_kv_heads + h
+    K16, V16 = unit_inputs(run, b, h, r0, T)
+    ref = orc.compress_unit(po, T, r0, K16, V16, unit_qw(run, b, h), a_in=a_ref, s_in=s_ref)
+    assert ref["status"] == 0
+    nseg = ref["nseg"]
+    desc = run.cc.desc[u].cpu().numpy().view(np.uint64)
+    seg0 = r0 // S
+    strat_gpu = ((desc[seg0:seg0 + nseg] >> np.uint64(32)) & np.uint64(255)).astype(np.int32)
+    agree = int(np.sum(strat_gpu == ref["strat"]))
+    # decode of q over the oracle's own arena (segments of this call) and the
+    # dense tail after them; only units compressed in one call are compared
+    assert r0 == 0, "end-to-end decode compares units compressed in one call"
+    Tn = int(run.seq_len[b])
+    ce = nseg * S
+    Kt, Vt = unit_inputs(run, b, h, ce, Tn)
+    G = wl.group
+    o_ref = orc.decode_unit(po, ref["arena"], ref["offs"], ref["strat"], Kt, Vt,
+                            q[b, h * G:(h + 1) * G].cpu().numpy())
+    return (agree, nseg), o_ref
+
+
 def check_compress_unit(orc, run: GpuRun, b: int, h: int, independent: bool = True,
-                        arena_before=None):
-    """Parity of one unit after the latest compress() call."""
+                        arena_before=None, scores=None):
+    """Parity of one unit after the latest compress() call.  With scores
+    (the oracle's (a, lse, s), e.g. from oracle_scores) those are compared
+    instead of scoring the unit again."""
     wl, p = run.wl, run.p
     po = oracle_params(orc, p)
     u = b * wl.num_kv_heads + h
@@ -132,7 +213,9 @@ def check_compress_unit(orc, run: GpuRun, b: int, h: int, independent: bool = Tr
     E_gpu = run.dbg["E"][u, :nseg].cpu().numpy()
     lse_gpu = run.dbg["lse"][b, h * wl.group:(h + 1) * wl.group].reshape(-1).double().cpu().numpy()
 
-    if independent:
+    if scores is not None:
+        check_scores(run, b, h, scores)
+    elif independent:
         a_ref = orc.win_stats(po, qw16.astype(np.float64))
         assert np.max(np.abs(a_gpu - a_ref) / np.maximum(np.abs(a_ref), 1e-30)) < 1e-5
         lse_ref, s_ref = orc.score(po, T, r0, K16.astype(np.float64), qw16.astype(np.float64))
@@ -168,7 +251,7 @@ def check_compress_unit(orc, run: GpuRun, b: int, h: int, independent: bool = Tr
 
 
 def gpu_decode(run: GpuRun, q: torch.Tensor, cc: B.CompressedCache | None = None,
-               max_seq=None):
+               max_seq=None, expect_bits=0):
     wl, p = run.wl, run.p
     cc = cc or run.cc
     out = torch.full((wl.batch, wl.num_q_heads, wl.head_dim), float("nan"),
@@ -177,7 +260,9 @@ def gpu_decode(run: GpuRun, q: torch.Tensor, cc: B.CompressedCache | None = None
     ws = B.workspace(B.kv2d_workspace_bytes(p, B.OP_DECODE, wl.batch, ms))
     B.kv2d_decode_attn(p, wl.batch, cc.struct, run.dv, run.seq_len, ms, q, out, ws)
     torch.cuda.synchronize()
-    assert B.kv2d_read_status(ws) == 0
+    bits = B.kv2d_read_status(ws)
+    if expect_bits is not None:
+        assert bits == expect_bits, f"device status bits {bits:#x}, expected {expect_bits:#x}"
     return out
 
 

@@ -177,3 +177,19 @@ def test_decode_table_cap_range(L):
             B.kv2d_set_decode_table_cap(bad)
     for good in (32, 4096, 0):
         B.kv2d_set_decode_table_cap(good)
+
+
+def test_noalloc_decode_rejects_oversize_before_launch(L):
+    """The scratch-array decode refuses, on the host, a shape whose scratch
+    would not fit its fixed array (8 MiB): 128 sequences x 64 KV heads with 8
+    query heads each need (8192 units + CTAs) x 8 x 132 x 4 bytes, about
+    35 MB.  The check runs before any CUDA call, so the fake pointers are
+    never used."""
+    lib = B.lib()
+    d = B.kv2d_dense(1 << 20, 2 << 20, 64 * 4096 * 128, 4096 * 128, 128, 4096, None, 0, 0, 0)
+    cc = _fake_cc()
+    big = B.params(128, 512, 64, 64, 64, 8, 32, 0.2)
+    rc = lib.kv2d_decode_attn_noalloc(C.byref(big), 128, C.byref(cc), C.byref(d), 1 << 22, 4096,
+                                      1 << 23, 1 << 24, None, None)
+    assert rc == 3
+    assert "scratch" in B.kv2d_last_error()

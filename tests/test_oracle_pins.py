@@ -135,6 +135,26 @@ def test_score_permutation_equivariance(orc):
     assert np.max(np.abs(s2 - s[perm])) < 1e-12
 
 
+def test_score_splits_by_query_head(orc):
+    """Each window row's softmax involves only its own query, so scoring the
+    G heads as G single-head problems gives the same lse rows, and s_t (a sum
+    over rows) is the sum of the heads' shares.  The full-size GPU tests rely
+    on this to score a large unit one head per host thread."""
+    rng = np.random.default_rng(3)
+    G, W, d, T, r0 = 4, 8, 128, 300, 64
+    K = f16(rng.standard_normal((T - r0, d))).astype(np.float64)
+    qw = f16(rng.standard_normal((G * W, d))).astype(np.float64)
+    p = orc.params(d, G, 16, W, 2, 32, 0.5)
+    lse, s = orc.score(p, T, r0, K, qw)
+    p1 = orc.params(d, 1, 16, W, 2, 32, 0.5)
+    s_sum = np.zeros_like(s)
+    for g in range(G):
+        lse_g, s_g = orc.score(p1, T, r0, K, qw[g * W:(g + 1) * W])
+        assert np.array_equal(lse_g, lse[g * W:(g + 1) * W])
+        s_sum += s_g
+    assert np.allclose(s_sum, s, rtol=1e-12, atol=0)
+
+
 def test_score_rejects_window_beyond_region(orc):
     p = orc.params(8, 1, 8, 10, 2, 2, 0.2)
     with pytest.raises(ValueError):
