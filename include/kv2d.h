@@ -257,19 +257,21 @@ KV2D_API kv2d_status kv2d_decode_attn(const kv2d_params* p, int batch, const kv2
  * interface convenience only.
  *   It takes no workspace.  Its per-CTA partials and per-unit tickets live
  *   in a fixed 8 MiB array in the library's own device memory, which every
- *   GPU that loads the library holds until the process exits.  The scratch
- *   a call needs is three regions, each rounded up to a multiple of 256
- *   bytes: 256 bytes, 4 bytes per unit, and (units + CTAs) x G x (d + 4) x 4
- *   bytes (CTAs <= the SM count); calls needing more than 8 MiB return
- *   KV2D_ERR_WORKSPACE before launching.
+ *   GPU that loads the library holds until the process exits.  Its layout
+ *   is the same for every call: a ticket per unit in a fixed 64 KiB region
+ *   (at most 16384 units, batch x Hkv), then the partials, (units + CTAs) x
+ *   G x (d + 4) x 4 bytes (CTAs <= the SM count) in the remaining
+ *   8 MiB - 64 KiB - 256 bytes; larger calls return KV2D_ERR_WORKSPACE
+ *   before launching.
  *   The first call on each device looks up the array's device address with
- *   the CUDA runtime (and makes the device's primary context current); make
- *   that first call outside any stream capture.  The address is kept per
- *   device together with the id of the context it belongs to, and looked up
- *   again when that context has changed (after cudaDeviceReset).
+ *   the CUDA runtime (which makes the device's primary context current) and
+ *   zeroes the ticket region with a synchronous cudaMemset; make that first
+ *   call outside any stream capture.  The address is kept per device
+ *   together with the id of the context it belongs to, and the set-up is
+ *   repeated when that context has changed (after cudaDeviceReset).
  *   All calls on a device share the one array and each leaves its partials
- *   behind; the array starts zeroed and every completed call leaves its
- *   per-unit tickets at zero again.  Calls whose
+ *   behind; every completed call leaves its per-unit tickets at zero again,
+ *   and no call writes anything else into the ticket region.  Calls whose
  *   kernels overlap on the GPU (two streams, or two host threads) race on the
  *   array and give wrong results: serialise them.
  *   status_dev: optional device uint32; device-side faults OR their

@@ -293,6 +293,14 @@ namespace {
 
 constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;   // 8 MiB per GPU
 constexpr int kNoAllocMaxDevices = 64;
+// Fixed layout, the same for every call: bytes [0, 256) are unused, the
+// per-unit tickets sit at [256, 256 + kNoAllocTicketBytes) and the per-CTA
+// partials after them.  The tickets must read zero when a call starts;
+// every completed call leaves the ones it used at zero, and no call ever
+// writes anything else there, whatever its shape.
+constexpr size_t kNoAllocTicketOff = 256;
+constexpr size_t kNoAllocTicketBytes = size_t(64) << 10;   // 16384 units
+constexpr size_t kNoAllocPartOff = kNoAllocTicketOff + kNoAllocTicketBytes;
 
 // Per device: the id of the context the address was looked up in, and the
 // address.  A device reset (cudaDeviceReset) ends that context and the
@@ -351,6 +359,11 @@ kv2d_status noalloc_scratch(void** out) {
             return fail(KV2D_ERR_CUDA, "cudaGetSymbolAddress of the decode scratch: %s",
                         cudaGetErrorString(e));
         if (!current_id(&id)) return fail(KV2D_ERR_CUDA, "cannot identify the current CUDA context");
+        // the tickets start at zero in a fresh context (one-time set-up,
+        // synchronous, before the array is first used)
+        e = cudaMemset(static_cast<uint8_t*>(ptr) + kNoAllocTicketOff, 0, kNoAllocTicketBytes);
+        if (e != cudaSuccess) return fail(KV2D_ERR_CUDA, "clearing the decode scratch tickets: %s",
+                                          cudaGetErrorString(e));
         slot.ctx_id = id;
         slot.ptr = ptr;
     }
@@ -719,15 +732,13 @@ kv2d_status kv2d_decode_attn_noalloc(const kv2d_params* p, int batch, const kv2d
     const int64_t units = static_cast<int64_t>(batch) * sh.Hkv;
     int kps = 0;
     const int nctas = decode_cta_count(static_cast<int>(units), max_seq_len_host, num_sms(), &kps);
-    Carver c;
-    c.take(256);                                               // status word
-    const size_t ticket_off = c.take(units * 4);
-    const size_t part_off = c.take((units + nctas) * sh.G * (kHeadDim + 4) * 4);
-    if (c.off > kNoAllocScratchBytes)
+    const size_t part_bytes = static_cast<size_t>(units + nctas) * sh.G * (kHeadDim + 4) * 4;
+    if (static_cast<size_t>(units) * 4 > kNoAllocTicketBytes || kNoAllocPartOff + part_bytes > kNoAllocScratchBytes)
         return fail(KV2D_ERR_WORKSPACE,
-                    "decode needs %zu bytes of scratch for %lld units on %d CTAs; the built-in "
-                    "scratch holds %zu bytes",
-                    c.off, static_cast<long long>(units), nctas, kNoAllocScratchBytes);
+                    "decode needs %zu bytes of scratch partials and %lld tickets for %lld units on %d "
+                    "CTAs; the built-in scratch holds %zu bytes of partials and %zu tickets",
+                    part_bytes, static_cast<long long>(units), static_cast<long long>(units), nctas,
+                    kNoAllocScratchBytes - kNoAllocPartOff, kNoAllocTicketBytes / 4);
     void* scratch = nullptr;
     if ((st = noalloc_scratch(&scratch)) != KV2D_OK) return st;
     uint8_t* w = static_cast<uint8_t*>(scratch);
@@ -749,8 +760,8 @@ kv2d_status kv2d_decode_attn_noalloc(const kv2d_params* p, int batch, const kv2d
     L.nctas = nctas;
     L.kps = kps;
     L.tbl_cap = g_dec_table_cap.load();
-    L.part = reinterpret_cast<float*>(w + part_off);
-    L.ticket = reinterpret_cast<uint32_t*>(w + ticket_off);   // left at zero by every call
+    L.part = reinterpret_cast<float*>(w + kNoAllocPartOff);
+    L.ticket = reinterpret_cast<uint32_t*>(w + kNoAllocTicketOff);   // left at zero by every call
     L.status = status_dev;   // NULL: device faults are not recorded anywhere
     cudaError_t e = launch_decode(L, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return fail(KV2D_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));

@@ -766,24 +766,40 @@ __device__ __forceinline__ void merge32_desc_f(float (&w)[32]) {
     }
 }
 
+// The key of channels 2e + {0, 1} of a 16-byte K chunk word: fp16 roundings
+// of the fp32 products |k_x| * a_x (a monotone function of the exact
+// product; see above).
+__device__ __forceinline__ __half2 key_pair(uint32_t w, float al, float ah) {
+    const float2 m = __half22float2(*reinterpret_cast<const __half2*>(&w));
+    return __floats2half2_rn(__fmul_rn(fabsf(m.x), al), __fmul_rn(fabsf(m.y), ah));
+}
+
 // Membership masks of one thread's 128 keys against v: bit x of M[x / 32]
-// is set iff key_x >= v, of Gt iff key_x > v.  ks[g][tid] holds the four key
-// registers of channels 8g..8g+7.  A compare yields 0xffff per half; one
-// AND-OR per register moves both flags to spare bit positions, and a final
-// shuffle puts each channel at its own bit.
-__device__ __forceinline__ void key_masks(const uint4 (*ks)[128], int tid, __half2 vv, uint32_t (&M)[4],
+// is set iff key_x >= v, of Gt iff key_x > v.  The keys are formed again
+// from the K row (the same operations as for the sort, so the same values)
+// rather than kept in shared memory, which leaves room for more resident
+// CTAs.  A compare yields 0xffff per half; one AND-OR per register moves
+// both flags to spare bit positions, and a final shuffle puts each channel
+// at its own bit.
+template <typename ChunkFn>
+__device__ __forceinline__ void key_masks(ChunkFn chunk, const float* af, __half2 vv, uint32_t (&M)[4],
                                           uint32_t (&Gt)[4]) {
 #pragma unroll
     for (int wd = 0; wd < 4; ++wd) {
         uint32_t lo = 0, hi = 0, glo = 0, ghi = 0;
 #pragma unroll
         for (int g4 = 0; g4 < 4; ++g4) {
-            const uint4 q = ks[wd * 4 + g4][tid];
+            const int gi = wd * 4 + g4;
+            const uint4 q = chunk(gi);
+            const float4 a0 = *reinterpret_cast<const float4*>(af + 8 * gi);
+            const float4 a1 = *reinterpret_cast<const float4*>(af + 8 * gi + 4);
             const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+            const float al[4] = {a0.x, a0.z, a1.x, a1.z};
+            const float ah[4] = {a0.y, a0.w, a1.y, a1.w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int s = g4 * 4 + e;        // channels 2s, 2s + 1 of this word
-                const __half2 kk = *reinterpret_cast<const __half2*>(&w[e]);
+                const __half2 kk = key_pair(w[e], al[e], ah[e]);
                 const uint32_t mk = __hge2_mask(kk, vv), gk = __hgt2_mask(kk, vv);
                 if (s < 8) {
                     const uint32_t bits = (1u << (2 * s)) | (1u << (2 * s + 17));
@@ -816,9 +832,15 @@ __device__ __forceinline__ double dfma_unless(double acc, double x, double y, ui
     return acc;
 }
 
+// An fp16 value (bits) widened to fp64 in one conversion (exact).
+__device__ __forceinline__ double h2d(uint16_t bits) {
+    double d;
+    asm("cvt.f64.f16 %0, %1;" : "=d"(d) : "h"(bits));
+    return d;
+}
+
 constexpr int kChanTile = 0;                  // 128 K rows, two 64-channel halves (SW128)
-constexpr int kChanKeys = kStage;             // uint4 [16][128]: the keys of each thread
-constexpr int kChanAf = kChanKeys + 32768;    // float [128]
+constexpr int kChanAf = kStage;               // float [128]
 constexpr int kChanAd = kChanAf + 512;        // double [128]
 constexpr int kChanBar = kChanAd + 1024;      // one mbarrier
 constexpr int kChanSmem = 1024 + kChanBar + 16;
@@ -828,13 +850,14 @@ constexpr int kChanSmem = 1024 + kChanBar + 16;
 // (row r, 16-byte chunk j of a 64-channel half at r * 128 + ((j ^ (r & 7))
 // << 4)), so the 8 threads of each quarter-warp read 8 different bank
 // groups.  K is never written by the kernels this one follows, so the
-// copy is issued before the wait on them and overlaps their tail.
+// copy is issued before the wait on them and overlaps their tail.  The
+// tile is the only large shared buffer (about 35 KB per CTA); at 96
+// registers five CTAs of 128 threads share an SM.
 __global__ void __launch_bounds__(128) chan_kernel_c32(const __grid_constant__ CUtensorMap kmap,
-                                                       const __grid_constant__ ChanArgs A) {
+                                                          const __grid_constant__ ChanArgs A) {
     extern __shared__ uint8_t chan_smem_raw[];
     uint8_t* sm = align1024(chan_smem_raw);
     uint8_t* tile = sm + kChanTile;
-    uint4 (*ks)[128] = reinterpret_cast<uint4 (*)[128]>(sm + kChanKeys);
     float* af = reinterpret_cast<float*>(sm + kChanAf);
     double* ad = reinterpret_cast<double*>(sm + kChanAd);
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + kChanBar);
@@ -869,9 +892,9 @@ __global__ void __launch_bounds__(128) chan_kernel_c32(const __grid_constant__ C
     auto chunk = [&](int j) {            // channels 8j .. 8j + 7
         return *reinterpret_cast<const uint4*>(myrow + (j >> 3) * 16384 + (((j & 7) ^ sw) << 4));
     };
-    auto kabs = [&](int x) {
-        const __half* p = reinterpret_cast<const __half*>(myrow + (x >> 6) * 16384 + ((((x >> 3) & 7) ^ sw) << 4));
-        return fabsf(__half2float(p[x & 7]));
+    auto kbits = [&](int x) {
+        const uint16_t* p = reinterpret_cast<const uint16_t*>(myrow + (x >> 6) * 16384 + ((((x >> 3) & 7) ^ sw) << 4));
+        return static_cast<uint16_t>(p[x & 7] & 0x7fffu);
     };
 
     __half2 srt[64];
@@ -880,18 +903,10 @@ __global__ void __launch_bounds__(128) chan_kernel_c32(const __grid_constant__ C
         const uint4 q = chunk(gi);
         const float4 a0 = *reinterpret_cast<const float4*>(af + 8 * gi);
         const float4 a1 = *reinterpret_cast<const float4*>(af + 8 * gi + 4);
-        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-        const float al[4] = {a0.x, a0.z, a1.x, a1.z};
-        const float ah[4] = {a0.y, a0.w, a1.y, a1.w};
-        uint32_t kw[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const float2 m = __half22float2(*reinterpret_cast<const __half2*>(&w[e]));
-            const __half2 kk = __floats2half2_rn(__fmul_rn(fabsf(m.x), al[e]), __fmul_rn(fabsf(m.y), ah[e]));
-            srt[4 * gi + e] = kk;
-            kw[e] = *reinterpret_cast<const uint32_t*>(&kk);
-        }
-        ks[gi][tid] = make_uint4(kw[0], kw[1], kw[2], kw[3]);
+        srt[4 * gi + 0] = key_pair(q.x, a0.x, a0.y);
+        srt[4 * gi + 1] = key_pair(q.y, a0.z, a0.w);
+        srt[4 * gi + 2] = key_pair(q.z, a1.x, a1.y);
+        srt[4 * gi + 3] = key_pair(q.w, a1.z, a1.w);
     }
     sort32_desc2<0>(srt);
     sort32_desc2<32>(srt);
@@ -918,26 +933,39 @@ __global__ void __launch_bounds__(128) chan_kernel_c32(const __grid_constant__ C
     }
     const __half2 vv = __float2half2_rn(vf);   // vf is a key value: exact in fp16
 
+    // the K tile is read again below; without this fence the compiler
+    // hoists those loads above the sort and keeps both live (160 registers
+    // instead of 96, three CTAs per SM instead of five)
     uint32_t M[4], G[4];
-    key_masks(ks, tid, vv, M, G);
+    asm volatile("" ::: "memory");
+    key_masks(chunk, af, vv, M, G);
     const int n_ge = __popc(M[0]) + __popc(M[1]) + __popc(M[2]) + __popc(M[3]);
     if (n_ge > c) {
         // the keys equal to v straddle the cut: keep the c - n_gt best of
-        // them by the exact product (e desc, x asc)
+        // them by (e desc, x asc).  The fp32 products f = fp32(|k| a) are
+        // correctly rounded, so f_y > f_x implies e_y > e_x; only equal f
+        // need the exact fp64 products.
         const int need = c - (__popc(G[0]) + __popc(G[1]) + __popc(G[2]) + __popc(G[3]));
         const uint32_t qm[4] = {M[0] & ~G[0], M[1] & ~G[1], M[2] & ~G[2], M[3] & ~G[3]};
         uint32_t keep[4] = {0, 0, 0, 0};
         for (int wi = 0; wi < 4; ++wi) {
             for (uint32_t m = qm[wi]; m; m &= m - 1) {
                 const int x = wi * 32 + __ffs(m) - 1;
-                const double ex = __dmul_rn(static_cast<double>(kabs(x)), ad[x]);
+                const double kx = h2d(kbits(x));
+                const float fx = __fmul_rn(static_cast<float>(kx), af[x]);
                 int rank = 0;
                 for (int wj = 0; wj < 4; ++wj) {
                     for (uint32_t m2 = qm[wj]; m2; m2 &= m2 - 1) {
                         const int y = wj * 32 + __ffs(m2) - 1;
                         if (y == x) continue;
-                        const double ey = __dmul_rn(static_cast<double>(kabs(y)), ad[y]);
-                        rank += (ey > ex) || (ey == ex && y < x);
+                        const double ky = h2d(kbits(y));
+                        const float fy = __fmul_rn(static_cast<float>(ky), af[y]);
+                        bool better = fy > fx;
+                        if (fy == fx) {
+                            const double ex = __dmul_rn(kx, ad[x]), ey = __dmul_rn(ky, ad[y]);
+                            better = (ey > ex) || (ey == ex && y < x);
+                        }
+                        rank += better;
                     }
                 }
                 if (rank < need) keep[wi] |= 1u << (x & 31);
@@ -947,21 +975,21 @@ __global__ void __launch_bounds__(128) chan_kernel_c32(const __grid_constant__ C
         for (int wi = 0; wi < 4; ++wi) M[wi] = G[wi] | keep[wi];
     }
 
-    // g_t: both fp64 sums ascending in x
+    // g_t: both fp64 sums ascending in x; |k| widened from fp16 in one
+    // conversion, and e = |k| a_x is exact in fp64, so each fused
+    // multiply-add rounds exactly as adding e does
     const int64_t slot = static_cast<int64_t>(u) * A.g_stride + t;
     double tot = 0.0, drop = 0.0;
 #pragma unroll 1
     for (int j = 0; j < 16; ++j) {
         const uint4 q = chunk(j);
         const uint32_t mw = ((j < 4) ? M[0] : (j < 8) ? M[1] : (j < 12) ? M[2] : M[3]) >> ((j & 3) * 8);
-        const uint32_t qw[4] = {q.x, q.y, q.z, q.w};
+        const uint32_t qw[4] = {q.x & 0x7fff7fffu, q.y & 0x7fff7fffu, q.z & 0x7fff7fffu, q.w & 0x7fff7fffu};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            const float2 f2 = __half22float2(__habs2(*reinterpret_cast<const __half2*>(&qw[e])));
             const double2 a2 = *reinterpret_cast<const double2*>(ad + 8 * j + 2 * e);
-            // e = |k| a_x is exact in fp64, so each fused multiply-add
-            // rounds exactly as adding e does
-            const double k0 = static_cast<double>(f2.x), k1 = static_cast<double>(f2.y);
+            const double k0 = h2d(static_cast<uint16_t>(qw[e] & 0xffffu));
+            const double k1 = h2d(static_cast<uint16_t>(qw[e] >> 16));
             tot = __fma_rn(k0, a2.x, tot);
             drop = dfma_unless(drop, k0, a2.x, mw, 1u << (2 * e));
             tot = __fma_rn(k1, a2.y, tot);
