@@ -521,14 +521,31 @@ kv2d_status kv2d_compress(const kv2d_params* p, int batch, const int32_t* seq_le
         }
         if (r != CUDA_SUCCESS) return fail(KV2D_ERR_CUDA, "key tensor map encode failed (%d)", int(r));
     }
-    // Grids fill whole waves: pass 1 runs two CTAs per SM, pass 2 one.
+    // Grids fill whole waves: pass 1 runs two CTAs per SM, pass 2 one.  A
+    // unit's keys are cut into ns splits so that the CTAs come as close as
+    // possible to a whole number of waves (few splits: each costs a
+    // pipeline fill and one lse partial per window row).
     const int nsm = num_sms();
     const int mtiles = sh.GWpad / 128;
+    auto pick_splits = [](int64_t groups, int64_t slots, int64_t max_ns) {
+        int64_t best = 1;
+        double best_eff = 0.0;
+        for (int64_t ns = 1; ns <= max_ns; ++ns) {
+            const int64_t ctas = groups * ns;
+            const int64_t waves = (ctas + slots - 1) / slots;
+            const double eff = static_cast<double>(ctas) / static_cast<double>(waves * slots);
+            if (eff > best_eff + 0.02) {
+                best_eff = eff;
+                best = ns;
+            }
+            if (eff >= 0.97 && ctas >= slots) break;
+        }
+        return best;
+    };
     {
         const int64_t max_tiles = (max_region + kKeyTile - 1) / kKeyTile;
-        const int groups = units * mtiles;
-        int64_t ns = std::max(1, (2 * nsm) / groups);
-        ns = std::max<int64_t>(1, std::min<int64_t>({ns, max_tiles, static_cast<int64_t>(kMaxSplit1)}));
+        const int64_t groups = static_cast<int64_t>(units) * mtiles;
+        const int64_t ns = pick_splits(groups, 2 * nsm, std::min<int64_t>(max_tiles, kMaxSplit1));
         const int64_t tiles_per = (max_tiles + ns - 1) / ns;
         SL.kps1 = static_cast<int>(tiles_per * kKeyTile);
         SL.nsplit1 = static_cast<int>((max_tiles + tiles_per - 1) / tiles_per);
@@ -536,8 +553,7 @@ kv2d_status kv2d_compress(const kv2d_params* p, int batch, const int32_t* seq_le
     {
         const int64_t seg_tok = static_cast<int64_t>(max_nseg) * sh.S;
         const int64_t max_tiles = (seg_tok + kKeyTile - 1) / kKeyTile;
-        int64_t ns = std::max(1, nsm / units);
-        ns = std::max<int64_t>(1, std::min<int64_t>(ns, max_tiles));
+        const int64_t ns = pick_splits(units, nsm, std::min<int64_t>(max_tiles, 256));
         const int64_t tiles_per = (max_tiles + ns - 1) / ns;
         SL.kps2 = static_cast<int>(tiles_per * kKeyTile);
         SL.nsplit2 = static_cast<int>((max_tiles + tiles_per - 1) / tiles_per);

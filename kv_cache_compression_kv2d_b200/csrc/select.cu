@@ -26,8 +26,12 @@ namespace kv2d {
 
 namespace {
 
-constexpr int kSegWarps = 32;   // segments per CTA (one warp each, then one lane each; <= 32)
-static_assert(kSegWarps <= 32, "phases 2 and 3 give each segment one lane of a warp");
+// Segments per CTA (one warp each, then one lane each).  Small CTAs: the
+// sequential phases 2 and 3 keep only three warps (then one) busy, so eight
+// CTAs of 8 warps per SM overlap one CTA's sequential phase with the
+// others' ranking.
+constexpr int kSegWarps = 8;
+static_assert(kSegWarps >= 3 && kSegWarps <= 32, "phase 2 needs three warps; phases 2 and 3 give each segment one lane");
 
 struct SegArgs {
     SeqPlan plan;
@@ -70,10 +74,10 @@ __global__ void __launch_bounds__(kSegWarps * 32) seg_select_kernel(const __grid
     const int jb = blockIdx.x * kSegWarps;
     if (jb >= nseg) return;
     const int S = A.S, r = A.r, RW = seg_row(S);
-    double* sgs = reinterpret_cast<double*>(seg_smem);                      // [32][RW]
-    double* sums = sgs + kSegWarps * RW;                                    // [3][32]
-    float* ss = reinterpret_cast<float*>(sums + 3 * kSegWarps);             // [32][RW]
-    uint8_t* kept = reinterpret_cast<uint8_t*>(ss + kSegWarps * RW);        // [32][RW]
+    double* sgs = reinterpret_cast<double*>(seg_smem);                      // [kSegWarps][RW]
+    double* sums = sgs + kSegWarps * RW;                                    // [3][kSegWarps]
+    float* ss = reinterpret_cast<float*>(sums + 3 * kSegWarps);             // [kSegWarps][RW]
+    uint8_t* kept = reinterpret_cast<uint8_t*>(ss + kSegWarps * RW);        // [kSegWarps][RW]
 
     const int j = jb + warp;
     if (j < nseg) {
@@ -117,6 +121,7 @@ __global__ void __launch_bounds__(kSegWarps * 32) seg_select_kernel(const __grid
         const double* grow = sgs + lane * RW;
         const float* srow = ss + lane * RW;
         const uint8_t* krow = kept + lane * RW;
+#pragma unroll 8
         for (int t = 0; t < S; ++t) {
             const bool kp = krow[t] != 0;
             if (warp == 0) acc = __dadd_rn(acc, grow[t]);
