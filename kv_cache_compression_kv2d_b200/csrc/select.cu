@@ -5,7 +5,8 @@
 // generation) chooses one compression pattern per KV-cache segment.  The
 // pages define no criterion; this library reads it as minimising lost
 // attention mass under a byte budget:
-//   seg_select (one warp per segment):
+//   seg_select (one thread per segment for r in {4, 8, 16}, S <= 128;
+//   otherwise one warp per segment):
 //     R_j = top-r tokens by s_t (ties to the lower token), ascending;
 //     E_FULL = 0, E_TOK = sum_{t not in R} s_t, E_CH = sum_t s_t g_t,
 //     E_BOTH = E_TOK + sum_{t in R} s_t g_t        (fp64, ascending t);
@@ -58,6 +59,55 @@ __host__ __device__ constexpr int seg_row(int S) { return S + 1; }
 inline int seg_smem_bytes(int S) {
     return kSegWarps * seg_row(S) * (8 + 4 + 1) + 3 * kSegWarps * 8 + 16;
 }
+
+// The error proxies of segment js of unit u from its three sums, written
+// out, and the lower convex hull of its options over (bytes, E).
+__device__ __forceinline__ void finish_segment(const SegArgs& A, int u, int js, double ech, double ekept,
+                                               double etok) {
+    const int64_t slot = static_cast<int64_t>(u) * A.max_nseg + js;
+    double E[4];
+    E[KV2D_FULL] = 0.0;
+    E[KV2D_TOK] = etok;
+    E[KV2D_CH] = ech;
+    E[KV2D_BOTH] = __dadd_rn(etok, ekept);
+    for (int k = 0; k < 4; ++k) A.E[slot * 4 + k] = E[k];
+    if (A.dbg_E)
+        for (int k = 0; k < 4; ++k)
+            A.dbg_E[(static_cast<int64_t>(u) * A.dbg_seg_stride + js) * 4 + k] = E[k];
+    // lower convex hull over (bytes, E), options visited by (bytes, id)
+    int hv[4];
+    int nh = 0;
+    hv[nh++] = A.order[0];
+    for (int i = 1; i < 4; ++i) {
+        const int o = A.order[i];
+        const int last = hv[nh - 1];
+        if (E[o] >= E[last]) continue;
+        if (A.bytes[o] == A.bytes[last]) {
+            hv[nh - 1] = o;
+            continue;
+        }
+        while (nh >= 2) {
+            const int pa = hv[nh - 2], pb = hv[nh - 1];
+            const double lhs = __dmul_rn(__dsub_rn(E[pa], E[pb]),
+                                         static_cast<double>(A.bytes[o] - A.bytes[pb]));
+            const double rhs = __dmul_rn(__dsub_rn(E[pb], E[o]),
+                                         static_cast<double>(A.bytes[pb] - A.bytes[pa]));
+            if (lhs <= rhs) --nh;
+            else break;
+        }
+        hv[nh++] = o;
+    }
+    uint8_t* H = A.hull + slot * 8;
+    H[0] = static_cast<uint8_t>(nh);
+    for (int k = 0; k < 4; ++k) H[1 + k] = static_cast<uint8_t>(k < nh ? hv[k] : 0);
+    for (int k = 1; k < nh; ++k) {
+        const int64_t db = A.bytes[hv[k]] - A.bytes[hv[k - 1]];
+        A.dbytes[slot * 3 + k - 1] = static_cast<int32_t>(db);
+        A.eff[slot * 3 + k - 1] =
+            __ddiv_rn(__dsub_rn(E[hv[k - 1]], E[hv[k]]), static_cast<double>(db));
+    }
+}
+
 
 // Phase 1, one warp per segment: R_j by rank counting (two tokens per lane
 // and pass), tidx, kept flags, and the products s_t g_t.  Phase 2, one lane
@@ -132,51 +182,160 @@ __global__ void __launch_bounds__(kSegWarps * 32) seg_select_kernel(const __grid
     }
     __syncthreads();
     if (warp != 0 || lane >= kSegWarps || jb + lane >= nseg) return;
-    const int js = jb + lane;
-    const int64_t slot = static_cast<int64_t>(u) * A.max_nseg + js;
-    const double ech = sums[lane], ekept = sums[kSegWarps + lane], etok = sums[2 * kSegWarps + lane];
-    double E[4];
-    E[KV2D_FULL] = 0.0;
-    E[KV2D_TOK] = etok;
-    E[KV2D_CH] = ech;
-    E[KV2D_BOTH] = __dadd_rn(etok, ekept);
-    for (int k = 0; k < 4; ++k) A.E[slot * 4 + k] = E[k];
-    if (A.dbg_E)
-        for (int k = 0; k < 4; ++k)
-            A.dbg_E[(static_cast<int64_t>(u) * A.dbg_seg_stride + js) * 4 + k] = E[k];
+    finish_segment(A, u, jb + lane, sums[lane], sums[kSegWarps + lane], sums[2 * kSegWarps + lane]);
+}
 
-    // lower convex hull over (bytes, E), options visited by (bytes, id)
-    int hv[4];
-    int nh = 0;
-    hv[nh++] = A.order[0];
-    for (int i = 1; i < 4; ++i) {
-        const int o = A.order[i];
-        const int last = hv[nh - 1];
-        if (E[o] >= E[last]) continue;
-        if (A.bytes[o] == A.bytes[last]) {
-            hv[nh - 1] = o;
-            continue;
+// One thread per segment, for r a power of two in {4, 8, 16} with S <= 128
+// (the default shapes: S = 64, r = 8 and S = 128, r = 16).  A warp stages
+// the s_t and g_t of its 32 consecutive segments (contiguous in memory)
+// through shared memory with coalesced 16-byte loads; rows are padded so
+// that each thread's 16-byte reads of its own row hit distinct bank groups.
+// Top-r: each token becomes one 64-bit key, bits(s_t) << 8 | (255 - t),
+// which orders by s_t (non-negative, so its bits are monotone) and then by
+// the lower t; read as an fp64 number the key is a positive subnormal whose
+// order is the key's, so fmax / fmin sort it exactly (min / max return one
+// of their operands).  Groups of R keys are sorted by a bitonic network and
+// merged into the running R largest (max against the reversed group, then
+// a bitonic merge).  Then the three sums in ascending t and the hull, as in
+// the general kernel.
+constexpr int kSmallSegs = 32;
+
+template <int N>
+__device__ __forceinline__ void bitonic_sort_desc(double (&v)[N]) {
+#pragma unroll
+    for (int k = 2; k <= N; k <<= 1) {
+#pragma unroll
+        for (int j = k >> 1; j > 0; j >>= 1) {
+#pragma unroll
+            for (int i = 0; i < N; ++i) {
+                const int l = i ^ j;
+                if (l > i) {
+                    const double hi = fmax(v[i], v[l]), lo = fmin(v[i], v[l]);
+                    v[i] = (i & k) == 0 ? hi : lo;
+                    v[l] = (i & k) == 0 ? lo : hi;
+                }
+            }
         }
-        while (nh >= 2) {
-            const int pa = hv[nh - 2], pb = hv[nh - 1];
-            const double lhs = __dmul_rn(__dsub_rn(E[pa], E[pb]),
-                                         static_cast<double>(A.bytes[o] - A.bytes[pb]));
-            const double rhs = __dmul_rn(__dsub_rn(E[pb], E[o]),
-                                         static_cast<double>(A.bytes[pb] - A.bytes[pa]));
-            if (lhs <= rhs) --nh;
-            else break;
+    }
+}
+
+template <int N>
+__device__ __forceinline__ void bitonic_merge_desc(double (&v)[N]) {
+#pragma unroll
+    for (int j = N >> 1; j > 0; j >>= 1) {
+#pragma unroll
+        for (int i = 0; i < N; ++i) {
+            const int l = i ^ j;
+            if (l > i) {
+                const double hi = fmax(v[i], v[l]), lo = fmin(v[i], v[l]);
+                v[i] = hi;
+                v[l] = lo;
+            }
         }
-        hv[nh++] = o;
     }
-    uint8_t* H = A.hull + slot * 8;
-    H[0] = static_cast<uint8_t>(nh);
-    for (int k = 0; k < 4; ++k) H[1 + k] = static_cast<uint8_t>(k < nh ? hv[k] : 0);
-    for (int k = 1; k < nh; ++k) {
-        const int64_t db = A.bytes[hv[k]] - A.bytes[hv[k - 1]];
-        A.dbytes[slot * 3 + k - 1] = static_cast<int32_t>(db);
-        A.eff[slot * 3 + k - 1] =
-            __ddiv_rn(__dsub_rn(E[hv[k - 1]], E[hv[k]]), static_cast<double>(db));
+}
+
+inline int seg_small_smem_bytes(int S) { return kSmallSegs * ((S + 4) * 4 + (S + 2) * 8); }
+
+template <int R>
+__global__ void __launch_bounds__(kSmallSegs) seg_select_small_kernel(const __grid_constant__ SegArgs A) {
+    pdl_wait();
+    extern __shared__ __align__(16) uint8_t seg_smem[];
+    const int lane = threadIdx.x;
+    const int u = blockIdx.y;
+    const int b = u / A.Hkv;
+    const int nseg = A.plan.nseg[b];
+    const int jb = blockIdx.x * kSmallSegs;
+    if (jb >= nseg) return;
+    const int S = A.S, SR = S + 4, GR = S + 2;
+    float* srows = reinterpret_cast<float*>(seg_smem);                          // [32][S + 4]
+    double* grows = reinterpret_cast<double*>(srows + kSmallSegs * SR);         // [32][S + 2]
+    const int nv = min(kSmallSegs, nseg - jb);
+    {
+        const float4* s4 = reinterpret_cast<const float4*>(A.s + static_cast<int64_t>(u) * A.s_stride +
+                                                           static_cast<int64_t>(jb) * S);
+        const int q4 = S / 4, n4 = nv * q4;
+        for (int i = lane; i < n4; i += kSmallSegs)
+            *reinterpret_cast<float4*>(srows + (i / q4) * SR + 4 * (i % q4)) = s4[i];
+        const double2* g2 = reinterpret_cast<const double2*>(A.g + static_cast<int64_t>(u) * A.g_stride +
+                                                             static_cast<int64_t>(jb) * S);
+        const int q2 = S / 2, n2 = nv * q2;
+        for (int i = lane; i < n2; i += kSmallSegs)
+            *reinterpret_cast<double2*>(grows + (i / q2) * GR + 2 * (i % q2)) = g2[i];
     }
+    __syncwarp();
+    if (lane >= nv) return;
+    const int js = jb + lane;
+    const float* srow = srows + lane * SR;
+    const double* grow = grows + lane * GR;
+    auto key_of = [&](float sv, int t) {
+        return __longlong_as_double(static_cast<long long>(
+            (static_cast<uint64_t>(__float_as_uint(sv)) << 8) | static_cast<uint64_t>(255 - t)));
+    };
+    double top[R];
+    for (int g0 = 0; g0 < S; g0 += R) {
+        double cur[R];
+#pragma unroll
+        for (int i = 0; i < R; i += 4) {
+            const float4 v4 = *reinterpret_cast<const float4*>(srow + g0 + i);
+            cur[i] = key_of(v4.x, g0 + i);
+            cur[i + 1] = key_of(v4.y, g0 + i + 1);
+            cur[i + 2] = key_of(v4.z, g0 + i + 2);
+            cur[i + 3] = key_of(v4.w, g0 + i + 3);
+        }
+        bitonic_sort_desc<R>(cur);
+        if (g0 == 0) {
+#pragma unroll
+            for (int i = 0; i < R; ++i) top[i] = cur[i];
+        } else {
+#pragma unroll
+            for (int i = 0; i < R; ++i) top[i] = fmax(top[i], cur[R - 1 - i]);
+            bitonic_merge_desc<R>(top);
+        }
+    }
+    // kept tokens as a 128-bit mask, then tidx ascending
+    uint64_t k0 = 0, k1 = 0;
+#pragma unroll
+    for (int i = 0; i < R; ++i) {
+        const int t = 255 - static_cast<int>(__double_as_longlong(top[i]) & 255);
+        if (t < 64) k0 |= 1ull << t;
+        else k1 |= 1ull << (t - 64);
+    }
+    const int64_t slot = static_cast<int64_t>(u) * A.max_nseg + js;
+    {
+        uint64_t m0 = k0, m1 = k1;
+#pragma unroll
+        for (int i = 0; i < R; ++i) {
+            int t;
+            if (m0) {
+                t = __ffsll(static_cast<long long>(m0)) - 1;
+                m0 &= m0 - 1;
+            } else {
+                t = 64 + __ffsll(static_cast<long long>(m1)) - 1;
+                m1 &= m1 - 1;
+            }
+            A.tidx[slot * R + i] = static_cast<uint8_t>(t);
+        }
+    }
+    // the three fp64 sums in ascending t (products and sums rounded once)
+    double ech = 0.0, ekept = 0.0, etok = 0.0;
+    for (int t0 = 0; t0 < S; t0 += 4) {
+        const float4 v4 = *reinterpret_cast<const float4*>(srow + t0);
+        const double2 ga = *reinterpret_cast<const double2*>(grow + t0);
+        const double2 gb = *reinterpret_cast<const double2*>(grow + t0 + 2);
+        const float sv[4] = {v4.x, v4.y, v4.z, v4.w};
+        const double gv[4] = {ga.x, ga.y, gb.x, gb.y};
+        const uint64_t kw = (t0 < 64) ? (k0 >> t0) : (k1 >> (t0 - 64));
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const double sd = static_cast<double>(sv[e]);
+            const double p = __dmul_rn(sd, gv[e]);
+            ech = __dadd_rn(ech, p);
+            if ((kw >> e) & 1) ekept = __dadd_rn(ekept, p);
+            else etok = __dadd_rn(etok, sd);
+        }
+    }
+    finish_segment(A, u, js, ech, ekept, etok);
 }
 
 // ---------------------------------------------------------------- budget
@@ -508,13 +667,26 @@ cudaError_t launch_selection(const SelectLaunch& L, cudaStream_t stream) {
         sa.dbytes = L.dbytes;
         sa.dbg_E = L.dbg_E;
         sa.dbg_seg_stride = L.dbg_seg_stride;
-        dim3 grid((L.max_nseg + kSegWarps - 1) / kSegWarps, units);
-        const int sm_bytes = seg_smem_bytes(sa.S);
-        cudaError_t e0 = cudaFuncSetAttribute(seg_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, sm_bytes);
-        if (e0 != cudaSuccess) return e0;
+        const int r = sa.r;
+        const bool small = sa.S <= 128 && (r == 4 || r == 8 || r == 16) && sa.S % r == 0;
         prof_begin(stream, kProfSegSelect);
-        cudaError_t e1 = launch_k(seg_select_kernel, grid, dim3(kSegWarps * 32), sm_bytes, stream, sa);
-        if (e1 != cudaSuccess) return e1;
+        if (small) {
+            dim3 grid((L.max_nseg + kSmallSegs - 1) / kSmallSegs, units);
+            const int sm_bytes = seg_small_smem_bytes(sa.S);
+            auto kern = r == 4 ? seg_select_small_kernel<4> : r == 8 ? seg_select_small_kernel<8>
+                                                                      : seg_select_small_kernel<16>;
+            cudaError_t e0 = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, sm_bytes);
+            if (e0 != cudaSuccess) return e0;
+            cudaError_t e1 = launch_k(kern, grid, dim3(kSmallSegs), sm_bytes, stream, sa);
+            if (e1 != cudaSuccess) return e1;
+        } else {
+            dim3 grid((L.max_nseg + kSegWarps - 1) / kSegWarps, units);
+            const int sm_bytes = seg_smem_bytes(sa.S);
+            cudaError_t e0 = cudaFuncSetAttribute(seg_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, sm_bytes);
+            if (e0 != cudaSuccess) return e0;
+            cudaError_t e1 = launch_k(seg_select_kernel, grid, dim3(kSegWarps * 32), sm_bytes, stream, sa);
+            if (e1 != cudaSuccess) return e1;
+        }
         prof_end(stream, kProfSegSelect);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;

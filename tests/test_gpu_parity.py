@@ -249,6 +249,23 @@ def test_channel_ties_parity(orc, keep_channels):
     _check_decode(orc, run)
 
 
+@pytest.mark.parametrize("keep_tokens", [3, 4, 8, 16])
+def test_token_ties_parity(orc, keep_tokens):
+    """Window queries of zero give every visible key the same logit, so the
+    token masses of all keys that every window row sees are equal: the top-r
+    of each segment is decided by the tie rule alone (lower token first),
+    and the zero channel weights make every channel tie as well (lower
+    channel first).  Covers both segment-select kernels (r = 3 runs the
+    warp-per-segment one, r = 4, 8, 16 the thread-per-segment one)."""
+    wl = Workload("token_ties", 2, 1, 4, 128, 1280, 64, 32, 0.3, ragged_min=900)
+    batch = synth.generate(wl, seed=4)
+    batch.qw.zero_()
+    run = H.make_run(wl, H.to_device(batch), H.params_for(wl, keep_tokens=keep_tokens))
+    H.compress(run)
+    _check_all_units(orc, run, independent=True)
+    _check_decode(orc, run)
+
+
 @pytest.mark.parametrize("cap", [32, 41])
 def test_decode_block_table_in_chunks(orc, cap):
     """With more units than half the SMs the batch's bytes are shared out
