@@ -284,9 +284,6 @@ __global__ void __launch_bounds__(kPassThreads, 1)
 
 // --------------------------------------------------------------- pass 2
 
-constexpr int kP2Threads = 576;      // 16 epilogue warps, 1 TMA warp, 1 MMA warp
-constexpr int kP2Epi = 512;          // epilogue threads (4 warpgroups)
-
 struct Pass2Args {
     SeqPlan plan;
     UnitShape shp;
@@ -303,15 +300,7 @@ struct Pass2Args {
     uint32_t* status;
 };
 
-// TMEM holds nbuf accumulator buffers of GWpad columns (two when GWpad <=
-// 256, else one of 512); column c of a buffer is window row c.  The four
-// epilogue warpgroups share the buffers: with two buffers, warpgroups 2b
-// and 2b + 1 take the two column halves of buffer b (tiles b, b + 2, ...);
-// with one, each warpgroup takes a quarter of every tile.  A thread owns one
-// key (TMEM lane) and sums exp2 over its columns; the partial sums of the
-// warpgroups sharing a buffer are added in column order through shared
-// memory.
-__global__ void __launch_bounds__(kP2Threads, 1)
+__global__ void __launch_bounds__(kPassThreads, 1)
     score_pass2_kernel(const __grid_constant__ CUtensorMap qmap,
                        const __grid_constant__ CUtensorMap kmap, const __grid_constant__ Pass2Args A) {
     const int sp = blockIdx.x, u = blockIdx.y;
@@ -325,10 +314,8 @@ __global__ void __launch_bounds__(kP2Threads, 1)
     if (nt == 0) return;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int NS = A.nstages, nqc = A.nqc, Nc = A.Nc;
-    const int nbuf = (GWpad <= 256) ? 2 : 1;
-    const int wpb = 4 / nbuf;                    // warpgroups per buffer
-    const int cpw = GWpad / wpb;                 // columns per warpgroup
-    const uint32_t ncols = 512u;
+    const bool split_cols = (nqc == 2);          // both WGs on every tile
+    const uint32_t ncols = split_cols ? 512u : (Nc == 256 ? 512u : 256u);
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
@@ -336,8 +323,8 @@ __global__ void __launch_bounds__(kP2Threads, 1)
     uint8_t* k_s = smem + GWpad * 256;
     float* lse_s = reinterpret_cast<float*>(k_s + NS * kStage);
     int* wpos_s = reinterpret_cast<int*>(lse_s + GWpad);
-    float* sb = reinterpret_cast<float*>(wpos_s + GWpad);          // [4][128] partial sums
-    uint64_t* full = reinterpret_cast<uint64_t*>(sb + 4 * 128);
+    float* sb = reinterpret_cast<float*>(wpos_s + GWpad);
+    uint64_t* full = reinterpret_cast<uint64_t*>(sb + 128);
     uint64_t* empty = full + 4;
     uint64_t* tfull = empty + 4;
     uint64_t* tempty = tfull + 2;
@@ -351,19 +338,19 @@ __global__ void __launch_bounds__(kP2Threads, 1)
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&tfull[i], 1);
-            mbar_init(&tempty[i], 128 * wpb);
+            mbar_init(&tempty[i], split_cols ? 256 : 128);
         }
         mbar_init(qbar, 1);
         mbar_fence_init();
     }
-    if (warp == 17) {
+    if (warp == 9) {
         tmem_alloc(tmem_slot, ncols);
         tmem_relinquish();
     }
     pdl_wait();
     // lse of every window row: merge the pass-1 split partials in split order
     // (padded rows get +inf so that they weigh nothing)
-    for (int i = tid; i < GWpad; i += kP2Threads) {
+    for (int i = tid; i < GWpad; i += kPassThreads) {
         float out = __int_as_float(0x7f800000);
         if (i < A.shp.GW) {
             const float2* p = A.part + (static_cast<int64_t>(u) * GWpad + i) * A.nsplit1;
@@ -396,7 +383,7 @@ __global__ void __launch_bounds__(kP2Threads, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 16) {
+    if (warp == 8) {
         if (lane == 0) {
             tma_prefetch_desc(&qmap);
             tma_prefetch_desc(&kmap);
@@ -415,20 +402,24 @@ __global__ void __launch_bounds__(kP2Threads, 1)
                               k_lo + i * kKeyTile, T, A.status);
             }
         }
-    } else if (warp == 17) {
+    } else if (warp == 9) {
         if (lane == 0) {
             const uint32_t idesc = idesc_f16_f32(128, Nc);
             const uint32_t qa = smem_u32(q_s);
             bool ok = mbar_wait(qbar, 0, A.status);
             for (int i = 0; ok && i < nt; ++i) {
                 const int s = i % NS;
-                const int buf = i % nbuf, k = i / nbuf;
+                const int buf = split_cols ? 0 : (i & 1);
                 if (!mbar_wait(&full[s], (i / NS) & 1, A.status)) break;
-                if (k >= 1 && !mbar_wait(&tempty[buf], (k - 1) & 1, A.status)) break;
+                if (split_cols) {
+                    if (i >= 1 && !mbar_wait(&tempty[0], (i - 1) & 1, A.status)) break;
+                } else if (i >= 2 && !mbar_wait(&tempty[buf], ((i >> 1) - 1) & 1, A.status)) {
+                    break;
+                }
                 tc_fence_after();
                 const uint32_t ka = smem_u32(k_s + s * kStage);
                 for (int qc = 0; qc < nqc; ++qc) {
-                    const uint32_t dcol = buf * GWpad + qc * Nc;
+                    const uint32_t dcol = split_cols ? qc * Nc : buf * Nc;
                     const uint32_t qb = qa + qc * Nc * 256;
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk) {
@@ -443,21 +434,22 @@ __global__ void __launch_bounds__(kP2Threads, 1)
             }
         }
     } else {
-        // epilogue: thread <-> key (TMEM lane), loop over its query columns
+        // epilogue: thread <-> key (TMEM lane), loop over query columns.
         const int wg = warp >> 2, lg = warp & 3;
         const int row = lg * 32 + lane;
-        const int buf = (nbuf == 2) ? (wg >> 1) : 0;
-        const int part = (nbuf == 2) ? (wg & 1) : wg;
-        const int col0 = part * cpw;
         const float c2 = A.shp.c2;
         const int tw = T - W;                 // keys <= tw are seen by every row
-        float* sbb = sb + (buf * wpb) * 128;  // this buffer's partial sums
-        for (int i = buf; i < nt; i += nbuf) {
-            const int k = i / nbuf;
+        const int step = split_cols ? 1 : 2;
+        for (int i = split_cols ? 0 : wg; i < nt; i += step) {
+            const int buf = split_cols ? 0 : wg;
+            const int k = split_cols ? i : (i >> 1);
             if (!mbar_wait(&tfull[buf], k & 1, A.status)) break;
             tc_fence_after();
             const int t = k_lo + i * kKeyTile + row;
-            const uint32_t taddr = tmem + (static_cast<uint32_t>(lg * 32) << 16) + buf * GWpad + col0;
+            const int qc = split_cols ? wg : 0;
+            const uint32_t taddr = tmem + (static_cast<uint32_t>(lg * 32) << 16) +
+                                   (split_cols ? qc * Nc : buf * Nc);
+            const int col0 = qc * Nc;
             const int need = t - tw;          // row visible iff wpos >= need
             float sacc = 0.f;
             // 32-column chunks, double-buffered: chunk c+1's TMEM load is in
@@ -485,7 +477,7 @@ __global__ void __launch_bounds__(kP2Threads, 1)
                 sacc += (a0 + a1) + (a2 + a3);
             };
             uint32_t ra[32], rb[32];
-            const int nch = cpw / 32;         // 2 or 4 chunks
+            const int nch = Nc / 32;          // 4, 6 or 8 chunks (Nc 128..256)
             tmem_ld32(taddr, ra);
             tmem_ld_wait(ra);
 #pragma unroll 1
@@ -500,25 +492,24 @@ __global__ void __launch_bounds__(kP2Threads, 1)
                 }
             }
             tc_fence_before();
-            // the buffer's partial sums, added in column order by its first
-            // warpgroup
-            if (part > 0) sbb[part * 128 + row] = sacc;
-            named_bar_sync(1 + buf, 128 * wpb);
-            if (part == 0)
-                for (int q = 1; q < wpb; ++q) sacc = sacc + sbb[q * 128 + row];
+            if (split_cols) {
+                if (wg == 1) sb[row] = sacc;
+                named_bar_sync(1, 256);
+                if (wg == 0) sacc = sacc + sb[row];
+                named_bar_sync(2, 256);
+            }
             mbar_arrive(&tempty[buf]);
-            if (part == 0 && t < k_hi) {
+            if ((!split_cols || wg == 0) && t < k_hi) {
                 const int64_t rel = t - r0;
                 A.s[static_cast<int64_t>(u) * A.s_stride + rel] = sacc;
                 if (A.dbg_s) A.dbg_s[static_cast<int64_t>(u) * A.dbg_stride + rel] = sacc;
             }
-            named_bar_sync(3 + buf, 128 * wpb);   // sbb is free again
         }
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 17) tmem_dealloc(tmem, ncols);
+    if (warp == 9) tmem_dealloc(tmem, ncols);
 }
 
 // ------------------------------------------------- channel top-c and g_t
@@ -1021,7 +1012,7 @@ int score_pass1_smem_bytes() {
 
 int score_pass2_smem_bytes(int gwpad) {
     const int ns = gwpad <= 256 ? 4 : 2;
-    return 1024 + gwpad * 256 + ns * kStage + gwpad * 8 + 4 * 128 * 4 + 256;
+    return 1024 + gwpad * 256 + ns * kStage + gwpad * 8 + 512 + 256;
 }
 
 cudaError_t launch_scoring(const ScoreLaunch& L, cudaStream_t stream) {
@@ -1071,7 +1062,7 @@ cudaError_t launch_scoring(const ScoreLaunch& L, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     dim3 g2(L.nsplit2, units);
     prof_begin(stream, kProfPass2);
-    e = launch_k(score_pass2_kernel, g2, dim3(kP2Threads), smem2, stream, L.qmap, L.kmap, p2);
+    e = launch_k(score_pass2_kernel, g2, dim3(kPassThreads), smem2, stream, L.qmap, L.kmap, p2);
     if (e != cudaSuccess) return e;
     prof_end(stream, kProfPass2);
     e = cudaGetLastError();
