@@ -29,6 +29,25 @@ namespace {
 constexpr int kPassThreads = 320;    // 8 epilogue warps, 1 TMA warp, 1 MMA warp
 constexpr int kStage = 128 * 256;    // one K tile: 128 keys x 128 fp16
 constexpr int kP1Stages = 2;   // ~99 KB of shared memory: two CTAs per SM
+// Every n-th exponential of a fully visible tile runs on the FMA pipe
+// (exp2_fma) instead of MUFU; 0: none.  Pass 2 sums 2^x of G*W columns per
+// key and leans on MUFU harder than pass 1, which also tracks row maxima.
+#ifndef KV2D_P1_FMA_EVERY
+#define KV2D_P1_FMA_EVERY 8
+#endif
+#ifndef KV2D_P2_FMA_EVERY
+#define KV2D_P2_FMA_EVERY 4
+#endif
+constexpr int kP1FmaEvery = KV2D_P1_FMA_EVERY;
+constexpr int kP2FmaEvery = KV2D_P2_FMA_EVERY;
+
+template <int EVERY>
+__device__ __forceinline__ float exp2_mixed(float x, int j) {
+    if constexpr (EVERY > 0) {
+        if (j % EVERY == EVERY - 1) return exp2_fma(x);
+    }
+    return fast_exp2(x);
+}
 constexpr uint32_t kNegInf = 0xff800000u;
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
@@ -210,10 +229,10 @@ __global__ void __launch_bounds__(kPassThreads, 1)
                 if (whole) {
 #pragma unroll
                     for (int j = 0; j < 32; j += 4) {
-                        a0 += fast_exp2(fmaf(__uint_as_float(r[j]), c2, nm));
-                        a1 += fast_exp2(fmaf(__uint_as_float(r[j + 1]), c2, nm));
-                        a2 += fast_exp2(fmaf(__uint_as_float(r[j + 2]), c2, nm));
-                        a3 += fast_exp2(fmaf(__uint_as_float(r[j + 3]), c2, nm));
+                        a0 += exp2_mixed<kP1FmaEvery>(fmaf(__uint_as_float(r[j]), c2, nm), j);
+                        a1 += exp2_mixed<kP1FmaEvery>(fmaf(__uint_as_float(r[j + 1]), c2, nm), j + 1);
+                        a2 += exp2_mixed<kP1FmaEvery>(fmaf(__uint_as_float(r[j + 2]), c2, nm), j + 2);
+                        a3 += exp2_mixed<kP1FmaEvery>(fmaf(__uint_as_float(r[j + 3]), c2, nm), j + 3);
                     }
                 } else {
                     const int t0 = t_base + cc * 32;
@@ -461,10 +480,10 @@ __global__ void __launch_bounds__(kPassThreads, 1)
 #pragma unroll
                     for (int j = 0; j < 32; j += 4) {
                         const float4 lz = l4[j >> 2];
-                        a0 += fast_exp2(fmaf(__uint_as_float(r[j]), c2, -lz.x));
-                        a1 += fast_exp2(fmaf(__uint_as_float(r[j + 1]), c2, -lz.y));
-                        a2 += fast_exp2(fmaf(__uint_as_float(r[j + 2]), c2, -lz.z));
-                        a3 += exp2_fma(fmaf(__uint_as_float(r[j + 3]), c2, -lz.w));
+                        a0 += exp2_mixed<kP2FmaEvery>(fmaf(__uint_as_float(r[j]), c2, -lz.x), j);
+                        a1 += exp2_mixed<kP2FmaEvery>(fmaf(__uint_as_float(r[j + 1]), c2, -lz.y), j + 1);
+                        a2 += exp2_mixed<kP2FmaEvery>(fmaf(__uint_as_float(r[j + 2]), c2, -lz.z), j + 2);
+                        a3 += exp2_mixed<kP2FmaEvery>(fmaf(__uint_as_float(r[j + 3]), c2, -lz.w), j + 3);
                     }
                 } else {
                     const int* wp = wpos_s + col0 + cc;

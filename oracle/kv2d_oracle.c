@@ -561,3 +561,156 @@ void orc_decode(const orc_params* p, int nseg, const uint8_t* arena,
     free(logit);
     free(vrows);
 }
+
+/* ------------------------------ decode-time token selection (stage 2) */
+
+/* [MosaicKV] Fig. 6 caption: "stage 2" (sequence compression) runs in the
+ * decode stage before each attention layer; Sec. 5.3: PackedAttention
+ * performs sequence compression and attention in each layer of the decode
+ * stage; Fig. 8: token selection rates of 6.25% and 12.5%.  The pages give no
+ * rule, so these readings are taken:
+ *   - candidates are the tokens the packed segments keep (S for FULL / CH, r
+ *     for TOK / BOTH), slot j*S + i for token i of segment j; the dense tail
+ *     [comp_end, T) is always attended;
+ *   - the score of a candidate is the largest over the G query heads of its
+ *     logit, scale * q_g . k (the stored key: whole for FULL / TOK, its kept
+ *     channels for CH / BOTH), so one selection serves the heads that share
+ *     the KV head;
+ *   - the rate rho counts tokens of the compressed context:
+ *     n_sel = min(candidates, ceil(rho * nseg * S));
+ *   - the n_sel largest scores are kept, ties to the lower slot;
+ *   - attention then runs over the kept candidates and the dense tail, the
+ *     others leaving the softmax. */
+
+/* Key of candidate i of segment j as doubles (dropped channels 0). */
+static void orc_candidate_key(const orc_params* p, const uint8_t* seg, int st, int i, double* k)
+{
+    int S = p->S, d = p->d, r = p->r, c = p->c;
+    int ntok = (st == ORC_TOK || st == ORC_BOTH) ? r : S;
+    const uint8_t* sec = seg + ((st == ORC_TOK || st == ORC_BOTH) ? pad16(r) : 0);
+    for (int x = 0; x < d; ++x) k[x] = 0.0;
+    if (st == ORC_FULL || st == ORC_TOK) {
+        const uint8_t* krow = sec + (int64_t)i * d * 2;
+        for (int x = 0; x < d; ++x)
+            k[x] = orc_half_to_double((uint16_t)(krow[2 * x] | (krow[2 * x + 1] << 8)));
+    } else {
+        const uint8_t* ci = sec + (int64_t)i * c;
+        const uint8_t* kv = sec + pad16((int64_t)ntok * c) + (int64_t)i * c * 2;
+        for (int x = 0; x < c; ++x)
+            k[ci[x]] = orc_half_to_double((uint16_t)(kv[2 * x] | (kv[2 * x + 1] << 8)));
+    }
+}
+
+/* score[j*S + i] = max_g scale * q_g . k_{j,i} for every candidate, -inf for
+ * slots past a segment's kept tokens.  Returns the number of candidates. */
+int64_t orc_select_scores(const orc_params* p, int nseg, const uint8_t* arena, const int64_t* offs,
+                          const int32_t* strat, const double* q, double* score)
+{
+    int S = p->S, d = p->d, G = p->G;
+    double* k = (double*)malloc(sizeof(double) * (size_t)d);
+    int64_t ncand = 0;
+    for (int j = 0; j < nseg; ++j) {
+        int st = strat[j];
+        int ntok = (st == ORC_TOK || st == ORC_BOTH) ? p->r : S;
+        for (int i = 0; i < S; ++i) {
+            double best = -INFINITY;
+            if (i < ntok) {
+                orc_candidate_key(p, arena + offs[j], st, i, k);
+                for (int g = 0; g < G; ++g) {
+                    double dot = 0.0;
+                    for (int x = 0; x < d; ++x) dot += q[(int64_t)g * d + x] * k[x];
+                    double l = p->scale * dot;
+                    if (l > best) best = l;
+                }
+                ++ncand;
+            }
+            score[(int64_t)j * S + i] = best;
+        }
+    }
+    free(k);
+    return ncand;
+}
+
+/* Tokens to keep at rate rho for nseg segments and ncand candidates. */
+int64_t orc_select_count(const orc_params* p, int nseg, int64_t ncand, double rho)
+{
+    double want = ceil(rho * (double)((int64_t)nseg * p->S));
+    int64_t n = (int64_t)want;
+    if (want >= (double)ncand) n = ncand;
+    return n < 0 ? 0 : n;
+}
+
+/* sel[slot] = 1 for the n_sel largest finite scores, ties to the lower
+ * slot (a plain repeated maximum search). */
+void orc_select_tokens(int64_t nslots, const double* score, int64_t n_sel, uint8_t* sel)
+{
+    for (int64_t s = 0; s < nslots; ++s) sel[s] = 0;
+    for (int64_t n = 0; n < n_sel; ++n) {
+        int64_t arg = -1;
+        for (int64_t s = 0; s < nslots; ++s) {
+            if (sel[s] || score[s] == -INFINITY) continue;
+            if (arg < 0 || score[s] > score[arg]) arg = s;
+        }
+        if (arg < 0) break;
+        sel[arg] = 1;
+    }
+}
+
+/* Attention of the G heads over the selected candidates and the dense tail:
+ * per head, softmax over that set of logits scale * q_g . k, output the
+ * weighted sum of the value rows. */
+void orc_decode_select(const orc_params* p, int nseg, const uint8_t* arena, const int64_t* offs,
+                       const int32_t* strat, const uint8_t* sel, int n_tail, const double* Kt,
+                       const double* Vt, const double* q, double* out)
+{
+    int S = p->S, d = p->d, r = p->r, c = p->c, G = p->G;
+    int64_t cap = (int64_t)nseg * S + n_tail;
+    double* logit = (double*)malloc(sizeof(double) * (size_t)(cap > 0 ? cap : 1));
+    double* vrows = (double*)malloc(sizeof(double) * (size_t)(cap > 0 ? cap : 1) * d);
+    double* k = (double*)malloc(sizeof(double) * (size_t)d);
+    for (int g = 0; g < G; ++g) {
+        const double* qg = q + (int64_t)g * d;
+        int64_t n = 0;
+        for (int j = 0; j < nseg; ++j) {
+            int st = strat[j];
+            int ntok = (st == ORC_TOK || st == ORC_BOTH) ? r : S;
+            const uint8_t* seg = arena + offs[j];
+            const uint8_t* sec = seg + ((st == ORC_TOK || st == ORC_BOTH) ? pad16(r) : 0);
+            const uint8_t* vsec = (st == ORC_FULL || st == ORC_TOK)
+                                      ? sec + (int64_t)ntok * d * 2
+                                      : sec + pad16((int64_t)ntok * c) + pad16((int64_t)ntok * c * 2);
+            for (int i = 0; i < ntok; ++i) {
+                if (!sel[(int64_t)j * S + i]) continue;
+                orc_candidate_key(p, seg, st, i, k);
+                double dot = 0.0;
+                for (int x = 0; x < d; ++x) dot += qg[x] * k[x];
+                logit[n] = p->scale * dot;
+                for (int x = 0; x < d; ++x) {
+                    const uint8_t* vb = vsec + ((int64_t)i * d + x) * 2;
+                    vrows[n * d + x] = orc_half_to_double((uint16_t)(vb[0] | (vb[1] << 8)));
+                }
+                ++n;
+            }
+        }
+        for (int t = 0; t < n_tail; ++t) {
+            double dot = 0.0;
+            for (int x = 0; x < d; ++x) dot += qg[x] * Kt[(int64_t)t * d + x];
+            logit[n] = p->scale * dot;
+            for (int x = 0; x < d; ++x) vrows[n * d + x] = Vt[(int64_t)t * d + x];
+            ++n;
+        }
+        for (int x = 0; x < d; ++x) out[(int64_t)g * d + x] = 0.0;
+        if (n == 0) continue;
+        double mx = -INFINITY;
+        for (int64_t t = 0; t < n; ++t) if (logit[t] > mx) mx = logit[t];
+        double z = 0.0;
+        for (int64_t t = 0; t < n; ++t) z += exp(logit[t] - mx);
+        for (int64_t t = 0; t < n; ++t) {
+            double w = exp(logit[t] - mx) / z;
+            for (int x = 0; x < d; ++x) out[(int64_t)g * d + x] += w * vrows[t * d + x];
+        }
+    }
+    free(k);
+    free(logit);
+    free(vrows);
+}

@@ -77,6 +77,13 @@ def lib():
                                             C.c_int64, i64p]
             L.orc_compress_unit.restype = C.c_int
             L.orc_decode.argtypes = [pp, C.c_int, u8p, i64p, i32p, C.c_int, dp, dp, dp, dp]
+            L.orc_select_scores.argtypes = [pp, C.c_int, u8p, i64p, i32p, dp, dp]
+            L.orc_select_scores.restype = C.c_int64
+            L.orc_select_count.argtypes = [pp, C.c_int, C.c_int64, C.c_double]
+            L.orc_select_count.restype = C.c_int64
+            L.orc_select_tokens.argtypes = [C.c_int64, dp, C.c_int64, u8p]
+            L.orc_decode_select.argtypes = [pp, C.c_int, u8p, i64p, i32p, u8p, C.c_int, dp, dp,
+                                            dp, dp]
             _lib = L
     return _lib
 
@@ -265,6 +272,65 @@ def decode_unit(p: Params, arena, offs, strat, Kt16, Vt16, q16) -> np.ndarray:
                      _p(strat_, C.c_int32), n_tail, _p(np.ascontiguousarray(Kt), C.c_double),
                      _p(np.ascontiguousarray(Vt), C.c_double), _p(q, C.c_double),
                      _p(out, C.c_double))
+    return out
+
+
+def _seg_args(arena, offs, strat):
+    arena = np.ascontiguousarray(arena, np.uint8)
+    if arena.size == 0:
+        arena = np.zeros(16, np.uint8)
+    offs = np.ascontiguousarray(offs, np.int64)
+    strat = np.ascontiguousarray(strat, np.int32)
+    nseg = strat.size
+    offs_ = offs if offs.size else np.zeros(1, np.int64)
+    strat_ = strat if strat.size else np.zeros(1, np.int32)
+    return arena, offs_, strat_, nseg
+
+
+def select_scores(p: Params, arena, offs, strat, q16):
+    """Decode-time selection scores of every candidate slot j*S + i: the
+    largest logit over the G heads (-inf past a segment's kept tokens).
+    Returns (score[nseg*S], number of candidates)."""
+    arena, offs_, strat_, nseg = _seg_args(arena, offs, strat)
+    q = np.ascontiguousarray(_u16(q16).view(np.float16).astype(np.float64).reshape(p.G, p.d))
+    score = np.zeros(max(nseg * p.S, 1))
+    n = lib().orc_select_scores(C.byref(p), nseg, _p(arena, C.c_uint8), _p(offs_, C.c_int64),
+                                _p(strat_, C.c_int32), _p(q, C.c_double), _p(score, C.c_double))
+    return score[:nseg * p.S], int(n)
+
+
+def select_count(p: Params, nseg: int, ncand: int, rho: float) -> int:
+    return int(lib().orc_select_count(C.byref(p), int(nseg), int(ncand), float(rho)))
+
+
+def select_tokens(score, n_sel: int) -> np.ndarray:
+    """Flags of the n_sel largest finite scores, ties to the lower slot."""
+    score = _f64(score)
+    sel = np.zeros(max(score.size, 1), np.uint8)
+    lib().orc_select_tokens(score.size, _p(score if score.size else np.zeros(1), C.c_double),
+                            int(n_sel), _p(sel, C.c_uint8))
+    return sel[:score.size]
+
+
+def decode_select(p: Params, arena, offs, strat, sel, Kt16, Vt16, q16) -> np.ndarray:
+    """Attention of the G heads over the selected candidates (flags per slot
+    j*S + i) and the dense tail rows."""
+    arena, offs_, strat_, nseg = _seg_args(arena, offs, strat)
+    sel = np.ascontiguousarray(sel, np.uint8)
+    sel_ = sel if sel.size else np.zeros(1, np.uint8)
+    Kt = _u16(Kt16).view(np.float16).astype(np.float64).reshape(-1, p.d)
+    Vt = _u16(Vt16).view(np.float16).astype(np.float64).reshape(-1, p.d)
+    n_tail = Kt.shape[0]
+    if n_tail == 0:
+        Kt = np.zeros((1, p.d))
+        Vt = np.zeros((1, p.d))
+    q = np.ascontiguousarray(_u16(q16).view(np.float16).astype(np.float64).reshape(p.G, p.d))
+    out = np.zeros((p.G, p.d))
+    lib().orc_decode_select(C.byref(p), nseg, _p(arena, C.c_uint8), _p(offs_, C.c_int64),
+                            _p(strat_, C.c_int32), _p(sel_, C.c_uint8), n_tail,
+                            _p(np.ascontiguousarray(Kt), C.c_double),
+                            _p(np.ascontiguousarray(Vt), C.c_double), _p(q, C.c_double),
+                            _p(out, C.c_double))
     return out
 
 
