@@ -359,6 +359,37 @@ def decode_bytes(wl, cc, seq):
     return used + 8 * nsegs + tail * wl.head_dim * 4 + 2 * wl.batch * wl.num_q_heads * wl.head_dim * 2
 
 
+def select_bytes(wl, cc, seq):
+    """Algorithmic bytes of one selection decode at a rate: every candidate's
+    stored key (dense row, or index + value pairs) and descriptor, a 4-byte
+    score written and read per candidate slot and a 4-byte index per kept
+    slot, the kept candidates' value rows (their keys were read already),
+    the dense tail's K and V rows, q and out."""
+    import numpy as np
+    S, r, c, d = wl.segment_len, wl.r, wl.c, wl.head_dim
+    desc = cc.desc.cpu().numpy().view(np.uint64)
+    nsg = cc.n_segs.cpu().numpy()
+    ce = cc.comp_end.cpu().tolist()
+    sq = seq.cpu().tolist()
+    key = {0: S * d * 2, 1: r * d * 2, 2: S * c * 3, 3: r * c * 3}
+    ntok = {0: S, 1: r, 2: S, 3: r}
+    kbytes = slots = 0
+    cands = []
+    for u in range(desc.shape[0]):
+        st = ((desc[u, :nsg[u]] >> np.uint64(32)) & np.uint64(255)).astype(int)
+        cnt = np.bincount(st, minlength=4)
+        kbytes += sum(int(cnt[k]) * key[k] for k in range(4)) + 8 * int(nsg[u])
+        slots += int(nsg[u]) * S
+        cands.append((int(nsg[u]) * S, sum(int(cnt[k]) * ntok[k] for k in range(4))))
+    tail = sum((sq[b] - ce[b]) * wl.num_kv_heads for b in range(wl.batch))
+
+    def at(rate):
+        kept = sum(min(nc, int(np.ceil(np.float64(np.float32(rate)) * ns))) for ns, nc in cands)
+        return (kbytes + 8 * slots + 4 * kept + kept * d * 2 + tail * d * 4 +
+                2 * wl.batch * wl.num_q_heads * d * 2)
+    return at
+
+
 def compress_alg_bytes(wl, lens, used):
     """Algorithmic bytes of kv2d_compress: K and V of the region read once,
     the window queries, the packed bytes written, and s (4 B) and g (8 B)
@@ -621,6 +652,21 @@ def main():
             dense_dec_us = 1e3 * timed(torch, stream, decode1, args.steps, flush=flush)
             del cc1
             torch.cuda.empty_cache()
+        # ---- decode with decode-time token selection at the pages' two
+        # rates (6.25 % and 12.5 % of the compressed context), L2 flushed
+        step()
+        sel_rec = {}
+        ws_s = B.workspace(B.kv2d_workspace_bytes(p, B.OP_DECODE_SELECT, wl.batch, cap), dev)
+        for rate in (0.0625, 0.125):
+            def decode_sel():
+                B.kv2d_decode_attn_select(p, wl.batch, cc.struct, dv, seq, cap, q, out, rate, ws_s,
+                                          stream=stream)
+
+            decode_sel()
+            sel_rec[str(rate)] = {"us_per_call": 1e3 * timed(torch, stream, decode_sel, args.steps,
+                                                             flush=flush)}
+        assert B.kv2d_read_status(ws_s, stream) == 0
+        del ws_s
         # leave the cache in its post-step state for the byte accounting
         step()
         torch.cuda.synchronize(dev)
@@ -637,6 +683,11 @@ def main():
     dec_bytes = decode_bytes(wl, cc, seq)
     dec_us = 1e3 * dec_ms
     comp_us = 1e3 * comp_ms
+    sel_bytes = select_bytes(wl, cc, seq)
+    for rate, rec in sel_rec.items():
+        nb = sel_bytes(float(rate))
+        rec.update({"alg_bytes": nb, "hbm_frac": nb / (rec["us_per_call"] * 1e-6) / 1e9 / hbm,
+                    "speedup_vs_plain_decode": dec_us / rec["us_per_call"]})
     flops_pass = 2.0 * wl.num_q_heads * wl.window * sum(lens) * wl.head_dim
     seg_tokens = sum((T // wl.segment_len) * wl.segment_len for T in lens)
     kv_seg_bytes = seg_tokens * wl.num_kv_heads * wl.head_dim * 2
@@ -753,6 +804,9 @@ def main():
                    "graph_note": "100 back-to-back calls in one CUDA graph, no flush between them",
                    "budget1_us": dense_dec_us,
                    "speedup_vs_budget1": (dense_dec_us / dec_us) if dense_dec_us else None},
+        "decode_select": {"rates": sel_rec,
+                          "note": "decode-time token selection: candidate scores, top-n per unit, "
+                                  "attention over the kept tokens and the dense tail; L2 flushed"},
         "compress": {"us": comp_us, "gbs": nbytes / (comp_us * 1e-6) / 1e9,
                      "alg_bytes": comp_alg, "hbm_frac": comp_alg / (comp_us * 1e-6) / 1e9 / hbm},
         "scoring": scoring,

@@ -85,7 +85,7 @@ typedef enum kv2d_status {
 enum { KV2D_FULL = 0, KV2D_TOK = 1, KV2D_CH = 2, KV2D_BOTH = 3 };
 
 /* Operations for kv2d_workspace_bytes. */
-enum { KV2D_OP_COMPRESS = 0, KV2D_OP_DECODE = 1, KV2D_OP_APPEND = 2 };
+enum { KV2D_OP_COMPRESS = 0, KV2D_OP_DECODE = 1, KV2D_OP_APPEND = 2, KV2D_OP_DECODE_SELECT = 3 };
 
 /* Device status bits (kv2d_read_status ORs them into *bits). */
 enum {
@@ -247,6 +247,42 @@ KV2D_API kv2d_status kv2d_decode_attn(const kv2d_params* p, int batch, const kv2
                              const kv2d_dense* kv, const int32_t* seq_len_dev,
                              int32_t max_seq_len_host, const void* q, void* out, void* ws,
                              size_t ws_bytes, void* stream);
+
+/* kv2d_decode_attn_select -- decode attention with decode-time,
+ * query-aware token selection over the packed segments (MosaicKV Fig. 6
+ * caption: stage 2 runs during the decode stage before each attention
+ * layer; Sec. 5.3, PackedAttention: sequence compression and attention in
+ * every decode layer; Fig. 8: token selection rates of 6.25 % and 12.5 %).
+ * Readings the library takes where the pages give no rule:
+ *   candidates  every token the unit's packed segments keep, slot j*S + i
+ *               for token i of segment j; the dense tail [comp_end,
+ *               seq_len) is always attended;
+ *   score       the largest over the unit's G query heads of the logit
+ *               scale * q_g . k (the stored key: whole for FULL / TOK, its
+ *               kept channels for CH / BOTH), in fp32;
+ *   count       n_sel = min(candidates, ceil(select_rate * n_segs * S)),
+ *               select_rate taken as the double of the float given;
+ *   choice      the n_sel largest scores, ties to the lower slot;
+ *   attention   softmax of each head over the kept candidates and the
+ *               dense tail; out = sum_t p_t v_t (fp16).
+ *   select_rate       > 0 and finite; >= 1 keeps every candidate (the
+ *                     result is then kv2d_decode_attn's, up to rounding).
+ *   ws, ws_bytes      kv2d_workspace_bytes(p, KV2D_OP_DECODE_SELECT, batch,
+ *                     max_seq_len_host) bytes, 256-byte aligned; zero it
+ *                     once before first use (tickets return to zero after
+ *                     every completed call).
+ *   dbg_score, dbg_sel  optional device outputs [units][slots], slots =
+ *                     (max_seq_len_host / S) * S rounded up to a multiple
+ *                     of 4: the fp32 score of every candidate slot (-inf
+ *                     past a segment's kept tokens) and a 0/1 flag per slot
+ *                     (1 = kept); written for slots < n_segs * S.
+ * Other arguments and errors as kv2d_decode_attn; G <= 8. */
+KV2D_API kv2d_status kv2d_decode_attn_select(const kv2d_params* p, int batch,
+                                             const kv2d_ccache* cc, const kv2d_dense* kv,
+                                             const int32_t* seq_len_dev, int32_t max_seq_len_host,
+                                             const void* q, void* out, float select_rate,
+                                             void* ws, size_t ws_bytes, float* dbg_score,
+                                             uint8_t* dbg_sel, void* stream);
 
 /* kv2d_decode_attn_noalloc -- the same decode attention as kv2d_decode_attn,
  * for callers that cannot obtain device memory at all: a plugin that runs

@@ -18,7 +18,7 @@ KV2D_OK = 0
 STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "BUDGET_INFEASIBLE", 3: "WORKSPACE", 4: "CUDA",
                 5: "DEVICE_FAULT", 6: "UNSUPPORTED", 7: "CAPACITY"}
 FULL, TOK, CH, BOTH = 0, 1, 2, 3
-OP_COMPRESS, OP_DECODE, OP_APPEND = 0, 1, 2
+OP_COMPRESS, OP_DECODE, OP_APPEND, OP_DECODE_SELECT = 0, 1, 2, 3
 MAX_BATCH = 128
 
 
@@ -55,7 +55,7 @@ class kv2d_debug(C.Structure):
 EXPORTS = ["kv2d_segment_bytes", "kv2d_arena_bytes", "kv2d_workspace_bytes", "kv2d_compress",
            "kv2d_append", "kv2d_decode_attn", "kv2d_read_status", "kv2d_last_error",
            "kv2d_version", "kv2d_profile_enable", "kv2d_profile_read", "kv2d_set_decode_table_cap",
-           "kv2d_profile_stage_name", "kv2d_decode_attn_noalloc"]
+           "kv2d_profile_stage_name", "kv2d_decode_attn_noalloc", "kv2d_decode_attn_select"]
 
 _lib = None
 
@@ -89,6 +89,11 @@ def lib():
                                                P(kv2d_dense), C.c_void_p, C.c_int32, C.c_void_p,
                                                C.c_void_p, C.c_void_p, C.c_void_p]
         L.kv2d_decode_attn_noalloc.restype = C.c_int
+        L.kv2d_decode_attn_select.argtypes = [P(kv2d_params), C.c_int, P(kv2d_ccache),
+                                              P(kv2d_dense), C.c_void_p, C.c_int32, C.c_void_p,
+                                              C.c_void_p, C.c_float, C.c_void_p, C.c_size_t,
+                                              C.c_void_p, C.c_void_p, C.c_void_p]
+        L.kv2d_decode_attn_select.restype = C.c_int
         L.kv2d_read_status.argtypes = [C.c_void_p, C.c_void_p, P(C.c_uint32)]
         L.kv2d_read_status.restype = C.c_int
         L.kv2d_last_error.argtypes = []
@@ -201,6 +206,19 @@ def kv2d_decode_attn(p, batch, cc, dense_view, seq_len_dev, max_seq_len_host, q,
                                 _ptr(seq_len_dev), int(max_seq_len_host), _ptr(q), _ptr(out),
                                 _ptr(ws), ws.numel() if hasattr(ws, "numel") else 0,
                                 _stream(stream))
+    return _check(rc) if check else rc
+
+
+def kv2d_decode_attn_select(p, batch, cc, dense_view, seq_len_dev, max_seq_len_host, q, out,
+                            select_rate, ws, dbg_score=None, dbg_sel=None, stream=None,
+                            check=True) -> int:
+    """Decode attention with decode-time token selection at select_rate
+    (dbg_score / dbg_sel: optional per-slot scores and kept flags)."""
+    rc = lib().kv2d_decode_attn_select(C.byref(p), int(batch), C.byref(cc), C.byref(dense_view),
+                                       _ptr(seq_len_dev), int(max_seq_len_host), _ptr(q),
+                                       _ptr(out), float(select_rate), _ptr(ws),
+                                       ws.numel() if hasattr(ws, "numel") else 0, _ptr(dbg_score),
+                                       _ptr(dbg_sel), _stream(stream))
     return _check(rc) if check else rc
 
 

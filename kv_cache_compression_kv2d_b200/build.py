@@ -9,7 +9,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libkv2d.so")
-SOURCES = ["api.cu", "score.cu", "select.cu", "pack.cu", "decode.cu"]
+SOURCES = ["api.cu", "score.cu", "select.cu", "pack.cu", "decode.cu", "stage2.cu"]
 HEADERS = ["common.cuh", "kernels.h"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 

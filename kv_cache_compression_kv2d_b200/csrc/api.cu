@@ -170,6 +170,30 @@ DecodeLayout decode_layout(const kv2d_params* p, int batch) {
     return L;
 }
 
+struct SelectLayout {
+    size_t score, sel, nsel, ticket, part, total;
+    int64_t slot_stride;
+};
+
+// Workspace of kv2d_decode_attn_select: per unit a score and a kept-slot
+// list over (max_seq_len / S) * S candidate slots, the kept count, a ticket,
+// and the attention partials of up to kSel2MaxChunks chunks.
+SelectLayout select_layout(const kv2d_params* p, int batch, int64_t max_seq_len) {
+    const UnitShape sh = shape_of(p);
+    const int64_t units = static_cast<int64_t>(batch) * sh.Hkv;
+    SelectLayout L;
+    L.slot_stride = round_up(std::max<int64_t>(max_seq_len / sh.S * sh.S, 1), 4);
+    Carver c;
+    c.take(256);
+    L.score = c.take(units * L.slot_stride * 4);
+    L.sel = c.take(units * L.slot_stride * 4);
+    L.nsel = c.take(units * 4);
+    L.ticket = c.take(units * 4);
+    L.part = c.take(units * kSel2MaxChunks * sh.G * (kHeadDim + 4) * 4);
+    L.total = c.off;
+    return L;
+}
+
 // blocks per chunk of the decode kernel's block table (kv2d_set_decode_table_cap)
 std::atomic<int> g_dec_table_cap{kDecTableMax};
 
@@ -251,9 +275,9 @@ bool g_prof_on = false;
 std::vector<ProfRec> g_prof_open;      // begun, not yet ended (one per stage)
 std::vector<ProfRec> g_prof_done;
 
-const char* const kStageNames[kProfStages] = {"score_pass1", "score_pass2", "chan_topc",
-                                              "seg_select",  "budget",      "pack",
-                                              "append",      "decode"};
+const char* const kStageNames[kProfStages] = {"score_pass1", "score_pass2", "chan_topc",  "seg_select",
+                                              "budget",      "pack",        "append",     "decode",
+                                              "sel_score",   "sel_topn",    "sel_attn"};
 
 }  // namespace
 
@@ -396,6 +420,7 @@ size_t kv2d_workspace_bytes(const kv2d_params* p, int op, int batch, int64_t max
     case KV2D_OP_COMPRESS: return compress_layout(p, batch, max_tokens).total;
     case KV2D_OP_DECODE: return decode_layout(p, batch).total;
     case KV2D_OP_APPEND: return 256;
+    case KV2D_OP_DECODE_SELECT: return select_layout(p, batch, max_tokens).total;
     default: return 0;
     }
 }
@@ -781,6 +806,64 @@ kv2d_status kv2d_decode_attn_noalloc(const kv2d_params* p, int batch, const kv2d
     L.status = status_dev;   // NULL: device faults are not recorded anywhere
     cudaError_t e = launch_decode(L, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return fail(KV2D_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
+    return ok();
+}
+
+kv2d_status kv2d_decode_attn_select(const kv2d_params* p, int batch, const kv2d_ccache* cc,
+                                    const kv2d_dense* kv, const int32_t* seq_len_dev,
+                                    int32_t max_seq_len_host, const void* q, void* out,
+                                    float select_rate, void* ws, size_t ws_bytes, float* dbg_score,
+                                    uint8_t* dbg_sel, void* stream) {
+    kv2d_status st = check_params(p);
+    if (st != KV2D_OK) return st;
+    const UnitShape sh = shape_of(p);
+    if (sh.G > 8) return fail(KV2D_ERR_UNSUPPORTED, "token-selection decode runs G <= 8, got %d", sh.G);
+    if (batch < 1 || batch > KV2D_MAX_BATCH)
+        return fail(KV2D_ERR_INVALID_ARG, "batch %d not in [1, %d]", batch, KV2D_MAX_BATCH);
+    if ((st = check_dense(p, batch, kv)) != KV2D_OK) return st;
+    if (!cc || !cc->arena || !cc->desc || !cc->n_segs || !cc->used_bytes || !cc->comp_end)
+        return fail(KV2D_ERR_INVALID_ARG, "compressed cache has a NULL pointer");
+    if (!aligned(cc->arena, 256) || cc->arena_stride % 256)
+        return fail(KV2D_ERR_INVALID_ARG, "arena must be 256-byte aligned with a multiple-of-256 stride");
+    if (!seq_len_dev || !q || !out || !aligned(q, 16) || !aligned(out, 16))
+        return fail(KV2D_ERR_INVALID_ARG, "seq_len / q / out must be 16-byte aligned device pointers");
+    if (max_seq_len_host < 0 || max_seq_len_host > dense_capacity(kv))
+        return fail(KV2D_ERR_INVALID_ARG, "max_seq_len %d outside [0, capacity]", max_seq_len_host);
+    if (!(select_rate > 0.f) || !std::isfinite(select_rate))
+        return fail(KV2D_ERR_INVALID_ARG, "select_rate must be a positive finite fraction");
+    const SelectLayout WL = select_layout(p, batch, max_seq_len_host);
+    if (!ws || !aligned(ws, 256) || ws_bytes < WL.total)
+        return fail(KV2D_ERR_WORKSPACE, "selection decode workspace %zu bytes, need %zu (256-byte aligned)",
+                    ws_bytes, WL.total);
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    DecodeSelectLaunch L;
+    L.shp = sh;
+    L.batch = batch;
+    L.scale = eff_scale(p);
+    L.rate = static_cast<double>(select_rate);
+    L.dv = view_of(p, kv);
+    L.arena = static_cast<const uint8_t*>(cc->arena);
+    L.arena_stride = cc->arena_stride;
+    L.desc = static_cast<const uint64_t*>(cc->desc);
+    L.max_segs = cc->max_segs;
+    L.n_segs = cc->n_segs;
+    L.used_bytes = cc->used_bytes;
+    L.comp_end = cc->comp_end;
+    L.seq_len = seq_len_dev;
+    L.q = static_cast<const __half*>(q);
+    L.out = static_cast<__half*>(out);
+    L.slot_stride = WL.slot_stride;
+    L.score = reinterpret_cast<float*>(w + WL.score);
+    L.sel = reinterpret_cast<int32_t*>(w + WL.sel);
+    L.nsel = reinterpret_cast<int32_t*>(w + WL.nsel);
+    L.part = reinterpret_cast<float*>(w + WL.part);
+    L.ticket = reinterpret_cast<uint32_t*>(w + WL.ticket);
+    L.nchunk = sel2_chunks(batch * sh.Hkv, num_sms());
+    L.dbg_score = dbg_score;
+    L.dbg_sel = dbg_sel;
+    L.status = reinterpret_cast<uint32_t*>(w);
+    cudaError_t e = launch_decode_select(L, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail(KV2D_ERR_CUDA, "selection decode launch: %s", cudaGetErrorString(e));
     return ok();
 }
 

@@ -22,6 +22,9 @@ enum ProfStage {
     kProfPack,
     kProfAppend,
     kProfDecode,
+    kProfSelScore,
+    kProfSelTop,
+    kProfSelAttn,
     kProfStages
 };
 
@@ -179,5 +182,37 @@ constexpr int kMaxDecCtas = 512;
 constexpr int kDecTableMax = 4096;
 cudaError_t launch_decode(const DecodeLaunch& L, cudaStream_t stream);
 int decode_cta_count(int units, int64_t max_seq_len, int num_sms, int* kps);
+
+// ---- decode with decode-time token selection (stage2.cu)
+struct DecodeSelectLaunch {
+    UnitShape shp;
+    int batch;
+    float scale;               // softmax scale (natural log domain)
+    double rate;               // token selection rate
+    DenseView dv;
+    const uint8_t* arena;
+    int64_t arena_stride;
+    const uint64_t* desc;
+    int32_t max_segs;
+    const int32_t* n_segs;
+    const int64_t* used_bytes;
+    const int32_t* comp_end;
+    const int32_t* seq_len;
+    const __half* q;
+    __half* out;
+    int64_t slot_stride;       // candidate slots per unit: (max_seq_len / S) * S
+    float* score;              // [units][slot_stride]
+    int32_t* sel;              // [units][slot_stride]
+    int32_t* nsel;             // [units]
+    float* part;               // [units][nchunk][G][4 + d]
+    uint32_t* ticket;          // [units]
+    int nchunk;                // attention chunks per unit, <= kSel2MaxChunks
+    float* dbg_score;
+    uint8_t* dbg_sel;
+    uint32_t* status;
+};
+constexpr int kSel2MaxChunks = 64;
+cudaError_t launch_decode_select(const DecodeSelectLaunch& L, cudaStream_t stream);
+int sel2_chunks(int units, int num_sms);
 
 }  // namespace kv2d

@@ -1,0 +1,576 @@
+// stage2.cu -- decode attention with decode-time token selection over the
+// packed segments (sm_100a).
+//
+// MosaicKV ("MosaicKV: Serving Long-Context LLM with Dynamic Two-D KV Cache
+// Compression", Fig. 6: stage 2 runs during the decode stage before each
+// attention layer; Sec. 5.3: PackedAttention performs sequence compression
+// and attention in every decode layer; Fig. 8: token selection rates of
+// 6.25 % and 12.5 %) selects tokens per step with the current query.  The
+// pages give no rule; this library reads it as:
+//   - candidates: the tokens the unit's packed segments keep, slot j*S + i
+//     for token i of segment j; the dense tail [comp_end, seq_len) is always
+//     attended;
+//   - score of a candidate: the largest over the unit's G query heads of the
+//     logit scale * q_g . k (the stored key; kept channels only for CH /
+//     BOTH), so one selection serves the heads that share the KV head;
+//   - count: n_sel = min(candidates, ceil(rate * n_segs * S));
+//   - the n_sel largest scores are kept, ties to the lower slot;
+//   - attention over the kept candidates and the dense tail.
+// Three kernels:
+//   sel_score : one thread per candidate slot, G fp32 dot products with q
+//               from shared memory, the maximum written per slot;
+//   sel_topn  : one CTA per unit, an exact radix select of the n_sel-th
+//               largest score key (8-bit digits), the tied keys taken in
+//               slot order by a block scan, the kept slots written ascending;
+//   sel_attn  : the unit's items (kept slots, then tail tokens) cut into
+//               equal chunks, one CTA per chunk; a warp per item with lanes
+//               over d (coalesced 8-byte key / value reads), online softmax
+//               per head, fixed-order warp and chunk merges (the last CTA of
+//               a unit, by atomic ticket, writes the fp16 output).
+#include <algorithm>
+
+#include "kernels.h"
+
+namespace kv2d {
+
+namespace {
+
+constexpr int kScoreThreads = 256;
+constexpr int kTopThreads = 1024;
+constexpr int kAttnWarps = 8;
+constexpr float kNegInf2 = -__builtin_huge_valf();
+
+struct Sel2Args {
+    int Hkv, Hq, G, S, r, c;
+    float scale, c2;
+    double rate;
+    DenseView dv;
+    const uint8_t* arena;
+    int64_t arena_stride;
+    const uint64_t* desc;
+    int32_t max_segs;
+    const int32_t* n_segs;
+    const int64_t* used_bytes;
+    const int32_t* comp_end;
+    const int32_t* seq_len;
+    const __half* q;
+    __half* out;
+    int64_t slot_stride;   // slots per unit in score / sel
+    float* score;          // [units][slot_stride]
+    int32_t* sel;          // [units][slot_stride]: kept slots, ascending
+    int32_t* nsel;         // [units]
+    float* part;           // [units][nchunk][G][4 + d]
+    uint32_t* ticket;      // [units]
+    int nchunk;
+    float* dbg_score;      // optional [units][slot_stride]
+    uint8_t* dbg_sel;      // optional [units][slot_stride]
+    uint32_t* status;
+};
+
+__host__ __device__ inline int64_t seg_payload(int st, int S, int r, int c) {
+    switch (st) {
+    case KV2D_FULL: return 4ll * S * kHeadDim;
+    case KV2D_TOK: return pad16(r) + 4ll * r * kHeadDim;
+    case KV2D_CH: return pad16(static_cast<int64_t>(S) * c) + pad16(2ll * S * c) + 2ll * S * kHeadDim;
+    default: return pad16(r) + pad16(static_cast<int64_t>(r) * c) + pad16(2ll * r * c) + 2ll * r * kHeadDim;
+    }
+}
+
+// Segments a unit holds, clamped to the slot range; a value out of range
+// sets KV2D_DEV_SEQ_RANGE (when report is set).
+__device__ __forceinline__ int unit_segs(const Sel2Args& A, int u, bool report) {
+    int n = A.n_segs[u];
+    const int lim = static_cast<int>(min(static_cast<int64_t>(A.max_segs), A.slot_stride / A.S));
+    if (n < 0 || n > lim) {
+        if (report) set_status(A.status, KV2D_DEV_SEQ_RANGE);
+        n = max(0, min(n, lim));
+    }
+    return n;
+}
+
+// Where candidate i of segment j of unit u lives.  kind 0: none (slot past
+// the segment's kept tokens, or the segment's bytes outside the arena);
+// 1: dense key row; 2: c (index, value) pairs.
+struct Cand {
+    int kind;
+    const uint8_t* key;    // key row, or the index bytes
+    const __half* kval;    // sparse key values
+    const __half* vrow;    // value row
+};
+
+__device__ __forceinline__ Cand candidate(const Sel2Args& A, int u, int j, int i, bool report) {
+    Cand cd{0, nullptr, nullptr, nullptr};
+    const uint64_t d = A.desc[static_cast<int64_t>(u) * A.max_segs + j];
+    const int st = static_cast<int>((d >> 32) & 255u);
+    const int64_t off = static_cast<int64_t>(d & 0xffffffffull) * 16;
+    const int S = A.S, r = A.r, c = A.c;
+    const bool tok = (st == KV2D_TOK || st == KV2D_BOTH);
+    const int ntok = tok ? r : S;
+    if (i >= ntok) return cd;
+    int64_t U = A.used_bytes[u];
+    U = max(static_cast<int64_t>(0), min(U, A.arena_stride));
+    if (st > KV2D_BOTH || off < 0 || off + seg_payload(st, S, r, c) > U) {
+        if (report) set_status(A.status, KV2D_DEV_CAPACITY);
+        return cd;
+    }
+    const uint8_t* sec = A.arena + static_cast<int64_t>(u) * A.arena_stride + off + (tok ? pad16(r) : 0);
+    if (st == KV2D_FULL || st == KV2D_TOK) {
+        cd.kind = 1;
+        cd.key = sec + static_cast<int64_t>(i) * kHeadDim * 2;
+        cd.vrow = reinterpret_cast<const __half*>(sec + static_cast<int64_t>(ntok + i) * kHeadDim * 2);
+    } else {
+        cd.kind = 2;
+        cd.key = sec + static_cast<int64_t>(i) * c;
+        cd.kval = reinterpret_cast<const __half*>(sec + pad16(static_cast<int64_t>(ntok) * c)) +
+                  static_cast<int64_t>(i) * c;
+        cd.vrow = reinterpret_cast<const __half*>(sec + pad16(static_cast<int64_t>(ntok) * c) +
+                                                  pad16(2ll * ntok * c)) +
+                  static_cast<int64_t>(i) * kHeadDim;
+    }
+    return cd;
+}
+
+// ------------------------------------------------------------- scores
+
+__global__ void __launch_bounds__(kScoreThreads) sel_score_kernel(const __grid_constant__ Sel2Args A) {
+    pdl_wait();
+    __shared__ __align__(16) float qs[8][kHeadDim];
+    const int u = blockIdx.y;
+    const int b = u / A.Hkv, h = u % A.Hkv;
+    const int G = A.G;
+    for (int x = threadIdx.x; x < G * kHeadDim; x += kScoreThreads)
+        qs[x / kHeadDim][x % kHeadDim] =
+            __half2float(A.q[(static_cast<int64_t>(b) * A.Hq + h * G + x / kHeadDim) * kHeadDim + x % kHeadDim]);
+    __syncthreads();
+    const int nsg = unit_segs(A, u, blockIdx.x == 0 && threadIdx.x == 0);
+    const int64_t slot = static_cast<int64_t>(blockIdx.x) * kScoreThreads + threadIdx.x;
+    if (slot >= static_cast<int64_t>(nsg) * A.S) return;
+    const int j = static_cast<int>(slot / A.S), i = static_cast<int>(slot % A.S);
+    const Cand cd = candidate(A, u, j, i, true);
+    float best = kNegInf2;
+    if (cd.kind != 0) {
+        float acc[8];
+#pragma unroll
+        for (int g = 0; g < 8; ++g) acc[g] = 0.f;
+        if (cd.kind == 1) {
+#pragma unroll 2
+            for (int ch = 0; ch < 16; ++ch) {
+                const uint4 w = *reinterpret_cast<const uint4*>(cd.key + ch * 16);
+                const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+                float kf[8];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&ws[e]));
+                    kf[2 * e] = f.x;
+                    kf[2 * e + 1] = f.y;
+                }
+#pragma unroll
+                for (int g = 0; g < 8; ++g) {
+                    if (g < G) {
+                        const float4 q0 = *reinterpret_cast<const float4*>(&qs[g][ch * 8]);
+                        const float4 q1 = *reinterpret_cast<const float4*>(&qs[g][ch * 8 + 4]);
+                        float a = acc[g];
+                        a = fmaf(q0.x, kf[0], a);
+                        a = fmaf(q0.y, kf[1], a);
+                        a = fmaf(q0.z, kf[2], a);
+                        a = fmaf(q0.w, kf[3], a);
+                        a = fmaf(q1.x, kf[4], a);
+                        a = fmaf(q1.y, kf[5], a);
+                        a = fmaf(q1.z, kf[6], a);
+                        a = fmaf(q1.w, kf[7], a);
+                        acc[g] = a;
+                    }
+                }
+            }
+        } else {
+            for (int x = 0; x < A.c; ++x) {
+                const int ci = cd.key[x] & 0x7f;     // indices are < 128; the mask keeps a bad byte in range
+                const float kv = __half2float(cd.kval[x]);
+#pragma unroll
+                for (int g = 0; g < 8; ++g)
+                    if (g < G) acc[g] = fmaf(qs[g][ci], kv, acc[g]);
+            }
+        }
+#pragma unroll
+        for (int g = 0; g < 8; ++g)
+            if (g < G) best = fmaxf(best, A.scale * acc[g]);
+    }
+    A.score[static_cast<int64_t>(u) * A.slot_stride + slot] = best;
+    if (A.dbg_score) A.dbg_score[static_cast<int64_t>(u) * A.slot_stride + slot] = best;
+}
+
+// ---------------------------------------------------------- selection
+
+// Order-preserving key of a score: larger score, larger key; -inf (no
+// candidate) is 0, every finite score is above it.
+__device__ __forceinline__ uint32_t score_key(float s) {
+    if (s == kNegInf2) return 0u;
+    const uint32_t b = __float_as_uint(s);
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+__device__ __forceinline__ long long block_exscan_ll(long long v, long long* red, long long* total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    long long inc = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const long long n = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += n;
+    }
+    __syncthreads();
+    if (lane == 31) red[warp] = inc;
+    __syncthreads();
+    if (warp == 0) {
+        const long long w = (lane < (blockDim.x >> 5)) ? red[lane] : 0;
+        long long wi = w;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const long long n = __shfl_up_sync(0xffffffffu, wi, o);
+            if (lane >= o) wi += n;
+        }
+        red[lane] = wi - w;
+        if (lane == 31) red[32] = wi;
+    }
+    __syncthreads();
+    const long long res = red[warp] + inc - v;
+    *total = red[32];
+    __syncthreads();
+    return res;
+}
+
+__global__ void __launch_bounds__(kTopThreads) sel_topn_kernel(const __grid_constant__ Sel2Args A) {
+    pdl_wait();
+    __shared__ unsigned int hist[256];
+    __shared__ long long red[33];
+    __shared__ uint32_t s_prefix;
+    __shared__ long long s_need;
+    const int u = blockIdx.x;
+    const int tid = threadIdx.x;
+    const int nsg = unit_segs(A, u, false);
+    const int64_t nslots = static_cast<int64_t>(nsg) * A.S;
+    const float* sc = A.score + static_cast<int64_t>(u) * A.slot_stride;
+    // candidates: kept tokens per segment from the descriptors
+    long long nc = 0;
+    for (int j = tid; j < nsg; j += kTopThreads) {
+        const int st = static_cast<int>((A.desc[static_cast<int64_t>(u) * A.max_segs + j] >> 32) & 255u);
+        nc += (st == KV2D_TOK || st == KV2D_BOTH) ? A.r : A.S;
+    }
+    long long ncand;
+    block_exscan_ll(nc, red, &ncand);
+    const double want = ceil(A.rate * static_cast<double>(nslots));
+    const long long n_sel = (want >= static_cast<double>(ncand)) ? ncand : static_cast<long long>(want);
+    // the n_sel-th largest key, 8 bits at a time from the top
+    if (tid == 0) {
+        s_prefix = 0u;
+        s_need = n_sel;
+    }
+    __syncthreads();
+    for (int pass = 0; pass < 4 && n_sel > 0; ++pass) {
+        const int shift = 24 - 8 * pass;
+        for (int i = tid; i < 256; i += kTopThreads) hist[i] = 0u;
+        __syncthreads();
+        const uint32_t pre = s_prefix;
+        const uint32_t hmask = pass == 0 ? 0u : (0xffffffffu << (shift + 8));
+        for (int64_t s = tid; s < nslots; s += kTopThreads) {
+            const uint32_t k = score_key(sc[s]);
+            if (k != 0u && (k & hmask) == (pre & hmask)) atomicAdd(&hist[(k >> shift) & 255u], 1u);
+        }
+        __syncthreads();
+        if (tid < 32) {
+            // lane l owns digits 255 - 8l .. 248 - 8l (largest first)
+            long long cnt = 0;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) cnt += hist[255 - (8 * tid + k)];
+            long long inc = cnt;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const long long n = __shfl_up_sync(0xffffffffu, inc, o);
+                if (tid >= o) inc += n;
+            }
+            const long long need = s_need;
+            long long above = inc - cnt;            // keys with larger digits
+            int found = -1;
+            long long above_found = 0;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const int dg = 255 - (8 * tid + k);
+                const long long hk = hist[dg];
+                if (found < 0 && above + hk >= need) {
+                    found = dg;
+                    above_found = above;
+                }
+                above += hk;
+            }
+            const uint32_t bal = __ballot_sync(0xffffffffu, found >= 0);
+            const int src = bal ? (__ffs(bal) - 1) : 0;
+            const int dg = __shfl_sync(0xffffffffu, found, src);
+            const long long ab = __shfl_sync(0xffffffffu, above_found, src);
+            if (tid == 0 && bal) {
+                s_prefix = pre | (static_cast<uint32_t>(dg) << shift);
+                s_need = need - ab;
+            }
+        }
+        __syncthreads();
+    }
+    const uint32_t v = s_prefix;            // the n_sel-th largest key (0: nothing kept)
+    const long long eq_take = s_need;       // keys equal to v to keep, lowest slots first
+    // thread tid scans its own contiguous range of slots, so block scans give slot order
+    const int64_t per = (nslots + kTopThreads - 1) / kTopThreads;
+    const int64_t s0 = min(nslots, per * tid), s1 = min(nslots, s0 + per);
+    long long n_gt = 0, n_eq = 0;
+    for (int64_t s = s0; s < s1; ++s) {
+        const uint32_t k = score_key(sc[s]);
+        n_gt += (n_sel > 0 && k > v);
+        n_eq += (n_sel > 0 && k == v && k != 0u);
+    }
+    long long tot_eq;
+    const long long eq_before = block_exscan_ll(n_eq, red, &tot_eq);
+    long long mine = n_gt + max(0ll, min(n_eq, eq_take - eq_before));
+    long long tot_sel;
+    long long pos = block_exscan_ll(mine, red, &tot_sel);
+    int32_t* out = A.sel + static_cast<int64_t>(u) * A.slot_stride;
+    long long eq_seen = eq_before;
+    for (int64_t s = s0; s < s1; ++s) {
+        const uint32_t k = score_key(sc[s]);
+        bool keep = false;
+        if (n_sel > 0 && k != 0u) {
+            if (k > v) keep = true;
+            else if (k == v) keep = (eq_seen++ < eq_take);
+        }
+        if (keep) out[pos++] = static_cast<int32_t>(s);
+        if (A.dbg_sel) A.dbg_sel[static_cast<int64_t>(u) * A.slot_stride + s] = keep ? 1 : 0;
+    }
+    if (tid == 0) {
+        A.nsel[u] = static_cast<int32_t>(tot_sel);
+        if (tot_sel != n_sel) set_status(A.status, KV2D_DEV_BAD_MASK);
+    }
+}
+
+// ---------------------------------------------------------- attention
+
+template <int G>
+__global__ void __launch_bounds__(kAttnWarps * 32) sel_attn_kernel(const __grid_constant__ Sel2Args A) {
+    pdl_wait();
+    constexpr int kRec = kHeadDim + 4;
+    __shared__ __align__(16) float qs[G][kHeadDim];
+    __shared__ float wm[kAttnWarps][G], wl[kAttnWarps][G];
+    __shared__ __align__(16) float wo[kAttnWarps][G][kHeadDim];
+    __shared__ int is_last;
+    const int c_id = blockIdx.x, u = blockIdx.y;
+    const int b = u / A.Hkv, h = u % A.Hkv;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    for (int x = tid; x < G * kHeadDim; x += kAttnWarps * 32)
+        qs[x / kHeadDim][x % kHeadDim] =
+            __half2float(A.q[(static_cast<int64_t>(b) * A.Hq + h * G + x / kHeadDim) * kHeadDim + x % kHeadDim]);
+    __syncthreads();
+    // the unit's items: kept candidates, then its dense tail tokens
+    const int cap = A.dv.block_table ? A.dv.max_blocks * A.dv.block_size : A.dv.capacity;
+    int T = A.seq_len[b], ce = A.comp_end[b];
+    if (T < 0 || T > cap || ce < 0 || ce > T) {
+        if (tid == 0 && c_id == 0) set_status(A.status, KV2D_DEV_SEQ_RANGE);
+        T = max(0, min(T, cap));
+        ce = max(0, min(ce, T));
+    }
+    const int64_t nsel = A.nsel[u];
+    const int64_t items = nsel + (T - ce);
+    const int64_t i_lo = items * c_id / A.nchunk, i_hi = items * (c_id + 1) / A.nchunk;
+    const int32_t* sl = A.sel + static_cast<int64_t>(u) * A.slot_stride;
+    // lane l holds dims 4l .. 4l + 3 of q (log2-domain scale folded in later)
+    float qv[G][4];
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) qv[g][e] = qs[g][4 * lane + e];
+    float m[G], l[G], o[G][4];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+        m[g] = kNegInf2;
+        l[g] = 0.f;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o[g][e] = 0.f;
+    }
+    for (int64_t it = i_lo + warp; it < i_hi; it += kAttnWarps) {
+        float dot[G];
+#pragma unroll
+        for (int g = 0; g < G; ++g) dot[g] = 0.f;
+        const __half* vrow = nullptr;
+        if (it < nsel) {
+            const int32_t slot = sl[it];
+            const Cand cd = candidate(A, u, slot / A.S, slot % A.S, lane == 0);
+            if (cd.kind == 0) continue;      // (status already set; warp-uniform)
+            vrow = cd.vrow;
+            if (cd.kind == 1) {
+                const uint2 kw = *reinterpret_cast<const uint2*>(cd.key + lane * 8);
+                const float2 k01 = __half22float2(*reinterpret_cast<const __half2*>(&kw.x));
+                const float2 k23 = __half22float2(*reinterpret_cast<const __half2*>(&kw.y));
+#pragma unroll
+                for (int g = 0; g < G; ++g)
+                    dot[g] = fmaf(qv[g][3], k23.y, fmaf(qv[g][2], k23.x, fmaf(qv[g][1], k01.y, qv[g][0] * k01.x)));
+            } else {
+                for (int x = lane; x < A.c; x += 32) {
+                    const int ci = cd.key[x] & 0x7f;
+                    const float kv = __half2float(cd.kval[x]);
+#pragma unroll
+                    for (int g = 0; g < G; ++g) dot[g] = fmaf(qs[g][ci], kv, dot[g]);
+                }
+            }
+        } else {
+            const int t = ce + static_cast<int>(it - nsel);
+            const __half* kr = dense_row(A.dv, A.dv.k, b, h, t, lane == 0 ? A.status : nullptr);
+            vrow = dense_row(A.dv, A.dv.v, b, h, t, nullptr);
+            if (!kr || !vrow) continue;      // warp-uniform
+            const uint2 kw = *reinterpret_cast<const uint2*>(kr + lane * 4);
+            const float2 k01 = __half22float2(*reinterpret_cast<const __half2*>(&kw.x));
+            const float2 k23 = __half22float2(*reinterpret_cast<const __half2*>(&kw.y));
+#pragma unroll
+            for (int g = 0; g < G; ++g)
+                dot[g] = fmaf(qv[g][3], k23.y, fmaf(qv[g][2], k23.x, fmaf(qv[g][1], k01.y, qv[g][0] * k01.x)));
+        }
+        // every lane gets the G logits (fixed butterfly order)
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) dot[g] += __shfl_xor_sync(0xffffffffu, dot[g], off);
+        const uint2 vw = *reinterpret_cast<const uint2*>(vrow + lane * 4);
+        const float2 v01 = __half22float2(*reinterpret_cast<const __half2*>(&vw.x));
+        const float2 v23 = __half22float2(*reinterpret_cast<const __half2*>(&vw.y));
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            const float x = dot[g] * A.c2;
+            const float mn = fmaxf(m[g], x);
+            const float alpha = (m[g] == kNegInf2) ? 0.f : fast_exp2(m[g] - mn);
+            const float p = fast_exp2(x - mn);
+            m[g] = mn;
+            l[g] = fmaf(l[g], alpha, p);
+            o[g][0] = fmaf(o[g][0], alpha, p * v01.x);
+            o[g][1] = fmaf(o[g][1], alpha, p * v01.y);
+            o[g][2] = fmaf(o[g][2], alpha, p * v23.x);
+            o[g][3] = fmaf(o[g][3], alpha, p * v23.y);
+        }
+    }
+    // warp partials -> the chunk's partial (warps merged in order)
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+        if (lane == 0) {
+            wm[warp][g] = m[g];
+            wl[warp][g] = l[g];
+        }
+        *reinterpret_cast<float4*>(&wo[warp][g][4 * lane]) = make_float4(o[g][0], o[g][1], o[g][2], o[g][3]);
+    }
+    __syncthreads();
+    float* myp = A.part + (static_cast<int64_t>(u) * A.nchunk + c_id) * G * kRec;
+    for (int x = tid; x < G * kHeadDim; x += kAttnWarps * 32) {
+        const int g = x / kHeadDim, dd = x % kHeadDim;
+        float M = kNegInf2;
+#pragma unroll
+        for (int w = 0; w < kAttnWarps; ++w) M = fmaxf(M, wm[w][g]);
+        float O = 0.f, L = 0.f;
+        if (M != kNegInf2) {
+#pragma unroll
+            for (int w = 0; w < kAttnWarps; ++w) {
+                if (wm[w][g] == kNegInf2) continue;
+                const float s = fast_exp2(wm[w][g] - M);
+                O = fmaf(wo[w][g][dd], s, O);
+                L = fmaf(wl[w][g], s, L);
+            }
+        }
+        myp[g * kRec + 4 + dd] = O;
+        if (dd == 0) {
+            myp[g * kRec] = M;
+            myp[g * kRec + 1] = L;
+        }
+    }
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) is_last = (atomicAdd(&A.ticket[u], 1u) == static_cast<uint32_t>(A.nchunk - 1));
+    __syncthreads();
+    if (!is_last) return;
+    __threadfence();
+    // the unit's chunks merged in order; a thread per (head, dim)
+    const float* up = A.part + static_cast<int64_t>(u) * A.nchunk * G * kRec;
+    for (int x = tid; x < G * kHeadDim; x += kAttnWarps * 32) {
+        const int g = x / kHeadDim, dd = x % kHeadDim;
+        float M = kNegInf2;
+        for (int k = 0; k < A.nchunk; ++k) M = fmaxf(M, __ldcg(up + (static_cast<int64_t>(k) * G + g) * kRec));
+        float O = 0.f, L = 0.f;
+        if (M != kNegInf2) {
+            for (int k = 0; k < A.nchunk; ++k) {
+                const float* rec = up + (static_cast<int64_t>(k) * G + g) * kRec;
+                const float mk = __ldcg(rec);
+                if (mk == kNegInf2) continue;
+                const float s = fast_exp2(mk - M);
+                O = fmaf(__ldcg(rec + 4 + dd), s, O);
+                L = fmaf(__ldcg(rec + 1), s, L);
+            }
+        }
+        A.out[(static_cast<int64_t>(b) * A.Hq + h * G + g) * kHeadDim + dd] = __float2half_rn(L > 0.f ? O / L : 0.f);
+    }
+    if (tid == 0) A.ticket[u] = 0;
+}
+
+}  // namespace
+
+int sel2_chunks(int units, int num_sms) {
+    return std::max(1, std::min(kSel2MaxChunks, (2 * num_sms + units - 1) / units));
+}
+
+cudaError_t launch_decode_select(const DecodeSelectLaunch& L, cudaStream_t stream) {
+    Sel2Args a;
+    a.Hkv = L.shp.Hkv;
+    a.Hq = L.shp.Hq;
+    a.G = L.shp.G;
+    a.S = L.shp.S;
+    a.r = L.shp.r;
+    a.c = L.shp.c;
+    a.scale = L.scale;
+    a.c2 = L.shp.c2;
+    a.rate = L.rate;
+    a.dv = L.dv;
+    a.arena = L.arena;
+    a.arena_stride = L.arena_stride;
+    a.desc = L.desc;
+    a.max_segs = L.max_segs;
+    a.n_segs = L.n_segs;
+    a.used_bytes = L.used_bytes;
+    a.comp_end = L.comp_end;
+    a.seq_len = L.seq_len;
+    a.q = L.q;
+    a.out = L.out;
+    a.slot_stride = L.slot_stride;
+    a.score = L.score;
+    a.sel = L.sel;
+    a.nsel = L.nsel;
+    a.part = L.part;
+    a.ticket = L.ticket;
+    a.nchunk = L.nchunk;
+    a.dbg_score = L.dbg_score;
+    a.dbg_sel = L.dbg_sel;
+    a.status = L.status;
+    const int units = L.batch * L.shp.Hkv;
+    cudaError_t e;
+    prof_begin(stream, kProfSelScore);
+    if (L.slot_stride > 0) {
+        dim3 g1(static_cast<unsigned>((L.slot_stride + kScoreThreads - 1) / kScoreThreads), units);
+        e = launch_k(sel_score_kernel, g1, dim3(kScoreThreads), 0, stream, a);
+        if (e != cudaSuccess) return e;
+    }
+    prof_end(stream, kProfSelScore);
+    prof_begin(stream, kProfSelTop);
+    e = launch_k(sel_topn_kernel, dim3(units), dim3(kTopThreads), 0, stream, a);
+    if (e != cudaSuccess) return e;
+    prof_end(stream, kProfSelTop);
+    prof_begin(stream, kProfSelAttn);
+    dim3 g3(L.nchunk, units);
+    switch (L.shp.G) {
+    case 1: e = launch_k(sel_attn_kernel<1>, g3, dim3(kAttnWarps * 32), 0, stream, a); break;
+    case 2: e = launch_k(sel_attn_kernel<2>, g3, dim3(kAttnWarps * 32), 0, stream, a); break;
+    case 4: e = launch_k(sel_attn_kernel<4>, g3, dim3(kAttnWarps * 32), 0, stream, a); break;
+    case 8: e = launch_k(sel_attn_kernel<8>, g3, dim3(kAttnWarps * 32), 0, stream, a); break;
+    default: return cudaErrorInvalidValue;
+    }
+    if (e != cudaSuccess) return e;
+    prof_end(stream, kProfSelAttn);
+    return cudaGetLastError();
+}
+
+}  // namespace kv2d

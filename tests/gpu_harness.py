@@ -286,3 +286,40 @@ def oracle_decode_unit(orc, run: GpuRun, b: int, h: int, q: torch.Tensor,
     G = wl.group
     qh = q[b, h * G:(h + 1) * G].cpu().numpy()
     return orc.decode_unit(po, arena, offs, strat, Kt, Vt, qh)
+
+
+def unit_cache(run: GpuRun, b: int, h: int, cc: B.CompressedCache | None = None):
+    """The packed bytes, offsets and strategies of unit (b, h) and the dense
+    tail rows after its segments."""
+    cc = cc or run.cc
+    u = b * run.wl.num_kv_heads + h
+    nsg = int(cc.n_segs[u])
+    used = int(cc.used_bytes[u])
+    ce = int(cc.comp_end[b])
+    T = int(run.seq_len[b])
+    desc = cc.desc[u, :nsg].cpu().numpy().view(np.uint64)
+    strat = ((desc >> np.uint64(32)) & np.uint64(255)).astype(np.int32)
+    offs = (desc & np.uint64(0xffffffff)).astype(np.int64) * 16
+    arena = cc.arena[u * cc.arena_stride: u * cc.arena_stride + used].cpu().numpy()
+    Kt, Vt = unit_inputs(run, b, h, ce, T)
+    return arena, offs, strat, Kt, Vt
+
+
+def gpu_decode_select(run: GpuRun, q: torch.Tensor, rate: float, max_seq=None):
+    """kv2d_decode_attn_select with its per-slot scores and kept flags."""
+    wl, p = run.wl, run.p
+    ms = max_seq or run.batch.capacity
+    units = wl.batch * wl.num_kv_heads
+    slots = -(-(ms // wl.segment_len * wl.segment_len) // 4) * 4
+    slots = max(slots, 4)
+    out = torch.full((wl.batch, wl.num_q_heads, wl.head_dim), float("nan"), dtype=torch.float16,
+                     device="cuda")
+    score = torch.full((units, slots), float("nan"), device="cuda")
+    sel = torch.full((units, slots), 7, dtype=torch.uint8, device="cuda")
+    ws = B.workspace(B.kv2d_workspace_bytes(p, B.OP_DECODE_SELECT, wl.batch, ms))
+    B.kv2d_decode_attn_select(p, wl.batch, run.cc.struct, run.dv, run.seq_len, ms, q, out, rate, ws,
+                              score, sel)
+    torch.cuda.synchronize()
+    bits = B.kv2d_read_status(ws)
+    assert bits == 0, f"device status bits {bits:#x}"
+    return out, score, sel
