@@ -665,6 +665,15 @@ def main():
             decode_sel()
             sel_rec[str(rate)] = {"us_per_call": 1e3 * timed(torch, stream, decode_sel, args.steps,
                                                              flush=flush)}
+            B.kv2d_profile_read()
+            B.kv2d_profile_enable(True)
+            for _ in range(3):
+                flush.zero_()
+                decode_sel()
+            torch.cuda.synchronize(dev)
+            B.kv2d_profile_enable(False)
+            sel_rec[str(rate)]["kernels_us"] = {k: 1e3 * t / n for k, (t, n) in B.kv2d_profile_read().items()
+                                                if n and k.startswith("sel_")}
         assert B.kv2d_read_status(ws_s, stream) == 0
         del ws_s
         # leave the cache in its post-step state for the byte accounting

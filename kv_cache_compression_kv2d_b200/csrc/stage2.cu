@@ -17,16 +17,18 @@
 //   - the n_sel largest scores are kept, ties to the lower slot;
 //   - attention over the kept candidates and the dense tail.
 // Three kernels:
-//   sel_score : one thread per candidate slot, G fp32 dot products with q
-//               from shared memory, the maximum written per slot;
+//   sel_score : one thread per candidate (a CTA scans its segments'
+//               kept-token counts), G fp32 dot products with q from shared
+//               memory, the maximum written per slot (-inf for empty slots);
 //   sel_topn  : one CTA per unit, an exact radix select of the n_sel-th
 //               largest score key (8-bit digits), the tied keys taken in
 //               slot order by a block scan, the kept slots written ascending;
 //   sel_attn  : the unit's items (kept slots, then tail tokens) cut into
-//               equal chunks, one CTA per chunk; a warp per item with lanes
-//               over d (coalesced 8-byte key / value reads), online softmax
-//               per head, fixed-order warp and chunk merges (the last CTA of
-//               a unit, by atomic ticket, writes the fp16 output).
+//               equal chunks, one CTA per chunk; groups of 8 (G <= 4) or 16
+//               lanes per item with lanes over d (16-byte key / value reads),
+//               online softmax per head, fixed-order group, warp and chunk
+//               merges (the last CTA of a unit, by atomic ticket, writes the
+//               fp16 output).
 #include <algorithm>
 
 #include "kernels.h"
@@ -132,71 +134,122 @@ __device__ __forceinline__ Cand candidate(const Sel2Args& A, int u, int j, int i
 
 // ------------------------------------------------------------- scores
 
+constexpr int kScoreSegs = 64;    // segments per CTA of the score kernel
+
+// One CTA per kScoreSegs segments of a unit.  The segments' kept-token
+// counts are scanned in shared memory, so that each thread takes real
+// candidates (not empty slots of TOK / BOTH segments); every slot past a
+// segment's kept tokens gets -inf.  A thread computes the G logits of its
+// candidate (fp32, dimensions in ascending order) and writes their maximum.
 __global__ void __launch_bounds__(kScoreThreads) sel_score_kernel(const __grid_constant__ Sel2Args A) {
     pdl_wait();
     __shared__ __align__(16) float qs[8][kHeadDim];
+    __shared__ int pre[kScoreSegs + 1];
     const int u = blockIdx.y;
     const int b = u / A.Hkv, h = u % A.Hkv;
-    const int G = A.G;
+    const int G = A.G, S = A.S;
+    const int nsg = unit_segs(A, u, blockIdx.x == 0 && threadIdx.x == 0);
+    const int j0 = blockIdx.x * kScoreSegs;
+    if (j0 >= nsg) return;
+    const int nj = min(kScoreSegs, nsg - j0);
     for (int x = threadIdx.x; x < G * kHeadDim; x += kScoreThreads)
         qs[x / kHeadDim][x % kHeadDim] =
             __half2float(A.q[(static_cast<int64_t>(b) * A.Hq + h * G + x / kHeadDim) * kHeadDim + x % kHeadDim]);
+    if (threadIdx.x < 32) {
+        // inclusive scan of the kept-token counts of the CTA's segments
+        const int lane = threadIdx.x;
+        int carry = 0;
+        for (int k0 = 0; k0 < kScoreSegs; k0 += 32) {
+            const int j = j0 + k0 + lane;
+            int n = 0;
+            if (k0 + lane < nj) {
+                const int st = static_cast<int>((A.desc[static_cast<int64_t>(u) * A.max_segs + j] >> 32) & 255u);
+                n = (st == KV2D_TOK || st == KV2D_BOTH) ? A.r : S;
+            }
+            int x = n;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, x, o);
+                if (lane >= o) x += y;
+            }
+            pre[k0 + lane + 1] = carry + x;
+            carry += __shfl_sync(0xffffffffu, x, 31);
+        }
+        if (lane == 0) pre[0] = 0;
+    }
     __syncthreads();
-    const int nsg = unit_segs(A, u, blockIdx.x == 0 && threadIdx.x == 0);
-    const int64_t slot = static_cast<int64_t>(blockIdx.x) * kScoreThreads + threadIdx.x;
-    if (slot >= static_cast<int64_t>(nsg) * A.S) return;
-    const int j = static_cast<int>(slot / A.S), i = static_cast<int>(slot % A.S);
-    const Cand cd = candidate(A, u, j, i, true);
-    float best = kNegInf2;
-    if (cd.kind != 0) {
-        float acc[8];
+    float* sc = A.score + static_cast<int64_t>(u) * A.slot_stride + static_cast<int64_t>(j0) * S;
+    float* dsc = A.dbg_score ? A.dbg_score + static_cast<int64_t>(u) * A.slot_stride + static_cast<int64_t>(j0) * S
+                             : nullptr;
+    // empty slots
+    for (int x = threadIdx.x; x < nj * S; x += kScoreThreads) {
+        const int k = x / S, i = x % S;
+        if (i >= pre[k + 1] - pre[k]) {
+            sc[x] = kNegInf2;
+            if (dsc) dsc[x] = kNegInf2;
+        }
+    }
+    const int ncand = pre[nj];
+    for (int cidx = threadIdx.x; cidx < ncand; cidx += kScoreThreads) {
+        int lo = 0, hi = nj;             // the segment k with pre[k] <= cidx < pre[k + 1]
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (pre[mid] <= cidx) lo = mid;
+            else hi = mid;
+        }
+        const int k = lo, i = cidx - pre[k];
+        const Cand cd = candidate(A, u, j0 + k, i, true);
+        float best = kNegInf2;
+        if (cd.kind != 0) {
+            float acc[8];
 #pragma unroll
-        for (int g = 0; g < 8; ++g) acc[g] = 0.f;
-        if (cd.kind == 1) {
+            for (int g = 0; g < 8; ++g) acc[g] = 0.f;
+            if (cd.kind == 1) {
 #pragma unroll 2
-            for (int ch = 0; ch < 16; ++ch) {
-                const uint4 w = *reinterpret_cast<const uint4*>(cd.key + ch * 16);
-                const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-                float kf[8];
+                for (int ch = 0; ch < 16; ++ch) {
+                    const uint4 w = *reinterpret_cast<const uint4*>(cd.key + ch * 16);
+                    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+                    float kf[8];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&ws[e]));
-                    kf[2 * e] = f.x;
-                    kf[2 * e + 1] = f.y;
-                }
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&ws[e]));
+                        kf[2 * e] = f.x;
+                        kf[2 * e + 1] = f.y;
+                    }
 #pragma unroll
-                for (int g = 0; g < 8; ++g) {
-                    if (g < G) {
-                        const float4 q0 = *reinterpret_cast<const float4*>(&qs[g][ch * 8]);
-                        const float4 q1 = *reinterpret_cast<const float4*>(&qs[g][ch * 8 + 4]);
-                        float a = acc[g];
-                        a = fmaf(q0.x, kf[0], a);
-                        a = fmaf(q0.y, kf[1], a);
-                        a = fmaf(q0.z, kf[2], a);
-                        a = fmaf(q0.w, kf[3], a);
-                        a = fmaf(q1.x, kf[4], a);
-                        a = fmaf(q1.y, kf[5], a);
-                        a = fmaf(q1.z, kf[6], a);
-                        a = fmaf(q1.w, kf[7], a);
-                        acc[g] = a;
+                    for (int g = 0; g < 8; ++g) {
+                        if (g < G) {
+                            const float4 q0 = *reinterpret_cast<const float4*>(&qs[g][ch * 8]);
+                            const float4 q1 = *reinterpret_cast<const float4*>(&qs[g][ch * 8 + 4]);
+                            float a = acc[g];
+                            a = fmaf(q0.x, kf[0], a);
+                            a = fmaf(q0.y, kf[1], a);
+                            a = fmaf(q0.z, kf[2], a);
+                            a = fmaf(q0.w, kf[3], a);
+                            a = fmaf(q1.x, kf[4], a);
+                            a = fmaf(q1.y, kf[5], a);
+                            a = fmaf(q1.z, kf[6], a);
+                            a = fmaf(q1.w, kf[7], a);
+                            acc[g] = a;
+                        }
                     }
                 }
-            }
-        } else {
-            for (int x = 0; x < A.c; ++x) {
-                const int ci = cd.key[x] & 0x7f;     // indices are < 128; the mask keeps a bad byte in range
-                const float kv = __half2float(cd.kval[x]);
+            } else {
+                for (int x = 0; x < A.c; ++x) {
+                    const int ci = cd.key[x] & 0x7f;     // indices are < 128; the mask keeps a bad byte in range
+                    const float kv = __half2float(cd.kval[x]);
 #pragma unroll
-                for (int g = 0; g < 8; ++g)
-                    if (g < G) acc[g] = fmaf(qs[g][ci], kv, acc[g]);
+                    for (int g = 0; g < 8; ++g)
+                        if (g < G) acc[g] = fmaf(qs[g][ci], kv, acc[g]);
+                }
             }
+#pragma unroll
+            for (int g = 0; g < 8; ++g)
+                if (g < G) best = fmaxf(best, A.scale * acc[g]);
         }
-#pragma unroll
-        for (int g = 0; g < 8; ++g)
-            if (g < G) best = fmaxf(best, A.scale * acc[g]);
+        sc[static_cast<int64_t>(k) * S + i] = best;
+        if (dsc) dsc[static_cast<int64_t>(k) * S + i] = best;
     }
-    A.score[static_cast<int64_t>(u) * A.slot_stride + slot] = best;
-    if (A.dbg_score) A.dbg_score[static_cast<int64_t>(u) * A.slot_stride + slot] = best;
 }
 
 // ---------------------------------------------------------- selection
@@ -348,9 +401,18 @@ __global__ void __launch_bounds__(kTopThreads) sel_topn_kernel(const __grid_cons
 
 // ---------------------------------------------------------- attention
 
+// A group of LPI lanes takes one item at a time (LPI = 8 for G <= 4, 16 for
+// G = 8), so a warp has 32 / LPI items in flight; lane k of a group owns
+// dimensions [k * 128 / LPI, (k + 1) * 128 / LPI).  The group's G logits are
+// summed with a butterfly inside the group (fixed order), then each head's
+// online softmax (log2 domain) updates the group's running max, sum and
+// output slice.  Groups, then warps, then chunks merge in a fixed order.
 template <int G>
-__global__ void __launch_bounds__(kAttnWarps * 32) sel_attn_kernel(const __grid_constant__ Sel2Args A) {
+__global__ void __launch_bounds__(kAttnWarps * 32, 2) sel_attn_kernel(const __grid_constant__ Sel2Args A) {
     pdl_wait();
+    constexpr int LPI = (G <= 4) ? 8 : 16;       // lanes per item
+    constexpr int DPL = kHeadDim / LPI;          // dims per lane (16 or 8)
+    constexpr int IPW = 32 / LPI;                // items per warp in flight
     constexpr int kRec = kHeadDim + 4;
     __shared__ __align__(16) float qs[G][kHeadDim];
     __shared__ float wm[kAttnWarps][G], wl[kAttnWarps][G];
@@ -359,6 +421,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32) sel_attn_kernel(const __grid_
     const int c_id = blockIdx.x, u = blockIdx.y;
     const int b = u / A.Hkv, h = u % A.Hkv;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int grp = lane / LPI, lg = lane % LPI;
     for (int x = tid; x < G * kHeadDim; x += kAttnWarps * 32)
         qs[x / kHeadDim][x % kHeadDim] =
             __half2float(A.q[(static_cast<int64_t>(b) * A.Hq + h * G + x / kHeadDim) * kHeadDim + x % kHeadDim]);
@@ -375,39 +438,31 @@ __global__ void __launch_bounds__(kAttnWarps * 32) sel_attn_kernel(const __grid_
     const int64_t items = nsel + (T - ce);
     const int64_t i_lo = items * c_id / A.nchunk, i_hi = items * (c_id + 1) / A.nchunk;
     const int32_t* sl = A.sel + static_cast<int64_t>(u) * A.slot_stride;
-    // lane l holds dims 4l .. 4l + 3 of q (log2-domain scale folded in later)
-    float qv[G][4];
-#pragma unroll
-    for (int g = 0; g < G; ++g)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) qv[g][e] = qs[g][4 * lane + e];
-    float m[G], l[G], o[G][4];
+    const unsigned gmask = (LPI == 32) ? 0xffffffffu : (((1u << LPI) - 1u) << (grp * LPI));
+    float m[G], l[G], o[G][DPL];
 #pragma unroll
     for (int g = 0; g < G; ++g) {
         m[g] = kNegInf2;
         l[g] = 0.f;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) o[g][e] = 0.f;
+        for (int e = 0; e < DPL; ++e) o[g][e] = 0.f;
     }
-    for (int64_t it = i_lo + warp; it < i_hi; it += kAttnWarps) {
+    const int d0 = lg * DPL;
+    for (int64_t it = i_lo + warp * IPW + grp; it < i_hi; it += kAttnWarps * IPW) {
         float dot[G];
 #pragma unroll
         for (int g = 0; g < G; ++g) dot[g] = 0.f;
         const __half* vrow = nullptr;
+        const __half* krow = nullptr;
         if (it < nsel) {
             const int32_t slot = sl[it];
-            const Cand cd = candidate(A, u, slot / A.S, slot % A.S, lane == 0);
-            if (cd.kind == 0) continue;      // (status already set; warp-uniform)
+            const Cand cd = candidate(A, u, slot / A.S, slot % A.S, lg == 0);
+            if (cd.kind == 0) continue;      // (status already set; uniform in the group)
             vrow = cd.vrow;
             if (cd.kind == 1) {
-                const uint2 kw = *reinterpret_cast<const uint2*>(cd.key + lane * 8);
-                const float2 k01 = __half22float2(*reinterpret_cast<const __half2*>(&kw.x));
-                const float2 k23 = __half22float2(*reinterpret_cast<const __half2*>(&kw.y));
-#pragma unroll
-                for (int g = 0; g < G; ++g)
-                    dot[g] = fmaf(qv[g][3], k23.y, fmaf(qv[g][2], k23.x, fmaf(qv[g][1], k01.y, qv[g][0] * k01.x)));
+                krow = reinterpret_cast<const __half*>(cd.key);
             } else {
-                for (int x = lane; x < A.c; x += 32) {
+                for (int x = lg; x < A.c; x += LPI) {
                     const int ci = cd.key[x] & 0x7f;
                     const float kv = __half2float(cd.kval[x]);
 #pragma unroll
@@ -416,24 +471,43 @@ __global__ void __launch_bounds__(kAttnWarps * 32) sel_attn_kernel(const __grid_
             }
         } else {
             const int t = ce + static_cast<int>(it - nsel);
-            const __half* kr = dense_row(A.dv, A.dv.k, b, h, t, lane == 0 ? A.status : nullptr);
+            krow = dense_row(A.dv, A.dv.k, b, h, t, lg == 0 ? A.status : nullptr);
             vrow = dense_row(A.dv, A.dv.v, b, h, t, nullptr);
-            if (!kr || !vrow) continue;      // warp-uniform
-            const uint2 kw = *reinterpret_cast<const uint2*>(kr + lane * 4);
-            const float2 k01 = __half22float2(*reinterpret_cast<const __half2*>(&kw.x));
-            const float2 k23 = __half22float2(*reinterpret_cast<const __half2*>(&kw.y));
-#pragma unroll
-            for (int g = 0; g < G; ++g)
-                dot[g] = fmaf(qv[g][3], k23.y, fmaf(qv[g][2], k23.x, fmaf(qv[g][1], k01.y, qv[g][0] * k01.x)));
+            if (!krow || !vrow) continue;    // uniform in the group
         }
-        // every lane gets the G logits (fixed butterfly order)
+        uint4 vw[DPL / 8];
+#pragma unroll
+        for (int k = 0; k < DPL / 8; ++k) vw[k] = *reinterpret_cast<const uint4*>(vrow + d0 + 8 * k);
+        if (krow) {
+#pragma unroll
+            for (int k = 0; k < DPL / 8; ++k) {
+                const uint4 kw = *reinterpret_cast<const uint4*>(krow + d0 + 8 * k);
+                const uint32_t ws[4] = {kw.x, kw.y, kw.z, kw.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&ws[e]));
+                    const int x = d0 + 8 * k + 2 * e;
+#pragma unroll
+                    for (int g = 0; g < G; ++g) dot[g] = fmaf(qs[g][x + 1], f.y, fmaf(qs[g][x], f.x, dot[g]));
+                }
+            }
+        }
+        // the group's G logits (butterfly inside the group, fixed order)
 #pragma unroll
         for (int g = 0; g < G; ++g)
 #pragma unroll
-            for (int off = 16; off > 0; off >>= 1) dot[g] += __shfl_xor_sync(0xffffffffu, dot[g], off);
-        const uint2 vw = *reinterpret_cast<const uint2*>(vrow + lane * 4);
-        const float2 v01 = __half22float2(*reinterpret_cast<const __half2*>(&vw.x));
-        const float2 v23 = __half22float2(*reinterpret_cast<const __half2*>(&vw.y));
+            for (int off = LPI / 2; off > 0; off >>= 1) dot[g] += __shfl_xor_sync(gmask, dot[g], off, LPI);
+        float vf[DPL];
+#pragma unroll
+        for (int k = 0; k < DPL / 8; ++k) {
+            const uint32_t ws[4] = {vw[k].x, vw[k].y, vw[k].z, vw[k].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&ws[e]));
+                vf[8 * k + 2 * e] = f.x;
+                vf[8 * k + 2 * e + 1] = f.y;
+            }
+        }
 #pragma unroll
         for (int g = 0; g < G; ++g) {
             const float x = dot[g] * A.c2;
@@ -442,20 +516,46 @@ __global__ void __launch_bounds__(kAttnWarps * 32) sel_attn_kernel(const __grid_
             const float p = fast_exp2(x - mn);
             m[g] = mn;
             l[g] = fmaf(l[g], alpha, p);
-            o[g][0] = fmaf(o[g][0], alpha, p * v01.x);
-            o[g][1] = fmaf(o[g][1], alpha, p * v01.y);
-            o[g][2] = fmaf(o[g][2], alpha, p * v23.x);
-            o[g][3] = fmaf(o[g][3], alpha, p * v23.y);
+#pragma unroll
+            for (int e = 0; e < DPL; ++e) o[g][e] = fmaf(o[g][e], alpha, p * vf[e]);
         }
     }
-    // warp partials -> the chunk's partial (warps merged in order)
+    // the warp's groups merged in order (butterfly over groups), then the
+    // warps, then the chunks
+#pragma unroll
+    for (int off = LPI; off < 32; off <<= 1) {
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            const float m2 = __shfl_xor_sync(0xffffffffu, m[g], off);
+            const float l2 = __shfl_xor_sync(0xffffffffu, l[g], off);
+            const float M = fmaxf(m[g], m2);
+            const float s1 = (m[g] == kNegInf2) ? 0.f : fast_exp2(m[g] - M);
+            const float s2 = (m2 == kNegInf2) ? 0.f : fast_exp2(m2 - M);
+            // the lower group's values first, whichever lane adds
+            const bool low = (lane & off) == 0;
+            const float sa = low ? s1 : s2, sb = low ? s2 : s1;
+            const float la = low ? l[g] : l2, lb = low ? l2 : l[g];
+            l[g] = fmaf(lb, sb, la * sa);
+#pragma unroll
+            for (int e = 0; e < DPL; ++e) {
+                const float o2 = __shfl_xor_sync(0xffffffffu, o[g][e], off);
+                const float oa = low ? o[g][e] : o2, ob = low ? o2 : o[g][e];
+                o[g][e] = fmaf(ob, sb, oa * sa);
+            }
+            m[g] = M;
+        }
+    }
 #pragma unroll
     for (int g = 0; g < G; ++g) {
         if (lane == 0) {
             wm[warp][g] = m[g];
             wl[warp][g] = l[g];
         }
-        *reinterpret_cast<float4*>(&wo[warp][g][4 * lane]) = make_float4(o[g][0], o[g][1], o[g][2], o[g][3]);
+        if (grp == 0) {
+#pragma unroll
+            for (int e = 0; e < DPL; e += 4)
+                *reinterpret_cast<float4*>(&wo[warp][g][d0 + e]) = make_float4(o[g][e], o[g][e + 1], o[g][e + 2], o[g][e + 3]);
+        }
     }
     __syncthreads();
     float* myp = A.part + (static_cast<int64_t>(u) * A.nchunk + c_id) * G * kRec;
@@ -550,7 +650,8 @@ cudaError_t launch_decode_select(const DecodeSelectLaunch& L, cudaStream_t strea
     cudaError_t e;
     prof_begin(stream, kProfSelScore);
     if (L.slot_stride > 0) {
-        dim3 g1(static_cast<unsigned>((L.slot_stride + kScoreThreads - 1) / kScoreThreads), units);
+        const int64_t segs = L.slot_stride / L.shp.S;
+        dim3 g1(static_cast<unsigned>((segs + kScoreSegs - 1) / kScoreSegs), units);
         e = launch_k(sel_score_kernel, g1, dim3(kScoreThreads), 0, stream, a);
         if (e != cudaSuccess) return e;
     }
