@@ -100,17 +100,21 @@ struct Cand {
     const __half* vrow;    // value row
 };
 
-__device__ __forceinline__ Cand candidate(const Sel2Args& A, int u, int j, int i, bool report) {
+// The unit's packed bytes, clamped into its arena.
+__device__ __forceinline__ int64_t unit_used(const Sel2Args& A, int u) {
+    const int64_t U = A.used_bytes[u];
+    return max(static_cast<int64_t>(0), min(U, A.arena_stride));
+}
+
+// Candidate i of the segment with descriptor d; U = the unit's used bytes.
+__device__ __forceinline__ Cand candidate_of(const Sel2Args& A, int u, int64_t U, uint64_t d, int i, bool report) {
     Cand cd{0, nullptr, nullptr, nullptr};
-    const uint64_t d = A.desc[static_cast<int64_t>(u) * A.max_segs + j];
     const int st = static_cast<int>((d >> 32) & 255u);
     const int64_t off = static_cast<int64_t>(d & 0xffffffffull) * 16;
     const int S = A.S, r = A.r, c = A.c;
     const bool tok = (st == KV2D_TOK || st == KV2D_BOTH);
     const int ntok = tok ? r : S;
     if (i >= ntok) return cd;
-    int64_t U = A.used_bytes[u];
-    U = max(static_cast<int64_t>(0), min(U, A.arena_stride));
     if (st > KV2D_BOTH || off < 0 || off + seg_payload(st, S, r, c) > U) {
         if (report) set_status(A.status, KV2D_DEV_CAPACITY);
         return cd;
@@ -130,6 +134,10 @@ __device__ __forceinline__ Cand candidate(const Sel2Args& A, int u, int j, int i
                   static_cast<int64_t>(i) * kHeadDim;
     }
     return cd;
+}
+
+__device__ __forceinline__ uint64_t seg_desc(const Sel2Args& A, int u, int j) {
+    return A.desc[static_cast<int64_t>(u) * A.max_segs + j];
 }
 
 // ------------------------------------------------------------- scores
@@ -190,6 +198,7 @@ __global__ void __launch_bounds__(kScoreThreads) sel_score_kernel(const __grid_c
         }
     }
     const int ncand = pre[nj];
+    const int64_t U = unit_used(A, u);
     for (int cidx = threadIdx.x; cidx < ncand; cidx += kScoreThreads) {
         int lo = 0, hi = nj;             // the segment k with pre[k] <= cidx < pre[k + 1]
         while (hi - lo > 1) {
@@ -198,7 +207,7 @@ __global__ void __launch_bounds__(kScoreThreads) sel_score_kernel(const __grid_c
             else hi = mid;
         }
         const int k = lo, i = cidx - pre[k];
-        const Cand cd = candidate(A, u, j0 + k, i, true);
+        const Cand cd = candidate_of(A, u, U, seg_desc(A, u, j0 + k), i, true);
         float best = kNegInf2;
         if (cd.kind != 0) {
             float acc[8];
@@ -324,9 +333,23 @@ __global__ void __launch_bounds__(kTopThreads) sel_topn_kernel(const __grid_cons
         __syncthreads();
         const uint32_t pre = s_prefix;
         const uint32_t hmask = pass == 0 ? 0u : (0xffffffffu << (shift + 8));
-        for (int64_t s = tid; s < nslots; s += kTopThreads) {
-            const uint32_t k = score_key(sc[s]);
-            if (k != 0u && (k & hmask) == (pre & hmask)) atomicAdd(&hist[(k >> shift) & 255u], 1u);
+        // lanes with the same digit add once (scores cluster in few digits,
+        // so plain shared atomics would serialise on one address)
+        const int lane = tid & 31;
+        for (int64_t s0 = tid - lane; s0 < nslots; s0 += 4 * kTopThreads) {
+            float v[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int64_t s = s0 + lane + static_cast<int64_t>(k) * kTopThreads;
+                v[k] = (s < nslots) ? sc[s] : kNegInf2;
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const uint32_t key = score_key(v[k]);
+                const int dg = (key != 0u && (key & hmask) == (pre & hmask)) ? static_cast<int>((key >> shift) & 255u) : -1;
+                const uint32_t peers = __match_any_sync(0xffffffffu, dg);
+                if (dg >= 0 && lane == __ffs(peers) - 1) atomicAdd(&hist[dg], static_cast<unsigned>(__popc(peers)));
+            }
         }
         __syncthreads();
         if (tid < 32) {
@@ -448,33 +471,50 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 2) sel_attn_kernel(const __gr
         for (int e = 0; e < DPL; ++e) o[g][e] = 0.f;
     }
     const int d0 = lg * DPL;
-    for (int64_t it = i_lo + warp * IPW + grp; it < i_hi; it += kAttnWarps * IPW) {
+    const int64_t U = unit_used(A, u);
+    constexpr int64_t kStep = kAttnWarps * IPW;
+    // the next item's slot and descriptor are loaded while this one is
+    // computed (the chain slot -> descriptor -> key / value is three loads)
+    int64_t it = i_lo + warp * IPW + grp;
+    int32_t slot_n = (it < i_hi && it < nsel) ? sl[it] : 0;
+    uint64_t desc_n = (it < i_hi && it < nsel) ? seg_desc(A, u, slot_n / A.S) : 0ull;
+    for (; it < i_hi; it += kStep) {
+        const int32_t slot = slot_n;
+        const uint64_t dsc = desc_n;
+        const int64_t it2 = it + kStep;
+        const bool next_sel = it2 < i_hi && it2 < nsel;
+        if (next_sel) slot_n = sl[it2];
         float dot[G];
 #pragma unroll
         for (int g = 0; g < G; ++g) dot[g] = 0.f;
         const __half* vrow = nullptr;
         const __half* krow = nullptr;
+        bool skip = false;
         if (it < nsel) {
-            const int32_t slot = sl[it];
-            const Cand cd = candidate(A, u, slot / A.S, slot % A.S, lg == 0);
-            if (cd.kind == 0) continue;      // (status already set; uniform in the group)
-            vrow = cd.vrow;
-            if (cd.kind == 1) {
-                krow = reinterpret_cast<const __half*>(cd.key);
+            const Cand cd = candidate_of(A, u, U, dsc, slot % A.S, lg == 0);
+            if (cd.kind == 0) {
+                skip = true;                 // (status already set; uniform in the group)
             } else {
-                for (int x = lg; x < A.c; x += LPI) {
-                    const int ci = cd.key[x] & 0x7f;
-                    const float kv = __half2float(cd.kval[x]);
+                vrow = cd.vrow;
+                if (cd.kind == 1) {
+                    krow = reinterpret_cast<const __half*>(cd.key);
+                } else {
+                    for (int x = lg; x < A.c; x += LPI) {
+                        const int ci = cd.key[x] & 0x7f;
+                        const float kv = __half2float(cd.kval[x]);
 #pragma unroll
-                    for (int g = 0; g < G; ++g) dot[g] = fmaf(qs[g][ci], kv, dot[g]);
+                        for (int g = 0; g < G; ++g) dot[g] = fmaf(qs[g][ci], kv, dot[g]);
+                    }
                 }
             }
         } else {
             const int t = ce + static_cast<int>(it - nsel);
             krow = dense_row(A.dv, A.dv.k, b, h, t, lg == 0 ? A.status : nullptr);
             vrow = dense_row(A.dv, A.dv.v, b, h, t, nullptr);
-            if (!krow || !vrow) continue;    // uniform in the group
+            skip = !krow || !vrow;           // uniform in the group
         }
+        if (next_sel) desc_n = seg_desc(A, u, slot_n / A.S);
+        if (skip) continue;
         uint4 vw[DPL / 8];
 #pragma unroll
         for (int k = 0; k < DPL / 8; ++k) vw[k] = *reinterpret_cast<const uint4*>(vrow + d0 + 8 * k);
