@@ -149,13 +149,14 @@ constexpr int kScoreSegs = 64;    // segments per CTA of the score kernel
 // candidates (not empty slots of TOK / BOTH segments); every slot past a
 // segment's kept tokens gets -inf.  A thread computes the G logits of its
 // candidate (fp32, dimensions in ascending order) and writes their maximum.
+template <int G>
 __global__ void __launch_bounds__(kScoreThreads) sel_score_kernel(const __grid_constant__ Sel2Args A) {
     pdl_wait();
-    __shared__ __align__(16) float qs[8][kHeadDim];
+    __shared__ __align__(16) float qs[G][kHeadDim];
     __shared__ int pre[kScoreSegs + 1];
     const int u = blockIdx.y;
     const int b = u / A.Hkv, h = u % A.Hkv;
-    const int G = A.G, S = A.S;
+    const int S = A.S;
     const int nsg = unit_segs(A, u, blockIdx.x == 0 && threadIdx.x == 0);
     const int j0 = blockIdx.x * kScoreSegs;
     if (j0 >= nsg) return;
@@ -210,9 +211,9 @@ __global__ void __launch_bounds__(kScoreThreads) sel_score_kernel(const __grid_c
         const Cand cd = candidate_of(A, u, U, seg_desc(A, u, j0 + k), i, true);
         float best = kNegInf2;
         if (cd.kind != 0) {
-            float acc[8];
+            float acc[G];
 #pragma unroll
-            for (int g = 0; g < 8; ++g) acc[g] = 0.f;
+            for (int g = 0; g < G; ++g) acc[g] = 0.f;
             if (cd.kind == 1) {
 #pragma unroll 2
                 for (int ch = 0; ch < 16; ++ch) {
@@ -226,21 +227,19 @@ __global__ void __launch_bounds__(kScoreThreads) sel_score_kernel(const __grid_c
                         kf[2 * e + 1] = f.y;
                     }
 #pragma unroll
-                    for (int g = 0; g < 8; ++g) {
-                        if (g < G) {
-                            const float4 q0 = *reinterpret_cast<const float4*>(&qs[g][ch * 8]);
-                            const float4 q1 = *reinterpret_cast<const float4*>(&qs[g][ch * 8 + 4]);
-                            float a = acc[g];
-                            a = fmaf(q0.x, kf[0], a);
-                            a = fmaf(q0.y, kf[1], a);
-                            a = fmaf(q0.z, kf[2], a);
-                            a = fmaf(q0.w, kf[3], a);
-                            a = fmaf(q1.x, kf[4], a);
-                            a = fmaf(q1.y, kf[5], a);
-                            a = fmaf(q1.z, kf[6], a);
-                            a = fmaf(q1.w, kf[7], a);
-                            acc[g] = a;
-                        }
+                    for (int g = 0; g < G; ++g) {
+                        const float4 q0 = *reinterpret_cast<const float4*>(&qs[g][ch * 8]);
+                        const float4 q1 = *reinterpret_cast<const float4*>(&qs[g][ch * 8 + 4]);
+                        float a = acc[g];
+                        a = fmaf(q0.x, kf[0], a);
+                        a = fmaf(q0.y, kf[1], a);
+                        a = fmaf(q0.z, kf[2], a);
+                        a = fmaf(q0.w, kf[3], a);
+                        a = fmaf(q1.x, kf[4], a);
+                        a = fmaf(q1.y, kf[5], a);
+                        a = fmaf(q1.z, kf[6], a);
+                        a = fmaf(q1.w, kf[7], a);
+                        acc[g] = a;
                     }
                 }
             } else {
@@ -248,13 +247,11 @@ __global__ void __launch_bounds__(kScoreThreads) sel_score_kernel(const __grid_c
                     const int ci = cd.key[x] & 0x7f;     // indices are < 128; the mask keeps a bad byte in range
                     const float kv = __half2float(cd.kval[x]);
 #pragma unroll
-                    for (int g = 0; g < 8; ++g)
-                        if (g < G) acc[g] = fmaf(qs[g][ci], kv, acc[g]);
+                    for (int g = 0; g < G; ++g) acc[g] = fmaf(qs[g][ci], kv, acc[g]);
                 }
             }
 #pragma unroll
-            for (int g = 0; g < 8; ++g)
-                if (g < G) best = fmaxf(best, A.scale * acc[g]);
+            for (int g = 0; g < G; ++g) best = fmaxf(best, A.scale * acc[g]);
         }
         sc[static_cast<int64_t>(k) * S + i] = best;
         if (dsc) dsc[static_cast<int64_t>(k) * S + i] = best;
@@ -437,7 +434,10 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 2) sel_attn_kernel(const __gr
     constexpr int DPL = kHeadDim / LPI;          // dims per lane (16 or 8)
     constexpr int IPW = 32 / LPI;                // items per warp in flight
     constexpr int kRec = kHeadDim + 4;
-    __shared__ __align__(16) float qs[G][kHeadDim];
+    // q rows padded by 4 floats per 16 dims, so that the 8 lanes of a group
+    // (16 dims each) read distinct bank groups
+    constexpr int kQRow = kHeadDim + kHeadDim / 4;
+    __shared__ __align__(16) float qs[G][kQRow];
     __shared__ float wm[kAttnWarps][G], wl[kAttnWarps][G];
     __shared__ __align__(16) float wo[kAttnWarps][G][kHeadDim];
     __shared__ int is_last;
@@ -445,8 +445,9 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 2) sel_attn_kernel(const __gr
     const int b = u / A.Hkv, h = u % A.Hkv;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int grp = lane / LPI, lg = lane % LPI;
+    auto qix = [](int x) { return x + 4 * (x >> 4); };
     for (int x = tid; x < G * kHeadDim; x += kAttnWarps * 32)
-        qs[x / kHeadDim][x % kHeadDim] =
+        qs[x / kHeadDim][qix(x % kHeadDim)] =
             __half2float(A.q[(static_cast<int64_t>(b) * A.Hq + h * G + x / kHeadDim) * kHeadDim + x % kHeadDim]);
     __syncthreads();
     // the unit's items: kept candidates, then its dense tail tokens
@@ -503,7 +504,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 2) sel_attn_kernel(const __gr
                         const int ci = cd.key[x] & 0x7f;
                         const float kv = __half2float(cd.kval[x]);
 #pragma unroll
-                        for (int g = 0; g < G; ++g) dot[g] = fmaf(qs[g][ci], kv, dot[g]);
+                        for (int g = 0; g < G; ++g) dot[g] = fmaf(qs[g][qix(ci)], kv, dot[g]);
                     }
                 }
             }
@@ -519,6 +520,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 2) sel_attn_kernel(const __gr
 #pragma unroll
         for (int k = 0; k < DPL / 8; ++k) vw[k] = *reinterpret_cast<const uint4*>(vrow + d0 + 8 * k);
         if (krow) {
+            float kf[DPL];
 #pragma unroll
             for (int k = 0; k < DPL / 8; ++k) {
                 const uint4 kw = *reinterpret_cast<const uint4*>(krow + d0 + 8 * k);
@@ -526,9 +528,16 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 2) sel_attn_kernel(const __gr
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&ws[e]));
-                    const int x = d0 + 8 * k + 2 * e;
+                    kf[8 * k + 2 * e] = f.x;
+                    kf[8 * k + 2 * e + 1] = f.y;
+                }
+            }
 #pragma unroll
-                    for (int g = 0; g < G; ++g) dot[g] = fmaf(qs[g][x + 1], f.y, fmaf(qs[g][x], f.x, dot[g]));
+            for (int g = 0; g < G; ++g) {
+#pragma unroll
+                for (int k4 = 0; k4 < DPL; k4 += 4) {
+                    const float4 q4 = *reinterpret_cast<const float4*>(&qs[g][qix(d0 + k4)]);
+                    dot[g] = fmaf(q4.w, kf[k4 + 3], fmaf(q4.z, kf[k4 + 2], fmaf(q4.y, kf[k4 + 1], fmaf(q4.x, kf[k4], dot[g]))));
                 }
             }
         }
@@ -692,7 +701,13 @@ cudaError_t launch_decode_select(const DecodeSelectLaunch& L, cudaStream_t strea
     if (L.slot_stride > 0) {
         const int64_t segs = L.slot_stride / L.shp.S;
         dim3 g1(static_cast<unsigned>((segs + kScoreSegs - 1) / kScoreSegs), units);
-        e = launch_k(sel_score_kernel, g1, dim3(kScoreThreads), 0, stream, a);
+        switch (L.shp.G) {
+        case 1: e = launch_k(sel_score_kernel<1>, g1, dim3(kScoreThreads), 0, stream, a); break;
+        case 2: e = launch_k(sel_score_kernel<2>, g1, dim3(kScoreThreads), 0, stream, a); break;
+        case 4: e = launch_k(sel_score_kernel<4>, g1, dim3(kScoreThreads), 0, stream, a); break;
+        case 8: e = launch_k(sel_score_kernel<8>, g1, dim3(kScoreThreads), 0, stream, a); break;
+        default: return cudaErrorInvalidValue;
+        }
         if (e != cudaSuccess) return e;
     }
     prof_end(stream, kProfSelScore);

@@ -49,6 +49,8 @@ typedef struct {
     int32_t c;       /* channels kept per key vector by CH / BOTH        */
     double beta;     /* byte budget as a fraction of the FULL bytes      */
     double scale;    /* softmax scale                                    */
+    int32_t chunk_len;     /* Token2Chunk: longest chunk (tokens); 0 = off */
+    int32_t chunk_budget;  /* Token2Chunk: tokens chunks may add per segment */
 } orc_params;
 
 enum { ORC_FULL = 0, ORC_TOK = 1, ORC_CH = 2, ORC_BOTH = 3 };
@@ -198,6 +200,87 @@ void orc_topr(const orc_params* p, const double* s_seg, uint8_t* tidx)
     for (int t = 0; t < S; ++t)
         if (sel[t]) tidx[w++] = (uint8_t)t;
     free(sel);
+}
+
+/* Token2Chunk variant of R_j ([Kara] "What carries the argument": high-score
+ * tokens are endpoints of candidate flexible chunks, the best kept under a
+ * length cap and a budget; free parameters: max chunk length gamma and
+ * chunk budget alpha).  The page gives no equations; the reading taken
+ * keeps exactly r tokens (so the TOK / BOTH byte layout does not change):
+ *   1. core: the r - alpha tokens with the largest s, ties to the lower t;
+ *   2. candidates: every gap between consecutive core positions a < b with
+ *      b - a - 1 >= 1 and b - a + 1 <= gamma; its merit is the sum of s over
+ *      the gap (fp64, ascending t);
+ *   3. candidates by (merit desc, a asc) are filled while their gap fits the
+ *      remaining budget (a gap that does not fit is skipped);
+ *   4. budget left over goes to the best tokens not yet kept, by (s desc,
+ *      t asc).
+ * Written ascending as segment-relative indices. */
+void orc_topr_chunks(const orc_params* p, const double* s_seg, uint8_t* tidx)
+{
+    int S = p->S, r = p->r, a = p->chunk_budget, gamma = p->chunk_len;
+    unsigned char* sel = (unsigned char*)calloc((size_t)S, 1);
+    int* order = (int*)malloc(sizeof(int) * (size_t)S);
+    /* all tokens by (s desc, t asc): repeated maximum search */
+    unsigned char* used = (unsigned char*)calloc((size_t)S, 1);
+    for (int k = 0; k < S; ++k) {
+        int best = -1;
+        for (int t = 0; t < S; ++t) {
+            if (used[t]) continue;
+            if (best < 0 || s_seg[t] > s_seg[best]) best = t;
+        }
+        used[best] = 1;
+        order[k] = best;
+    }
+    for (int k = 0; k < r - a; ++k) sel[order[k]] = 1;
+    /* candidate gaps between consecutive core positions */
+    int nc = 0;
+    int* ca = (int*)malloc(sizeof(int) * (size_t)S);
+    int* cg = (int*)malloc(sizeof(int) * (size_t)S);
+    double* cm = (double*)malloc(sizeof(double) * (size_t)S);
+    int prev = -1;
+    for (int t = 0; t < S; ++t) {
+        if (!sel[t]) continue;
+        if (prev >= 0 && t - prev - 1 >= 1 && t - prev + 1 <= gamma) {
+            double m = 0.0;
+            for (int x = prev + 1; x < t; ++x) m += s_seg[x];
+            ca[nc] = prev;
+            cg[nc] = t - prev - 1;
+            cm[nc] = m;
+            ++nc;
+        }
+        prev = t;
+    }
+    /* by (merit desc, start asc): selection sort */
+    for (int i = 0; i < nc; ++i) {
+        int best = i;
+        for (int k = i + 1; k < nc; ++k)
+            if (cm[k] > cm[best] || (cm[k] == cm[best] && ca[k] < ca[best])) best = k;
+        int ta = ca[i], tg = cg[i];
+        double tm = cm[i];
+        ca[i] = ca[best]; cg[i] = cg[best]; cm[i] = cm[best];
+        ca[best] = ta; cg[best] = tg; cm[best] = tm;
+    }
+    int rem = a;
+    for (int i = 0; i < nc; ++i) {
+        if (cg[i] > rem) continue;
+        for (int x = ca[i] + 1; x <= ca[i] + cg[i]; ++x) sel[x] = 1;
+        rem -= cg[i];
+    }
+    for (int k = 0; k < S && rem > 0; ++k) {
+        if (sel[order[k]]) continue;
+        sel[order[k]] = 1;
+        --rem;
+    }
+    int w = 0;
+    for (int t = 0; t < S; ++t)
+        if (sel[t]) tidx[w++] = (uint8_t)t;
+    free(sel);
+    free(order);
+    free(used);
+    free(ca);
+    free(cg);
+    free(cm);
 }
 
 /* Error proxy of the four strategies of one segment, read as LOST ATTENTION
@@ -458,7 +541,10 @@ int orc_compress_unit(const orc_params* p, int T, int r0,
     double* eff = (double*)malloc(sizeof(double) * 3 * (size_t)(nseg + 1));
     int64_t* db = (int64_t*)malloc(sizeof(int64_t) * 3 * (size_t)(nseg + 1));
     for (int j = 0; j < nseg; ++j) {
-        orc_topr(p, s + (int64_t)j * S, tidx + (int64_t)j * p->r);
+        if (p->chunk_len > 0)
+            orc_topr_chunks(p, s + (int64_t)j * S, tidx + (int64_t)j * p->r);
+        else
+            orc_topr(p, s + (int64_t)j * S, tidx + (int64_t)j * p->r);
         orc_segment_errors(p, s + (int64_t)j * S, g + (int64_t)j * S,
                            tidx + (int64_t)j * p->r, E + 4 * (int64_t)j);
         nv[j] = orc_hull(p, E + 4 * (int64_t)j, verts + 4 * j, eff + 3 * j, db + 3 * j);

@@ -38,7 +38,8 @@ def build(force: bool = False) -> str:
 
 class Params(C.Structure):
     _fields_ = [("d", C.c_int32), ("G", C.c_int32), ("S", C.c_int32), ("W", C.c_int32),
-                ("r", C.c_int32), ("c", C.c_int32), ("beta", C.c_double), ("scale", C.c_double)]
+                ("r", C.c_int32), ("c", C.c_int32), ("beta", C.c_double), ("scale", C.c_double),
+                ("chunk_len", C.c_int32), ("chunk_budget", C.c_int32)]
 
 
 _lib = None
@@ -61,6 +62,7 @@ def lib():
             L.orc_score.restype = C.c_int
             L.orc_channel.argtypes = [pp, C.c_int, dp, dp, u8p, dp]
             L.orc_topr.argtypes = [pp, dp, u8p]
+            L.orc_topr_chunks.argtypes = [pp, dp, u8p]
             L.orc_segment_errors.argtypes = [pp, dp, dp, u8p, dp]
             L.orc_segment_bytes.argtypes = [pp, C.c_int]
             L.orc_segment_bytes.restype = C.c_int64
@@ -88,10 +90,11 @@ def lib():
     return _lib
 
 
-def params(d, G, S, W, r, c, beta, scale=None) -> Params:
+def params(d, G, S, W, r, c, beta, scale=None, chunk_len=0, chunk_budget=0) -> Params:
     if scale is None:
         scale = 1.0 / np.sqrt(d)
-    return Params(int(d), int(G), int(S), int(W), int(r), int(c), float(beta), float(scale))
+    return Params(int(d), int(G), int(S), int(W), int(r), int(c), float(beta), float(scale),
+                  int(chunk_len), int(chunk_budget))
 
 
 def _p(a, ct):
@@ -146,6 +149,14 @@ def topr(p: Params, s_seg) -> np.ndarray:
     s_seg = _f64(s_seg)
     t = np.zeros(p.r, np.uint8)
     lib().orc_topr(C.byref(p), _p(s_seg, C.c_double), _p(t, C.c_uint8))
+    return t
+
+
+def topr_chunks(p: Params, s_seg) -> np.ndarray:
+    """The Token2Chunk variant of the kept tokens of one segment."""
+    s_seg = _f64(s_seg)
+    t = np.zeros(p.r, np.uint8)
+    lib().orc_topr_chunks(C.byref(p), _p(s_seg, C.c_double), _p(t, C.c_uint8))
     return t
 
 
