@@ -27,6 +27,10 @@
  *   C_t    = the c channels of largest |k_t,d| * a_d, ties to the lower d
  *   g_t    = share of sum_d |k_t,d| a_d carried by the dropped channels
  *   R_j    = the r tokens of segment j with the largest s_t, ties to lower t
+ *            (or, with chunk_len > 0, Kara's Token2Chunk variant: the top
+ *            r - alpha tokens, then whole gaps between consecutive ones of
+ *            span <= gamma by summed s_t while they fit alpha, then the best
+ *            tokens left; "KARA" page, "What carries the argument")
  *   E_FULL = 0, E_TOK = sum_{t not in R} s_t, E_CH = sum_t s_t g_t,
  *   E_BOTH = E_TOK + sum_{t in R} s_t g_t            (lost attention mass)
  *   choice = greedy over each segment's lower convex hull in (bytes, E),
@@ -108,6 +112,11 @@ typedef struct kv2d_params {
     int32_t keep_channels;  /* c: 1 <= c <= d                                */
     float budget;           /* beta > 0: byte budget / FULL bytes            */
     float scale;            /* softmax scale; 0 selects 1/sqrt(d)            */
+    int32_t chunk_len;      /* Token2Chunk: longest chunk gamma in tokens,
+                               3 <= gamma <= S; 0 = plain top-r              */
+    int32_t chunk_budget;   /* Token2Chunk: tokens alpha that chunks may add
+                               per segment, 1 <= alpha < r and r - alpha <=
+                               33 (ignored when chunk_len is 0)              */
 } kv2d_params;
 
 /* Dense (uncompressed) K/V view of one layer.  Two layouts:

@@ -31,7 +31,8 @@ class Kv2dError(RuntimeError):
 class kv2d_params(C.Structure):
     _fields_ = [("head_dim", C.c_int32), ("num_q_heads", C.c_int32), ("num_kv_heads", C.c_int32),
                 ("segment_len", C.c_int32), ("window", C.c_int32), ("keep_tokens", C.c_int32),
-                ("keep_channels", C.c_int32), ("budget", C.c_float), ("scale", C.c_float)]
+                ("keep_channels", C.c_int32), ("budget", C.c_float), ("scale", C.c_float),
+                ("chunk_len", C.c_int32), ("chunk_budget", C.c_int32)]
 
 
 class kv2d_dense(C.Structure):
@@ -147,9 +148,10 @@ def _i32_host(x, n):
 
 
 def params(head_dim, num_q_heads, num_kv_heads, segment_len, window, keep_tokens, keep_channels,
-           budget, scale=0.0) -> kv2d_params:
+           budget, scale=0.0, chunk_len=0, chunk_budget=0) -> kv2d_params:
     return kv2d_params(int(head_dim), int(num_q_heads), int(num_kv_heads), int(segment_len),
-                       int(window), int(keep_tokens), int(keep_channels), float(budget), float(scale))
+                       int(window), int(keep_tokens), int(keep_channels), float(budget), float(scale),
+                       int(chunk_len), int(chunk_budget))
 
 
 def dense(k: torch.Tensor, v: torch.Tensor, block_table: torch.Tensor | None = None,

@@ -67,6 +67,17 @@ kv2d_status check_params(const kv2d_params* p) {
         return fail(KV2D_ERR_INVALID_ARG, "budget must be a positive finite fraction");
     if (!(p->scale >= 0.f) || !std::isfinite(p->scale))
         return fail(KV2D_ERR_INVALID_ARG, "scale must be finite and >= 0 (0 selects 1/sqrt(d))");
+    if (p->chunk_len != 0) {
+        if (p->chunk_len < 3 || p->chunk_len > p->segment_len)
+            return fail(KV2D_ERR_INVALID_ARG, "chunk_len %d: need 0 (off) or 3 <= chunk_len <= S = %d",
+                        p->chunk_len, p->segment_len);
+        if (p->chunk_budget < 1 || p->chunk_budget >= p->keep_tokens)
+            return fail(KV2D_ERR_INVALID_ARG, "chunk_budget %d: need 1 <= chunk_budget < r = %d",
+                        p->chunk_budget, p->keep_tokens);
+        if (p->keep_tokens - p->chunk_budget > 33)
+            return fail(KV2D_ERR_UNSUPPORTED, "Token2Chunk runs r - chunk_budget <= 33 core tokens, got %d",
+                        p->keep_tokens - p->chunk_budget);
+    }
     if (p->head_dim != kHeadDim)
         return fail(KV2D_ERR_UNSUPPORTED, "this build runs head_dim = %d only", kHeadDim);
     return KV2D_OK;
@@ -99,6 +110,8 @@ UnitShape shape_of(const kv2d_params* p) {
     s.r = p->keep_tokens;
     s.c = p->keep_channels;
     s.c2 = eff_scale(p) * kLog2e;
+    s.chunk_len = p->chunk_len;
+    s.chunk_budget = p->chunk_len ? p->chunk_budget : 0;
     return s;
 }
 

@@ -56,6 +56,7 @@ struct UnitShape {
     int32_t Hkv, Hq, G, W, GW, GWpad;
     int32_t S, r, c;
     float c2;   // softmax scale * log2(e)
+    int32_t chunk_len, chunk_budget;   // Token2Chunk (chunk_len 0: plain top-r)
 };
 
 // ---- scoring (score.cu)

@@ -6,7 +6,7 @@
 // pages define no criterion; this library reads it as minimising lost
 // attention mass under a byte budget:
 //   seg_select (one thread per segment for r in {4, 8, 16}, S <= 128;
-//   otherwise one warp per segment):
+//   otherwise, and for the Token2Chunk variant, one warp per segment):
 //     R_j = top-r tokens by s_t (ties to the lower token), ascending;
 //     E_FULL = 0, E_TOK = sum_{t not in R} s_t, E_CH = sum_t s_t g_t,
 //     E_BOTH = E_TOK + sum_{t in R} s_t g_t        (fp64, ascending t);
@@ -37,6 +37,7 @@ static_assert(kSegWarps >= 3 && kSegWarps <= 32, "phase 2 needs three warps; pha
 struct SegArgs {
     SeqPlan plan;
     int Hkv, S, r, max_nseg;
+    int chunk_len, chunk_budget;   // Token2Chunk; chunk_len 0: plain top-r
     int64_t bytes[4];
     int32_t order[4];
     const float* s;
@@ -57,7 +58,58 @@ struct SegArgs {
 // reads spread over the banks; then the three sums per segment.
 __host__ __device__ constexpr int seg_row(int S) { return S + 1; }
 inline int seg_smem_bytes(int S) {
-    return kSegWarps * seg_row(S) * (8 + 4 + 1) + 3 * kSegWarps * 8 + 16;
+    return kSegWarps * seg_row(S) * (8 + 4 + 1 + 2) + 3 * kSegWarps * 8 + 16;
+}
+
+// Token2Chunk on one segment by one lane (Kara, "What carries the
+// argument"; the steps follow the library's reading): rk[t] is the rank of
+// token t by (s desc, t asc) and inv[k] the token of rank k.  Writes kept[t].
+__device__ void chunk_select(const float* srow, const uint8_t* rk, const uint8_t* inv, uint8_t* kept,
+                             int S, int r, int alpha, int gamma) {
+    const int ncore = r - alpha;
+    for (int t = 0; t < S; ++t) kept[t] = rk[t] < ncore ? 1 : 0;
+    // candidate gaps between consecutive core tokens (at most ncore - 1)
+    double cm[32];
+    int ca[32], cg[32];
+    int nc = 0, prev = -1;
+    for (int t = 0; t < S; ++t) {
+        if (!kept[t]) continue;
+        if (prev >= 0 && t - prev - 1 >= 1 && t - prev + 1 <= gamma && nc < 32) {
+            double m = 0.0;
+            for (int x = prev + 1; x < t; ++x) m = __dadd_rn(m, static_cast<double>(srow[x]));
+            cm[nc] = m;
+            ca[nc] = prev;
+            cg[nc] = t - prev - 1;
+            ++nc;
+        }
+        prev = t;
+    }
+    // by (merit desc, start asc)
+    for (int i = 0; i < nc; ++i) {
+        int best = i;
+        for (int k = i + 1; k < nc; ++k)
+            if (cm[k] > cm[best] || (cm[k] == cm[best] && ca[k] < ca[best])) best = k;
+        const double tm = cm[i];
+        const int ta = ca[i], tg = cg[i];
+        cm[i] = cm[best];
+        ca[i] = ca[best];
+        cg[i] = cg[best];
+        cm[best] = tm;
+        ca[best] = ta;
+        cg[best] = tg;
+    }
+    int rem = alpha;
+    for (int i = 0; i < nc; ++i) {
+        if (cg[i] > rem) continue;
+        for (int x = ca[i] + 1; x <= ca[i] + cg[i]; ++x) kept[x] = 1;
+        rem -= cg[i];
+    }
+    for (int k = 0; k < S && rem > 0; ++k) {
+        const int t = inv[k];
+        if (kept[t]) continue;
+        kept[t] = 1;
+        --rem;
+    }
 }
 
 // The error proxies of segment js of unit u from its three sums, written
@@ -128,6 +180,9 @@ __global__ void __launch_bounds__(kSegWarps * 32) seg_select_kernel(const __grid
     double* sums = sgs + kSegWarps * RW;                                    // [3][kSegWarps]
     float* ss = reinterpret_cast<float*>(sums + 3 * kSegWarps);             // [kSegWarps][RW]
     uint8_t* kept = reinterpret_cast<uint8_t*>(ss + kSegWarps * RW);        // [kSegWarps][RW]
+    uint8_t* rks = kept + kSegWarps * RW;                                   // [kSegWarps][RW] ranks
+    uint8_t* invs = rks + kSegWarps * RW;                                   // [kSegWarps][RW] rank -> t
+    const bool chunk = A.chunk_len > 0;
 
     const int j = jb + warp;
     if (j < nseg) {
@@ -152,6 +207,17 @@ __global__ void __launch_bounds__(kSegWarps * 32) seg_select_kernel(const __grid
                 ra += (v2 > va) || (v2 == va && t2 < ta);
                 rc += (v2 > vc) || (v2 == vc && t2 < tc);
             }
+            if (chunk) {
+                if (ta < S) {
+                    rks[warp * RW + ta] = static_cast<uint8_t>(ra);
+                    invs[warp * RW + ra] = static_cast<uint8_t>(ta);
+                }
+                if (tc < S) {
+                    rks[warp * RW + tc] = static_cast<uint8_t>(rc);
+                    invs[warp * RW + rc] = static_cast<uint8_t>(tc);
+                }
+                continue;
+            }
             const bool ka = ta < S && ra < r, kc = tc < S && rc < r;
             if (ta < S) kept[warp * RW + ta] = ka ? 1 : 0;
             if (tc < S) kept[warp * RW + tc] = kc ? 1 : 0;
@@ -162,6 +228,16 @@ __global__ void __launch_bounds__(kSegWarps * 32) seg_select_kernel(const __grid
             const uint32_t bc = __ballot_sync(0xffffffffu, kc);
             if (kc) A.tidx[slot * r + before + __popc(bc & lt)] = static_cast<uint8_t>(tc);
             before += __popc(bc);
+        }
+        if (chunk) {
+            __syncwarp();
+            if (lane == 0) {
+                chunk_select(srow, rks + warp * RW, invs + warp * RW, kept + warp * RW, S, r,
+                             A.chunk_budget, A.chunk_len);
+                int w = 0;
+                for (int t = 0; t < S; ++t)
+                    if (kept[warp * RW + t]) A.tidx[slot * r + w++] = static_cast<uint8_t>(t);
+            }
         }
     }
     __syncthreads();
@@ -652,6 +728,8 @@ cudaError_t launch_selection(const SelectLaunch& L, cudaStream_t stream) {
         sa.S = L.shp.S;
         sa.r = L.shp.r;
         sa.max_nseg = L.max_nseg;
+        sa.chunk_len = L.shp.chunk_len;
+        sa.chunk_budget = L.shp.chunk_budget;
         for (int k = 0; k < 4; ++k) {
             sa.bytes[k] = L.bytes[k];
             sa.order[k] = L.order[k];
@@ -668,7 +746,7 @@ cudaError_t launch_selection(const SelectLaunch& L, cudaStream_t stream) {
         sa.dbg_E = L.dbg_E;
         sa.dbg_seg_stride = L.dbg_seg_stride;
         const int r = sa.r;
-        const bool small = sa.S <= 128 && (r == 4 || r == 8 || r == 16) && sa.S % r == 0;
+        const bool small = sa.chunk_len == 0 && sa.S <= 128 && (r == 4 || r == 8 || r == 16) && sa.S % r == 0;
         prof_begin(stream, kProfSegSelect);
         if (small) {
             dim3 grid((L.max_nseg + kSmallSegs - 1) / kSmallSegs, units);

@@ -38,17 +38,18 @@ class GpuRun:
     ws: torch.Tensor
 
 
-def params_for(wl: synth.Workload, budget=None, keep_channels=None, keep_tokens=None):
+def params_for(wl: synth.Workload, budget=None, keep_channels=None, keep_tokens=None,
+               chunk_len=0, chunk_budget=0):
     scale = float(np.float32(1.0 / math.sqrt(wl.head_dim)))
     return B.params(wl.head_dim, wl.num_q_heads, wl.num_kv_heads, wl.segment_len, wl.window,
                     keep_tokens or wl.r, keep_channels or wl.c,
-                    wl.budget if budget is None else budget, scale)
+                    wl.budget if budget is None else budget, scale, chunk_len, chunk_budget)
 
 
 def oracle_params(orc, p: B.kv2d_params):
     return orc.params(p.head_dim, p.num_q_heads // p.num_kv_heads, p.segment_len, p.window,
                       p.keep_tokens, p.keep_channels, float(np.float32(p.budget)),
-                      float(np.float32(p.scale)))
+                      float(np.float32(p.scale)), p.chunk_len, p.chunk_budget if p.chunk_len else 0)
 
 
 def to_device(batch: synth.Batch, device="cuda") -> synth.Batch:

@@ -89,6 +89,7 @@ def _compress(p, batch, seq, ce, dense=None, cc=None, ws_bytes=1 << 30, q=8 << 2
     ("window", 0, 1), ("window", 129, 1), ("keep_tokens", 0, 1), ("keep_tokens", 65, 1),
     ("keep_channels", 129, 1), ("keep_channels", 0, 1), ("budget", 0.0, 1),
     ("budget", float("nan"), 1), ("num_kv_heads", 3, 1), ("scale", -1.0, 1),
+    ("chunk_len", 2, 1), ("chunk_len", 65, 1), ("chunk_len", -1, 1),
 ])
 def test_invalid_params_rejected(L, field, value, code):
     p = B.params(128, 32, 8, 64, 64, 8, 32, 0.2)
@@ -193,3 +194,14 @@ def test_noalloc_decode_rejects_oversize_before_launch(L):
                                       1 << 23, 1 << 24, None, None)
     assert rc == 3
     assert "scratch" in B.kv2d_last_error()
+
+
+def test_chunk_params_checked(L):
+    """Token2Chunk needs 1 <= chunk_budget < r when chunk_len is set, and at
+    most 33 core tokens; chunk_budget is ignored when chunk_len is 0."""
+    for (r, alpha, code) in [(8, 0, 1), (8, 8, 1), (8, 4, 0), (40, 6, 6), (40, 7, 0)]:
+        p = B.params(128, 32, 8, 64, 64, r, 32, 0.2, chunk_len=8, chunk_budget=alpha)
+        rc = _compress(p, 1, [63], [0])          # nothing complete: OK without a launch
+        assert rc == code, (r, alpha, rc)
+    p = B.params(128, 32, 8, 64, 64, 8, 32, 0.2, chunk_len=0, chunk_budget=99)
+    assert _compress(p, 1, [63], [0]) == 0

@@ -266,6 +266,23 @@ def test_token_ties_parity(orc, keep_tokens):
     _check_decode(orc, run)
 
 
+@pytest.mark.parametrize("name,gamma,alpha", [("tiny", 8, 4), ("mix4", 6, 3), ("g2_small_rc", 4, 1),
+                                               ("gw512_s128", 8, 8), ("paged", 5, 2)])
+def test_token2chunk_parity(orc, name, gamma, alpha):
+    """Kara's Token2Chunk variant of the kept tokens (core top r - alpha,
+    gaps of span <= gamma filled by summed mass within the budget alpha,
+    the rest from the best tokens left): the whole compression against the
+    oracle -- scores independently, and with the GPU's scores fed in the
+    kept tokens, strategies and every packed byte bit for bit -- then
+    decode."""
+    wl = CASES[name]
+    run = _run(wl, chunk_len=gamma, chunk_budget=alpha)
+    H.compress(run)
+    strats = _check_all_units(orc, run, independent=True)
+    assert len(strats) > 0
+    _check_decode(orc, run)
+
+
 @pytest.mark.parametrize("cap", [32, 41])
 def test_decode_block_table_in_chunks(orc, cap):
     """With more units than half the SMs the batch's bytes are shared out
