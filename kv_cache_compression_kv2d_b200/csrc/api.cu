@@ -184,22 +184,28 @@ DecodeLayout decode_layout(const kv2d_params* p, int batch) {
 }
 
 struct SelectLayout {
-    size_t score, sel, nsel, ticket, part, total;
+    size_t cscore, cslot, ccount, gather, nsel, ticket, part, total;
     int64_t slot_stride;
+    int nreg;
 };
 
-// Workspace of kv2d_decode_attn_select: per unit a score and a kept-slot
-// list over (max_seq_len / S) * S candidate slots, the kept count, a ticket,
-// and the attention partials of up to kSel2MaxChunks chunks.
+// Workspace of kv2d_decode_attn_select: per unit the candidate scores and
+// their slots compacted per region of 64 segments over (max_seq_len / S) * S
+// candidate slots, the regions' counts, the kept items' gather entries, the
+// kept count, a ticket, and the attention partials of up to kSel2MaxChunks
+// chunks.
 SelectLayout select_layout(const kv2d_params* p, int batch, int64_t max_seq_len) {
     const UnitShape sh = shape_of(p);
     const int64_t units = static_cast<int64_t>(batch) * sh.Hkv;
     SelectLayout L;
     L.slot_stride = round_up(std::max<int64_t>(max_seq_len / sh.S * sh.S, 1), 4);
+    L.nreg = std::max(1, sel2_regions(L.slot_stride, sh.S));
     Carver c;
     c.take(256);
-    L.score = c.take(units * L.slot_stride * 4);
-    L.sel = c.take(units * L.slot_stride * 4);
+    L.cscore = c.take(units * L.slot_stride * 4);
+    L.cslot = c.take(units * L.slot_stride * 4);
+    L.ccount = c.take(units * L.nreg * 4);
+    L.gather = c.take(units * L.slot_stride * 8);
     L.nsel = c.take(units * 4);
     L.ticket = c.take(units * 4);
     L.part = c.take(units * kSel2MaxChunks * sh.G * (kHeadDim + 4) * 4);
@@ -844,6 +850,8 @@ kv2d_status kv2d_decode_attn_select(const kv2d_params* p, int batch, const kv2d_
         return fail(KV2D_ERR_INVALID_ARG, "max_seq_len %d outside [0, capacity]", max_seq_len_host);
     if (!(select_rate > 0.f) || !std::isfinite(select_rate))
         return fail(KV2D_ERR_INVALID_ARG, "select_rate must be a positive finite fraction");
+    if (cc->arena_stride >= (int64_t(1) << 36))
+        return fail(KV2D_ERR_UNSUPPORTED, "selection decode runs arenas below 64 GB per unit");
     const SelectLayout WL = select_layout(p, batch, max_seq_len_host);
     if (!ws || !aligned(ws, 256) || ws_bytes < WL.total)
         return fail(KV2D_ERR_WORKSPACE, "selection decode workspace %zu bytes, need %zu (256-byte aligned)",
@@ -866,8 +874,11 @@ kv2d_status kv2d_decode_attn_select(const kv2d_params* p, int batch, const kv2d_
     L.q = static_cast<const __half*>(q);
     L.out = static_cast<__half*>(out);
     L.slot_stride = WL.slot_stride;
-    L.score = reinterpret_cast<float*>(w + WL.score);
-    L.sel = reinterpret_cast<int32_t*>(w + WL.sel);
+    L.cscore = reinterpret_cast<float*>(w + WL.cscore);
+    L.cslot = reinterpret_cast<int32_t*>(w + WL.cslot);
+    L.ccount = reinterpret_cast<int32_t*>(w + WL.ccount);
+    L.nreg_max = WL.nreg;
+    L.gather = reinterpret_cast<uint2*>(w + WL.gather);
     L.nsel = reinterpret_cast<int32_t*>(w + WL.nsel);
     L.part = reinterpret_cast<float*>(w + WL.part);
     L.ticket = reinterpret_cast<uint32_t*>(w + WL.ticket);

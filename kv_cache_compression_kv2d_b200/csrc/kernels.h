@@ -202,8 +202,11 @@ struct DecodeSelectLaunch {
     const __half* q;
     __half* out;
     int64_t slot_stride;       // candidate slots per unit: (max_seq_len / S) * S
-    float* score;              // [units][slot_stride]
-    int32_t* sel;              // [units][slot_stride]
+    float* cscore;             // [units][slot_stride]: scores compacted per region
+    int32_t* cslot;            // [units][slot_stride]
+    int32_t* ccount;           // [units][nreg_max]
+    int nreg_max;              // regions of 64 segments per unit
+    uint2* gather;             // [units][slot_stride]: kept items
     int32_t* nsel;             // [units]
     float* part;               // [units][nchunk][G][4 + d]
     uint32_t* ticket;          // [units]
@@ -215,5 +218,6 @@ struct DecodeSelectLaunch {
 constexpr int kSel2MaxChunks = 64;
 cudaError_t launch_decode_select(const DecodeSelectLaunch& L, cudaStream_t stream);
 int sel2_chunks(int units, int num_sms);
+int sel2_regions(int64_t slot_stride, int S);
 
 }  // namespace kv2d

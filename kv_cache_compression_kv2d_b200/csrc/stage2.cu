@@ -57,9 +57,12 @@ struct Sel2Args {
     const int32_t* seq_len;
     const __half* q;
     __half* out;
-    int64_t slot_stride;   // slots per unit in score / sel
-    float* score;          // [units][slot_stride]
-    int32_t* sel;          // [units][slot_stride]: kept slots, ascending
+    int64_t slot_stride;   // slots per unit: (max_seq_len / S) * S, multiple of 4
+    float* cscore;         // [units][slot_stride]: scores, compacted per region
+    int32_t* cslot;        // [units][slot_stride]: the slot of each compacted score
+    int32_t* ccount;       // [units][nreg_max]: candidates of each region
+    int nreg_max;
+    uint2* gather;         // [units][slot_stride]: kept items {desc low word, strategy | i << 8}
     int32_t* nsel;         // [units]
     float* part;           // [units][nchunk][G][4 + d]
     uint32_t* ticket;      // [units]
@@ -142,39 +145,51 @@ __device__ __forceinline__ uint64_t seg_desc(const Sel2Args& A, int u, int j) {
 
 // ------------------------------------------------------------- scores
 
-constexpr int kScoreSegs = 64;    // segments per CTA of the score kernel
+constexpr int kScoreSegs = 64;    // segments per region (one CTA of the score kernel)
+constexpr int kQRow = kHeadDim + kHeadDim / 4;
 
-// One CTA per kScoreSegs segments of a unit.  The segments' kept-token
-// counts are scanned in shared memory, so that each thread takes real
-// candidates (not empty slots of TOK / BOTH segments); every slot past a
-// segment's kept tokens gets -inf.  A thread computes the G logits of its
-// candidate (fp32, dimensions in ascending order) and writes their maximum.
+// q rows padded by 4 floats per 16 dims, so that the 8 lanes of a group
+// (16 dims each) read distinct bank groups.
+__device__ __forceinline__ int qix(int x) { return x + 4 * (x >> 4); }
+
+// One CTA per region of kScoreSegs segments of a unit.  The segments'
+// kept-token counts are scanned in shared memory and the region's
+// candidates numbered 0..n-1 in slot order; a group of 8 lanes takes one
+// candidate (lane k: dims 16k .. 16k + 15, coalesced 32-byte reads of the
+// key row, or every 8th (index, value) pair of a sparse key), the group's G
+// dot products are summed by a butterfly, and the largest logit is written
+// at the candidate's number in the region, with its slot beside it.
 template <int G>
 __global__ void __launch_bounds__(kScoreThreads) sel_score_kernel(const __grid_constant__ Sel2Args A) {
     pdl_wait();
-    __shared__ __align__(16) float qs[G][kHeadDim];
+    __shared__ __align__(16) float qs[G][kQRow];
     __shared__ int pre[kScoreSegs + 1];
+    __shared__ uint64_t dsc[kScoreSegs];
     const int u = blockIdx.y;
     const int b = u / A.Hkv, h = u % A.Hkv;
     const int S = A.S;
-    const int nsg = unit_segs(A, u, blockIdx.x == 0 && threadIdx.x == 0);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int grp = lane >> 3, lg = lane & 7;
+    const int nsg = unit_segs(A, u, blockIdx.x == 0 && tid == 0);
     const int j0 = blockIdx.x * kScoreSegs;
     if (j0 >= nsg) return;
     const int nj = min(kScoreSegs, nsg - j0);
-    for (int x = threadIdx.x; x < G * kHeadDim; x += kScoreThreads)
-        qs[x / kHeadDim][x % kHeadDim] =
+    for (int x = tid; x < G * kHeadDim; x += kScoreThreads)
+        qs[x / kHeadDim][qix(x % kHeadDim)] =
             __half2float(A.q[(static_cast<int64_t>(b) * A.Hq + h * G + x / kHeadDim) * kHeadDim + x % kHeadDim]);
-    if (threadIdx.x < 32) {
-        // inclusive scan of the kept-token counts of the CTA's segments
-        const int lane = threadIdx.x;
+    if (tid < 32) {
+        // inclusive scan of the kept-token counts of the region's segments
         int carry = 0;
         for (int k0 = 0; k0 < kScoreSegs; k0 += 32) {
             const int j = j0 + k0 + lane;
             int n = 0;
+            uint64_t d = 0;
             if (k0 + lane < nj) {
-                const int st = static_cast<int>((A.desc[static_cast<int64_t>(u) * A.max_segs + j] >> 32) & 255u);
+                d = seg_desc(A, u, j);
+                const int st = static_cast<int>((d >> 32) & 255u);
                 n = (st == KV2D_TOK || st == KV2D_BOTH) ? A.r : S;
             }
+            dsc[k0 + lane] = d;
             int x = n;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
@@ -187,74 +202,77 @@ __global__ void __launch_bounds__(kScoreThreads) sel_score_kernel(const __grid_c
         if (lane == 0) pre[0] = 0;
     }
     __syncthreads();
-    float* sc = A.score + static_cast<int64_t>(u) * A.slot_stride + static_cast<int64_t>(j0) * S;
-    float* dsc = A.dbg_score ? A.dbg_score + static_cast<int64_t>(u) * A.slot_stride + static_cast<int64_t>(j0) * S
-                             : nullptr;
-    // empty slots
-    for (int x = threadIdx.x; x < nj * S; x += kScoreThreads) {
-        const int k = x / S, i = x % S;
-        if (i >= pre[k + 1] - pre[k]) {
-            sc[x] = kNegInf2;
-            if (dsc) dsc[x] = kNegInf2;
+    const int ncand = pre[nj];
+    const int64_t rbase = static_cast<int64_t>(u) * A.slot_stride + static_cast<int64_t>(j0) * S;
+    if (tid == 0) A.ccount[static_cast<int64_t>(u) * A.nreg_max + blockIdx.x] = ncand;
+    if (A.dbg_score) {
+        // empty slots of the debug copy (indexed by slot)
+        for (int x = tid; x < nj * S; x += kScoreThreads) {
+            const int k = x / S, i = x % S;
+            if (i >= pre[k + 1] - pre[k]) A.dbg_score[rbase + x] = kNegInf2;
         }
     }
-    const int ncand = pre[nj];
     const int64_t U = unit_used(A, u);
-    for (int cidx = threadIdx.x; cidx < ncand; cidx += kScoreThreads) {
-        int lo = 0, hi = nj;             // the segment k with pre[k] <= cidx < pre[k + 1]
-        while (hi - lo > 1) {
-            const int mid = (lo + hi) >> 1;
-            if (pre[mid] <= cidx) lo = mid;
-            else hi = mid;
+    for (int cb = warp * 4; cb < ncand; cb += kScoreThreads / 8) {
+        const int c = cb + grp;
+        const bool on = c < ncand;
+        int k = 0;
+        if (on) {
+            int lo = 0, hi = nj;             // the segment k with pre[k] <= c < pre[k + 1]
+            while (hi - lo > 1) {
+                const int mid = (lo + hi) >> 1;
+                if (pre[mid] <= c) lo = mid;
+                else hi = mid;
+            }
+            k = lo;
         }
-        const int k = lo, i = cidx - pre[k];
-        const Cand cd = candidate_of(A, u, U, seg_desc(A, u, j0 + k), i, true);
-        float best = kNegInf2;
-        if (cd.kind != 0) {
-            float acc[G];
+        const int i = c - pre[k];
+        const Cand cd = on ? candidate_of(A, u, U, dsc[k], i, lg == 0) : Cand{0, nullptr, nullptr, nullptr};
+        float dot[G];
 #pragma unroll
-            for (int g = 0; g < G; ++g) acc[g] = 0.f;
-            if (cd.kind == 1) {
-#pragma unroll 2
-                for (int ch = 0; ch < 16; ++ch) {
-                    const uint4 w = *reinterpret_cast<const uint4*>(cd.key + ch * 16);
-                    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-                    float kf[8];
+        for (int g = 0; g < G; ++g) dot[g] = 0.f;
+        if (cd.kind == 1) {
+            const uint4* kp = reinterpret_cast<const uint4*>(cd.key + lg * 32);
+            const uint4 w0 = kp[0], w1 = kp[1];
+            const uint32_t ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+            float kf[16];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&ws[e]));
-                        kf[2 * e] = f.x;
-                        kf[2 * e + 1] = f.y;
-                    }
-#pragma unroll
-                    for (int g = 0; g < G; ++g) {
-                        const float4 q0 = *reinterpret_cast<const float4*>(&qs[g][ch * 8]);
-                        const float4 q1 = *reinterpret_cast<const float4*>(&qs[g][ch * 8 + 4]);
-                        float a = acc[g];
-                        a = fmaf(q0.x, kf[0], a);
-                        a = fmaf(q0.y, kf[1], a);
-                        a = fmaf(q0.z, kf[2], a);
-                        a = fmaf(q0.w, kf[3], a);
-                        a = fmaf(q1.x, kf[4], a);
-                        a = fmaf(q1.y, kf[5], a);
-                        a = fmaf(q1.z, kf[6], a);
-                        a = fmaf(q1.w, kf[7], a);
-                        acc[g] = a;
-                    }
-                }
-            } else {
-                for (int x = 0; x < A.c; ++x) {
-                    const int ci = cd.key[x] & 0x7f;     // indices are < 128; the mask keeps a bad byte in range
-                    const float kv = __half2float(cd.kval[x]);
-#pragma unroll
-                    for (int g = 0; g < G; ++g) acc[g] = fmaf(qs[g][ci], kv, acc[g]);
-                }
+            for (int e = 0; e < 8; ++e) {
+                const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&ws[e]));
+                kf[2 * e] = f.x;
+                kf[2 * e + 1] = f.y;
             }
 #pragma unroll
-            for (int g = 0; g < G; ++g) best = fmaxf(best, A.scale * acc[g]);
+            for (int g = 0; g < G; ++g) {
+#pragma unroll
+                for (int k4 = 0; k4 < 16; k4 += 4) {
+                    const float4 q4 = *reinterpret_cast<const float4*>(&qs[g][qix(lg * 16 + k4)]);
+                    dot[g] = fmaf(q4.w, kf[k4 + 3], fmaf(q4.z, kf[k4 + 2], fmaf(q4.y, kf[k4 + 1], fmaf(q4.x, kf[k4], dot[g]))));
+                }
+            }
+        } else if (cd.kind == 2) {
+            for (int x = lg; x < A.c; x += 8) {
+                const int ci = cd.key[x] & 0x7f;      // indices are < 128; the mask keeps a bad byte in range
+                const float kv = __half2float(cd.kval[x]);
+#pragma unroll
+                for (int g = 0; g < G; ++g) dot[g] = fmaf(qs[g][qix(ci)], kv, dot[g]);
+            }
         }
-        sc[static_cast<int64_t>(k) * S + i] = best;
-        if (dsc) dsc[static_cast<int64_t>(k) * S + i] = best;
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+#pragma unroll
+            for (int off = 4; off > 0; off >>= 1) dot[g] += __shfl_xor_sync(0xffffffffu, dot[g], off);
+        if (on && lg == 0) {
+            float best = kNegInf2;
+            if (cd.kind != 0) {
+#pragma unroll
+                for (int g = 0; g < G; ++g) best = fmaxf(best, A.scale * dot[g]);
+            }
+            const int slot = (j0 + k) * S + i;
+            A.cscore[rbase + c] = best;
+            A.cslot[rbase + c] = slot;
+            if (A.dbg_score) A.dbg_score[static_cast<int64_t>(u) * A.slot_stride + slot] = best;
+        }
     }
 }
 
@@ -303,20 +321,29 @@ __global__ void __launch_bounds__(kTopThreads) sel_topn_kernel(const __grid_cons
     __shared__ long long red[33];
     __shared__ uint32_t s_prefix;
     __shared__ long long s_need;
+    extern __shared__ int rp[];            // [nreg + 1]: region prefix of candidate counts
     const int u = blockIdx.x;
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31;
+    const int S = A.S;
     const int nsg = unit_segs(A, u, false);
-    const int64_t nslots = static_cast<int64_t>(nsg) * A.S;
-    const float* sc = A.score + static_cast<int64_t>(u) * A.slot_stride;
-    // candidates: kept tokens per segment from the descriptors
-    long long nc = 0;
-    for (int j = tid; j < nsg; j += kTopThreads) {
-        const int st = static_cast<int>((A.desc[static_cast<int64_t>(u) * A.max_segs + j] >> 32) & 255u);
-        nc += (st == KV2D_TOK || st == KV2D_BOTH) ? A.r : A.S;
+    const int nreg = (nsg + kScoreSegs - 1) / kScoreSegs;
+    const int64_t RS = static_cast<int64_t>(kScoreSegs) * S;
+    const int64_t ubase = static_cast<int64_t>(u) * A.slot_stride;
+    const float* sc = A.cscore + ubase;
+    // region counts -> prefix (one block scan per 1024 regions)
+    long long carry = 0;
+    for (int k0 = 0; k0 < nreg; k0 += kTopThreads) {
+        const int k = k0 + tid;
+        const long long n = (k < nreg) ? A.ccount[static_cast<int64_t>(u) * A.nreg_max + k] : 0;
+        long long tot;
+        const long long ex = block_exscan_ll(n, red, &tot);
+        if (k < nreg) rp[k] = static_cast<int>(carry + ex);
+        carry += tot;
     }
-    long long ncand;
-    block_exscan_ll(nc, red, &ncand);
-    const double want = ceil(A.rate * static_cast<double>(nslots));
+    if (tid == 0) rp[nreg] = static_cast<int>(carry);
+    __syncthreads();
+    const long long ncand = carry;
+    const double want = ceil(A.rate * static_cast<double>(static_cast<int64_t>(nsg) * S));
     const long long n_sel = (want >= static_cast<double>(ncand)) ? ncand : static_cast<long long>(want);
     // the n_sel-th largest key, 8 bits at a time from the top
     if (tid == 0) {
@@ -330,19 +357,14 @@ __global__ void __launch_bounds__(kTopThreads) sel_topn_kernel(const __grid_cons
         __syncthreads();
         const uint32_t pre = s_prefix;
         const uint32_t hmask = pass == 0 ? 0u : (0xffffffffu << (shift + 8));
-        // lanes with the same digit add once (scores cluster in few digits,
-        // so plain shared atomics would serialise on one address)
-        const int lane = tid & 31;
-        for (int64_t s0 = tid - lane; s0 < nslots; s0 += 4 * kTopThreads) {
-            float v[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int64_t s = s0 + lane + static_cast<int64_t>(k) * kTopThreads;
-                v[k] = (s < nslots) ? sc[s] : kNegInf2;
-            }
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const uint32_t key = score_key(v[k]);
+        // region by region; lanes with the same digit add once (scores
+        // cluster in few digits, so plain shared atomics would serialise)
+        for (int k = 0; k < nreg; ++k) {
+            const int cnt = rp[k + 1] - rp[k];
+            const float* rs = sc + k * RS;
+            for (int i0 = tid - lane; i0 < cnt; i0 += kTopThreads) {
+                const int i = i0 + lane;
+                const uint32_t key = (i < cnt) ? score_key(rs[i]) : 0u;
                 const int dg = (key != 0u && (key & hmask) == (pre & hmask)) ? static_cast<int>((key >> shift) & 255u) : -1;
                 const uint32_t peers = __match_any_sync(0xffffffffu, dg);
                 if (dg >= 0 && lane == __ffs(peers) - 1) atomicAdd(&hist[dg], static_cast<unsigned>(__popc(peers)));
@@ -387,31 +409,59 @@ __global__ void __launch_bounds__(kTopThreads) sel_topn_kernel(const __grid_cons
     }
     const uint32_t v = s_prefix;            // the n_sel-th largest key (0: nothing kept)
     const long long eq_take = s_need;       // keys equal to v to keep, lowest slots first
-    // thread tid scans its own contiguous range of slots, so block scans give slot order
-    const int64_t per = (nslots + kTopThreads - 1) / kTopThreads;
-    const int64_t s0 = min(nslots, per * tid), s1 = min(nslots, s0 + per);
+    if (A.dbg_sel) {
+        for (int64_t s = tid; s < static_cast<int64_t>(nsg) * S; s += kTopThreads) A.dbg_sel[ubase + s] = 0;
+        __syncthreads();
+    }
+    // thread tid scans its own contiguous range of candidate numbers (flat
+    // over the regions), so block scans give slot order
+    const int64_t per = (ncand + kTopThreads - 1) / kTopThreads;
+    const int64_t f0 = min(static_cast<int64_t>(ncand), per * tid), f1 = min(static_cast<int64_t>(ncand), f0 + per);
+    auto region_of = [&](int64_t f) {
+        int lo = 0, hi = nreg;
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (rp[mid] <= f) lo = mid;
+            else hi = mid;
+        }
+        return lo;
+    };
     long long n_gt = 0, n_eq = 0;
-    for (int64_t s = s0; s < s1; ++s) {
-        const uint32_t k = score_key(sc[s]);
-        n_gt += (n_sel > 0 && k > v);
-        n_eq += (n_sel > 0 && k == v && k != 0u);
+    {
+        int k = (f0 < f1) ? region_of(f0) : 0;
+        for (int64_t f = f0; f < f1; ++f) {
+            while (f >= rp[k + 1]) ++k;
+            const uint32_t key = score_key(sc[k * RS + (f - rp[k])]);
+            n_gt += (n_sel > 0 && key > v);
+            n_eq += (n_sel > 0 && key == v && key != 0u);
+        }
     }
     long long tot_eq;
     const long long eq_before = block_exscan_ll(n_eq, red, &tot_eq);
-    long long mine = n_gt + max(0ll, min(n_eq, eq_take - eq_before));
+    const long long mine = n_gt + max(0ll, min(n_eq, eq_take - eq_before));
     long long tot_sel;
     long long pos = block_exscan_ll(mine, red, &tot_sel);
-    int32_t* out = A.sel + static_cast<int64_t>(u) * A.slot_stride;
+    uint2* out = A.gather + ubase;
     long long eq_seen = eq_before;
-    for (int64_t s = s0; s < s1; ++s) {
-        const uint32_t k = score_key(sc[s]);
-        bool keep = false;
-        if (n_sel > 0 && k != 0u) {
-            if (k > v) keep = true;
-            else if (k == v) keep = (eq_seen++ < eq_take);
+    {
+        int k = (f0 < f1) ? region_of(f0) : 0;
+        for (int64_t f = f0; f < f1; ++f) {
+            while (f >= rp[k + 1]) ++k;
+            const int64_t at = k * RS + (f - rp[k]);
+            const uint32_t key = score_key(sc[at]);
+            bool keep = false;
+            if (n_sel > 0 && key != 0u) {
+                if (key > v) keep = true;
+                else if (key == v) keep = (eq_seen++ < eq_take);
+            }
+            if (keep) {
+                const int slot = A.cslot[ubase + at];
+                const uint64_t d = seg_desc(A, u, slot / S);
+                out[pos++] = make_uint2(static_cast<uint32_t>(d),
+                                        static_cast<uint32_t>((d >> 32) & 255u) | (static_cast<uint32_t>(slot % S) << 8));
+                if (A.dbg_sel) A.dbg_sel[ubase + slot] = 1;
+            }
         }
-        if (keep) out[pos++] = static_cast<int32_t>(s);
-        if (A.dbg_sel) A.dbg_sel[static_cast<int64_t>(u) * A.slot_stride + s] = keep ? 1 : 0;
     }
     if (tid == 0) {
         A.nsel[u] = static_cast<int32_t>(tot_sel);
@@ -434,9 +484,6 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 2) sel_attn_kernel(const __gr
     constexpr int DPL = kHeadDim / LPI;          // dims per lane (16 or 8)
     constexpr int IPW = 32 / LPI;                // items per warp in flight
     constexpr int kRec = kHeadDim + 4;
-    // q rows padded by 4 floats per 16 dims, so that the 8 lanes of a group
-    // (16 dims each) read distinct bank groups
-    constexpr int kQRow = kHeadDim + kHeadDim / 4;
     __shared__ __align__(16) float qs[G][kQRow];
     __shared__ float wm[kAttnWarps][G], wl[kAttnWarps][G];
     __shared__ __align__(16) float wo[kAttnWarps][G][kHeadDim];
@@ -445,7 +492,6 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 2) sel_attn_kernel(const __gr
     const int b = u / A.Hkv, h = u % A.Hkv;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int grp = lane / LPI, lg = lane % LPI;
-    auto qix = [](int x) { return x + 4 * (x >> 4); };
     for (int x = tid; x < G * kHeadDim; x += kAttnWarps * 32)
         qs[x / kHeadDim][qix(x % kHeadDim)] =
             __half2float(A.q[(static_cast<int64_t>(b) * A.Hq + h * G + x / kHeadDim) * kHeadDim + x % kHeadDim]);
@@ -461,7 +507,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 2) sel_attn_kernel(const __gr
     const int64_t nsel = A.nsel[u];
     const int64_t items = nsel + (T - ce);
     const int64_t i_lo = items * c_id / A.nchunk, i_hi = items * (c_id + 1) / A.nchunk;
-    const int32_t* sl = A.sel + static_cast<int64_t>(u) * A.slot_stride;
+    const uint2* gl = A.gather + static_cast<int64_t>(u) * A.slot_stride;
     const unsigned gmask = (LPI == 32) ? 0xffffffffu : (((1u << LPI) - 1u) << (grp * LPI));
     float m[G], l[G], o[G][DPL];
 #pragma unroll
@@ -474,17 +520,13 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 2) sel_attn_kernel(const __gr
     const int d0 = lg * DPL;
     const int64_t U = unit_used(A, u);
     constexpr int64_t kStep = kAttnWarps * IPW;
-    // the next item's slot and descriptor are loaded while this one is
-    // computed (the chain slot -> descriptor -> key / value is three loads)
+    // the next item's gather entry is loaded while this one is computed
     int64_t it = i_lo + warp * IPW + grp;
-    int32_t slot_n = (it < i_hi && it < nsel) ? sl[it] : 0;
-    uint64_t desc_n = (it < i_hi && it < nsel) ? seg_desc(A, u, slot_n / A.S) : 0ull;
+    uint2 ge_n = (it < i_hi && it < nsel) ? gl[it] : make_uint2(0u, 0u);
     for (; it < i_hi; it += kStep) {
-        const int32_t slot = slot_n;
-        const uint64_t dsc = desc_n;
+        const uint2 ge = ge_n;
         const int64_t it2 = it + kStep;
-        const bool next_sel = it2 < i_hi && it2 < nsel;
-        if (next_sel) slot_n = sl[it2];
+        if (it2 < i_hi && it2 < nsel) ge_n = gl[it2];
         float dot[G];
 #pragma unroll
         for (int g = 0; g < G; ++g) dot[g] = 0.f;
@@ -492,7 +534,8 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 2) sel_attn_kernel(const __gr
         const __half* krow = nullptr;
         bool skip = false;
         if (it < nsel) {
-            const Cand cd = candidate_of(A, u, U, dsc, slot % A.S, lg == 0);
+            const uint64_t dsc = static_cast<uint64_t>(ge.x) | (static_cast<uint64_t>(ge.y & 255u) << 32);
+            const Cand cd = candidate_of(A, u, U, dsc, static_cast<int>(ge.y >> 8), lg == 0);
             if (cd.kind == 0) {
                 skip = true;                 // (status already set; uniform in the group)
             } else {
@@ -514,7 +557,6 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 2) sel_attn_kernel(const __gr
             vrow = dense_row(A.dv, A.dv.v, b, h, t, nullptr);
             skip = !krow || !vrow;           // uniform in the group
         }
-        if (next_sel) desc_n = seg_desc(A, u, slot_n / A.S);
         if (skip) continue;
         uint4 vw[DPL / 8];
 #pragma unroll
@@ -659,6 +701,10 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 2) sel_attn_kernel(const __gr
 
 }  // namespace
 
+int sel2_regions(int64_t slot_stride, int S) {
+    return static_cast<int>((slot_stride / S + kScoreSegs - 1) / kScoreSegs);
+}
+
 int sel2_chunks(int units, int num_sms) {
     return std::max(1, std::min(kSel2MaxChunks, (2 * num_sms + units - 1) / units));
 }
@@ -686,8 +732,11 @@ cudaError_t launch_decode_select(const DecodeSelectLaunch& L, cudaStream_t strea
     a.q = L.q;
     a.out = L.out;
     a.slot_stride = L.slot_stride;
-    a.score = L.score;
-    a.sel = L.sel;
+    a.cscore = L.cscore;
+    a.cslot = L.cslot;
+    a.ccount = L.ccount;
+    a.nreg_max = L.nreg_max;
+    a.gather = L.gather;
     a.nsel = L.nsel;
     a.part = L.part;
     a.ticket = L.ticket;
@@ -699,8 +748,7 @@ cudaError_t launch_decode_select(const DecodeSelectLaunch& L, cudaStream_t strea
     cudaError_t e;
     prof_begin(stream, kProfSelScore);
     if (L.slot_stride > 0) {
-        const int64_t segs = L.slot_stride / L.shp.S;
-        dim3 g1(static_cast<unsigned>((segs + kScoreSegs - 1) / kScoreSegs), units);
+        dim3 g1(static_cast<unsigned>(L.nreg_max), units);
         switch (L.shp.G) {
         case 1: e = launch_k(sel_score_kernel<1>, g1, dim3(kScoreThreads), 0, stream, a); break;
         case 2: e = launch_k(sel_score_kernel<2>, g1, dim3(kScoreThreads), 0, stream, a); break;
@@ -712,7 +760,7 @@ cudaError_t launch_decode_select(const DecodeSelectLaunch& L, cudaStream_t strea
     }
     prof_end(stream, kProfSelScore);
     prof_begin(stream, kProfSelTop);
-    e = launch_k(sel_topn_kernel, dim3(units), dim3(kTopThreads), 0, stream, a);
+    e = launch_k(sel_topn_kernel, dim3(units), dim3(kTopThreads), (L.nreg_max + 1) * sizeof(int), stream, a);
     if (e != cudaSuccess) return e;
     prof_end(stream, kProfSelTop);
     prof_begin(stream, kProfSelAttn);
