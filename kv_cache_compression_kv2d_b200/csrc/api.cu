@@ -190,7 +190,7 @@ struct SelectLayout {
 };
 
 // Workspace of kv2d_decode_attn_select: per unit the candidate scores and
-// their slots compacted per region of 64 segments over (max_seq_len / S) * S
+// their slots compacted per region of 16 segments over (max_seq_len / S) * S
 // candidate slots, the regions' counts, the kept items' gather entries, the
 // kept count, a ticket, and the attention partials of up to kSel2MaxChunks
 // chunks.
@@ -853,6 +853,8 @@ kv2d_status kv2d_decode_attn_select(const kv2d_params* p, int batch, const kv2d_
     if (cc->arena_stride >= (int64_t(1) << 36))
         return fail(KV2D_ERR_UNSUPPORTED, "selection decode runs arenas below 64 GB per unit");
     const SelectLayout WL = select_layout(p, batch, max_seq_len_host);
+    if (WL.nreg > 12000)
+        return fail(KV2D_ERR_UNSUPPORTED, "selection decode runs at most 12000 x 16 segments per sequence");
     if (!ws || !aligned(ws, 256) || ws_bytes < WL.total)
         return fail(KV2D_ERR_WORKSPACE, "selection decode workspace %zu bytes, need %zu (256-byte aligned)",
                     ws_bytes, WL.total);

@@ -205,7 +205,7 @@ struct DecodeSelectLaunch {
     float* cscore;             // [units][slot_stride]: scores compacted per region
     int32_t* cslot;            // [units][slot_stride]
     int32_t* ccount;           // [units][nreg_max]
-    int nreg_max;              // regions of 64 segments per unit
+    int nreg_max;              // regions of 16 segments per unit
     uint2* gather;             // [units][slot_stride]: kept items
     int32_t* nsel;             // [units]
     float* part;               // [units][nchunk][G][4 + d]

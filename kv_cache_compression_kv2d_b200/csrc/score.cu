@@ -836,6 +836,21 @@ __device__ __forceinline__ void key_masks(ChunkFn chunk, const float* af, __half
     }
 }
 
+// fp64 acc + x * y unless (m & bit) != 0, as one fused multiply-add: the
+// callers' products are exact in fp64 (an fp16 magnitude times an fp32
+// weight: 11 x 24 significant bits), so rounding x * y + acc once equals
+// adding the exact product with one rounding.  One compare into a predicate
+// and one guarded instruction, so the skipped add costs no 64-bit select.
+__device__ __forceinline__ double dfma_unless(double acc, double x, double y, uint32_t m, uint32_t bit) {
+    asm("{\n\t.reg .pred p;\n\t.reg .b32 t;\n\t"
+        "and.b32 t, %3, %4;\n\t"
+        "setp.eq.u32 p, t, 0;\n\t"
+        "@p fma.rn.f64 %0, %1, %2, %0;\n\t}"
+        : "+d"(acc)
+        : "d"(x), "d"(y), "r"(m), "r"(bit));
+    return acc;
+}
+
 // An fp16 value (bits) widened to fp64 in one conversion (exact).
 __device__ __forceinline__ double h2d(uint16_t bits) {
     double d;
@@ -980,10 +995,8 @@ __global__ void __launch_bounds__(128) chan_kernel_c32(const __grid_constant__ C
     }
 
     // g_t: both fp64 sums ascending in x; |k| widened from fp16 in one
-    // conversion per half (the halves taken as 16-bit registers, no shift),
-    // and e = |k| a_x is exact in fp64, so each fused multiply-add rounds
-    // exactly as adding e does.  Bit x of the keep mask is moved to the sign
-    // bit by an integer multiply (FMA pipe) and tested there.
+    // conversion, and e = |k| a_x is exact in fp64, so each fused
+    // multiply-add rounds exactly as adding e does
     const int64_t slot = static_cast<int64_t>(u) * A.g_stride + t;
     double tot = 0.0, drop = 0.0;
 #pragma unroll 1
@@ -994,20 +1007,12 @@ __global__ void __launch_bounds__(128) chan_kernel_c32(const __grid_constant__ C
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             const double2 a2 = *reinterpret_cast<const double2*>(ad + 8 * j + 2 * e);
-            asm("{\n\t.reg .b16 lo, hi;\n\t.reg .f64 k0, k1;\n\t.reg .b32 t0, t1;\n\t.reg .pred p0, p1;\n\t"
-                "mov.b32 {lo, hi}, %2;\n\t"
-                "cvt.f64.f16 k0, lo;\n\t"
-                "cvt.f64.f16 k1, hi;\n\t"
-                "mul.lo.u32 t0, %5, %6;\n\t"
-                "mul.lo.u32 t1, %5, %7;\n\t"
-                "setp.ge.s32 p0, t0, 0;\n\t"
-                "setp.ge.s32 p1, t1, 0;\n\t"
-                "fma.rn.f64 %0, k0, %3, %0;\n\t"
-                "@p0 fma.rn.f64 %1, k0, %3, %1;\n\t"
-                "fma.rn.f64 %0, k1, %4, %0;\n\t"
-                "@p1 fma.rn.f64 %1, k1, %4, %1;\n\t}"
-                : "+d"(tot), "+d"(drop)
-                : "r"(qw[e]), "d"(a2.x), "d"(a2.y), "r"(mw), "r"(1u << (31 - 2 * e)), "r"(1u << (30 - 2 * e)));
+            const double k0 = h2d(static_cast<uint16_t>(qw[e] & 0xffffu));
+            const double k1 = h2d(static_cast<uint16_t>(qw[e] >> 16));
+            tot = __fma_rn(k0, a2.x, tot);
+            drop = dfma_unless(drop, k0, a2.x, mw, 1u << (2 * e));
+            tot = __fma_rn(k1, a2.y, tot);
+            drop = dfma_unless(drop, k1, a2.y, mw, 2u << (2 * e));
         }
     }
     A.cmask[slot] = make_uint4(M[0], M[1], M[2], M[3]);

@@ -145,7 +145,7 @@ __device__ __forceinline__ uint64_t seg_desc(const Sel2Args& A, int u, int j) {
 
 // ------------------------------------------------------------- scores
 
-constexpr int kScoreSegs = 64;    // segments per region (one CTA of the score kernel)
+constexpr int kScoreSegs = 16;    // segments per region (one CTA of the score kernel)
 constexpr int kQRow = kHeadDim + kHeadDim / 4;
 
 // q rows padded by 4 floats per 16 dims, so that the 8 lanes of a group
@@ -189,14 +189,16 @@ __global__ void __launch_bounds__(kScoreThreads) sel_score_kernel(const __grid_c
                 const int st = static_cast<int>((d >> 32) & 255u);
                 n = (st == KV2D_TOK || st == KV2D_BOTH) ? A.r : S;
             }
-            dsc[k0 + lane] = d;
             int x = n;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 const int y = __shfl_up_sync(0xffffffffu, x, o);
                 if (lane >= o) x += y;
             }
-            pre[k0 + lane + 1] = carry + x;
+            if (k0 + lane < kScoreSegs) {
+                dsc[k0 + lane] = d;
+                pre[k0 + lane + 1] = carry + x;
+            }
             carry += __shfl_sync(0xffffffffu, x, 31);
         }
         if (lane == 0) pre[0] = 0;
