@@ -219,6 +219,42 @@ KV2D_API kv2d_status kv2d_compress(const kv2d_params* p, int batch, const int32_
                           const void* q_window, kv2d_ccache* cc, void* ws, size_t ws_bytes,
                           const kv2d_debug* dbg, void* stream);
 
+/* Staged bookkeeping of a compression that is not yet published (device
+ * memory, caller-owned): n_segs [units], used_bytes [units] (8-byte
+ * aligned), comp_end [batch]. */
+typedef struct kv2d_staged {
+    int32_t* n_segs;
+    int64_t* used_bytes;
+    int32_t* comp_end;
+} kv2d_staged;
+
+/* kv2d_compress_staged / kv2d_switch -- compression that does not block
+ * decode (MosaicKV Fig. 1 and Fig. 5: a switching mechanism replaces the
+ * temporary version of a new segment with the compressed one without
+ * blocking the decode stage; here the temporary version is the dense view
+ * itself, so no CPU copy is involved).
+ *   kv2d_compress_staged does what kv2d_compress does, but writes the new
+ *   segments' bookkeeping into *staged and leaves cc->n_segs, used_bytes
+ *   and comp_end untouched: the new packed bytes go past used_bytes and the
+ *   new descriptors past n_segs, which decode never reads.  It may run on
+ *   a second stream while kv2d_decode_attn / kv2d_append run on the decode
+ *   stream: decode keeps attending the old segments and reads the tokens
+ *   being compressed from the dense view (the region [comp_end, seq_len) a
+ *   compression reads is never written by append).  *staged first receives
+ *   the live values (stream-ordered copies), then the new ones.
+ *   kv2d_switch publishes *staged as the live bookkeeping with one small
+ *   kernel on the given stream.  The caller orders it after the staged
+ *   compression (an event) and before the next decode that should see the
+ *   new segments, and issues no other compression of the same cache until
+ *   the switch.  Arguments and errors otherwise as kv2d_compress. */
+KV2D_API kv2d_status kv2d_compress_staged(const kv2d_params* p, int batch,
+                                          const int32_t* seq_len_host, const int32_t* comp_end_host,
+                                          const kv2d_dense* kv, const void* q_window,
+                                          kv2d_ccache* cc, const kv2d_staged* staged, void* ws,
+                                          size_t ws_bytes, const kv2d_debug* dbg, void* stream);
+KV2D_API kv2d_status kv2d_switch(const kv2d_params* p, int batch, kv2d_ccache* cc,
+                                 const kv2d_staged* staged, void* stream);
+
 /* kv2d_append -- write one new token per (sequence, KV head) into the dense
  * view at position seq_len_dev[b], then increment seq_len_dev[b] (the
  * decode stage's KV growth that later compressions consume; MosaicKV

@@ -48,6 +48,10 @@ class kv2d_ccache(C.Structure):
                 ("comp_end", C.c_void_p)]
 
 
+class kv2d_staged(C.Structure):
+    _fields_ = [("n_segs", C.c_void_p), ("used_bytes", C.c_void_p), ("comp_end", C.c_void_p)]
+
+
 class kv2d_debug(C.Structure):
     _fields_ = [("a", C.c_void_p), ("lse", C.c_void_p), ("s", C.c_void_p), ("g", C.c_void_p),
                 ("E", C.c_void_p), ("region_stride", C.c_int64), ("seg_stride", C.c_int32)]
@@ -56,7 +60,8 @@ class kv2d_debug(C.Structure):
 EXPORTS = ["kv2d_segment_bytes", "kv2d_arena_bytes", "kv2d_workspace_bytes", "kv2d_compress",
            "kv2d_append", "kv2d_decode_attn", "kv2d_read_status", "kv2d_last_error",
            "kv2d_version", "kv2d_profile_enable", "kv2d_profile_read", "kv2d_set_decode_table_cap",
-           "kv2d_profile_stage_name", "kv2d_decode_attn_noalloc", "kv2d_decode_attn_select"]
+           "kv2d_profile_stage_name", "kv2d_decode_attn_noalloc", "kv2d_decode_attn_select",
+           "kv2d_compress_staged", "kv2d_switch"]
 
 _lib = None
 
@@ -79,6 +84,13 @@ def lib():
                                     P(kv2d_dense), C.c_void_p, P(kv2d_ccache), C.c_void_p,
                                     C.c_size_t, P(kv2d_debug), C.c_void_p]
         L.kv2d_compress.restype = C.c_int
+        L.kv2d_compress_staged.argtypes = [P(kv2d_params), C.c_int, P(C.c_int32), P(C.c_int32),
+                                           P(kv2d_dense), C.c_void_p, P(kv2d_ccache),
+                                           P(kv2d_staged), C.c_void_p, C.c_size_t, P(kv2d_debug),
+                                           C.c_void_p]
+        L.kv2d_compress_staged.restype = C.c_int
+        L.kv2d_switch.argtypes = [P(kv2d_params), C.c_int, P(kv2d_ccache), P(kv2d_staged), C.c_void_p]
+        L.kv2d_switch.restype = C.c_int
         L.kv2d_append.argtypes = [P(kv2d_params), C.c_int, P(kv2d_dense), C.c_void_p, C.c_void_p,
                                   C.c_void_p, C.c_void_p, C.c_size_t, C.c_void_p]
         L.kv2d_append.restype = C.c_int
@@ -194,6 +206,25 @@ def kv2d_compress(p, batch, seq_len_host, comp_end_host, dense_view, q_window, c
     return _check(rc) if check else rc
 
 
+def kv2d_compress_staged(p, batch, seq_len_host, comp_end_host, dense_view, q_window, cc, staged,
+                         ws, dbg=None, stream=None, check=True) -> int:
+    """kv2d_compress whose bookkeeping goes to `staged` (a StagedRecord)
+    until kv2d_switch publishes it."""
+    rc = lib().kv2d_compress_staged(C.byref(p), int(batch), _i32_host(seq_len_host, batch),
+                                    _i32_host(comp_end_host, batch), C.byref(dense_view),
+                                    _ptr(q_window), C.byref(cc), C.byref(staged.struct), _ptr(ws),
+                                    ws.numel() if hasattr(ws, "numel") else 0,
+                                    C.byref(dbg) if dbg is not None else None, _stream(stream))
+    return _check(rc) if check else rc
+
+
+def kv2d_switch(p, batch, cc, staged, stream=None, check=True) -> int:
+    """Publishes a staged compression as the cache's live bookkeeping."""
+    rc = lib().kv2d_switch(C.byref(p), int(batch), C.byref(cc), C.byref(staged.struct),
+                           _stream(stream))
+    return _check(rc) if check else rc
+
+
 def kv2d_append(p, batch, dense_view, k_new, v_new, seq_len_dev, ws, stream=None,
                 check=True) -> int:
     rc = lib().kv2d_append(C.byref(p), int(batch), C.byref(dense_view), _ptr(k_new), _ptr(v_new),
@@ -292,6 +323,17 @@ class CompressedCache:
         """Forget every compressed segment (the arena bytes are left as they
         are; descriptors past n_segs are never read)."""
         self.book.zero_()
+
+
+class StagedRecord:
+    """Device buffers of a staged compression's bookkeeping (caller-owned)."""
+
+    def __init__(self, p: kv2d_params, batch: int, device="cuda"):
+        units = batch * p.num_kv_heads
+        self.used_bytes = torch.zeros(units, dtype=torch.int64, device=device)
+        self.n_segs = torch.zeros(units, dtype=torch.int32, device=device)
+        self.comp_end = torch.zeros(batch, dtype=torch.int32, device=device)
+        self.struct = kv2d_staged(_ptr(self.n_segs), _ptr(self.used_bytes), _ptr(self.comp_end))
 
 
 def workspace(nbytes: int, device="cuda") -> torch.Tensor:

@@ -190,7 +190,7 @@ struct SelectLayout {
 };
 
 // Workspace of kv2d_decode_attn_select: per unit the candidate scores and
-// their slots compacted per region of 16 segments over (max_seq_len / S) * S
+// their slots compacted per region of 64 segments over (max_seq_len / S) * S
 // candidate slots, the regions' counts, the kept items' gather entries, the
 // kept count, a ticket, and the attention partials of up to kSel2MaxChunks
 // chunks.
@@ -444,10 +444,18 @@ size_t kv2d_workspace_bytes(const kv2d_params* p, int op, int batch, int64_t max
     }
 }
 
-kv2d_status kv2d_compress(const kv2d_params* p, int batch, const int32_t* seq_len_host,
+}  // extern "C"
+
+namespace {
+
+// The compression of kv2d_compress; with staged != NULL the new bookkeeping
+// (n_segs, used_bytes, comp_end) goes to the staged record instead of the
+// live one (the record is first set to the live values, so sequences
+// without a new segment keep theirs).
+kv2d_status compress_impl(const kv2d_params* p, int batch, const int32_t* seq_len_host,
                           const int32_t* comp_end_host, const kv2d_dense* kv, const void* q_window,
-                          kv2d_ccache* cc, void* ws, size_t ws_bytes, const kv2d_debug* dbg,
-                          void* stream) {
+                          kv2d_ccache* cc, const kv2d_staged* staged, void* ws, size_t ws_bytes,
+                          const kv2d_debug* dbg, void* stream) {
     kv2d_status st = check_params(p);
     if (st != KV2D_OK) return st;
     if (batch < 1 || batch > KV2D_MAX_BATCH)
@@ -500,6 +508,19 @@ kv2d_status kv2d_compress(const kv2d_params* p, int batch, const int32_t* seq_le
                         b, static_cast<long long>(need), static_cast<long long>(cc->arena_stride));
         if (nseg > 0) max_region = std::max<int64_t>(max_region, region);
         max_nseg = std::max(max_nseg, nseg);
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (staged) {
+        if (!staged->n_segs || !staged->used_bytes || !staged->comp_end || !aligned(staged->used_bytes, 8))
+            return fail(KV2D_ERR_INVALID_ARG, "staged record has a NULL or misaligned pointer");
+        const size_t units = static_cast<size_t>(batch) * sh.Hkv;
+        cudaError_t e0 = cudaMemcpyAsync(staged->n_segs, cc->n_segs, units * 4, cudaMemcpyDeviceToDevice, s);
+        if (e0 == cudaSuccess)
+            e0 = cudaMemcpyAsync(staged->used_bytes, cc->used_bytes, units * 8, cudaMemcpyDeviceToDevice, s);
+        if (e0 == cudaSuccess)
+            e0 = cudaMemcpyAsync(staged->comp_end, cc->comp_end, static_cast<size_t>(batch) * 4,
+                                 cudaMemcpyDeviceToDevice, s);
+        if (e0 != cudaSuccess) return fail(KV2D_ERR_CUDA, "staging copy: %s", cudaGetErrorString(e0));
     }
     if (max_nseg == 0) return ok();   // nothing complete to compress
 
@@ -617,7 +638,6 @@ kv2d_status kv2d_compress(const kv2d_params* p, int batch, const int32_t* seq_le
         SL.dbg_g = dbg->g;
         SL.dbg_stride = dbg->region_stride;
     }
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e = launch_scoring(SL, s);
     if (e != cudaSuccess) return fail(KV2D_ERR_CUDA, "scoring launch: %s", cudaGetErrorString(e));
 
@@ -658,6 +678,11 @@ kv2d_status kv2d_compress(const kv2d_params* p, int batch, const int32_t* seq_le
     XL.n_segs = cc->n_segs;
     XL.used_bytes = cc->used_bytes;
     XL.comp_end = cc->comp_end;
+    if (staged) {
+        XL.out_n_segs = staged->n_segs;
+        XL.out_used_bytes = staged->used_bytes;
+        XL.out_comp_end = staged->comp_end;
+    }
     XL.arena_stride = cc->arena_stride;
     XL.status = SL.status;
     if (dbg) {
@@ -687,6 +712,44 @@ kv2d_status kv2d_compress(const kv2d_params* p, int batch, const int32_t* seq_le
     e = launch_pack(PL, s);
     if (e != cudaSuccess) return fail(KV2D_ERR_CUDA, "pack launch: %s", cudaGetErrorString(e));
     (void)units;
+    return ok();
+}
+
+}  // namespace
+
+extern "C" {
+
+kv2d_status kv2d_compress(const kv2d_params* p, int batch, const int32_t* seq_len_host,
+                          const int32_t* comp_end_host, const kv2d_dense* kv, const void* q_window,
+                          kv2d_ccache* cc, void* ws, size_t ws_bytes, const kv2d_debug* dbg,
+                          void* stream) {
+    return compress_impl(p, batch, seq_len_host, comp_end_host, kv, q_window, cc, nullptr, ws, ws_bytes,
+                         dbg, stream);
+}
+
+kv2d_status kv2d_compress_staged(const kv2d_params* p, int batch, const int32_t* seq_len_host,
+                                 const int32_t* comp_end_host, const kv2d_dense* kv,
+                                 const void* q_window, kv2d_ccache* cc, const kv2d_staged* staged,
+                                 void* ws, size_t ws_bytes, const kv2d_debug* dbg, void* stream) {
+    if (!staged) return fail(KV2D_ERR_INVALID_ARG, "staged record is NULL");
+    return compress_impl(p, batch, seq_len_host, comp_end_host, kv, q_window, cc, staged, ws, ws_bytes,
+                         dbg, stream);
+}
+
+kv2d_status kv2d_switch(const kv2d_params* p, int batch, kv2d_ccache* cc, const kv2d_staged* staged,
+                        void* stream) {
+    kv2d_status st = check_params(p);
+    if (st != KV2D_OK) return st;
+    if (batch < 1 || batch > KV2D_MAX_BATCH)
+        return fail(KV2D_ERR_INVALID_ARG, "batch %d not in [1, %d]", batch, KV2D_MAX_BATCH);
+    if (!cc || !cc->n_segs || !cc->used_bytes || !cc->comp_end)
+        return fail(KV2D_ERR_INVALID_ARG, "compressed cache has a NULL pointer");
+    if (!staged || !staged->n_segs || !staged->used_bytes || !staged->comp_end)
+        return fail(KV2D_ERR_INVALID_ARG, "staged record has a NULL pointer");
+    const int units = batch * p->num_kv_heads;
+    cudaError_t e = launch_publish(units, batch, staged->n_segs, staged->used_bytes, staged->comp_end,
+                                   cc->n_segs, cc->used_bytes, cc->comp_end, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail(KV2D_ERR_CUDA, "switch launch: %s", cudaGetErrorString(e));
     return ok();
 }
 
@@ -854,7 +917,7 @@ kv2d_status kv2d_decode_attn_select(const kv2d_params* p, int batch, const kv2d_
         return fail(KV2D_ERR_UNSUPPORTED, "selection decode runs arenas below 64 GB per unit");
     const SelectLayout WL = select_layout(p, batch, max_seq_len_host);
     if (WL.nreg > 12000)
-        return fail(KV2D_ERR_UNSUPPORTED, "selection decode runs at most 12000 x 16 segments per sequence");
+        return fail(KV2D_ERR_UNSUPPORTED, "selection decode runs at most 12000 x 64 segments per sequence");
     if (!ws || !aligned(ws, 256) || ws_bytes < WL.total)
         return fail(KV2D_ERR_WORKSPACE, "selection decode workspace %zu bytes, need %zu (256-byte aligned)",
                     ws_bytes, WL.total);

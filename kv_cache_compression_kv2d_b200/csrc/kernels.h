@@ -118,12 +118,20 @@ struct SelectLaunch {
     int32_t* n_segs;
     int64_t* used_bytes;
     int32_t* comp_end;
+    // where the new bookkeeping goes; NULL: the live fields above (a staged
+    // compression leaves the live ones untouched until it is published)
+    int32_t* out_n_segs;
+    int64_t* out_used_bytes;
+    int32_t* out_comp_end;
     int64_t arena_stride;
     uint32_t* status;
     double* dbg_E;
     int32_t dbg_seg_stride;
 };
 cudaError_t launch_selection(const SelectLaunch& L, cudaStream_t stream);
+cudaError_t launch_publish(int units, int batch, const int32_t* st_n_segs, const int64_t* st_used,
+                           const int32_t* st_comp_end, int32_t* n_segs, int64_t* used, int32_t* comp_end,
+                           cudaStream_t stream);
 
 // ---- packing (pack.cu)
 struct PackLaunch {
@@ -205,7 +213,7 @@ struct DecodeSelectLaunch {
     float* cscore;             // [units][slot_stride]: scores compacted per region
     int32_t* cslot;            // [units][slot_stride]
     int32_t* ccount;           // [units][nreg_max]
-    int nreg_max;              // regions of 16 segments per unit
+    int nreg_max;              // regions of 64 segments per unit
     uint2* gather;             // [units][slot_stride]: kept items
     int32_t* nsel;             // [units]
     float* part;               // [units][nchunk][G][4 + d]

@@ -21,6 +21,8 @@
 // Every fp64 sum, product and quotient uses the _rn intrinsics so that no
 // multiply-add is fused and the results are bit-identical to the same
 // operations done one at a time in IEEE double precision.
+#include <algorithm>
+
 #include "kernels.h"
 
 namespace kv2d {
@@ -430,9 +432,10 @@ struct BudgetArgs {
     int32_t* unit_ok;
     uint64_t* desc;
     int32_t max_segs;
-    int32_t* n_segs;
-    int64_t* used_bytes;
-    int32_t* comp_end;
+    const int64_t* used_bytes;     // live: where this call's segments start
+    int32_t* out_n_segs;           // where the new bookkeeping goes (live or staged)
+    int64_t* out_used_bytes;
+    int32_t* out_comp_end;
     int64_t arena_stride;
     uint32_t* status;
 };
@@ -710,14 +713,44 @@ __global__ void __launch_bounds__(kBudgetThreads) budget_kernel(const __grid_con
         __syncthreads();
     }
     if (tid == 0) {
-        A.used_bytes[u] = used0 + total;
-        A.n_segs[u] = segbase + nseg;
-        if (h == 0) A.comp_end[b] = A.plan.r0[b] + nseg * A.S;
+        A.out_used_bytes[u] = used0 + total;
+        A.out_n_segs[u] = segbase + nseg;
+        if (h == 0) A.out_comp_end[b] = A.plan.r0[b] + nseg * A.S;
         A.unit_ok[u] = 1;
     }
 }
 
+// Publishes a staged compression: the staged bookkeeping becomes the live
+// one (one thread per unit, and per sequence for comp_end).
+struct PublishArgs {
+    int units, batch;
+    const int32_t* st_n_segs;
+    const int64_t* st_used_bytes;
+    const int32_t* st_comp_end;
+    int32_t* n_segs;
+    int64_t* used_bytes;
+    int32_t* comp_end;
+};
+
+__global__ void publish_kernel(const __grid_constant__ PublishArgs A) {
+    pdl_wait();
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < A.units) {
+        A.n_segs[i] = A.st_n_segs[i];
+        A.used_bytes[i] = A.st_used_bytes[i];
+    }
+    if (i < A.batch) A.comp_end[i] = A.st_comp_end[i];
+}
+
 }  // namespace
+
+cudaError_t launch_publish(int units, int batch, const int32_t* st_n_segs, const int64_t* st_used,
+                           const int32_t* st_comp_end, int32_t* n_segs, int64_t* used, int32_t* comp_end,
+                           cudaStream_t stream) {
+    PublishArgs a{units, batch, st_n_segs, st_used, st_comp_end, n_segs, used, comp_end};
+    const int n = std::max(units, batch);
+    return launch_k(publish_kernel, dim3((n + 255) / 256), dim3(256), 0, stream, a);
+}
 
 cudaError_t launch_selection(const SelectLaunch& L, cudaStream_t stream) {
     const int units = L.batch * L.shp.Hkv;
@@ -783,9 +816,10 @@ cudaError_t launch_selection(const SelectLaunch& L, cudaStream_t stream) {
     ba.unit_ok = L.unit_ok;
     ba.desc = L.desc;
     ba.max_segs = L.max_segs;
-    ba.n_segs = L.n_segs;
     ba.used_bytes = L.used_bytes;
-    ba.comp_end = L.comp_end;
+    ba.out_n_segs = L.out_n_segs ? L.out_n_segs : L.n_segs;
+    ba.out_used_bytes = L.out_used_bytes ? L.out_used_bytes : L.used_bytes;
+    ba.out_comp_end = L.out_comp_end ? L.out_comp_end : L.comp_end;
     ba.arena_stride = L.arena_stride;
     ba.status = L.status;
     prof_begin(stream, kProfBudget);

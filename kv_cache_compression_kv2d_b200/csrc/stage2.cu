@@ -145,7 +145,7 @@ __device__ __forceinline__ uint64_t seg_desc(const Sel2Args& A, int u, int j) {
 
 // ------------------------------------------------------------- scores
 
-constexpr int kScoreSegs = 16;    // segments per region (one CTA of the score kernel)
+constexpr int kScoreSegs = 64;    // segments per region (one CTA of the score kernel)
 constexpr int kQRow = kHeadDim + kHeadDim / 4;
 
 // q rows padded by 4 floats per 16 dims, so that the 8 lanes of a group
