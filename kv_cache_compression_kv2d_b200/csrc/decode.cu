@@ -931,12 +931,8 @@ int decode_cta_count(int units, int64_t max_seq_len, int num_sms, int* kps) {
     // out evenly.
     const int sms = std::min(num_sms, kMaxDecCtas);
     const int64_t by_len = std::max<int64_t>(1, std::min<int64_t>(64, (max_seq_len + 255) / 256));
-#ifndef KV2D_DEC_MAX_KPS
-#define KV2D_DEC_MAX_KPS 64
-#endif
     if (2 * static_cast<int64_t>(units) <= sms) {
-        *kps = static_cast<int>(std::min<int64_t>(std::min<int64_t>(sms / units, by_len),
-                                                  static_cast<int64_t>(KV2D_DEC_MAX_KPS)));
+        *kps = static_cast<int>(std::min<int64_t>(sms / units, by_len));
         return units * *kps;
     }
     *kps = 0;

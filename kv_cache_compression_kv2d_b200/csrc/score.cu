@@ -800,21 +800,14 @@ __device__ __forceinline__ __half2 key_pair(uint32_t w, float al, float ah) {
 // CTAs.  A compare yields 0xffff per half; one AND-OR per register moves
 // both flags to spare bit positions, and a final shuffle puts each channel
 // at its own bit.
-#ifndef KV2D_CHAN_ROLL
-#define KV2D_CHAN_ROLL 0
-#endif
 template <typename ChunkFn>
 __device__ __forceinline__ void key_masks(ChunkFn chunk, const float* af, __half2 vv, uint32_t (&M)[4],
                                           uint32_t (&Gt)[4]) {
-#if KV2D_CHAN_ROLL & 2
-    // one copy of the loop body (instruction-cache footprint); the words
-    // move through M[0..3] / Gt[0..3] as a queue
+    // one copy of the loop body: the unrolled networks and masks of this
+    // kernel overflow the instruction cache (instruction-fetch stalls were
+    // its largest); the words move through M[0..3] / Gt[0..3] as a queue
 #pragma unroll 1
     for (int wd = 0; wd < 4; ++wd) {
-#else
-#pragma unroll
-    for (int wd = 0; wd < 4; ++wd) {
-#endif
         uint32_t lo = 0, hi = 0, glo = 0, ghi = 0;
 #pragma unroll
         for (int g4 = 0; g4 < 4; ++g4) {
@@ -843,7 +836,6 @@ __device__ __forceinline__ void key_masks(ChunkFn chunk, const float* af, __half
         }
         const uint32_t mw = (lo & 0x5555u) | ((lo >> 16) & 0xAAAAu) | ((hi << 16) & 0x55550000u) | (hi & 0xAAAA0000u);
         const uint32_t gw = (glo & 0x5555u) | ((glo >> 16) & 0xAAAAu) | ((ghi << 16) & 0x55550000u) | (ghi & 0xAAAA0000u);
-#if KV2D_CHAN_ROLL & 2
         M[0] = M[1];
         M[1] = M[2];
         M[2] = M[3];
@@ -852,10 +844,6 @@ __device__ __forceinline__ void key_masks(ChunkFn chunk, const float* af, __half
         Gt[1] = Gt[2];
         Gt[2] = Gt[3];
         Gt[3] = gw;
-#else
-        M[wd] = mw;
-        Gt[wd] = gw;
-#endif
     }
 }
 
@@ -893,12 +881,9 @@ constexpr int kChanSmem = 1024 + kChanBar + 16;
 // << 4)), so the 8 threads of each quarter-warp read 8 different bank
 // groups.  K is never written by the kernels this one follows, so the
 // copy is issued before the wait on them and overlaps their tail.  The
-// tile is the only large shared buffer (about 35 KB per CTA); at 96
-// registers five CTAs of 128 threads share an SM.
-#ifndef KV2D_CHAN_MINB
-#define KV2D_CHAN_MINB 1
-#endif
-__global__ void __launch_bounds__(128, KV2D_CHAN_MINB) chan_kernel_c32(const __grid_constant__ CUtensorMap kmap,
+// tile is the only large shared buffer (about 35 KB per CTA), and the
+// kernel is held to 96 registers, so five CTAs of 128 threads share an SM.
+__global__ void __launch_bounds__(128, 5) chan_kernel_c32(const __grid_constant__ CUtensorMap kmap,
                                                           const __grid_constant__ ChanArgs A) {
     extern __shared__ uint8_t chan_smem_raw[];
     uint8_t* sm = align1024(chan_smem_raw);
@@ -953,9 +938,9 @@ __global__ void __launch_bounds__(128, KV2D_CHAN_MINB) chan_kernel_c32(const __g
         srt[4 * gi + 2] = key_pair(q.z, a1.x, a1.y);
         srt[4 * gi + 3] = key_pair(q.w, a1.z, a1.w);
     }
-#if KV2D_CHAN_ROLL & 1
     // one copy of the 32-key network, run on each half in turn (the halves
-    // swap places between the runs and are back in place after the second)
+    // swap places between the runs and are back in place after the second):
+    // half the code of two unrolled copies, for 32 register swaps
 #pragma unroll 1
     for (int rep = 0; rep < 2; ++rep) {
         sort32_desc2<0>(srt);
@@ -966,10 +951,6 @@ __global__ void __launch_bounds__(128, KV2D_CHAN_MINB) chan_kernel_c32(const __g
             srt[32 + i] = tmp;
         }
     }
-#else
-    sort32_desc2<0>(srt);
-    sort32_desc2<32>(srt);
-#endif
 #pragma unroll
     for (int i = 0; i < 32; ++i) srt[i] = __hmax2(srt[i], srt[63 - i]);
     merge32_desc2<16>(srt);          // low halves: 32 largest even channels (L),
