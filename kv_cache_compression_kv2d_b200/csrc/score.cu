@@ -574,14 +574,11 @@ struct ChanArgs {
     uint32_t* status;
 };
 
-// a_x = (sum of the row-tile partial sums, in tile order) / (G * W); the
-// first CTA of a unit also writes it to the debug output.
+// a_x = (sum of the row-tile partial sums, in tile order) / (G * W).
 __device__ __forceinline__ float chan_weight(const ChanArgs& A, int u, int x) {
     float s = 0.f;
     for (int mt = 0; mt < A.mtiles; ++mt) s += A.apart[(static_cast<int64_t>(u) * A.mtiles + mt) * kHeadDim + x];
-    const float v = s / static_cast<float>(A.GW);
-    if (A.dbg_a && blockIdx.x == 0) A.dbg_a[static_cast<int64_t>(u) * kHeadDim + x] = v;
-    return v;
+    return s / static_cast<float>(A.GW);
 }
 
 // One thread per key.  The block's 128 key rows sit in shared memory with
@@ -606,6 +603,7 @@ __global__ void __launch_bounds__(128) chan_kernel_generic(const __grid_constant
     __shared__ float as[128];
     const int tid = threadIdx.x;
     as[tid] = chan_weight(A, u, tid);
+    if (A.dbg_a && blockIdx.x == 0) A.dbg_a[static_cast<int64_t>(u) * kHeadDim + tid] = as[tid];
     for (int idx = tid; idx < 128 * 16; idx += 128) {
         const int rr = idx >> 4, ch = idx & 15;
         uint4 val = make_uint4(0, 0, 0, 0);
@@ -735,30 +733,30 @@ __device__ __forceinline__ void ce2(__half2& a, __half2& b) {
     b = lo;
 }
 
-// One (p, k) stage of Batcher's odd-even merge sort of registers O..O+31
-// into descending order, then the next stage; every register index is a
+// One (p, k) stage of Batcher's odd-even merge sort of 32 registers into
+// descending order, then the next stage; every register index is a
 // compile-time constant after unrolling.
-template <int O, int P, int K>
-__device__ __forceinline__ void oem32_pass(__half2 (&v)[64]) {
+template <int P, int K>
+__device__ __forceinline__ void oem32_pass(__half2 (&v)[32]) {
 #pragma unroll
     for (int j = K % P; j + K < 32; j += 2 * K) {
 #pragma unroll
         for (int i = 0; i < K; ++i) {
             if (i < 32 - j - K && (i + j) / (2 * P) == (i + j + K) / (2 * P))
-                ce2(v[O + i + j], v[O + i + j + K]);
+                ce2(v[i + j], v[i + j + K]);
         }
     }
-    if constexpr (K > 1) oem32_pass<O, P, K / 2>(v);
-    else if constexpr (P < 16) oem32_pass<O, P * 2, P * 2>(v);
+    if constexpr (K > 1) oem32_pass<P, K / 2>(v);
+    else if constexpr (P < 16) oem32_pass<P * 2, P * 2>(v);
 }
 
-template <int O>
-__device__ __forceinline__ void sort32_desc2(__half2 (&v)[64]) {
-    oem32_pass<O, 1, 1>(v);
+__device__ __forceinline__ void sort32_desc2(__half2 (&v)[32]) {
+    oem32_pass<1, 1>(v);
 }
 
+// Sorts a bitonic sequence of 32 registers into descending order.
 template <int J>
-__device__ __forceinline__ void merge32_desc2(__half2 (&v)[64]) {
+__device__ __forceinline__ void merge32_desc2(__half2 (&v)[32]) {
     if constexpr (J > 0) {
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
@@ -869,19 +867,186 @@ __device__ __forceinline__ double h2d(uint16_t bits) {
     return d;
 }
 
+// Rows of a 128-row K tile in the 128-byte-swizzled layout of the scoring
+// passes: row r, 16-byte chunk j of a 64-channel half at
+// half * 16384 + r * 128 + ((j ^ (r & 7)) << 4), so the 8 threads of each
+// quarter-warp (consecutive rows) read 8 different bank groups.
+struct ChanRow {
+    const uint8_t* row;   // tile + r * 128
+    int sw;               // r & 7
+    __device__ __forceinline__ uint4 chunk(int j) const {     // channels 8j .. 8j + 7
+        return *reinterpret_cast<const uint4*>(row + (j >> 3) * 16384 + (((j & 7) ^ sw) << 4));
+    }
+    __device__ __forceinline__ uint16_t kbits(int x) const {  // |k_x| as fp16 bits
+        const uint16_t* p = reinterpret_cast<const uint16_t*>(row + (x >> 6) * 16384 + ((((x >> 3) & 7) ^ sw) << 4));
+        return static_cast<uint16_t>(p[x & 7] & 0x7fffu);
+    }
+};
+
+// Keep mask of one key row (bit x set iff channel x is kept), c <= 32;
+// af / ad hold the weights a_x in fp32 and fp64.
+__device__ __forceinline__ uint4 chan_row_mask(const ChanRow R, const float* af, const double* ad, int c) {
+    auto chunk = [&](int j) { return R.chunk(j); };
+    // the 32 largest keys of the even channels (low halves, L) and of the odd
+    // channels (high halves, H), as bitonic sequences in srt[0..31]
+    __half2 srt[32];
+    {
+        __half2 hi[32];
+#pragma unroll
+        for (int gi = 0; gi < 16; ++gi) {
+            const uint4 q = chunk(gi);
+            const float4 a0 = *reinterpret_cast<const float4*>(af + 8 * gi);
+            const float4 a1 = *reinterpret_cast<const float4*>(af + 8 * gi + 4);
+            __half2* d = gi < 8 ? srt + 4 * gi : hi + 4 * (gi - 8);
+            d[0] = key_pair(q.x, a0.x, a0.y);
+            d[1] = key_pair(q.y, a0.z, a0.w);
+            d[2] = key_pair(q.z, a1.x, a1.y);
+            d[3] = key_pair(q.w, a1.z, a1.w);
+        }
+        // one copy of the 32-key network, run on each half in turn (the
+        // halves swap places between the runs and are back in place after
+        // the second): half the code of two unrolled copies
+#pragma unroll 1
+        for (int rep = 0; rep < 2; ++rep) {
+            sort32_desc2(srt);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const __half2 tmp = srt[i];
+                srt[i] = hi[i];
+                hi[i] = tmp;
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < 32; ++i) srt[i] = __hmax2(srt[i], hi[31 - i]);
+    }
+    merge32_desc2<16>(srt);          // low halves: L, high halves: H, descending
+    float vf;
+    if (c == 32) {
+        // the 32 largest of all are max(L_i, H_{31-i}); with the halves of
+        // register 31-i swapped, one __hmax2 forms the pairs for i and 31-i
+        __half2 mn = __half2half2(__ushort_as_half(0x7c00));   // +inf
+#pragma unroll
+        for (int i = 0; i < 16; ++i) mn = __hmin2(mn, __hmax2(srt[i], __lowhigh2highlow(srt[31 - i])));
+        vf = fminf(__low2float(mn), __high2float(mn));
+    } else {
+        float w[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) w[i] = fmaxf(__low2float(srt[i]), __high2float(srt[31 - i]));
+        merge32_desc_f<16>(w);       // 32 largest of all 128, descending
+        vf = w[0];
+#pragma unroll
+        for (int i = 1; i < 32; ++i) vf = (i < c) ? w[i] : vf;
+    }
+    const __half2 vv = __float2half2_rn(vf);   // vf is a key value: exact in fp16
+
+    // the K tile is read again below; without this fence the compiler
+    // hoists those loads above the sort and keeps both live (160 registers
+    // instead of 96)
+    uint32_t M[4], G[4];
+    asm volatile("" ::: "memory");
+    key_masks(chunk, af, vv, M, G);
+    const int n_ge = __popc(M[0]) + __popc(M[1]) + __popc(M[2]) + __popc(M[3]);
+    if (n_ge > c) {
+        // the keys equal to v straddle the cut: keep the c - n_gt best of
+        // them by (e desc, x asc).  The fp32 products f = fp32(|k| a) are
+        // correctly rounded, so f_y > f_x implies e_y > e_x; only equal f
+        // need the exact fp64 products.
+        const int n_gt = __popc(G[0]) + __popc(G[1]) + __popc(G[2]) + __popc(G[3]);
+        const int need = c - n_gt;
+        const uint32_t qm[4] = {M[0] & ~G[0], M[1] & ~G[1], M[2] & ~G[2], M[3] & ~G[3]};
+        uint32_t keep[4] = {0, 0, 0, 0};
+        // y ranks above x: f_y > f_x, or equal f and (e_y > e_x, or equal e and y < x)
+        auto above = [&](int y, double ky, float fy, int x, double kx, float fx) {
+            if (fy != fx) return fy > fx;
+            const double ex = __dmul_rn(kx, ad[x]), ey = __dmul_rn(ky, ad[y]);
+            return (ey > ex) || (ey == ex && y < x);
+        };
+        if (need == 1 || need == n_ge - n_gt - 1) {
+            // one pass over the tied channels: keep the single best one, or
+            // keep all but the single worst one
+            const bool best = need == 1;
+            int bx = -1;
+            double bk = 0.0;
+            float bf = 0.f;
+            for (int wi = 0; wi < 4; ++wi) {
+                for (uint32_t m = qm[wi]; m; m &= m - 1) {
+                    const int x = wi * 32 + __ffs(m) - 1;
+                    const double kx = h2d(R.kbits(x));
+                    const float fx = __fmul_rn(static_cast<float>(kx), af[x]);
+                    if (bx < 0 || above(x, kx, fx, bx, bk, bf) == best) {
+                        bx = x;
+                        bk = kx;
+                        bf = fx;
+                    }
+                }
+            }
+#pragma unroll
+            for (int wi = 0; wi < 4; ++wi) {
+                const uint32_t bit = (bx >> 5) == wi ? 1u << (bx & 31) : 0u;
+                keep[wi] = best ? bit : (qm[wi] & ~bit);
+            }
+        } else {
+            for (int wi = 0; wi < 4; ++wi) {
+                for (uint32_t m = qm[wi]; m; m &= m - 1) {
+                    const int x = wi * 32 + __ffs(m) - 1;
+                    const double kx = h2d(R.kbits(x));
+                    const float fx = __fmul_rn(static_cast<float>(kx), af[x]);
+                    int rank = 0;
+                    for (int wj = 0; wj < 4; ++wj) {
+                        for (uint32_t m2 = qm[wj]; m2; m2 &= m2 - 1) {
+                            const int y = wj * 32 + __ffs(m2) - 1;
+                            if (y == x) continue;
+                            const double ky = h2d(R.kbits(y));
+                            rank += above(y, ky, __fmul_rn(static_cast<float>(ky), af[y]), x, kx, fx);
+                        }
+                    }
+                    if (rank < need) keep[wi] |= 1u << (x & 31);
+                }
+            }
+        }
+#pragma unroll
+        for (int wi = 0; wi < 4; ++wi) M[wi] = G[wi] | keep[wi];
+    }
+    return make_uint4(M[0], M[1], M[2], M[3]);
+}
+
+// g_t of one key row under keep mask m: both fp64 sums ascending in x; |k|
+// widened exactly, and e = |k| a_x is exact in fp64, so each fused
+// multiply-add rounds exactly as adding e does.
+__device__ __forceinline__ double chan_row_g(const ChanRow R, const double* ad, uint4 m) {
+    const uint32_t M[4] = {m.x, m.y, m.z, m.w};
+    double tot = 0.0, drop = 0.0;
+#pragma unroll 1
+    for (int j = 0; j < 16; ++j) {
+        const uint4 q = R.chunk(j);
+        const uint32_t mw = ((j < 4) ? M[0] : (j < 8) ? M[1] : (j < 12) ? M[2] : M[3]) >> ((j & 3) * 8);
+        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const double2 a2 = *reinterpret_cast<const double2*>(ad + 8 * j + 2 * e);
+            // fp16 -> fp32 on the FMA pipe, then |.| and fp32 -> fp64: all exact
+            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[e]));
+            const double k0 = static_cast<double>(fabsf(f.x));
+            const double k1 = static_cast<double>(fabsf(f.y));
+            tot = __fma_rn(k0, a2.x, tot);
+            drop = dfma_unless(drop, k0, a2.x, mw, 1u << (2 * e));
+            tot = __fma_rn(k1, a2.y, tot);
+            drop = dfma_unless(drop, k1, a2.y, mw, 2u << (2 * e));
+        }
+    }
+    return tot > 0.0 ? __ddiv_rn(drop, tot) : 0.0;
+}
+
 constexpr int kChanTile = 0;                  // 128 K rows, two 64-channel halves (SW128)
 constexpr int kChanAf = kStage;               // float [128]
 constexpr int kChanAd = kChanAf + 512;        // double [128]
 constexpr int kChanBar = kChanAd + 1024;      // one mbarrier
 constexpr int kChanSmem = 1024 + kChanBar + 16;
 
-// One CTA per 128 tokens of a unit, one thread per token.  The K tile
-// arrives by TMA in the 128-byte-swizzled layout of the scoring passes
-// (row r, 16-byte chunk j of a 64-channel half at r * 128 + ((j ^ (r & 7))
-// << 4)), so the 8 threads of each quarter-warp read 8 different bank
-// groups.  K is never written by the kernels this one follows, so the
-// copy is issued before the wait on them and overlaps their tail.  The
-// tile is the only large shared buffer (about 35 KB per CTA), and the
+// One CTA per 128 tokens of a unit, one thread per token, for short
+// regions.  K is never written by the kernels this one follows, so the
+// tile's copy is issued before the wait on them and overlaps their tail.
+// The tile is the only large shared buffer (about 35 KB per CTA), and the
 // kernel is held to 96 registers, so five CTAs of 128 threads share an SM.
 __global__ void __launch_bounds__(128, 5) chan_kernel_c32(const __grid_constant__ CUtensorMap kmap,
                                                           const __grid_constant__ ChanArgs A) {
@@ -909,6 +1074,7 @@ __global__ void __launch_bounds__(128, 5) chan_kernel_c32(const __grid_constant_
     pdl_wait();
     {
         const float av = chan_weight(A, u, tid);
+        if (A.dbg_a && blockIdx.x == 0) A.dbg_a[static_cast<int64_t>(u) * kHeadDim + tid] = av;
         af[tid] = av;
         ad[tid] = static_cast<double>(av);
     }
@@ -916,129 +1082,11 @@ __global__ void __launch_bounds__(128, 5) chan_kernel_c32(const __grid_constant_
     if (!mbar_wait(bar, 0, A.status)) return;
     const int t = base + tid;
     if (t >= ntok) return;
-    const int c = A.c;
-    const uint8_t* myrow = tile + tid * 128;
-    const int sw = tid & 7;
-    auto chunk = [&](int j) {            // channels 8j .. 8j + 7
-        return *reinterpret_cast<const uint4*>(myrow + (j >> 3) * 16384 + (((j & 7) ^ sw) << 4));
-    };
-    auto kbits = [&](int x) {
-        const uint16_t* p = reinterpret_cast<const uint16_t*>(myrow + (x >> 6) * 16384 + ((((x >> 3) & 7) ^ sw) << 4));
-        return static_cast<uint16_t>(p[x & 7] & 0x7fffu);
-    };
-
-    __half2 srt[64];
-#pragma unroll
-    for (int gi = 0; gi < 16; ++gi) {
-        const uint4 q = chunk(gi);
-        const float4 a0 = *reinterpret_cast<const float4*>(af + 8 * gi);
-        const float4 a1 = *reinterpret_cast<const float4*>(af + 8 * gi + 4);
-        srt[4 * gi + 0] = key_pair(q.x, a0.x, a0.y);
-        srt[4 * gi + 1] = key_pair(q.y, a0.z, a0.w);
-        srt[4 * gi + 2] = key_pair(q.z, a1.x, a1.y);
-        srt[4 * gi + 3] = key_pair(q.w, a1.z, a1.w);
-    }
-    // one copy of the 32-key network, run on each half in turn (the halves
-    // swap places between the runs and are back in place after the second):
-    // half the code of two unrolled copies, for 32 register swaps
-#pragma unroll 1
-    for (int rep = 0; rep < 2; ++rep) {
-        sort32_desc2<0>(srt);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            const __half2 tmp = srt[i];
-            srt[i] = srt[32 + i];
-            srt[32 + i] = tmp;
-        }
-    }
-#pragma unroll
-    for (int i = 0; i < 32; ++i) srt[i] = __hmax2(srt[i], srt[63 - i]);
-    merge32_desc2<16>(srt);          // low halves: 32 largest even channels (L),
-                                     // high halves: 32 largest odd channels (H), descending
-    float vf;
-    if (c == 32) {
-        // the 32 largest of all are max(L_i, H_{31-i}); with the halves of
-        // register 31-i swapped, one __hmax2 forms the pairs for i and 31-i
-        __half2 mn = __half2half2(__ushort_as_half(0x7c00));   // +inf
-#pragma unroll
-        for (int i = 0; i < 16; ++i) mn = __hmin2(mn, __hmax2(srt[i], __lowhigh2highlow(srt[31 - i])));
-        vf = fminf(__low2float(mn), __high2float(mn));
-    } else {
-        float w[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) w[i] = fmaxf(__low2float(srt[i]), __high2float(srt[31 - i]));
-        merge32_desc_f<16>(w);       // 32 largest of all 128, descending
-        vf = w[0];
-#pragma unroll
-        for (int i = 1; i < 32; ++i) vf = (i < c) ? w[i] : vf;
-    }
-    const __half2 vv = __float2half2_rn(vf);   // vf is a key value: exact in fp16
-
-    // the K tile is read again below; without this fence the compiler
-    // hoists those loads above the sort and keeps both live (160 registers
-    // instead of 96, three CTAs per SM instead of five)
-    uint32_t M[4], G[4];
-    asm volatile("" ::: "memory");
-    key_masks(chunk, af, vv, M, G);
-    const int n_ge = __popc(M[0]) + __popc(M[1]) + __popc(M[2]) + __popc(M[3]);
-    if (n_ge > c) {
-        // the keys equal to v straddle the cut: keep the c - n_gt best of
-        // them by (e desc, x asc).  The fp32 products f = fp32(|k| a) are
-        // correctly rounded, so f_y > f_x implies e_y > e_x; only equal f
-        // need the exact fp64 products.
-        const int need = c - (__popc(G[0]) + __popc(G[1]) + __popc(G[2]) + __popc(G[3]));
-        const uint32_t qm[4] = {M[0] & ~G[0], M[1] & ~G[1], M[2] & ~G[2], M[3] & ~G[3]};
-        uint32_t keep[4] = {0, 0, 0, 0};
-        for (int wi = 0; wi < 4; ++wi) {
-            for (uint32_t m = qm[wi]; m; m &= m - 1) {
-                const int x = wi * 32 + __ffs(m) - 1;
-                const double kx = h2d(kbits(x));
-                const float fx = __fmul_rn(static_cast<float>(kx), af[x]);
-                int rank = 0;
-                for (int wj = 0; wj < 4; ++wj) {
-                    for (uint32_t m2 = qm[wj]; m2; m2 &= m2 - 1) {
-                        const int y = wj * 32 + __ffs(m2) - 1;
-                        if (y == x) continue;
-                        const double ky = h2d(kbits(y));
-                        const float fy = __fmul_rn(static_cast<float>(ky), af[y]);
-                        bool better = fy > fx;
-                        if (fy == fx) {
-                            const double ex = __dmul_rn(kx, ad[x]), ey = __dmul_rn(ky, ad[y]);
-                            better = (ey > ex) || (ey == ex && y < x);
-                        }
-                        rank += better;
-                    }
-                }
-                if (rank < need) keep[wi] |= 1u << (x & 31);
-            }
-        }
-#pragma unroll
-        for (int wi = 0; wi < 4; ++wi) M[wi] = G[wi] | keep[wi];
-    }
-
-    // g_t: both fp64 sums ascending in x; |k| widened from fp16 in one
-    // conversion, and e = |k| a_x is exact in fp64, so each fused
-    // multiply-add rounds exactly as adding e does
+    const ChanRow R{tile + tid * 128, tid & 7};
+    const uint4 m = chan_row_mask(R, af, ad, A.c);
+    const double gv = chan_row_g(R, ad, m);
     const int64_t slot = static_cast<int64_t>(u) * A.g_stride + t;
-    double tot = 0.0, drop = 0.0;
-#pragma unroll 1
-    for (int j = 0; j < 16; ++j) {
-        const uint4 q = chunk(j);
-        const uint32_t mw = ((j < 4) ? M[0] : (j < 8) ? M[1] : (j < 12) ? M[2] : M[3]) >> ((j & 3) * 8);
-        const uint32_t qw[4] = {q.x & 0x7fff7fffu, q.y & 0x7fff7fffu, q.z & 0x7fff7fffu, q.w & 0x7fff7fffu};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const double2 a2 = *reinterpret_cast<const double2*>(ad + 8 * j + 2 * e);
-            const double k0 = h2d(static_cast<uint16_t>(qw[e] & 0xffffu));
-            const double k1 = h2d(static_cast<uint16_t>(qw[e] >> 16));
-            tot = __fma_rn(k0, a2.x, tot);
-            drop = dfma_unless(drop, k0, a2.x, mw, 1u << (2 * e));
-            tot = __fma_rn(k1, a2.y, tot);
-            drop = dfma_unless(drop, k1, a2.y, mw, 2u << (2 * e));
-        }
-    }
-    A.cmask[slot] = make_uint4(M[0], M[1], M[2], M[3]);
-    const double gv = tot > 0.0 ? __ddiv_rn(drop, tot) : 0.0;
+    A.cmask[slot] = m;
     A.g[slot] = gv;
     if (A.dbg_g) A.dbg_g[static_cast<int64_t>(u) * A.dbg_stride + t] = gv;
 }
