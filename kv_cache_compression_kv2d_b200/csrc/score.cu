@@ -13,7 +13,9 @@
 //   pass 2    : merges the lse partials in split order, then
 //               s_t = sum_rows exp(l - lse) from the transposed product
 //               K Q_w^T (M = 128 keys, N = window rows) so that each TMEM lane
-//               owns one key and sums over queries in-thread
+//               owns one key and sums over queries in-thread; the two
+//               epilogue warpgroups take alternate tiles, each accumulator
+//               split in two column halves with their own barriers
 //   chan      : a_d = (sum of the |q_d| tile sums) / (G*W); per key: top-c
 //               channels of |k_d| a_d and g_t in fp64 (a
 //               packed 16-bit SIMD selection network for c <= 32, a full
@@ -122,8 +124,8 @@ __global__ void __launch_bounds__(kPassThreads, 1)
     uint64_t* full = reinterpret_cast<uint64_t*>(k_s + kP1Stages * kStage);
     uint64_t* empty = full + kP1Stages;
     uint64_t* tfull = empty + kP1Stages;
-    uint64_t* tempty = tfull + 2;
-    uint64_t* qbar = tempty + 2;
+    uint64_t* tempty = tfull + 4;
+    uint64_t* qbar = tempty + 4;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(qbar + 1);
     float* xm = reinterpret_cast<float*>(tmem_slot + 4);   // [256]
     float* xl = xm + 256;
@@ -133,7 +135,7 @@ __global__ void __launch_bounds__(kPassThreads, 1)
             mbar_init(&full[i], 1);
             mbar_init(&empty[i], 1);
         }
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < 4; ++i) {
             mbar_init(&tfull[i], 1);
             mbar_init(&tempty[i], 128);
         }
@@ -170,28 +172,39 @@ __global__ void __launch_bounds__(kPassThreads, 1)
         }
     } else if (warp == 9) {
         if (lane == 0) {
-            constexpr uint32_t idesc = idesc_f16_f32(128, 128);
+            // each warpgroup's accumulator is two 64-key halves with their
+            // own barriers, so the MMA refills the first half while the
+            // epilogue still reads the second
+            constexpr uint32_t idesc = idesc_f16_f32(128, 64);
             const uint32_t qa = smem_u32(q_s);
             bool ok = mbar_wait(qbar, 0, A.status);
             for (int i = 0; ok && i < nt; ++i) {
                 const int s = i % kP1Stages, buf = i & 1;
                 if (!mbar_wait(&full[s], (i / kP1Stages) & 1, A.status)) break;
-                if (i >= 2 && !mbar_wait(&tempty[buf], ((i >> 1) - 1) & 1, A.status)) break;
-                tc_fence_after();
                 const uint32_t ka = smem_u32(k_s + s * kStage);
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int hb = 2 * buf + hh;
+                    if (i >= 2 && !mbar_wait(&tempty[hb], ((i >> 1) - 1) & 1, A.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                    umma_f16(tmem + buf * 128, sw128_kmajor_desc(qa + off),
-                             sw128_kmajor_desc(ka + off), idesc, kk > 0 ? 1u : 0u);
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                        umma_f16(tmem + hb * 64, sw128_kmajor_desc(qa + off),
+                                 sw128_kmajor_desc(ka + hh * 8192 + off), idesc, kk > 0 ? 1u : 0u);
+                    }
+                    umma_commit(&tfull[hb]);
                 }
+                if (!ok) break;
                 umma_commit(&empty[s]);
-                umma_commit(&tfull[buf]);
             }
         }
     } else {
         // epilogue: warps 0-3 take even tiles (TMEM columns 0..127), warps
-        // 4-7 odd tiles (columns 128..255); thread <-> window row.
+        // 4-7 odd tiles (columns 128..255), each as two 64-column halves;
+        // thread <-> window row.
         const int wg = warp >> 2, lg = warp & 3;
         const int row = lg * 32 + lane;
         const int rho = mt * 128 + row;
@@ -200,7 +213,7 @@ __global__ void __launch_bounds__(kPassThreads, 1)
         const float c2 = A.shp.c2;
         float m = __uint_as_float(kNegInf), l = 0.f;
         for (int i = wg; i < nt; i += 2) {
-            if (!mbar_wait(&tfull[wg], (i >> 1) & 1, A.status)) break;
+            if (!mbar_wait(&tfull[2 * wg], (i >> 1) & 1, A.status)) break;
             tc_fence_after();
             const int t_base = k_lo + i * kKeyTile;
             const uint32_t taddr = tmem + (static_cast<uint32_t>(lg * 32) << 16) + wg * 128;
@@ -244,21 +257,27 @@ __global__ void __launch_bounds__(kPassThreads, 1)
                 }
                 l += (a0 + a1) + (a2 + a3);
             };
+            // half buffer 2 wg holds chunks 0, 1 (columns wg * 128 + 0..63),
+            // half buffer 2 wg + 1 chunks 2, 3
             uint32_t ra[32], rb[32];
             tmem_ld32(taddr, ra);
             tmem_ld_wait(ra);
             tmem_ld32(taddr + 32, rb);
             proc(ra, 0);
             tmem_ld_wait(rb);
+            if (!mbar_wait(&tfull[2 * wg + 1], (i >> 1) & 1, A.status)) break;
+            tc_fence_after();
             tmem_ld32(taddr + 64, ra);
             proc(rb, 1);
+            tc_fence_before();
+            mbar_arrive(&tempty[2 * wg]);
             tmem_ld_wait(ra);
             tmem_ld32(taddr + 96, rb);
             proc(ra, 2);
             tmem_ld_wait(rb);
             proc(rb, 3);
             tc_fence_before();
-            mbar_arrive(&tempty[wg]);
+            mbar_arrive(&tempty[2 * wg + 1]);
         }
         if (wg == 1) {
             xm[row] = m;
@@ -346,8 +365,8 @@ __global__ void __launch_bounds__(kPassThreads, 1)
     uint64_t* full = reinterpret_cast<uint64_t*>(sb + 128);
     uint64_t* empty = full + 4;
     uint64_t* tfull = empty + 4;
-    uint64_t* tempty = tfull + 2;
-    uint64_t* qbar = tempty + 2;
+    uint64_t* tempty = tfull + 4;
+    uint64_t* qbar = tempty + 4;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(qbar + 1);
 
     if (tid == 0) {
@@ -355,7 +374,7 @@ __global__ void __launch_bounds__(kPassThreads, 1)
             mbar_init(&full[i], 1);
             mbar_init(&empty[i], 1);
         }
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < 4; ++i) {
             mbar_init(&tfull[i], 1);
             mbar_init(&tempty[i], split_cols ? 256 : 128);
         }
@@ -426,19 +445,46 @@ __global__ void __launch_bounds__(kPassThreads, 1)
             const uint32_t idesc = idesc_f16_f32(128, Nc);
             const uint32_t qa = smem_u32(q_s);
             bool ok = mbar_wait(qbar, 0, A.status);
-            for (int i = 0; ok && i < nt; ++i) {
+            // G*W <= 256: each warpgroup's accumulator is two half-width
+            // buffers with their own barriers, so the MMA refills the first
+            // half while the epilogue still reads the second
+            const bool halves = !split_cols;
+            const uint32_t idesc_h = idesc_f16_f32(128, Nc / 2);
+            for (int i = 0; ok && halves && i < nt; ++i) {
+                // tile i into the half buffers 2 (i & 1) + h, Nc / 2 columns each
                 const int s = i % NS;
-                const int buf = split_cols ? 0 : (i & 1);
                 if (!mbar_wait(&full[s], (i / NS) & 1, A.status)) break;
-                if (split_cols) {
-                    if (i >= 1 && !mbar_wait(&tempty[0], (i - 1) & 1, A.status)) break;
-                } else if (i >= 2 && !mbar_wait(&tempty[buf], ((i >> 1) - 1) & 1, A.status)) {
-                    break;
+                const uint32_t ka = smem_u32(k_s + s * kStage);
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int hb = 2 * (i & 1) + hh;
+                    if (i >= 2 && !mbar_wait(&tempty[hb], ((i >> 1) - 1) & 1, A.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t qb = qa + hh * (Nc / 2) * 128;
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint32_t aoff = (kk >> 2) * 16384 + (kk & 3) * 32;
+                        const uint32_t boff = (kk >> 2) * (Nc * 128) + (kk & 3) * 32;
+                        umma_f16(tmem + hb * (Nc / 2), sw128_kmajor_desc(ka + aoff),
+                                 sw128_kmajor_desc(qb + boff), idesc_h, kk > 0 ? 1u : 0u);
+                    }
+                    umma_commit(&tfull[hb]);
                 }
+                if (!ok) break;
+                umma_commit(&empty[s]);
+            }
+            // split-column mode: both column halves of every tile into one
+            // buffer pair
+            for (int i = 0; ok && split_cols && i < nt; ++i) {
+                const int s = i % NS;
+                if (!mbar_wait(&full[s], (i / NS) & 1, A.status)) break;
+                if (i >= 1 && !mbar_wait(&tempty[0], (i - 1) & 1, A.status)) break;
                 tc_fence_after();
                 const uint32_t ka = smem_u32(k_s + s * kStage);
                 for (int qc = 0; qc < nqc; ++qc) {
-                    const uint32_t dcol = split_cols ? qc * Nc : buf * Nc;
+                    const uint32_t dcol = qc * Nc;
                     const uint32_t qb = qa + qc * Nc * 256;
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk) {
@@ -449,7 +495,7 @@ __global__ void __launch_bounds__(kPassThreads, 1)
                     }
                 }
                 umma_commit(&empty[s]);
-                umma_commit(&tfull[buf]);
+                umma_commit(&tfull[0]);
             }
         }
     } else {
@@ -459,65 +505,76 @@ __global__ void __launch_bounds__(kPassThreads, 1)
         const float c2 = A.shp.c2;
         const int tw = T - W;                 // keys <= tw are seen by every row
         const int step = split_cols ? 1 : 2;
+        const bool halves = !split_cols;
+        const int nparts = halves ? 2 : 1;
+        const int ncol = halves ? Nc / 2 : Nc;    // columns per TMEM buffer
         for (int i = split_cols ? 0 : wg; i < nt; i += step) {
-            const int buf = split_cols ? 0 : wg;
             const int k = split_cols ? i : (i >> 1);
-            if (!mbar_wait(&tfull[buf], k & 1, A.status)) break;
-            tc_fence_after();
             const int t = k_lo + i * kKeyTile + row;
-            const int qc = split_cols ? wg : 0;
-            const uint32_t taddr = tmem + (static_cast<uint32_t>(lg * 32) << 16) +
-                                   (split_cols ? qc * Nc : buf * Nc);
-            const int col0 = qc * Nc;
             const int need = t - tw;          // row visible iff wpos >= need
             float sacc = 0.f;
-            // 32-column chunks, double-buffered: chunk c+1's TMEM load is in
-            // flight while chunk c is summed
-            auto proc = [&](const uint32_t (&r)[32], int cc) {
-                const float4* l4 = reinterpret_cast<const float4*>(lse_s + col0 + cc);
-                float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-                if (need <= 0) {
-#pragma unroll
-                    for (int j = 0; j < 32; j += 4) {
-                        const float4 lz = l4[j >> 2];
-                        a0 += exp2_mixed<kP2FmaEvery>(fmaf(__uint_as_float(r[j]), c2, -lz.x), j);
-                        a1 += exp2_mixed<kP2FmaEvery>(fmaf(__uint_as_float(r[j + 1]), c2, -lz.y), j + 1);
-                        a2 += exp2_mixed<kP2FmaEvery>(fmaf(__uint_as_float(r[j + 2]), c2, -lz.z), j + 2);
-                        a3 += exp2_mixed<kP2FmaEvery>(fmaf(__uint_as_float(r[j + 3]), c2, -lz.w), j + 3);
-                    }
-                } else {
-                    const int* wp = wpos_s + col0 + cc;
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const float e = fast_exp2(fmaf(__uint_as_float(r[j]), c2, -lse_s[col0 + cc + j]));
-                        a0 += (wp[j] >= need) ? e : 0.f;
-                    }
+            bool ok = true;
+            for (int part = 0; part < nparts; ++part) {
+                const int buf = split_cols ? 0 : 2 * wg + part;
+                if (!mbar_wait(&tfull[buf], k & 1, A.status)) {
+                    ok = false;
+                    break;
                 }
-                sacc += (a0 + a1) + (a2 + a3);
-            };
-            uint32_t ra[32], rb[32];
-            const int nch = Nc / 32;          // 4, 6 or 8 chunks (Nc 128..256)
-            tmem_ld32(taddr, ra);
-            tmem_ld_wait(ra);
+                tc_fence_after();
+                const int qc = split_cols ? wg : 0;
+                const uint32_t taddr = tmem + (static_cast<uint32_t>(lg * 32) << 16) +
+                                       (split_cols ? qc * Nc : buf * ncol);
+                const int col0 = split_cols ? qc * Nc : part * ncol;
+                // 32-column chunks, double-buffered: chunk c+1's TMEM load is
+                // in flight while chunk c is summed
+                auto proc = [&](const uint32_t (&r)[32], int cc) {
+                    const float4* l4 = reinterpret_cast<const float4*>(lse_s + col0 + cc);
+                    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+                    if (need <= 0) {
+#pragma unroll
+                        for (int j = 0; j < 32; j += 4) {
+                            const float4 lz = l4[j >> 2];
+                            a0 += exp2_mixed<kP2FmaEvery>(fmaf(__uint_as_float(r[j]), c2, -lz.x), j);
+                            a1 += exp2_mixed<kP2FmaEvery>(fmaf(__uint_as_float(r[j + 1]), c2, -lz.y), j + 1);
+                            a2 += exp2_mixed<kP2FmaEvery>(fmaf(__uint_as_float(r[j + 2]), c2, -lz.z), j + 2);
+                            a3 += exp2_mixed<kP2FmaEvery>(fmaf(__uint_as_float(r[j + 3]), c2, -lz.w), j + 3);
+                        }
+                    } else {
+                        const int* wp = wpos_s + col0 + cc;
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            const float e = fast_exp2(fmaf(__uint_as_float(r[j]), c2, -lse_s[col0 + cc + j]));
+                            a0 += (wp[j] >= need) ? e : 0.f;
+                        }
+                    }
+                    sacc += (a0 + a1) + (a2 + a3);
+                };
+                uint32_t ra[32], rb[32];
+                const int nch = ncol / 32;        // 2 .. 8 chunks
+                tmem_ld32(taddr, ra);
+                tmem_ld_wait(ra);
 #pragma unroll 1
-            for (int ch = 0; ch < nch; ch += 2) {
-                if (ch + 1 < nch) tmem_ld32(taddr + (ch + 1) * 32, rb);
-                proc(ra, ch * 32);
-                if (ch + 1 < nch) {
-                    tmem_ld_wait(rb);
-                    if (ch + 2 < nch) tmem_ld32(taddr + (ch + 2) * 32, ra);
-                    proc(rb, (ch + 1) * 32);
-                    if (ch + 2 < nch) tmem_ld_wait(ra);
+                for (int ch = 0; ch < nch; ch += 2) {
+                    if (ch + 1 < nch) tmem_ld32(taddr + (ch + 1) * 32, rb);
+                    proc(ra, ch * 32);
+                    if (ch + 1 < nch) {
+                        tmem_ld_wait(rb);
+                        if (ch + 2 < nch) tmem_ld32(taddr + (ch + 2) * 32, ra);
+                        proc(rb, (ch + 1) * 32);
+                        if (ch + 2 < nch) tmem_ld_wait(ra);
+                    }
                 }
+                tc_fence_before();
+                if (!split_cols) mbar_arrive(&tempty[buf]);
             }
-            tc_fence_before();
+            if (!ok) break;
             if (split_cols) {
                 if (wg == 1) sb[row] = sacc;
                 named_bar_sync(1, 256);
                 if (wg == 0) sacc = sacc + sb[row];
                 named_bar_sync(2, 256);
+                mbar_arrive(&tempty[0]);
             }
-            mbar_arrive(&tempty[buf]);
             if ((!split_cols || wg == 0) && t < k_hi) {
                 const int64_t rel = t - r0;
                 A.s[static_cast<int64_t>(u) * A.s_stride + rel] = sacc;
