@@ -238,17 +238,78 @@ __device__ __forceinline__ float fast_exp2(float x) {
 // fp32 Horner steps), and n added to the exponent bits.  Used for part of
 // the exponentials of the scoring epilogues so that the MUFU pipe is not the
 // only one busy.
+// Coefficients of the degree-5 fit on [-0.5, 0.5], highest degree first.
+constexpr float kExp2P5 = 1.327646780e-03f;
+constexpr float kExp2P4 = 9.675540961e-03f;
+constexpr float kExp2P3 = 5.550713465e-02f;
+constexpr float kExp2P2 = 2.402212024e-01f;
+constexpr float kExp2P1 = 6.931469440e-01f;
+constexpr float kExp2P0 = 1.000000119e+00f;
+
 __device__ __forceinline__ float exp2_fma(float x) {
     x = fmaxf(x, -126.f);
     const float t = x + 12582912.f;
     const float f = x - (t - 12582912.f);
-    float p = 1.327646780e-03f;
-    p = fmaf(p, f, 9.675540961e-03f);
-    p = fmaf(p, f, 5.550713465e-02f);
-    p = fmaf(p, f, 2.402212024e-01f);
-    p = fmaf(p, f, 6.931469440e-01f);
-    p = fmaf(p, f, 1.000000119e+00f);
+    float p = kExp2P5;
+    p = fmaf(p, f, kExp2P4);
+    p = fmaf(p, f, kExp2P3);
+    p = fmaf(p, f, kExp2P2);
+    p = fmaf(p, f, kExp2P1);
+    p = fmaf(p, f, kExp2P0);
     return __int_as_float(__float_as_int(p) + ((__float_as_int(t) - 0x4B400000) << 23));
+}
+
+// Packed fp32 pairs (sm_100): each lane is rounded exactly as the scalar
+// fused multiply-add / add / subtract of the same operands.
+__device__ __forceinline__ float2 f2_fma(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\t"
+        "mov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+
+__device__ __forceinline__ float2 f2_add(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rd, ra, rb;\n\t"
+        "mov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+
+__device__ __forceinline__ float2 f2_sub(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "sub.rn.f32x2 rd, ra, rb;\n\t"
+        "mov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+
+// exp2_fma on a pair, the floating-point steps on packed pairs (each lane
+// identical to exp2_fma).
+__device__ __forceinline__ float2 exp2_fma2(float2 x) {
+    x.x = fmaxf(x.x, -126.f);
+    x.y = fmaxf(x.y, -126.f);
+    const float2 sh = make_float2(12582912.f, 12582912.f);
+    const float2 t = f2_add(x, sh);
+    const float2 f = f2_sub(x, f2_sub(t, sh));
+    float2 p = make_float2(kExp2P5, kExp2P5);
+    p = f2_fma(p, f, make_float2(kExp2P4, kExp2P4));
+    p = f2_fma(p, f, make_float2(kExp2P3, kExp2P3));
+    p = f2_fma(p, f, make_float2(kExp2P2, kExp2P2));
+    p = f2_fma(p, f, make_float2(kExp2P1, kExp2P1));
+    p = f2_fma(p, f, make_float2(kExp2P0, kExp2P0));
+    return make_float2(__int_as_float(__float_as_int(p.x) + ((__float_as_int(t.x) - 0x4B400000) << 23)),
+                       __int_as_float(__float_as_int(p.y) + ((__float_as_int(t.y) - 0x4B400000) << 23)));
 }
 
 // Programmatic dependent launch: wait until the grids this one depends on

@@ -31,17 +31,18 @@ namespace {
 constexpr int kPassThreads = 320;    // 8 epilogue warps, 1 TMA warp, 1 MMA warp
 constexpr int kStage = 128 * 256;    // one K tile: 128 keys x 128 fp16
 constexpr int kP1Stages = 2;   // ~99 KB of shared memory: two CTAs per SM
-// Every n-th exponential of a fully visible tile runs on the FMA pipe
-// (exp2_fma) instead of MUFU; 0: none.  Pass 2 sums 2^x of G*W columns per
-// key and leans on MUFU harder than pass 1, which also tracks row maxima.
+// Part of the exponentials of a fully visible tile run on the FMA pipe
+// (exp2_fma) instead of MUFU.  Pass 1: every n-th (0: none).  Pass 2, which
+// sums 2^x of G*W columns per key and leans on MUFU harder than pass 1 (that
+// also tracks row maxima): this many pairs of each 8 columns (exp2_fma2).
 #ifndef KV2D_P1_FMA_EVERY
 #define KV2D_P1_FMA_EVERY 8
 #endif
-#ifndef KV2D_P2_FMA_EVERY
-#define KV2D_P2_FMA_EVERY 4
+#ifndef KV2D_P2_POLY_PAIRS
+#define KV2D_P2_POLY_PAIRS 1
 #endif
 constexpr int kP1FmaEvery = KV2D_P1_FMA_EVERY;
-constexpr int kP2FmaEvery = KV2D_P2_FMA_EVERY;
+constexpr int kP2PolyPairs = KV2D_P2_POLY_PAIRS;
 
 template <int EVERY>
 __device__ __forceinline__ float exp2_mixed(float x, int j) {
@@ -240,13 +241,25 @@ __global__ void __launch_bounds__(kPassThreads, 1)
                 const float nm = -m;
                 float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
                 if (whole) {
+                    // packed pairs: (a0, a1) and (a2, a3) accumulate columns
+                    // 4q + {0, 1} and 4q + {2, 3}, each lane as the scalar
+                    // multiply-add / add would
+                    const float2 c2v = make_float2(c2, c2), nmv = make_float2(nm, nm);
+                    float2 a01 = make_float2(0.f, 0.f), a23 = make_float2(0.f, 0.f);
 #pragma unroll
                     for (int j = 0; j < 32; j += 4) {
-                        a0 += exp2_mixed<kP1FmaEvery>(fmaf(__uint_as_float(r[j]), c2, nm), j);
-                        a1 += exp2_mixed<kP1FmaEvery>(fmaf(__uint_as_float(r[j + 1]), c2, nm), j + 1);
-                        a2 += exp2_mixed<kP1FmaEvery>(fmaf(__uint_as_float(r[j + 2]), c2, nm), j + 2);
-                        a3 += exp2_mixed<kP1FmaEvery>(fmaf(__uint_as_float(r[j + 3]), c2, nm), j + 3);
+                        const float2 x01 = f2_fma(make_float2(__uint_as_float(r[j]), __uint_as_float(r[j + 1])), c2v, nmv);
+                        const float2 x23 =
+                            f2_fma(make_float2(__uint_as_float(r[j + 2]), __uint_as_float(r[j + 3])), c2v, nmv);
+                        a01 = f2_add(a01, make_float2(exp2_mixed<kP1FmaEvery>(x01.x, j),
+                                                      exp2_mixed<kP1FmaEvery>(x01.y, j + 1)));
+                        a23 = f2_add(a23, make_float2(exp2_mixed<kP1FmaEvery>(x23.x, j + 2),
+                                                      exp2_mixed<kP1FmaEvery>(x23.y, j + 3)));
                     }
+                    a0 = a01.x;
+                    a1 = a01.y;
+                    a2 = a23.x;
+                    a3 = a23.y;
                 } else {
                     const int t0 = t_base + cc * 32;
 #pragma unroll
@@ -359,8 +372,8 @@ __global__ void __launch_bounds__(kPassThreads, 1)
     uint8_t* smem = align1024(smem_raw);
     uint8_t* q_s = smem;                                  // GWpad x 256 B
     uint8_t* k_s = smem + GWpad * 256;
-    float* lse_s = reinterpret_cast<float*>(k_s + NS * kStage);
-    int* wpos_s = reinterpret_cast<int*>(lse_s + GWpad);
+    float* nlse_s = reinterpret_cast<float*>(k_s + NS * kStage);   // -lse per column
+    int* wpos_s = reinterpret_cast<int*>(nlse_s + GWpad);
     float* sb = reinterpret_cast<float*>(wpos_s + GWpad);
     uint64_t* full = reinterpret_cast<uint64_t*>(sb + 128);
     uint64_t* empty = full + 4;
@@ -413,7 +426,7 @@ __global__ void __launch_bounds__(kPassThreads, 1)
                     out * 0.69314718055994531f;
             }
         }
-        lse_s[i] = out;
+        nlse_s[i] = -out;
         wpos_s[i] = i % W;
     }
     tc_fence_before();
@@ -528,26 +541,47 @@ __global__ void __launch_bounds__(kPassThreads, 1)
                 // 32-column chunks, double-buffered: chunk c+1's TMEM load is
                 // in flight while chunk c is summed
                 auto proc = [&](const uint32_t (&r)[32], int cc) {
-                    const float4* l4 = reinterpret_cast<const float4*>(lse_s + col0 + cc);
-                    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+                    const float4* l4 = reinterpret_cast<const float4*>(nlse_s + col0 + cc);
                     if (need <= 0) {
+                        // packed pairs: (a0, a1) and (a2, a3) accumulate
+                        // columns 4q + {0, 1} and 4q + {2, 3}; of each 8
+                        // columns the last kP2PolyPairs pairs take exp2 on
+                        // the FMA pipe, the rest on MUFU
+                        const float2 c2v = make_float2(c2, c2);
+                        float2 a01 = make_float2(0.f, 0.f), a23 = make_float2(0.f, 0.f);
 #pragma unroll
-                        for (int j = 0; j < 32; j += 4) {
-                            const float4 lz = l4[j >> 2];
-                            a0 += exp2_mixed<kP2FmaEvery>(fmaf(__uint_as_float(r[j]), c2, -lz.x), j);
-                            a1 += exp2_mixed<kP2FmaEvery>(fmaf(__uint_as_float(r[j + 1]), c2, -lz.y), j + 1);
-                            a2 += exp2_mixed<kP2FmaEvery>(fmaf(__uint_as_float(r[j + 2]), c2, -lz.z), j + 2);
-                            a3 += exp2_mixed<kP2FmaEvery>(fmaf(__uint_as_float(r[j + 3]), c2, -lz.w), j + 3);
+                        for (int j = 0; j < 32; j += 8) {
+                            const float4 n0 = l4[j >> 2], n1 = l4[(j >> 2) + 1];
+                            float2 x[4];
+                            x[0] = f2_fma(make_float2(__uint_as_float(r[j]), __uint_as_float(r[j + 1])), c2v,
+                                          make_float2(n0.x, n0.y));
+                            x[1] = f2_fma(make_float2(__uint_as_float(r[j + 2]), __uint_as_float(r[j + 3])), c2v,
+                                          make_float2(n0.z, n0.w));
+                            x[2] = f2_fma(make_float2(__uint_as_float(r[j + 4]), __uint_as_float(r[j + 5])), c2v,
+                                          make_float2(n1.x, n1.y));
+                            x[3] = f2_fma(make_float2(__uint_as_float(r[j + 6]), __uint_as_float(r[j + 7])), c2v,
+                                          make_float2(n1.z, n1.w));
+                            float2 e[4];
+#pragma unroll
+                            for (int q = 0; q < 4; ++q)
+                                e[q] = (q >= 4 - kP2PolyPairs) ? exp2_fma2(x[q])
+                                                               : make_float2(fast_exp2(x[q].x), fast_exp2(x[q].y));
+                            a01 = f2_add(a01, e[0]);
+                            a23 = f2_add(a23, e[1]);
+                            a01 = f2_add(a01, e[2]);
+                            a23 = f2_add(a23, e[3]);
                         }
+                        sacc += (a01.x + a01.y) + (a23.x + a23.y);
                     } else {
                         const int* wp = wpos_s + col0 + cc;
+                        float a0 = 0.f;
 #pragma unroll
                         for (int j = 0; j < 32; ++j) {
-                            const float e = fast_exp2(fmaf(__uint_as_float(r[j]), c2, -lse_s[col0 + cc + j]));
+                            const float e = fast_exp2(fmaf(__uint_as_float(r[j]), c2, nlse_s[col0 + cc + j]));
                             a0 += (wp[j] >= need) ? e : 0.f;
                         }
+                        sacc += a0;
                     }
-                    sacc += (a0 + a1) + (a2 + a3);
                 };
                 uint32_t ra[32], rb[32];
                 const int nch = ncol / 32;        // 2 .. 8 chunks

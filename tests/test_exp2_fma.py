@@ -1,4 +1,5 @@
-"""The FMA-pipe exp2 of the scoring epilogues (csrc/common.cuh: exp2_fma),
+"""The FMA-pipe exp2 of the scoring epilogues (csrc/common.cuh: exp2_fma,
+and exp2_fma2, the same steps on packed pairs with the same coefficients),
 replayed step by step in numpy float32 (each multiply-add rounded once, as a
 fused multiply-add is) and compared with the exact 2^x: relative error at
 most 3e-7 on [-126, 0], the same order as the hardware approximation it
@@ -14,9 +15,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 def _coeffs():
     with open(os.path.join(ROOT, "kv_cache_compression_kv2d_b200", "csrc", "common.cuh")) as f:
         src = f.read()
-    body = src[src.index("float exp2_fma(float x)"):]
-    body = body[:body.index("\n}\n")]
-    vals = [float(v) for v in re.findall(r"([0-9]\.[0-9]+e[-+][0-9]+)f", body)]
+    vals = [float(re.search(r"constexpr float kExp2P%d = ([0-9]\.[0-9]+e[-+][0-9]+)f;" % k, src).group(1))
+            for k in range(5, -1, -1)]
     return np.float32(vals[0]), [np.float32(v) for v in vals[1:]]
 
 
