@@ -278,6 +278,12 @@ __global__ void __launch_bounds__(kSegWarps * 32) seg_select_kernel(const __grid
 // the general kernel.
 constexpr int kSmallSegs = 32;
 
+// 16 bytes global -> shared by this thread, asynchronously (cached in L2
+// only); both addresses 16-byte aligned.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+
 template <int N>
 __device__ __forceinline__ void bitonic_sort_desc(double (&v)[N]) {
 #pragma unroll
@@ -330,16 +336,20 @@ __global__ void __launch_bounds__(kSmallSegs) seg_select_small_kernel(const __gr
     double* grows = reinterpret_cast<double*>(srows + kSmallSegs * SR);         // [32][S + 2]
     const int nv = min(kSmallSegs, nseg - jb);
     {
+        // every 16-byte piece is an asynchronous copy issued back to back,
+        // then one wait: the warp pays the L2 latency once, not once per
+        // load (at small sizes it is alone on its SM)
         const float4* s4 = reinterpret_cast<const float4*>(A.s + static_cast<int64_t>(u) * A.s_stride +
                                                            static_cast<int64_t>(jb) * S);
         const int q4 = S / 4, n4 = nv * q4;
         for (int i = lane; i < n4; i += kSmallSegs)
-            *reinterpret_cast<float4*>(srows + (i / q4) * SR + 4 * (i % q4)) = s4[i];
+            cp_async16(srows + (i / q4) * SR + 4 * (i % q4), s4 + i);
         const double2* g2 = reinterpret_cast<const double2*>(A.g + static_cast<int64_t>(u) * A.g_stride +
                                                              static_cast<int64_t>(jb) * S);
         const int q2 = S / 2, n2 = nv * q2;
         for (int i = lane; i < n2; i += kSmallSegs)
-            *reinterpret_cast<double2*>(grows + (i / q2) * GR + 2 * (i % q2)) = g2[i];
+            cp_async16(grows + (i / q2) * GR + 2 * (i % q2), g2 + i);
+        asm volatile("cp.async.wait_all;" ::: "memory");
     }
     __syncwarp();
     if (lane >= nv) return;
