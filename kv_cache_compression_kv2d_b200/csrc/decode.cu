@@ -155,15 +155,14 @@ constexpr int kTbl = kDecTableMax;                 // blocks in the block table 
 
 __device__ __forceinline__ void mma16816(float& d0, float& d1, uint32_t a0, uint32_t a2, uint32_t b0,
                                          uint32_t b1) {
-    float x2, x3;   // rows 8..15 of the tile: never used
+    // rows 8..15 of the tile (accumulators 2, 3) are never used: they go to
+    // scratch registers declared inside the asm
     asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
-        "{%8, %9}, {%10, %11, %12, %13};"
-        : "=f"(d0), "=f"(d1), "=f"(x2), "=f"(x3)
-        : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1), "f"(d0), "f"(d1), "f"(0.f),
-          "f"(0.f));
-    (void)x2;
-    (void)x3;
+        "{\n\t.reg .f32 x2, x3;\n\t"
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, x2, x3}, {%2, %3, %4, %5}, "
+        "{%6, %7}, {%8, %9, %10, %11};\n\t}"
+        : "=f"(d0), "=f"(d1)
+        : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1), "f"(d0), "f"(d1), "f"(0.f), "f"(0.f));
 }
 
 // m16n8k8, all four accumulators live: D[16 x 8] += A[16 x 8] B[8 x 8].

@@ -278,10 +278,16 @@ __global__ void __launch_bounds__(kSegWarps * 32) seg_select_kernel(const __grid
 // the general kernel.
 constexpr int kSmallSegs = 32;
 
-// 16 bytes global -> shared by this thread, asynchronously (cached in L2
-// only); both addresses 16-byte aligned.
+// 16 / 8 / 4 bytes global -> shared by this thread, asynchronously; both
+// addresses aligned to the size.
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async8(void* dst, const void* src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
 }
 
 template <int N>
@@ -528,12 +534,15 @@ __global__ void __launch_bounds__(kBudgetThreads) budget_kernel(const __grid_con
         double* efs = reinterpret_cast<double*>(budget_smem);
         int32_t* dbs = reinterpret_cast<int32_t*>(efs + 3 * kBudgetCacheSegs);
         uint8_t* hs = reinterpret_cast<uint8_t*>(dbs + 3 * kBudgetCacheSegs);
+        // asynchronous copies issued back to back, one wait: the L2 latency
+        // is paid once, not once per iteration
         for (int i = tid; i < nseg * 3; i += kBudgetThreads) {
-            efs[i] = EF[i];
-            dbs[i] = DB[i];
+            cp_async8(efs + i, EF + i);
+            cp_async4(dbs + i, DB + i);
         }
         for (int i = tid; i < nseg * 2; i += kBudgetThreads)
-            reinterpret_cast<uint32_t*>(hs)[i] = reinterpret_cast<const uint32_t*>(H)[i];
+            cp_async4(reinterpret_cast<uint32_t*>(hs) + i, reinterpret_cast<const uint32_t*>(H) + i);
+        asm volatile("cp.async.wait_all;" ::: "memory");
         __syncthreads();
         H = hs;
         EF = efs;
