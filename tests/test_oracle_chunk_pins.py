@@ -63,6 +63,21 @@ def test_hand_worked_merit_order_and_budget_skip(orc):
     assert orc.topr_chunks(_p(orc, 32, 6, 6, 2), s).tolist() == [1, 4, 8, 9, 10, 20]
 
 
+def test_hand_worked_span_cap_is_inclusive(orc):
+    # S = 16, r = 6, alpha = 3.  Core (top 3): tokens 2, 6, 12.  The chunk
+    # from 2 to 6 holds the gap 3, 4, 5 and spans 6 - 2 + 1 = 5 tokens,
+    # endpoints included; (6, 12) spans 7.  With gamma = 5 the first gap is
+    # a candidate and fills the whole budget: 2, 3, 4, 5, 6, 12.  With
+    # gamma = 4 neither gap is, and the budget goes to the best tokens left:
+    # 14, 0, 15.
+    s = np.zeros(16)
+    s[[2, 6, 12]] = [9.0, 8.0, 7.0]
+    s[3], s[4], s[5] = 0.1, 0.1, 0.1
+    s[14], s[0], s[15] = 0.9, 0.8, 0.7
+    assert orc.topr_chunks(_p(orc, 16, 6, 5, 3), s).tolist() == [2, 3, 4, 5, 6, 12]
+    assert orc.topr_chunks(_p(orc, 16, 6, 4, 3), s).tolist() == [0, 2, 6, 12, 14, 15]
+
+
 @pytest.mark.parametrize("seed", range(6))
 def test_structure_on_random_segments(orc, seed):
     rng = np.random.default_rng(100 + seed)
