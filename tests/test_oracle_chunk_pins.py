@@ -78,6 +78,17 @@ def test_hand_worked_span_cap_is_inclusive(orc):
     assert orc.topr_chunks(_p(orc, 16, 6, 4, 3), s).tolist() == [0, 2, 6, 12, 14, 15]
 
 
+def test_hand_worked_equal_merits_go_to_the_lower_gap(orc):
+    # S = 16, r = 5, alpha = 1, gamma = 3.  Core (top 4): 1, 3, 9, 11.  Gaps
+    # (1, 3) and (9, 11) hold one token each (2 and 10) with the same merit
+    # 0.5; the budget of 1 fills the one that starts lower: token 2.
+    s = np.zeros(16)
+    s[[1, 3, 9, 11]] = [9.0, 8.0, 7.0, 6.0]
+    s[2] = s[10] = 0.5
+    s[14] = 0.9
+    assert orc.topr_chunks(_p(orc, 16, 5, 3, 1), s).tolist() == [1, 2, 3, 9, 11]
+
+
 @pytest.mark.parametrize("seed", range(6))
 def test_structure_on_random_segments(orc, seed):
     rng = np.random.default_rng(100 + seed)

@@ -305,6 +305,31 @@ def test_budget_each_strategy_wins(orc):
     assert abs(sum(E_all[j, k] for j, k in enumerate(strat)) - _brute(p, orc, E_all, used)) < 1e-15
 
 
+def test_budget_bytes_closed_form(orc):
+    """floor(beta * nseg * FULL bytes): 0.3 * 32768 = 9830.4 -> 9830 and
+    0.15 * 3 * 32768 = 14745.6 -> 14745 (one rounding, then the floor)."""
+    assert orc.budget_bytes(orc.params(128, 4, 64, 8, 8, 32, 0.3), 1) == 9830
+    assert orc.budget_bytes(orc.params(128, 4, 64, 8, 8, 32, 0.15), 3) == 14745
+
+
+def test_budget_equal_efficiency_goes_to_the_lower_segment(orc):
+    """Two segments with the same errors have the same hull steps; a budget
+    that pays for one upgrade past the cheapest points gives it to segment 0
+    (ties in efficiency by the lower segment)."""
+    p = orc.params(128, 4, 64, 8, 8, 32, 0.6)
+    b = [orc.segment_bytes(p, k) for k in range(4)]       # FULL, TOK, CH, BOTH
+    E_all = np.array([[0.0, 0.2, 3.0, 1.0]] * 2)           # hull BOTH -> TOK -> FULL
+    verts, _, _ = orc.hull(p, E_all[0])
+    assert list(verts) == [BOTH, TOK, FULL]
+    nseg = 2
+    Bu = orc.budget_bytes(p, nseg)                         # 39321
+    assert 2 * b[TOK] + (b[FULL] - b[TOK]) <= Bu < 2 * b[FULL]
+    st, strat, used = orc.budget(p, E_all)
+    assert st == 0
+    # both BOTH -> TOK steps fit; then only one TOK -> FULL step: segment 0's
+    assert list(strat) == [FULL, TOK]
+
+
 def test_budget_beta_one_is_all_full(orc):
     p = orc.params(128, 4, 64, 8, 8, 32, 1.0)
     E_all = np.random.default_rng(9).random((5, 4))
@@ -330,6 +355,10 @@ def test_hull_steps(orc):
     # TOK lies above the chord BOTH -> CH -> popped
     verts, _, _ = orc.hull(p, np.array([0.0, 1.999, 0.2, 2.0]))
     assert list(verts) == [BOTH, CH, FULL]
+    # an option with the same error as the last hull point and more bytes
+    # is no better: TOK (= BOTH) and FULL (= CH) stay off the hull
+    verts, _, _ = orc.hull(p, np.array([0.0, 0.5, 0.0, 0.5]))
+    assert list(verts) == [BOTH, CH]
     # collinear middle point is popped (the <= in the pop rule)
     b = [32768, 4112, 22528, 2832]
     e_tok = 2.0 - 2.0 * (b[1] - b[3]) / (b[0] - b[3])

@@ -60,6 +60,39 @@ def test_scores_are_max_over_heads_of_kept_key_logits(orc):
     assert np.max(np.abs(score[fin] - want[fin])) < 1e-12
 
 
+def test_scores_over_every_strategy(orc):
+    """Segments packed as FULL, CH, TOK, BOTH, CH, BOTH (the oracle's own
+    packer, its selection steps not involved): every candidate's score is
+    the max over heads of the logit of its key as the test's parser reads
+    it, dropped channels zero."""
+    S, d, G, r, c = 8, 32, 4, 3, 5
+    p = orc.params(d, G, S, 8, r, c, 0.3)
+    rng = np.random.default_rng(57)
+    strat = np.array([FULL, CH, TOK, BOTH, CH, BOTH], np.int32)
+    nseg = len(strat)
+    K16 = f16(rng.standard_normal((nseg * S, d)))
+    V16 = f16(rng.standard_normal((nseg * S, d)))
+    q16 = f16(rng.standard_normal((G, d)))
+    arena, offs, o = [], [], 0
+    for j in range(nseg):
+        tidx = np.sort(rng.choice(S, r, replace=False)).astype(np.uint8)
+        cidx_all = np.stack([np.sort(rng.choice(d, c, replace=False)) for _ in range(S)]).astype(np.uint8)
+        buf = orc.pack_segment(p, strat[j], K16[j * S:(j + 1) * S], V16[j * S:(j + 1) * S], tidx, cidx_all)
+        offs.append(o)
+        arena.append(buf)
+        o += buf.size
+    res = {"nseg": nseg, "strat": strat, "arena": np.concatenate(arena), "offs": np.array(offs),
+           "used": o}
+    score, ncand = orc.select_scores(p, res["arena"], res["offs"], res["strat"], q16)
+    keys, _, slots = _candidates(orc, p, res)
+    assert ncand == len(slots) == 3 * S + 3 * r   # FULL, CH, CH keep S; TOK, BOTH, BOTH keep r
+    want = np.full(nseg * S, -np.inf)
+    want[slots] = (p.scale * (q16.astype(np.float64) @ keys.T)).max(axis=0)
+    assert np.array_equal(np.isinf(score), np.isinf(want))
+    fin = np.isfinite(want)
+    assert np.max(np.abs(score[fin] - want[fin])) < 1e-12
+
+
 def test_selection_is_a_stable_sort_by_score(orc):
     rng = np.random.default_rng(32)
     score = rng.standard_normal(200)
