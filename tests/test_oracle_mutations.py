@@ -67,10 +67,19 @@ MUTATIONS = [
     ("stage-2 candidate keys not cleared", "for (int x = 0; x < d; ++x) k[x] = 0.0;", "", 0),
     ("channel values packed from the wrong token", "kv[(int64_t)j * c + x] = K16[(int64_t)tok[j] * d + ch];",
      "kv[(int64_t)j * c + x] = K16[(int64_t)j * d + ch];", 0),
+    ("sparse keys decoded at their position, not their channel", "dot += qg[ci[x]] * orc_half_to_double(h);",
+     "dot += qg[x] * orc_half_to_double(h);", 0),
+    ("beta = 1 through the greedy, not all FULL", "if (p->beta >= 1.0) {", "if (p->beta > 1.0) {", 0),
+    ("E_TOK over the kept tokens", "if (!kept[t]) etok += s_seg[t];", "if (kept[t]) etok += s_seg[t];", 0),
+    ("hull efficiency with its sign flipped", "eff[k - 1] = (E[h[k - 1]] - E[h[k]]) / (double)dbytes[k - 1];",
+     "eff[k - 1] = (E[h[k]] - E[h[k - 1]]) / (double)dbytes[k - 1];", 0),
+    ("channel importance from k, not |k|", "e[x] = fabs(k[x]) * a[x];", "e[x] = k[x] * a[x];", 0),
+    ("lse without the max", "double lz = mx + log(sum);", "double lz = log(sum);", 0),
 ]
-# Not listed: the budget's tie rule on the step index cannot change a
-# result (a segment's hull steps have strictly decreasing efficiency, so two
-# of them never tie), so no pin can tell it apart.
+# Not listed, because they cannot change a result: the budget's tie rule on
+# the step index (a segment's hull steps have strictly decreasing
+# efficiency, so two of them never tie), and Token2Chunk gaps of length 0
+# as candidates (filling one keeps nothing more).
 
 
 def _replace_nth(src, old, new, n):

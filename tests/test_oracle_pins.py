@@ -334,6 +334,9 @@ def test_budget_beta_one_is_all_full(orc):
     p = orc.params(128, 4, 64, 8, 8, 32, 1.0)
     E_all = np.random.default_rng(9).random((5, 4))
     E_all[:, 0] = 0
+    # a segment whose channel-sparse form loses nothing: still FULL at
+    # beta = 1 (every segment is kept whole, whatever the errors)
+    E_all[2, CH] = 0.0
     st, strat, used = orc.budget(p, E_all)
     assert st == 0 and list(strat) == [FULL] * 5 and used == 5 * 32768
 
@@ -520,6 +523,50 @@ def test_decode_matches_independent_masked_dense(orc):
     Vs.append(V16[nc:].astype(np.float64))
     ref = _textbook(q16.astype(np.float64), np.concatenate(Ks), np.concatenate(Vs), p.scale)
     out = orc.decode_unit(p, res["arena"], res["offs"], res["strat"], K16[nc:], V16[nc:], q16)
+    assert np.max(np.abs(out - ref)) < 1e-12
+
+
+def test_decode_over_every_layout_with_sparse_channels(orc):
+    """Segments packed as FULL, CH, TOK, BOTH, CH, BOTH with random kept
+    tokens and random channel sets (the oracle's own packer, its selection
+    steps not involved), plus a dense tail: the decode equals softmax
+    attention over the keys the test's parser rebuilds (dropped channels
+    zero, each kept value at its own channel)."""
+    S, d, G, r, c = 8, 32, 4, 3, 5
+    p = orc.params(d, G, S, 8, r, c, 0.3)
+    rng = np.random.default_rng(58)
+    strat = np.array([FULL, CH, TOK, BOTH, CH, BOTH], np.int32)
+    nseg, tail = len(strat), 3
+    K16 = f16(rng.standard_normal((nseg * S + tail, d)))
+    V16 = f16(rng.standard_normal((nseg * S + tail, d)))
+    q16 = f16(rng.standard_normal((G, d)))
+    arena, offs, o = [], [], 0
+    for j in range(nseg):
+        tidx = np.sort(rng.choice(S, r, replace=False)).astype(np.uint8)
+        cidx_all = np.stack([np.sort(rng.choice(d, c, replace=False)) for _ in range(S)]).astype(np.uint8)
+        buf = orc.pack_segment(p, strat[j], K16[j * S:(j + 1) * S], V16[j * S:(j + 1) * S], tidx, cidx_all)
+        offs.append(o)
+        arena.append(buf)
+        o += buf.size
+    arena = np.concatenate(arena)
+    Ks, Vs = [], []
+    for j in range(nseg):
+        end = offs[j + 1] if j + 1 < nseg else o
+        t_, K_, ci_, kv_, V_ = _parse(p, orc, int(strat[j]), arena[offs[j]:end])
+        n = V_.shape[0]
+        if K_ is not None:
+            Kd = K_.view(np.float16).astype(np.float64)
+        else:
+            Kd = np.zeros((n, d))
+            for t in range(n):
+                Kd[t, ci_[t].astype(np.int64)] = kv_[t].view(np.float16).astype(np.float64)
+        Ks.append(Kd)
+        Vs.append(V_.view(np.float16).astype(np.float64))
+    nc = nseg * S
+    Ks.append(K16[nc:].astype(np.float64))
+    Vs.append(V16[nc:].astype(np.float64))
+    ref = _textbook(q16.astype(np.float64), np.concatenate(Ks), np.concatenate(Vs), p.scale)
+    out = orc.decode_unit(p, arena, np.array(offs), strat, K16[nc:], V16[nc:], q16)
     assert np.max(np.abs(out - ref)) < 1e-12
 
 
