@@ -68,7 +68,13 @@ __device__ __forceinline__ void copy_rows2(const __half* const* kr, int nk, uint
     }
 }
 
-__global__ void __launch_bounds__(128) pack_kernel(const __grid_constant__ PackArgs A) {
+// 64 threads per segment: a TOK segment's 4 KB is one 16-byte load per
+// thread and load slot, and up to 32 CTAs share an SM, so twice the bytes
+// are in flight per SM as with 128-thread CTAs (measured: 580 -> 493 us at
+// batch 16 x 128K).
+constexpr int kPackThreads = 64;
+
+__global__ void __launch_bounds__(kPackThreads) pack_kernel(const __grid_constant__ PackArgs A) {
     pdl_wait();
     const int j = blockIdx.x, u = blockIdx.y;
     const int b = u / A.Hkv, h = u % A.Hkv;
@@ -162,7 +168,7 @@ cudaError_t launch_pack(const PackLaunch& L, cudaStream_t stream) {
     a.status = L.status;
     dim3 grid(L.max_nseg, L.batch * L.shp.Hkv);
     prof_begin(stream, kProfPack);
-    cudaError_t e = launch_k(pack_kernel, grid, dim3(128), 0, stream, a);
+    cudaError_t e = launch_k(pack_kernel, grid, dim3(kPackThreads), 0, stream, a);
     if (e != cudaSuccess) return e;
     prof_end(stream, kProfPack);
     return cudaGetLastError();
