@@ -126,6 +126,39 @@ def peaks():
         return 6650.0, 1590.0, 1400.0, "fallback"
 
 
+def roofline_of(kind, amount, avg_s, hbm, tf_burst, tf_sust, src):
+    """Roofline of one kernel: `amount` algorithmic bytes ("hbm") or flops
+    ("tensor") per launch over its average launch time `avg_s`.  A tensor
+    kernel timed inside the step is held to the sustained bf16 GEMM figure
+    (the burst one, or the fallback, when no sustained figure exists), with
+    the burst fraction beside it."""
+    if kind == "tensor":
+        achieved = amount / avg_s / 1e12
+        tf_s = tf_sust if tf_sust > 0 else tf_burst
+        return {"bound": "tensor", "achieved": achieved, "peak": tf_s, "unit": "TFLOP/s",
+                "frac": achieved / tf_s,
+                "peak_source": (f"{src} bf16 sustained" if tf_sust > 0 else f"{src} bf16 burst") +
+                               " (fp16 runs at the bf16 rate; timed inside the step)",
+                "frac_of_burst": achieved / tf_burst}
+    achieved = amount / avg_s / 1e9
+    return {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+            "frac": achieved / hbm, "peak_source": f"{src} HBM copy"}
+
+
+def scoring_of(flops1, flops2, us1, us2, tf_burst, tf_sust, src):
+    """Both scoring passes together (executed MMA flops = algorithmic flops):
+    TFLOP/s over the sum of their average launch times, as a fraction of the
+    sustained bf16 figure (the passes run inside multi-millisecond steps
+    under the power cap) and of the burst figure."""
+    t12 = (us1 + us2) * 1e-6
+    tflops = (flops1 + flops2) / t12 / 1e12
+    tf_s = tf_sust if tf_sust > 0 else tf_burst
+    return {"tflops": tflops, "frac": tflops / tf_s, "peak": tf_s,
+            "peak_source": f"{src} bf16 sustained" if tf_sust > 0 else f"{src} bf16 burst",
+            "frac_of_burst": tflops / tf_burst, "burst_peak": tf_burst,
+            "pass1_tflops": flops1 / (us1 * 1e-6) / 1e12, "pass2_tflops": flops2 / (us2 * 1e-6) / 1e12}
+
+
 def dense_bytes(wl, lens):
     return sum(int(T) for T in lens) * wl.num_kv_heads * wl.head_dim * 2 * 2
 
@@ -719,36 +752,16 @@ def main():
     kind, amount, toks = work.get(dominant, ("hbm", 0.0, None))
     avg_s = kernels[dominant]["avg_us"] * 1e-6
     traffic, traffic_note = profiled_traffic(dominant, toks) if toks else (None, "not captured")
-    if kind == "tensor":
-        achieved = amount / avg_s / 1e12
-        tf_s = tf_sust if tf_sust > 0 else tf_burst
-        roof = {"bound": "tensor", "achieved": achieved, "peak": tf_s, "unit": "TFLOP/s",
-                "frac": achieved / tf_s, "traffic": traffic, "kernel": dominant,
-                "peak_source": (f"{src} bf16 sustained" if tf_sust > 0 else f"{src} bf16 burst") +
-                               " (fp16 runs at the bf16 rate; timed inside the step)",
-                "frac_of_burst": achieved / tf_burst}
-    else:
-        achieved = amount / avg_s / 1e9
-        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                "frac": achieved / hbm, "traffic": traffic, "kernel": dominant,
-                "peak_source": f"{src} HBM copy"}
+    roof = roofline_of(kind, amount, avg_s, hbm, tf_burst, tf_sust, src)
+    roof.update({"traffic": traffic, "kernel": dominant})
     roof["algorithmic_per_launch"] = amount
     roof["traffic_source"] = traffic_note
     gpu_launches = sum(v_["launches"] for v_ in kernels.values())
     # the scoring contraction, both passes (executed MMA flops = algorithmic)
     scoring = None
     if "score_pass1" in kernels and "score_pass2" in kernels:
-        t12 = (kernels["score_pass1"]["avg_us"] + kernels["score_pass2"]["avg_us"]) * 1e-6
-        sflops = flops_pass + work["score_pass2"][1]
-        # the passes run inside multi-millisecond steps under the power cap:
-        # the sustained GEMM figure is the denominator, the burst one beside it
-        tf_s = tf_sust if tf_sust > 0 else tf_burst
-        scoring = {"tflops": sflops / t12 / 1e12, "frac": sflops / t12 / 1e12 / tf_s,
-                   "peak": tf_s,
-                   "peak_source": f"{src} bf16 sustained" if tf_sust > 0 else f"{src} bf16 burst",
-                   "frac_of_burst": sflops / t12 / 1e12 / tf_burst, "burst_peak": tf_burst,
-                   "pass1_tflops": flops_pass / (kernels["score_pass1"]["avg_us"] * 1e-6) / 1e12,
-                   "pass2_tflops": work["score_pass2"][1] / (kernels["score_pass2"]["avg_us"] * 1e-6) / 1e12}
+        scoring = scoring_of(flops_pass, work["score_pass2"][1], kernels["score_pass1"]["avg_us"],
+                             kernels["score_pass2"]["avg_us"], tf_burst, tf_sust, src)
     comp_alg = compress_alg_bytes(wl, lens, used)
 
     # ---- end to end through the public API with host buffers

@@ -57,3 +57,32 @@ def test_cpu_record_extrapolates_by_units():
     assert abs(rec["extrapolated_step_s"] - 10.0 * 128 / 8) < 1e-9
     assert abs(rec["value"] - 8 * 131072 * 512 / 10.0 / 1e9) < 1e-12
     assert abs(rec["phase_share"]["scoring"] - 0.75) < 1e-12
+
+
+def test_roofline_hbm_and_tensor_peaks():
+    import bench
+    # 4.7 GB in 2.676 ms against a 6555.5 GB/s copy
+    r = bench.roofline_of("hbm", 4.7e9, 2.676e-3, 6555.5, 1595.8, 1385.2, "measured")
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s" and r["peak"] == 6555.5
+    assert abs(r["achieved"] - 4.7e9 / 2.676e-3 / 1e9) < 1e-9
+    assert abs(r["frac"] - r["achieved"] / 6555.5) < 1e-15
+    # a tensor kernel timed inside the step: sustained peak, burst beside it
+    t = bench.roofline_of("tensor", 1.1e12, 1.4e-3, 6555.5, 1595.8, 1385.2, "measured")
+    assert t["peak"] == 1385.2 and "sustained" in t["peak_source"]
+    assert abs(t["achieved"] - 1.1e12 / 1.4e-3 / 1e12) < 1e-9
+    assert abs(t["frac"] * 1385.2 - t["frac_of_burst"] * 1595.8) < 1e-9
+    # without a sustained figure the burst one is the peak
+    b = bench.roofline_of("tensor", 1.1e12, 1.4e-3, 6555.5, 1595.8, 0.0, "fallback")
+    assert b["peak"] == 1595.8 and "burst" in b["peak_source"] and b["frac"] == b["frac_of_burst"]
+
+
+def test_scoring_both_passes():
+    import bench
+    # two passes of 1.1 TFLOP in 1.4 ms and 1.6 ms: 2.2 TFLOP / 3.0 ms
+    s = bench.scoring_of(1.1e12, 1.1e12, 1400.0, 1600.0, 1595.8, 1385.2, "measured")
+    assert abs(s["tflops"] - 2.2e12 / 3.0e-3 / 1e12) < 1e-9
+    assert abs(s["frac"] - s["tflops"] / 1385.2) < 1e-15
+    assert abs(s["frac_of_burst"] - s["tflops"] / 1595.8) < 1e-15
+    assert abs(s["pass1_tflops"] - 1.1e12 / 1.4e-3 / 1e12) < 1e-9
+    assert abs(s["pass2_tflops"] - 1.1e12 / 1.6e-3 / 1e12) < 1e-9
+    assert s["peak"] == 1385.2 and s["burst_peak"] == 1595.8
