@@ -205,3 +205,47 @@ def test_chunk_params_checked(L):
         assert rc == code, (r, alpha, rc)
     p = B.params(128, 32, 8, 64, 64, 8, 32, 0.2, chunk_len=0, chunk_budget=99)
     assert _compress(p, 1, [63], [0]) == 0
+
+
+def test_switch_and_staged_host_checks(L):
+    """The staged compression and the switch reject a missing staged record,
+    an out-of-range batch and NULL bookkeeping pointers on the host, before
+    anything is launched (the fake addresses are never used)."""
+    lib = B.lib()
+    p = B.params(128, 32, 8, 64, 64, 8, 32, 0.2)
+    cc = _fake_cc()
+    st = B.kv2d_staged(8 << 20, 9 << 20, 10 << 20)
+    assert lib.kv2d_switch(C.byref(p), 1, C.byref(cc), None, None) == 1
+    assert lib.kv2d_switch(C.byref(p), 0, C.byref(cc), C.byref(st), None) == 1
+    assert lib.kv2d_switch(C.byref(p), 129, C.byref(cc), C.byref(st), None) == 1
+    assert lib.kv2d_switch(C.byref(p), 1, C.byref(cc), C.byref(B.kv2d_staged(None, 9 << 20, 10 << 20)),
+                           None) == 1
+    cc0 = B.kv2d_ccache(3 << 20, 1 << 24, 4 << 20, 1 << 12, None, 6 << 20, 7 << 20)
+    assert lib.kv2d_switch(C.byref(p), 1, C.byref(cc0), C.byref(st), None) == 1
+    bad = B.params(128, 30, 8, 64, 64, 8, 32, 0.2)          # Hq not a multiple of Hkv
+    assert lib.kv2d_switch(C.byref(bad), 1, C.byref(cc), C.byref(st), None) == 1
+    seq = (C.c_int32 * 1)(4096)
+    ce = (C.c_int32 * 1)(0)
+    d = _fake_dense()
+    assert lib.kv2d_compress_staged(C.byref(p), 1, seq, ce, C.byref(d), 8 << 20, C.byref(cc), None,
+                                    9 << 20, 1 << 30, None, None) == 1
+    assert "staged" in B.kv2d_last_error()
+
+
+def test_select_decode_host_checks(L):
+    """The selection decode rejects a non-positive or non-finite rate, a
+    group wider than 8 and a length beyond the capacity on the host, before
+    anything is launched."""
+    lib = B.lib()
+    p = B.params(128, 32, 8, 64, 64, 8, 32, 0.2)
+    cc = _fake_cc()
+    d = _fake_dense()
+    args = (1 << 22, 4096, 1 << 23, 1 << 24)
+    for rate in (0.0, -0.1, float("nan"), float("inf")):
+        assert lib.kv2d_decode_attn_select(C.byref(p), 1, C.byref(cc), C.byref(d), *args, rate,
+                                           9 << 20, 1 << 30, None, None, None) == 1
+    assert lib.kv2d_decode_attn_select(C.byref(p), 1, C.byref(cc), C.byref(d), 1 << 22, 5000,
+                                       1 << 23, 1 << 24, 0.1, 9 << 20, 1 << 30, None, None, None) == 1
+    wide = B.params(128, 128, 8, 64, 16, 8, 32, 0.2)        # G = 16
+    assert lib.kv2d_decode_attn_select(C.byref(wide), 1, C.byref(cc), C.byref(d), *args, 0.1,
+                                       9 << 20, 1 << 30, None, None, None) == 6
