@@ -26,7 +26,7 @@ TOL_OUT = 2e-3
 
 
 @dataclass
-class GpuRun:
+class GpuCase:
     wl: synth.Workload
     batch: synth.Batch
     p: B.kv2d_params
@@ -69,10 +69,10 @@ def make_run(wl, batch_dev, p, max_tokens=None):
         dv = B.dense(batch_dev.k, batch_dev.v)
     seq = batch_dev.seq_len.to(torch.int32).cuda()
     ws = B.workspace(B.kv2d_workspace_bytes(p, B.OP_COMPRESS, B_, max_tokens))
-    return GpuRun(wl, batch_dev, p, cc, dv, seq, [0] * B_, {}, ws)
+    return GpuCase(wl, batch_dev, p, cc, dv, seq, [0] * B_, {}, ws)
 
 
-def compress(run: GpuRun, seq_host=None, expect_bits=0):
+def compress(run: GpuCase, seq_host=None, expect_bits=0):
     wl, p = run.wl, run.p
     Bn = wl.batch
     seq_host = [int(x) for x in (seq_host if seq_host is not None else run.seq_len.cpu().tolist())]
@@ -102,17 +102,17 @@ def compress(run: GpuRun, seq_host=None, expect_bits=0):
     return run
 
 
-def unit_inputs(run: GpuRun, b: int, h: int, t0: int, t1: int):
+def unit_inputs(run: GpuCase, b: int, h: int, t0: int, t1: int):
     k, v = synth.dense_rows(run.batch, b, h, t0, t1)
     return k.cpu().numpy(), v.cpu().numpy()
 
 
-def unit_qw(run: GpuRun, b: int, h: int):
+def unit_qw(run: GpuCase, b: int, h: int):
     G, W, d = run.wl.group, run.wl.window, run.wl.head_dim
     return run.batch.qw[b, h * G:(h + 1) * G].reshape(G * W, d).cpu().numpy()
 
 
-def oracle_scores(orc, run: GpuRun, b: int, h: int, threads=None):
+def oracle_scores(orc, run: GpuCase, b: int, h: int, threads=None):
     """The oracle's own a_d, lse and s_t of unit (b, h) for the latest
     compress() call, scored one query head at a time on host threads: head
     g's W window rows are an independent single-head problem over the same
@@ -137,7 +137,7 @@ def oracle_scores(orc, run: GpuRun, b: int, h: int, threads=None):
     return orc.win_stats(po, qw), lse, s
 
 
-def check_scores(run: GpuRun, b: int, h: int, scores):
+def check_scores(run: GpuCase, b: int, h: int, scores):
     """a_d, lse and s_t of unit (b, h) against the oracle's (a, lse, s)."""
     wl = run.wl
     a_ref, lse_ref, s_ref = scores
@@ -157,7 +157,7 @@ def check_scores(run: GpuRun, b: int, h: int, scores):
     return float(np.max(err))
 
 
-def end_to_end_unit(orc, run: GpuRun, b: int, h: int, scores, q: torch.Tensor):
+def end_to_end_unit(orc, run: GpuCase, b: int, h: int, scores, q: torch.Tensor):
     """The fully independent end-to-end oracle for unit (b, h): the oracle's
     own a_d and s_t (scores), its own selection and packing of the region of
     the latest compress() call, and its decode of q over that arena plus the
@@ -191,7 +191,7 @@ def end_to_end_unit(orc, run: GpuRun, b: int, h: int, scores, q: torch.Tensor):
     return (agree, nseg), o_ref
 
 
-def check_compress_unit(orc, run: GpuRun, b: int, h: int, independent: bool = True,
+def check_compress_unit(orc, run: GpuCase, b: int, h: int, independent: bool = True,
                         arena_before=None, scores=None):
     """Parity of one unit after the latest compress() call.  With scores
     (the oracle's (a, lse, s), e.g. from oracle_scores) those are compared
@@ -251,7 +251,7 @@ def check_compress_unit(orc, run: GpuRun, b: int, h: int, independent: bool = Tr
     return dict(strat=ref["strat"], nseg=nseg)
 
 
-def gpu_decode(run: GpuRun, q: torch.Tensor, cc: B.CompressedCache | None = None,
+def gpu_decode(run: GpuCase, q: torch.Tensor, cc: B.CompressedCache | None = None,
                max_seq=None, expect_bits=0):
     wl, p = run.wl, run.p
     cc = cc or run.cc
@@ -267,7 +267,7 @@ def gpu_decode(run: GpuRun, q: torch.Tensor, cc: B.CompressedCache | None = None
     return out
 
 
-def oracle_decode_unit(orc, run: GpuRun, b: int, h: int, q: torch.Tensor,
+def oracle_decode_unit(orc, run: GpuCase, b: int, h: int, q: torch.Tensor,
                        cc: B.CompressedCache | None = None):
     """Oracle decode of unit (b, h) over the arena and descriptors the cache
     holds (bytes already proven equal to the oracle's own packing)."""
@@ -289,7 +289,7 @@ def oracle_decode_unit(orc, run: GpuRun, b: int, h: int, q: torch.Tensor,
     return orc.decode_unit(po, arena, offs, strat, Kt, Vt, qh)
 
 
-def unit_cache(run: GpuRun, b: int, h: int, cc: B.CompressedCache | None = None):
+def unit_cache(run: GpuCase, b: int, h: int, cc: B.CompressedCache | None = None):
     """The packed bytes, offsets and strategies of unit (b, h) and the dense
     tail rows after its segments."""
     cc = cc or run.cc
@@ -306,7 +306,7 @@ def unit_cache(run: GpuRun, b: int, h: int, cc: B.CompressedCache | None = None)
     return arena, offs, strat, Kt, Vt
 
 
-def gpu_decode_select(run: GpuRun, q: torch.Tensor, rate: float, max_seq=None):
+def gpu_decode_select(run: GpuCase, q: torch.Tensor, rate: float, max_seq=None):
     """kv2d_decode_attn_select with its per-slot scores and kept flags."""
     wl, p = run.wl, run.p
     ms = max_seq or run.batch.capacity
