@@ -814,9 +814,11 @@ __global__ void __launch_bounds__(128) chan_kernel_generic(const __grid_constant
 // largest, which a bitonic merge sorts again; one more such split gives the
 // 32 largest keys of all 128 and v, the c-th largest.  Channels with key > v
 // are in and those below are out.  When more than c keys are >= v, the keys
-// equal to v straddle the cut and are ranked exactly by (e desc, x asc) with
-// the fp64 products.  The keys stay in shared memory between the sort and
-// the membership pass, so the sort alone holds the registers.
+// equal to v straddle the cut and are ranked exactly by (e desc, x asc): by
+// their fp32 products, and by the exact fp64 products only where those tie
+// (one pass over them when a single one is kept or dropped).  The membership
+// pass forms the keys again from the K tile instead of keeping them, so
+// only the sort holds them in registers.
 
 __device__ __forceinline__ void ce2(__half2& a, __half2& b) {
     const __half2 hi = __hmax2(a, b), lo = __hmin2(a, b);
